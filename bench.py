@@ -1,0 +1,482 @@
+"""Benchmark of the block-sparse attention forward path on B200.
+
+One step = the whole path over one batch of synthetic input already resident
+in HBM: layout build, reorder of Q, K, V, mask prediction (pooling, similarity
+guard, compressed softmax + TopCdf, forced blocks, CSR lists, work order),
+block-sparse attention with the PV skip, inverse reorder of O and LSE.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload video]
+                    [--impl ours|reference]
+
+Default workload: the video DiT attention (B=1, 24 heads, latent [13,30,52]
++ 226 text tokens, N = 20,506, d = 128, bf16, [2,8,8] windows, first-frame
+sink, text forced, bq = 128, bk = 64, block sparsity 0.80, lambda = -5).
+
+The metric is kept-block TFLOP/s: 4*d*(valid query x key pairs of the kept
+tiles), the PV half counted only for tiles whose PV product ran, divided by
+the device time of one step (CUDA events, L2 flushed between steps).  N > 1
+ranks (torchrun) run independent replicas (the path has no exchange step);
+value = all ranks' FLOPs / the slowest rank's time.
+
+--impl reference times the fp64 CPU oracle (the plain restatement of the
+method that the tests check the kernels against) on the same workload, one
+bounded sample of query blocks per step, on this host's cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse attn fwd ms & TFLOP/s (kept blocks) vs dense, N=20.5K video, 1×B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per launch of the attention kernel from the ncu capture recorded
+# in profiles/attn_tc_video.md, keyed by the sha1 of the kernel source it was
+# taken on; any other source reports null.
+TRAFFIC = {}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def src_sha1(name):
+    with open(os.path.join(ROOT, "long_context_mean_b200", "csrc", name), "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# FLOP accounting (algorithmic, from the mask lists and the PV-skip log)
+# ----------------------------------------------------------------------------
+
+def kept_flops(w, row_ptr, col_idx, skip, nqb):
+    """4 * d * pairs split in QK (all kept tiles) and PV (unskipped tiles),
+    pairs = valid query rows x valid (causally visible) keys of each tile."""
+    import numpy as np
+    N, bq, bk = w.N, w.bq, w.bk
+    R = len(row_ptr) - 1
+    qb = np.arange(R) % nqb
+    counts = np.diff(row_ptr)
+    rows = np.repeat(np.minimum(bq, N - qb * bq), counts)
+    qbs = np.repeat(qb, counts)
+    kb = col_idx[:row_ptr[-1]].astype(np.int64)
+    cols = np.minimum(bk, N - kb * bk)
+    if w.causal:
+        i0 = qbs * bq
+        pairs = np.zeros_like(kb)
+        for r in range(bq):                      # rows of the block, vectorised over tiles
+            i = i0 + r
+            ok = i < N
+            vis = np.clip(i - kb * bk + 1, 0, cols)
+            pairs += np.where(ok, vis, 0)
+    else:
+        pairs = rows * cols
+    qk = 2.0 * w.d * float(pairs.sum())
+    pv = 2.0 * w.dv * float(pairs[skip[:row_ptr[-1]] == 0].sum())
+    return qk, pv
+
+
+# ----------------------------------------------------------------------------
+# Our arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from long_context_mean_b200 import inputs as I
+    from long_context_mean_b200 import sa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = I.WORKLOADS[args.workload]
+    g = I.gen_qkv(w)
+    host = {n: torch.from_numpy(g[n + "_bits"].view(np.int16)).view(torch.bfloat16).pin_memory() for n in "qkv"}
+    q, k, v = (host[n].to(dev) for n in "qkv")
+    stream = torch.cuda.current_stream(dev)
+    pipe = sa.pipeline_for(w, device=dev, log_skips=True)
+
+    # Calibration pass (untimed): mask, skip log, FLOPs, sparsity.
+    pipe.run(q, k, v)
+    st = pipe.status()
+    if st != sa.SA_OK:
+        raise RuntimeError(f"device status {sa.STATUS_NAMES.get(st, st)}")
+    rp = pipe.mask.row_ptr.cpu().numpy().astype(np.int64)
+    ci = pipe.mask.col_idx.cpu().numpy()
+    skip = pipe.skip_log.cpu().numpy()
+    nqb, nkb = pipe.mask.struct.nqb, pipe.mask.struct.nkb
+    qk_flops, pv_flops = kept_flops(w, rp, ci, skip, nqb)
+    flops = qk_flops + pv_flops
+    kept = int(rp[-1])
+    R = w.B * w.Hq * nqb
+    if w.causal:
+        valid_tiles = w.B * w.Hq * sum(min(nkb, (min(w.N, (qb + 1) * w.bq) - 1) // w.bk + 1) for qb in range(nqb))
+    else:
+        valid_tiles = R * nkb
+    sparsity = 1.0 - kept / valid_tiles
+    pv_skipped = int(skip[:kept].sum())
+    pipe.skip_log = None                      # timed steps run without the log
+
+    # L2 flush buffer (larger than the 126 MB L2).
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def l2_flush():
+        flush.fill_(1.0)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step_timed():
+        """One step with per-stage events; returns (total_ms, attn_ms)."""
+        e = [ev() for _ in range(4)]
+        e[0].record(stream)
+        if not pipe.identity:
+            sa.layout_build(pipe.layout, pipe.perm, pipe.inv, pipe.layout_ws)
+            sa.reorder(pipe.perm, q, pipe.qr)
+            sa.reorder(pipe.perm, k, pipe.kr)
+            sa.reorder(pipe.perm, v, pipe.vr)
+            qr, kr, vr, out_r, lse_r = pipe.qr, pipe.kr, pipe.vr, pipe.out_r, pipe.lse_r
+        else:
+            qr, kr, vr, out_r, lse_r = q, k, v, pipe.out, pipe.lse
+        sa.predict_mask(qr, kr, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
+        e[1].record(stream)
+        sa.block_sparse_attn(qr, kr, vr, pipe.shape, pipe.mask.struct, pipe.lam, pipe.scale, out_r, lse_r)
+        e[2].record(stream)
+        if not pipe.identity:
+            sa.unreorder(pipe.perm, out_r, pipe.out)
+            sa.unreorder(pipe.perm, lse_r, pipe.lse)
+        e[3].record(stream)
+        return e
+
+    launches_per_step = (0 if pipe.identity else (1 if w.order != "hilbert" else 3) + 3 + 2) + 6 + 1
+
+    for _ in range(args.warmup):
+        l2_flush()
+        step_timed()
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    recs = []
+    wall0 = time.perf_counter()
+    for _ in range(args.steps):
+        l2_flush()
+        recs.append(step_timed())
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop() if clocks else None
+    step_ms = [r[0].elapsed_time(r[3]) for r in recs]
+    attn_ms = [r[1].elapsed_time(r[2]) for r in recs]
+    pre_ms = [r[0].elapsed_time(r[1]) for r in recs]
+    post_ms = [r[2].elapsed_time(r[3]) for r in recs]
+    total_ms = sum(step_ms)
+    st = pipe.status()
+    if st != sa.SA_OK:
+        raise RuntimeError(f"device status after timing {sa.STATUS_NAMES.get(st, st)}")
+
+    # Dense reference kernel at the same shape (the speedup's denominator).
+    od = torch.empty_like(pipe.out)
+    ld = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=dev)
+    dst = torch.zeros(1, dtype=torch.int32, device=dev)
+    qr, kr, vr = (pipe.qr, pipe.kr, pipe.vr) if not pipe.identity else (q, k, v)
+    dense = []
+    for i in range(args.warmup + max(3, min(args.steps, 10))):
+        l2_flush()
+        a, b = ev(), ev()
+        a.record(stream)
+        sa.dense_attn(qr, kr, vr, pipe.shape, w.causal, 0.0, od, ld, dst)
+        b.record(stream)
+        if i >= args.warmup:
+            dense.append((a, b))
+    torch.cuda.synchronize(dev)
+    dense_ms = statistics.median(x[0].elapsed_time(x[1]) for x in dense)
+
+    # End to end through the public API with host buffers: pinned H2D of
+    # Q, K, V, the step, D2H of O and LSE.
+    out_host = torch.empty(pipe.out.shape, dtype=pipe.out.dtype).pin_memory()
+    lse_host = torch.empty(pipe.lse.shape, dtype=pipe.lse.dtype).pin_memory()
+    qd, kd, vd = (torch.empty_like(x) for x in (q, k, v))
+
+    def e2e_step():
+        qd.copy_(host["q"], non_blocking=True)
+        kd.copy_(host["k"], non_blocking=True)
+        vd.copy_(host["v"], non_blocking=True)
+        out, lse = pipe.run(qd, kd, vd)
+        out_host.copy_(out, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e = []
+    for _ in range(args.steps):
+        l2_flush()
+        a, b = ev(), ev()
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        e2e.append((a, b))
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(x[0].elapsed_time(x[1]) for x in e2e) / len(e2e)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in "qkv")
+    d2h = out_host.numel() * out_host.element_size() + lse_host.numel() * lse_host.element_size()
+
+    # Max over ranks.
+    mean_ms = total_ms / args.steps
+    vals = torch.tensor([mean_ms, statistics.mean(attn_ms), e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    mean_ms, attn_mean, e2e_ms = (float(x) for x in vals.tolist())
+    if rank != 0:
+        return None
+
+    pk, pk_src = peaks()
+    peak_tf = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    attn_tf = flops / (attn_mean * 1e-3) / 1e12
+    sha = src_sha1("attn_tc.cu")
+    traffic = TRAFFIC.get((sha, args.workload))
+    res = {
+        "metric": METRIC,
+        "value": round(world * flops / (mean_ms * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(mean_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded smooth-field generator, bf16)",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.Hq} N={w.N} ([{w.T},{w.H},{w.W}]+{w.txt_len} text) "
+                               f"d={w.d} {w.order}{list(w.win) if w.order == 'window' else ''} sink_frames={w.sink_frames} "
+                               f"bq={w.bq} bk={w.bk} tau={w.tau} theta={w.theta} lambda={w.lam}",
+                   "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (256 MB write)"},
+        "stages_ms": {"layout_reorder_predict": round(statistics.mean(pre_ms), 4),
+                      "attention": round(statistics.mean(attn_ms), 4),
+                      "unreorder": round(statistics.mean(post_ms), 4)},
+        "attn_ms": round(attn_mean, 4),
+        "attn_tflops": round(attn_tf, 2),
+        "dense_ms": round(dense_ms, 4),
+        "speedup_vs_dense": round(dense_ms / attn_mean, 3),
+        "speedup_vs_dense_whole_step": round(dense_ms / mean_ms, 3),
+        "block_sparsity": round(sparsity, 4),
+        "kept_tiles": kept,
+        "pv_skipped_tiles": pv_skipped,
+        "flops_per_step": {"qk": qk_flops, "pv": pv_flops},
+        "roofline": {"bound": "tensor", "achieved": round(attn_tf, 2), "peak": peak_tf,
+                     "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4), "traffic": traffic,
+                     "peak_source": f"{pk_src} bf16 dense (burst)", "kernel": "attn_tc_kernel<64>"},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "wall_s": round(wall, 3),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, g, seconds=args.cpu_seconds)
+    return res
+
+
+# ----------------------------------------------------------------------------
+# The oracle on the host cores (CPU baseline and the reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_sample_setup(w, g):
+    """Oracle layout + mask for the first kv head (one predict pass, fp64)."""
+    import numpy as np
+    from oracle import layout as Y
+    from oracle import predict as Pr
+    perm, _ = Y.build_layout(w.order, w.T, w.H, w.W, w.win, w.sink_frames, w.txt_len)
+    q = Y.reorder(g["q"][:1, :1], perm)
+    k = Y.reorder(g["k"][:1, :1], perm)
+    v = Y.reorder(g["v"][:1, :1], perm)
+    r = Pr.predict_mask(q, k, w.bq, w.bk, w.tau, w.theta, w.causal, w.sink_tokens, w.txt_len,
+                        w.local_window, w.anchor_tokens)
+    return q, k, v, r["mask"]
+
+
+def oracle_step(w, qkvm, qblocks):
+    """The oracle's block-sparse attention on the given q-blocks of head 0;
+    returns its kept-block FLOPs (QK + unskipped PV)."""
+    from oracle import attention as A
+    q, k, v, m = qkvm
+    res = A.block_sparse_attention(q[0, 0], k[0, 0], v[0, 0], m[0, 0], w.bq, w.bk, w.causal, w.lam,
+                                   qblocks=qblocks)
+    fl = 0.0
+    for (qb, kb), sk in res["skips"].items():
+        rows = min(w.bq, w.N - qb * w.bq)
+        cols = min(w.bk, w.N - kb * w.bk)
+        fl += 2.0 * w.d * rows * cols + (0.0 if sk else 2.0 * w.dv * rows * cols)
+    return fl
+
+
+def cores_used():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, g, seconds=15.0):
+    import numpy as np
+    qkvm = oracle_sample_setup(w, g)
+    nqb = -(-w.N // w.bq)
+    order = list(np.random.default_rng(0).permutation(nqb))
+    fl, blocks, t0 = 0.0, 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds and blocks < nqb:
+        fl += oracle_step(w, qkvm, [int(order[blocks])])
+        blocks += 1
+    dt = time.perf_counter() - t0
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
+            "sample": f"fp64 oracle block-sparse attention of {blocks} random query blocks of head 0 "
+                      f"(mask predicted by the oracle for that head), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from long_context_mean_b200 import inputs as I
+    w = I.WORKLOADS[args.workload]
+    g = I.gen_qkv(w, heads=[0], batches=[0])
+    qkvm = oracle_sample_setup(w, g)
+    nqb = -(-w.N // w.bq)
+    per_step = max(1, args.ref_qblocks)
+    for i in range(args.warmup):
+        oracle_step(w, qkvm, [(i * 7) % nqb])
+    fl, t0 = 0.0, time.perf_counter()
+    for s in range(args.steps):
+        fl += oracle_step(w, qkvm, [((s * per_step + j) * 13) % nqb for j in range(per_step)])
+    dt = time.perf_counter() - t0
+    value = fl / dt / 1e12
+    sample = (f"fp64 oracle block-sparse attention, {per_step} query blocks of head 0 per step "
+              f"(mask predicted by the oracle for that head)")
+    return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "seq_len": w.N, "parallelism": "host cores"},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="video")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-qblocks", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local_rank))
+        try:
+            res = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

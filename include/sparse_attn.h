@@ -1,0 +1,228 @@
+/*
+ * sparse_attn.h -- C ABI of libsparseattn.so: training-free block-sparse
+ * attention forward on NVIDIA B200 (sm_100a).
+ *
+ * The path, in call order:
+ *   sa_layout_build  -> token permutation (identity, [t,h,w] windows, Hilbert)
+ *   sa_reorder       -> Q, K, V gathered into the permuted order
+ *   sa_predict_mask  -> block mask M_g + CSR kept lists + work order
+ *   sa_block_sparse_attn -> O and per-row LSE over the kept blocks
+ *   sa_unreorder     -> O (and LSE) scattered back to the original order
+ *   sa_dense_attn    -> the same kernel with every block kept (reference)
+ *
+ * Sources of the operations (page title, section):
+ *   [P1] "AIGC 基本功｜视频稀疏注意力的误差与布局" (jefxiong.cn)
+ *        3.1 restricted softmax, 3.4 permutation equivariance, 4 block ledger.
+ *   [P2] MindIE-SD documentation "稀疏": rf_v2 block representatives,
+ *        [t,h,w] window reorder, first-frame sink; sparse_attention(q, k, v,
+ *        head_num, input_layout="BNSD", sparsity, txt_len, latent_shape...).
+ *   [P3] "SpargeAttention：中文精读笔记": 2.1 sparse FlashAttention (online
+ *        softmax m/l/O, M_g), 2.2 selective token compression (mean pooling,
+ *        CosSim guard theta, TopCdf tau, forced rows/columns), 2.3 PV skip
+ *        with lambda, 2.5 Hilbert permutation.
+ *   [P4] "44. Local Sliding and Sparse Attention": local causal window,
+ *        block pairs with causal filter.
+ *   [P5] "78. Attention Access Pattern Benchmark": window + anchor keys.
+ *
+ * Conventions (every entry point):
+ *   - Tensors are BNSD and contiguous: q [B, Hq, N, d], k [B, Hkv, N, d],
+ *     v [B, Hkv, N, dv], out [B, Hq, N, dv], lse [B, Hq, N] (fp32, natural
+ *     log).  Query head h reads kv head h / (Hq / Hkv).
+ *   - Every pointer argument to data is a DEVICE pointer unless stated;
+ *     struct arguments are HOST pointers.  The caller owns all memory; the
+ *     library never allocates device memory and keeps no state between
+ *     calls except a thread-local error string.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     enqueued asynchronously on it.  Argument errors are detected on the
+ *     host and returned synchronously before anything is enqueued; errors
+ *     found by a kernel (empty row, list capacity, wait timeout) are written
+ *     to a device status word and read back with sa_read_status().
+ *   - Nothing falls back to the CPU: without a usable CUDA device every
+ *     compute entry point returns SA_ERR_CUDA.
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,   /* bad pointer, size, or parameter value        */
+  SA_ERR_UNSUPPORTED = 2,   /* valid, but outside the kernels' shapes       */
+  SA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than queried    */
+  SA_ERR_EMPTY_ROW = 4,     /* a query row would keep no key ([P1] 3.1)     */
+  SA_ERR_TIMEOUT = 5,       /* a bounded device wait gave up                */
+  SA_ERR_CUDA = 6,          /* a CUDA runtime call failed (see last_error)  */
+  SA_ERR_CAPACITY = 7       /* kept blocks exceed mask->col_capacity        */
+} sa_status;
+
+typedef enum { SA_BF16 = 0, SA_FP32 = 1 } sa_dtype;
+
+/* Problem shape.  dtype applies to q, k, v and out. */
+typedef struct {
+  int64_t B, Hq, Hkv, N, d, dv;
+  int32_t dtype;
+  int32_t reserved;
+} sa_shape;
+
+typedef enum {
+  SA_ORDER_IDENTITY = 0,
+  SA_ORDER_WINDOW = 1,   /* [P2] [t,h,w] windows of size win[0..2]          */
+  SA_ORDER_HILBERT = 2   /* [P3] 2.5; Skilling's curve on the 2^b cube      */
+} sa_order;
+
+/* Token layout: N = T*H*W + txt_len tokens, raster frame-major video tokens
+ * (i = t*H*W + h*W + w) followed by text tokens.  The first sink_frames
+ * frames and the text tokens keep their positions; the remaining frames are
+ * reordered.  Window mode: windows tile the frames after the sink in raster
+ * order of window coordinates, tokens raster-ordered inside a window, edge
+ * windows smaller.  Hilbert mode: tokens sorted by the index of (t', h, w)
+ * on the 2^b cube, b = ceil(log2(max(T - sink_frames, H, W))), t' most
+ * significant; b <= 9. */
+typedef struct {
+  int64_t T, H, W, txt_len, sink_frames;
+  int64_t win[3];
+  int32_t mode;          /* sa_order */
+  int32_t reserved;
+} sa_layout_desc;
+
+/* Mask prediction parameters ([P3] 2.2, [P2], [P5]).
+ *   bq, bk        query / key block sizes (1..128).
+ *   tau           TopCdf threshold in (0, 1]: a block is kept iff the
+ *                 probability mass sorted before it is < tau * row total.
+ *   theta         similarity guard; blocks whose mean pairwise cosine is
+ *                 < theta get forced full rows (queries) or columns (keys)
+ *                 and key blocks below theta leave the compressed softmax.
+ *                 theta <= 0 disables the guard.
+ *   sink_tokens   tokens at the front whose blocks get full rows+columns.
+ *   txt_len       tokens at the back whose blocks get full rows+columns.
+ *   local_window  w > 0 keeps every block pair holding some (i, j) with
+ *                 0 <= i - j < w ([P4], block level); 0 = off.
+ *   anchor_tokens tokens at the front whose key blocks get full columns.
+ *   causal        1 = key j visible to query i only if j <= i. */
+typedef struct {
+  int32_t bq, bk;
+  float tau, theta;
+  int64_t sink_tokens, txt_len, local_window, anchor_tokens;
+  int32_t causal;
+  int32_t reserved;
+} sa_mask_params;
+
+/* A block mask and its compacted lists.  All pointers are device buffers
+ * owned by the caller and sized by the caller:
+ *   block_mask  uint8 [B*Hq, nqb, nkb], 1 = kept
+ *   row_ptr     int32 [B*Hq*nqb + 1], CSR offsets into col_idx
+ *   col_idx     int32 [col_capacity], kept key blocks, ascending per row
+ *   order       int32 [B*Hq*nqb], rows by descending kept count, ties by
+ *               ascending row index (work order of the attention kernel)
+ *   kept_total  int64 [1]
+ *   status      int32 [1], device status word (sa_status code, 0 = OK)
+ * The producer (sa_predict_mask / sa_mask_from_blocks) fills nqb, nkb, bq,
+ * bk, causal.  A row index is (b*Hq + h)*nqb + qb.  col_capacity of
+ * B*Hq*nqb*nkb always suffices. */
+typedef struct {
+  uint8_t* block_mask;
+  int32_t* row_ptr;
+  int32_t* col_idx;
+  int32_t* order;
+  int64_t* kept_total;
+  int32_t* status;
+  int64_t col_capacity;
+  int64_t nqb, nkb;
+  int32_t bq, bk, causal;
+  int32_t reserved;
+} sa_mask;
+
+/* Flags for the attention entry points. */
+#define SA_FLAG_FORCE_SIMT 1   /* use the portable CUDA-core kernel even where
+                                  the tensor-core kernel applies (testing) */
+
+/* Library version string and the calling thread's last error message. */
+const char* sa_version(void);
+const char* sa_last_error(void);
+
+/* Which attention kernel serves a shape: 1 = tcgen05 tensor-core kernel
+ * (bf16, d = dv = 128, bq = 128, bk in {64, 128}), 0 = CUDA-core kernel,
+ * -1 = unsupported. */
+int32_t sa_attn_kernel_path(const sa_shape* shape, int32_t bq, int32_t bk, int32_t flags);
+
+/* ---- a0: layout ([P2] window reorder; [P3] 2.5 Hilbert) ----------------
+ * perm[n] = source index of output position n; inv[perm[n]] = n.  Both are
+ * int32 [N] device buffers.  Window and identity modes need no workspace;
+ * Hilbert mode needs sa_layout_workspace() bytes (256-byte aligned). */
+size_t sa_layout_workspace(const sa_layout_desc* desc);
+sa_status sa_layout_build(const sa_layout_desc* desc, int32_t* perm, int32_t* inv,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* ---- a1/a7: reorder ([P1] 3.4) -------------------------------------------
+ * x, y are [outer, N, row] arrays of `row` elements of `dtype` per token
+ * (outer = B*H).  sa_reorder: y[o, n, :] = x[o, perm[n], :].
+ * sa_unreorder: x[o, perm[n], :] = y[o, n, :] (pass the same perm).
+ * x and y must not overlap.  row = 1 with SA_FP32 reorders LSE. */
+sa_status sa_reorder(const int32_t* perm, const void* x, void* y, int64_t outer,
+                     int64_t N, int64_t row, int32_t dtype, void* stream);
+sa_status sa_unreorder(const int32_t* perm, const void* y, void* x, int64_t outer,
+                       int64_t N, int64_t row, int32_t dtype, void* stream);
+
+/* ---- a2-a4: mask prediction ([P3] 2.2) -----------------------------------
+ * Pools q and k per block (mean over the block's real tokens), computes the
+ * mean pairwise cosine of each block, scores the compressed matrix
+ * q_hat k_hat^T / sqrt(d) (ineligible key blocks -inf), softmaxes and
+ * TopCdf-selects each row, ORs in the forced rows/columns, sink, text,
+ * anchors and local window, ANDs causal validity, checks that every query
+ * row keeps a key, and builds the CSR lists and work order into *out.
+ * Needs d a power of two with d*elem_size a multiple of 16 and d <= 256,
+ * N/bk <= 4095.  ws: sa_predict_mask_workspace() bytes, 256-byte aligned;
+ * its layout (pooled means and similarities, fp32) is reported by
+ * sa_predict_mask_ws_layout() for inspection. */
+size_t sa_predict_mask_workspace(const sa_shape* shape, const sa_mask_params* params);
+sa_status sa_predict_mask_ws_layout(const sa_shape* shape, const sa_mask_params* params,
+                                    size_t offsets[6]);
+sa_status sa_predict_mask(const void* q, const void* k, const sa_shape* shape,
+                          const sa_mask_params* params, void* ws, size_t ws_bytes,
+                          sa_mask* out, void* stream);
+
+/* A caller-supplied block mask (uint8 [B*Hq, nqb, nkb], nonzero = kept) is
+ * ANDed with causal validity, copied to out->block_mask (may alias), checked
+ * for empty rows and compacted into lists exactly as sa_predict_mask does. */
+size_t sa_mask_from_blocks_workspace(const sa_shape* shape, int32_t bq, int32_t bk);
+sa_status sa_mask_from_blocks(const uint8_t* block_mask, const sa_shape* shape, int32_t bq,
+                              int32_t bk, int32_t causal, void* ws, size_t ws_bytes,
+                              sa_mask* out, void* stream);
+
+/* ---- a5/a6: block-sparse attention ([P3] 2.1, 2.3) -----------------------
+ * For every query block, visits its kept key blocks in ascending order with
+ * the online-softmax recurrence; skips P~V of a tile when the largest
+ * (tile row max - running row max) over the block's rows is < lambda
+ * (lambda = -INFINITY disables the skip; the normaliser l still counts the
+ * tile).  scale = 0 means 1/sqrt(d).  out gets O / l in the input dtype,
+ * lse (nullable) gets m + ln l.  pv_skip_log (nullable) gets one byte per
+ * kept tile in CSR order, 1 = PV skipped.  The mask's status word also
+ * receives kernel errors. */
+sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v,
+                               const sa_shape* shape, const sa_mask* mask, float lambda,
+                               float scale, void* out, float* lse, uint8_t* pv_skip_log,
+                               int32_t flags, void* stream);
+
+/* ---- a8: dense reference --------------------------------------------------
+ * The same recurrence with every (causally valid) key visible and no lists
+ * (lambda = -inf); the library picks the tile shape.  status (device int32,
+ * nullable) receives kernel errors. */
+sa_status sa_dense_attn(const void* q, const void* k, const void* v, const sa_shape* shape,
+                        int32_t causal, float scale, void* out, float* lse, int32_t* status,
+                        int32_t flags, void* stream);
+
+/* Synchronises `stream` and returns the device status word's code (0 =
+ * SA_OK).  The word is not cleared. */
+sa_status sa_read_status(const int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

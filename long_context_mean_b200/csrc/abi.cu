@@ -1,0 +1,315 @@
+// The C ABI of libsparseattn.so: argument validation, workspace sizing and
+// dispatch to the kernels.  Every check here runs on the host before any
+// work is enqueued; nothing allocates device memory.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+
+#include "sa_internal.cuh"
+
+namespace sa {
+
+namespace {
+thread_local char g_err[768] = "";
+}
+
+sa_status set_error(sa_status code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+sa_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(SA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return SA_OK;
+}
+
+}  // namespace sa
+
+using namespace sa;
+
+namespace {
+
+sa_status check_shape(const sa_shape* s) {
+  if (!s) return set_error(SA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B <= 0 || s->Hq <= 0 || s->Hkv <= 0 || s->N <= 0 || s->d <= 0 || s->dv <= 0)
+    return set_error(SA_ERR_INVALID_ARG, "shape sizes must be positive");
+  if (s->Hq % s->Hkv != 0) return set_error(SA_ERR_INVALID_ARG, "Hq must be a multiple of Hkv");
+  if (s->dtype != SA_BF16 && s->dtype != SA_FP32) return set_error(SA_ERR_INVALID_ARG, "unknown dtype");
+  if (s->N > (int64_t)INT32_MAX / 2) return set_error(SA_ERR_UNSUPPORTED, "N too large");
+  return SA_OK;
+}
+
+sa_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return set_error(SA_ERR_CUDA, "no usable CUDA device");
+  }
+  return SA_OK;
+}
+
+bool is_sm100() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  return major == 10;
+}
+
+int elem_size(int32_t dtype) { return dtype == SA_BF16 ? 2 : 4; }
+
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+sa_status check_blocks(int32_t bq, int32_t bk, int64_t N) {
+  if (bq < 1 || bq > 128 || bk < 1 || bk > 128)
+    return set_error(SA_ERR_INVALID_ARG, "bq and bk must lie in [1, 128]");
+  if (ceil_div(N, bk) > 4095) return set_error(SA_ERR_UNSUPPORTED, "N / bk must be <= 4095");
+  return SA_OK;
+}
+
+sa_status check_mask_out(const sa_mask* m) {
+  if (!m) return set_error(SA_ERR_INVALID_ARG, "mask is NULL");
+  if (!m->block_mask || !m->row_ptr || !m->col_idx || !m->order || !m->kept_total || !m->status)
+    return set_error(SA_ERR_INVALID_ARG, "mask buffers must all be non-NULL");
+  if (m->col_capacity <= 0) return set_error(SA_ERR_INVALID_ARG, "mask col_capacity must be positive");
+  return SA_OK;
+}
+
+sa_status check_predict_dims(const sa_shape* s) {
+  const int es = elem_size(s->dtype);
+  if (!is_pow2(s->d) || s->d > 256 || (s->d * es) % 16 != 0 || (s->d * es) / 16 > 32)
+    return set_error(SA_ERR_UNSUPPORTED,
+                     "mask prediction needs d a power of two, d*elem_size a multiple of 16, d <= 256");
+  return SA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sa_version(void) { return "libsparseattn 0.1 (sm_100a)"; }
+
+const char* sa_last_error(void) { return g_err; }
+
+int32_t sa_attn_kernel_path(const sa_shape* shape, int32_t bq, int32_t bk, int32_t flags) {
+  if (check_shape(shape) != SA_OK) return -1;
+  if (bq < 1 || bq > 128 || bk < 1 || bk > 128) return -1;
+  if (!(flags & SA_FLAG_FORCE_SIMT) && attn_tc_supported(*shape, bq, bk)) return 1;
+  const size_t smem = ((size_t)bq * shape->dv + (size_t)bq * bk + 3 * (size_t)bq) * 4;
+  return smem <= 227 * 1024 ? 0 : -1;
+}
+
+size_t sa_layout_workspace(const sa_layout_desc* desc) {
+  if (!desc) return 0;
+  return layout_ws_bytes(*desc);
+}
+
+sa_status sa_layout_build(const sa_layout_desc* desc, int32_t* perm, int32_t* inv, void* ws,
+                          size_t ws_bytes, void* stream) {
+  if (!desc || !perm || !inv) return set_error(SA_ERR_INVALID_ARG, "NULL argument to sa_layout_build");
+  const sa_layout_desc& d = *desc;
+  if (d.T < 1 || d.H < 1 || d.W < 1 || d.txt_len < 0 || d.sink_frames < 0 || d.sink_frames > d.T)
+    return set_error(SA_ERR_INVALID_ARG, "bad layout sizes");
+  if (d.T * d.H * d.W + d.txt_len > (int64_t)INT32_MAX / 2)
+    return set_error(SA_ERR_UNSUPPORTED, "too many tokens");
+  if (d.mode != SA_ORDER_IDENTITY && d.mode != SA_ORDER_WINDOW && d.mode != SA_ORDER_HILBERT)
+    return set_error(SA_ERR_INVALID_ARG, "unknown layout mode");
+  if (d.mode == SA_ORDER_WINDOW && (d.win[0] < 1 || d.win[1] < 1 || d.win[2] < 1))
+    return set_error(SA_ERR_INVALID_ARG, "window sizes must be positive");
+  if (d.mode == SA_ORDER_HILBERT) {
+    const int64_t m = std::max(std::max(d.T - d.sink_frames, d.H), d.W);
+    if (m > 512) return set_error(SA_ERR_UNSUPPORTED, "Hilbert layout supports dimensions up to 512");
+    if (!ws || ws_bytes < layout_ws_bytes(d) || (uintptr_t)ws % 256)
+      return set_error(SA_ERR_WORKSPACE, "Hilbert layout needs %zu bytes of 256-byte aligned workspace",
+                       layout_ws_bytes(d));
+  }
+  if (sa_status e = check_device()) return e;
+  return launch_layout(d, perm, inv, ws, static_cast<cudaStream_t>(stream));
+}
+
+static sa_status reorder_common(const int32_t* perm, const void* src, void* dst, int64_t outer,
+                                int64_t N, int64_t row, int32_t dtype, bool scatter, void* stream) {
+  if (!perm || !src || !dst) return set_error(SA_ERR_INVALID_ARG, "NULL argument to sa_reorder");
+  if (outer <= 0 || N <= 0 || row <= 0) return set_error(SA_ERR_INVALID_ARG, "sizes must be positive");
+  if (dtype != SA_BF16 && dtype != SA_FP32) return set_error(SA_ERR_INVALID_ARG, "unknown dtype");
+  if (src == dst) return set_error(SA_ERR_INVALID_ARG, "reorder cannot run in place");
+  const int64_t bytes = row * elem_size(dtype);
+  if ((uintptr_t)src % 2 || (uintptr_t)dst % 2) return set_error(SA_ERR_INVALID_ARG, "misaligned tensor");
+  if (sa_status e = check_device()) return e;
+  return launch_reorder(perm, src, dst, outer, N, bytes, scatter, static_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_reorder(const int32_t* perm, const void* x, void* y, int64_t outer, int64_t N, int64_t row,
+                     int32_t dtype, void* stream) {
+  return reorder_common(perm, x, y, outer, N, row, dtype, false, stream);
+}
+
+sa_status sa_unreorder(const int32_t* perm, const void* y, void* x, int64_t outer, int64_t N,
+                       int64_t row, int32_t dtype, void* stream) {
+  return reorder_common(perm, y, x, outer, N, row, dtype, true, stream);
+}
+
+size_t sa_predict_mask_workspace(const sa_shape* shape, const sa_mask_params* p) {
+  if (check_shape(shape) != SA_OK || !p || p->bq < 1 || p->bk < 1) return 0;
+  size_t off[6];
+  return predict_ws_bytes(*shape, p->bq, p->bk, off);
+}
+
+sa_status sa_predict_mask_ws_layout(const sa_shape* shape, const sa_mask_params* p, size_t offsets[6]) {
+  if (sa_status e = check_shape(shape)) return e;
+  if (!p || !offsets || p->bq < 1 || p->bk < 1) return set_error(SA_ERR_INVALID_ARG, "bad arguments");
+  predict_ws_bytes(*shape, p->bq, p->bk, offsets);
+  return SA_OK;
+}
+
+sa_status sa_predict_mask(const void* q, const void* k, const sa_shape* shape,
+                          const sa_mask_params* params, void* ws, size_t ws_bytes, sa_mask* out,
+                          void* stream) {
+  if (sa_status e = check_shape(shape)) return e;
+  if (!q || !k || !params) return set_error(SA_ERR_INVALID_ARG, "NULL argument to sa_predict_mask");
+  const sa_mask_params& p = *params;
+  if (sa_status e = check_blocks(p.bq, p.bk, shape->N)) return e;
+  if (sa_status e = check_predict_dims(shape)) return e;
+  if (!(p.tau > 0.f && p.tau <= 1.f)) return set_error(SA_ERR_INVALID_ARG, "tau must lie in (0, 1]");
+  if (std::isnan(p.theta)) return set_error(SA_ERR_INVALID_ARG, "theta is NaN");
+  if (p.sink_tokens < 0 || p.txt_len < 0 || p.local_window < 0 || p.anchor_tokens < 0)
+    return set_error(SA_ERR_INVALID_ARG, "token counts must be non-negative");
+  if (p.causal != 0 && p.causal != 1) return set_error(SA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (sa_status e = check_mask_out(out)) return e;
+  if ((uintptr_t)q % 16 || (uintptr_t)k % 16) return set_error(SA_ERR_INVALID_ARG, "q and k must be 16-byte aligned");
+  size_t off[6];
+  const size_t need = predict_ws_bytes(*shape, p.bq, p.bk, off);
+  if (!ws || ws_bytes < need || (uintptr_t)ws % 256)
+    return set_error(SA_ERR_WORKSPACE, "sa_predict_mask needs %zu bytes of 256-byte aligned workspace", need);
+  if (sa_status e = check_device()) return e;
+  out->nqb = ceil_div(shape->N, p.bq);
+  out->nkb = ceil_div(shape->N, p.bk);
+  out->bq = p.bq;
+  out->bk = p.bk;
+  out->causal = p.causal;
+  return launch_predict(q, k, *shape, p, predict_ws_carve(ws, *shape, p.bq, p.bk), *out,
+                        static_cast<cudaStream_t>(stream));
+}
+
+size_t sa_mask_from_blocks_workspace(const sa_shape* shape, int32_t bq, int32_t bk) {
+  if (check_shape(shape) != SA_OK || bq < 1 || bk < 1) return 0;
+  return lists_ws_bytes(*shape, bq, bk);
+}
+
+sa_status sa_mask_from_blocks(const uint8_t* block_mask, const sa_shape* shape, int32_t bq, int32_t bk,
+                              int32_t causal, void* ws, size_t ws_bytes, sa_mask* out, void* stream) {
+  if (sa_status e = check_shape(shape)) return e;
+  if (!block_mask) return set_error(SA_ERR_INVALID_ARG, "block_mask is NULL");
+  if (sa_status e = check_blocks(bq, bk, shape->N)) return e;
+  if (causal != 0 && causal != 1) return set_error(SA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (sa_status e = check_mask_out(out)) return e;
+  const size_t need = lists_ws_bytes(*shape, bq, bk);
+  if (!ws || ws_bytes < need || (uintptr_t)ws % 256)
+    return set_error(SA_ERR_WORKSPACE, "sa_mask_from_blocks needs %zu bytes of 256-byte aligned workspace", need);
+  if (sa_status e = check_device()) return e;
+  out->nqb = ceil_div(shape->N, bq);
+  out->nkb = ceil_div(shape->N, bk);
+  out->bq = bq;
+  out->bk = bk;
+  out->causal = causal;
+  const int64_t R = shape->B * shape->Hq * out->nqb;
+  int32_t* counts = static_cast<int32_t*>(ws);
+  int32_t* tmp = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align_up((size_t)R * 4, 256));
+  return launch_mask_from_blocks(block_mask, *shape, bq, bk, causal, counts, tmp, *out,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+static sa_status attn_common(const void* q, const void* k, const void* v, const sa_shape* shape,
+                             const sa_mask* mask, int32_t causal, float lambda, float scale, void* out,
+                             float* lse, uint8_t* skip_log, int32_t* status, int32_t flags,
+                             void* stream) {
+  if (sa_status e = check_shape(shape)) return e;
+  if (!q || !k || !v || !out) return set_error(SA_ERR_INVALID_ARG, "NULL tensor argument");
+  if (std::isnan(lambda) || lambda > 0.f)
+    return set_error(SA_ERR_INVALID_ARG, "lambda must be <= 0 (or -INFINITY to disable the PV skip)");
+  if (!(scale >= 0.f) || std::isinf(scale)) return set_error(SA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  AttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.lse = lse;
+  a.skip_log = skip_log;
+  a.B = shape->B;
+  a.Hq = shape->Hq;
+  a.Hkv = shape->Hkv;
+  a.N = shape->N;
+  a.d = shape->d;
+  a.dv = shape->dv;
+  a.dtype = shape->dtype;
+  a.scale = scale > 0.f ? scale : 1.0f / std::sqrt((float)shape->d);
+  a.lambda = lambda;
+  if (mask) {
+    if (sa_status e = check_mask_out(mask)) return e;
+    if (mask->bq < 1 || mask->bq > 128 || mask->bk < 1 || mask->bk > 128 ||
+        mask->nqb != ceil_div(shape->N, mask->bq) || mask->nkb != ceil_div(shape->N, mask->bk))
+      return set_error(SA_ERR_INVALID_ARG, "mask does not match the shape (was it built for this shape?)");
+    a.row_ptr = mask->row_ptr;
+    a.col_idx = mask->col_idx;
+    a.order = mask->order;
+    a.status = mask->status;
+    a.bq = mask->bq;
+    a.bk = mask->bk;
+    a.causal = mask->causal;
+  } else {
+    a.status = status;
+    a.causal = causal;
+  }
+  const bool tc_ok = !(flags & SA_FLAG_FORCE_SIMT) && is_sm100();
+  if (!mask) {
+    if (tc_ok && attn_tc_supported(*shape, 128, 128)) {
+      a.bq = 128;
+      a.bk = 128;
+    } else {
+      a.bq = 64;
+      a.bk = 64;
+    }
+  }
+  a.nqb = ceil_div(a.N, a.bq);
+  a.nkb = ceil_div(a.N, a.bk);
+  if (sa_status e = check_device()) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_ok && attn_tc_supported(*shape, a.bq, a.bk)) return launch_attn_tc(a, st);
+  if (sa_attn_kernel_path(shape, a.bq, a.bk, SA_FLAG_FORCE_SIMT) < 0)
+    return set_error(SA_ERR_UNSUPPORTED, "no attention kernel for this shape");
+  return launch_attn_simt(a, st);
+}
+
+sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v, const sa_shape* shape,
+                               const sa_mask* mask, float lambda, float scale, void* out, float* lse,
+                               uint8_t* pv_skip_log, int32_t flags, void* stream) {
+  if (!mask) return set_error(SA_ERR_INVALID_ARG, "mask is NULL");
+  return attn_common(q, k, v, shape, mask, 0, lambda, scale, out, lse, pv_skip_log, nullptr, flags,
+                     stream);
+}
+
+sa_status sa_dense_attn(const void* q, const void* k, const void* v, const sa_shape* shape, int32_t causal,
+                        float scale, void* out, float* lse, int32_t* status, int32_t flags, void* stream) {
+  if (causal != 0 && causal != 1) return set_error(SA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  return attn_common(q, k, v, shape, nullptr, causal, -INFINITY, scale, out, lse, nullptr, status, flags,
+                     stream);
+}
+
+sa_status sa_read_status(const int32_t* status, void* stream) {
+  if (!status) return set_error(SA_ERR_INVALID_ARG, "status is NULL");
+  if (sa_status e = check_device()) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess)
+    return set_error(SA_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(cudaGetLastError()));
+  int32_t h = 0;
+  if (cudaMemcpy(&h, status, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return set_error(SA_ERR_CUDA, "reading the status word failed");
+  if (h < 0 || h > SA_ERR_CAPACITY) return set_error(SA_ERR_CUDA, "corrupt status word %d", h);
+  if (h != SA_OK) set_error((sa_status)h, "device status %d", h);
+  return (sa_status)h;
+}
+
+}  // extern "C"

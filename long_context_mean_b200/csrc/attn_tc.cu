@@ -1,0 +1,622 @@
+// Block-sparse FlashAttention forward on the sm_100a tensor cores.
+//
+// [P3] SpargeAttention notes, 2.1: per query block, the kept key blocks are
+// visited in ascending order with the online softmax (m, l, O); 2.3: the P V
+// product of a tile is skipped when max over the block's rows of
+// (rowmax S - running max) < lambda, l still counting the tile.
+//
+// Design (bf16, d = dv = 128, bq = 128, bk = 64 or 128):
+//   * persistent grid, one CTA per SM, work units (b, h, q-block) taken in
+//     the work order of the mask (rows by descending kept count);
+//   * warp 0 (one lane): TMA producer -- Q tile once per unit, K and V tiles
+//     of the unit's kept key blocks through a STAGES-deep ring;
+//   * warp 1 (one lane): tcgen05.mma issuer -- S = Q K^T into one of two
+//     TMEM S buffers, then O += P V into the TMEM O accumulator, one tile
+//     behind, so the tensor core works on S(t+1) and PV(t) while the softmax
+//     warps work on S(t+1)'s predecessor;
+//   * warps 4..7 (one thread per query row, TMEM lanes 0..127): load S from
+//     TMEM, mask, running max, the lambda decision for the whole block (a
+//     named barrier across the four warps), exp2, P to shared memory in the
+//     SW128 K-major layout the MMA reads, O rescale in TMEM when the reference
+//     maximum moves, and the epilogue O / l, LSE.
+//   The exact running max drives the lambda test; O and l use a reference
+//   maximum that is only moved when the running max exceeds it by more than
+//   2^8 (the final O / l is the same quotient).
+// Every mbarrier wait is bounded (2 s); on expiry the kernel raises
+// SA_ERR_TIMEOUT, every later wait returns at once, the producer drains its
+// own loads (bounded) and the TMEM allocation is released.
+#include <cuda.h>
+
+#include "sa_internal.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kThreadsTC = 256;
+constexpr int kWarpTMA = 0;
+constexpr int kWarpMMA = 1;
+constexpr int kWarpSoftmax0 = 4;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int BK>
+struct Cfg {
+  static constexpr int STAGES = BK == 64 ? 3 : 2;
+  static constexpr int Q_BYTES = 128 * 128 * 2;
+  static constexpr int KV_BYTES = BK * 128 * 2;
+  static constexpr int KV_CHUNK = BK * 128;          // one 64-column chunk: BK rows x 128 B
+  static constexpr int P_BYTES = 128 * BK * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_CTL = OFF_P + 2 * P_BYTES;
+  static constexpr int CTL_BYTES = 1024;
+  static constexpr int SMEM = OFF_CTL + CTL_BYTES + 1024;   // + alignment slack
+  static constexpr int TMEM_COLS = (128 + 2 * BK) <= 256 ? 256 : 512;
+  static constexpr int S_COL = 128;                          // O occupies columns 0..127
+};
+
+// Control block at OFF_CTL (8-byte mbarriers first).
+struct Ctl {
+  uint64_t q_full, q_empty, o_free;
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
+  uint32_t tmem_base;
+  volatile uint32_t abort;
+  volatile uint32_t skip_flag[2];
+  float gapw[2][4];
+};
+
+struct TcParams {
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  const int32_t* order;
+  uint16_t* out;
+  float* lse;
+  uint8_t* skip_log;
+  int32_t* status;
+  int64_t N, nqb, nkb;
+  int32_t Hq, Hkv;
+  int32_t num_units;
+  int32_t causal;
+  float scale_log2;
+  float lam_log2;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait.  Returns false when the CTA is aborting (a wait elsewhere
+// expired) or this wait expired (then it raises the abort itself).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl* ctl, int32_t* status) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (ctl->abort) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        ctl->abort = 1;
+        raise_status(status, SA_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+// Bounded wait that ignores the abort flag (draining in-flight copies).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try(bar, parity)) {
+    if (globaltimer() - t0 > kWaitLimitNs) return;
+  }
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 version 1).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor, kind::f16: bf16 x bf16 -> f32, A K-major.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, int b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+struct Unit {
+  int64_t bh, qb, kvh;
+  int64_t lo, n;
+};
+
+__device__ __forceinline__ Unit unit_at(const TcParams& p, int i, int BK) {
+  Unit u;
+  const int64_t id = p.order ? p.order[i] : i;
+  u.bh = id / p.nqb;
+  u.qb = id % p.nqb;
+  const int64_t b = u.bh / p.Hq, h = u.bh % p.Hq;
+  u.kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
+  if (p.row_ptr) {
+    u.lo = p.row_ptr[id];
+    u.n = p.row_ptr[id + 1] - u.lo;
+  } else {
+    u.lo = 0;
+    const int64_t last_row = min64(p.N, (u.qb + 1) * 128) - 1;
+    u.n = p.causal ? (last_row / BK + 1) : p.nkb;
+  }
+  return u;
+}
+
+__device__ __forceinline__ int64_t kblock_at(const TcParams& p, const Unit& u, int64_t t) {
+  return p.row_ptr ? p.col_idx[u.lo + t] : t;
+}
+
+template <int BK>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, TcParams p) {
+  using C = Cfg<BK>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::OFF_CTL);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctl->q_full, 1);
+    mbar_init(&ctl->q_empty, 1);
+    mbar_init(&ctl->o_free, 128);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&ctl->k_full[s], 1);
+      mbar_init(&ctl->k_empty[s], 1);
+      mbar_init(&ctl->v_full[s], 1);
+      mbar_init(&ctl->v_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->s_full[b], 1);
+      mbar_init(&ctl->s_empty[b], 128);
+      mbar_init(&ctl->p_full[b], 128);
+      mbar_init(&ctl->pv_done[b], 1);
+      ctl->skip_flag[b] = 0;
+    }
+    ctl->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kWarpMMA) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&ctl->tmem_base)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp == kWarpTMA) {
+    if (lane == 0) {
+      // ------------------------------------------------------------- producer
+      uint32_t kv_it = 0, nq = 0;   // tiles and Q tiles loaded so far
+      for (int i = blockIdx.x; i < p.num_units; i += gridDim.x) {
+        const Unit u = unit_at(p, i, BK);
+        if (u.n <= 0) continue;
+        mbar_wait(&ctl->q_empty, (nq & 1) ^ 1, ctl, p.status);
+        ++nq;
+        mbar_expect_tx(&ctl->q_full, C::Q_BYTES);
+        tma_load_3d(sb + C::OFF_Q, &tmQ, 0, (int)(u.qb * 128), (int)u.bh, &ctl->q_full);
+        tma_load_3d(sb + C::OFF_Q + C::Q_BYTES / 2, &tmQ, 64, (int)(u.qb * 128), (int)u.bh, &ctl->q_full);
+        for (int64_t t = 0; t < u.n; ++t, ++kv_it) {
+          const int kb = (int)kblock_at(p, u, t);
+          const int s = kv_it % C::STAGES;
+          const uint32_t ph = (kv_it / C::STAGES) & 1;
+          const uint32_t kdst = sb + C::OFF_K + s * C::KV_BYTES;
+          const uint32_t vdst = sb + C::OFF_V + s * C::KV_BYTES;
+          mbar_wait(&ctl->k_empty[s], ph ^ 1, ctl, p.status);
+          mbar_expect_tx(&ctl->k_full[s], C::KV_BYTES);
+          tma_load_3d(kdst, &tmK, 0, kb * BK, (int)u.kvh, &ctl->k_full[s]);
+          tma_load_3d(kdst + C::KV_CHUNK, &tmK, 64, kb * BK, (int)u.kvh, &ctl->k_full[s]);
+          mbar_wait(&ctl->v_empty[s], ph ^ 1, ctl, p.status);
+          mbar_expect_tx(&ctl->v_full[s], C::KV_BYTES);
+          tma_load_3d(vdst, &tmV, 0, kb * BK, (int)u.kvh, &ctl->v_full[s]);
+          tma_load_3d(vdst + C::KV_CHUNK, &tmV, 64, kb * BK, (int)u.kvh, &ctl->v_full[s]);
+        }
+      }
+      // Drain: the last loads of every stage (and the last Q) have landed.
+      if (nq > 0) mbar_drain(&ctl->q_full, (nq - 1) & 1);  // no-op unless a wait was abandoned
+      for (uint32_t j = kv_it > (uint32_t)C::STAGES ? kv_it - C::STAGES : 0; j < kv_it; ++j) {
+        mbar_drain(&ctl->k_full[j % C::STAGES], (j / C::STAGES) & 1);
+        mbar_drain(&ctl->v_full[j % C::STAGES], (j / C::STAGES) & 1);
+      }
+    }
+  } else if (warp == kWarpMMA) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc_s = make_idesc(128, BK, 0);
+      constexpr uint32_t idesc_pv = make_idesc(128, 128, 1);
+      uint32_t kv_it = 0, g = 0, unit_it = 0;   // unit_it counts units with work
+      for (int i = blockIdx.x; i < p.num_units; i += gridDim.x) {
+        const Unit u = unit_at(p, i, BK);
+        if (u.n <= 0) continue;
+        mbar_wait(&ctl->q_full, unit_it & 1, ctl, p.status);
+        tc_fence_after();
+        bool first_pv = true;
+        auto do_pv = [&](int64_t tt) {
+          const uint32_t it = kv_it + (uint32_t)tt, gt = g + (uint32_t)tt;
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          const int gb = gt & 1;
+          mbar_wait(&ctl->p_full[gb], (gt >> 1) & 1, ctl, p.status);
+          tc_fence_after();
+          const uint32_t skip = ctl->skip_flag[gb];
+          if (tt == 0) {
+            mbar_wait(&ctl->o_free, (unit_it & 1) ^ 1, ctl, p.status);
+            tc_fence_after();
+          }
+          mbar_wait(&ctl->v_full[s], ph, ctl, p.status);
+          tc_fence_after();
+          if (!skip) {
+            const uint32_t pbase = sb + C::OFF_P + gb * C::P_BYTES;
+            const uint32_t vbase = sb + C::OFF_V + s * C::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t a = desc_sw128(pbase + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+              const uint64_t b = desc_sw128(vbase + kk * 2048, C::KV_CHUNK, 1024);
+              umma_f16(tmem, a, b, idesc_pv, (first_pv && kk == 0) ? 0u : 1u);
+            }
+            first_pv = false;
+          }
+          umma_commit(&ctl->v_empty[s]);
+          umma_commit(&ctl->pv_done[gb]);
+        };
+        for (int64_t t = 0; t < u.n; ++t) {
+          const uint32_t it = kv_it + (uint32_t)t, gt = g + (uint32_t)t;
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          const int gb = gt & 1;
+          mbar_wait(&ctl->k_full[s], ph, ctl, p.status);
+          mbar_wait(&ctl->s_empty[gb], ((gt >> 1) & 1) ^ 1, ctl, p.status);
+          tc_fence_after();
+          const uint32_t kbase = sb + C::OFF_K + s * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = desc_sw128(sb + C::OFF_Q + (kk >> 2) * (C::Q_BYTES / 2) + (kk & 3) * 32, 16, 1024);
+            const uint64_t b = desc_sw128(kbase + (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32, 16, 1024);
+            umma_f16(tmem + C::S_COL + gb * BK, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&ctl->s_full[gb]);
+          umma_commit(&ctl->k_empty[s]);
+          if (t == u.n - 1) umma_commit(&ctl->q_empty);
+          if (t >= 1) do_pv(t - 1);
+        }
+        do_pv(u.n - 1);
+        kv_it += (uint32_t)u.n;
+        g += (uint32_t)u.n;
+        ++unit_it;
+      }
+    }
+    __syncwarp();
+  } else if (warp >= kWarpSoftmax0) {
+    // ------------------------------------------------------------- softmax
+    const int wq = warp - kWarpSoftmax0;        // == warp % 4: TMEM lanes 32*wq ..
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    uint32_t g = 0;
+    for (int i = blockIdx.x; i < p.num_units; i += gridDim.x) {
+      const Unit u = unit_at(p, i, BK);
+      const int64_t row_g = u.qb * 128 + row;
+      const bool row_valid = row_g < p.N;
+      if (u.n <= 0) {
+        if (row_valid) raise_status(p.status, SA_ERR_EMPTY_ROW);
+        continue;
+      }
+      float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
+      for (int64_t t = 0; t < u.n; ++t) {
+        const uint32_t gt = g + (uint32_t)t;
+        const int gb = gt & 1;
+        const int64_t kb = kblock_at(p, u, t);
+        mbar_wait(&ctl->s_full[gb], (gt >> 1) & 1, ctl, p.status);
+        tc_fence_after();
+        float s[BK];
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) tmem_ld32(tmem + lane_off + C::S_COL + gb * BK + c * 32, s + c * 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&ctl->s_empty[gb]);
+
+        const int64_t k0 = kb * BK;
+        const bool need_mask = (k0 + BK > p.N) || (p.causal && k0 + BK - 1 > u.qb * 128);
+        float mloc = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < BK; ++j) {
+          float x = s[j] * p.scale_log2;
+          if (need_mask) {
+            const int64_t key = k0 + j;
+            if (key >= p.N || (p.causal && key > row_g)) x = -INFINITY;
+          }
+          s[j] = x;
+          mloc = fmaxf(mloc, x);
+        }
+        const float m_new = fmaxf(m_run, mloc);
+        float gap = (row_valid && mloc > -INFINITY) ? mloc - m_new : -INFINITY;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) gap = fmaxf(gap, __shfl_xor_sync(0xffffffffu, gap, off));
+        if (lane == 0) ctl->gapw[gb][wq] = gap;
+        named_bar(1, 128);
+        const float G = fmaxf(fmaxf(ctl->gapw[gb][0], ctl->gapw[gb][1]), fmaxf(ctl->gapw[gb][2], ctl->gapw[gb][3]));
+        const bool skip = G < p.lam_log2;
+        m_run = m_new;
+        float corr = 1.f;
+        bool resc = false;
+        if (m_new > -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kRescaleThreshold)) {
+          corr = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
+          m_ref = m_new;
+          resc = (t > 0);
+        }
+        float rs = 0.f;
+        if (m_ref > -INFINITY) {
+#pragma unroll
+          for (int j = 0; j < BK; ++j) {
+            s[j] = ex2(s[j] - m_ref);
+            rs += s[j];
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < BK; ++j) s[j] = 0.f;
+        }
+        l = l * corr + rs;
+        if (!skip) {
+          if (gt >= 2) mbar_wait(&ctl->pv_done[gb], ((gt - 2) >> 1) & 1, ctl, p.status);
+          // tcgen05.ld/st are warp-collective: a warp rescales when any of
+          // its rows needs it (corr is 1 for the others).
+          if (__any_sync(0xffffffffu, resc)) {
+            const uint32_t gp = gt - 1;
+            mbar_wait(&ctl->pv_done[gp & 1], (gp >> 1) & 1, ctl, p.status);
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float o[32];
+              tmem_ld32(tmem + lane_off + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] *= corr;
+              tmem_st32(tmem + lane_off + c * 32, o);
+            }
+            tmem_wait_st();
+          }
+          uint8_t* prow = smem + C::OFF_P + gb * C::P_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < BK / 8; ++c) {
+            uint4 v;
+            v.x = pack_bf16(s[8 * c + 0], s[8 * c + 1]);
+            v.y = pack_bf16(s[8 * c + 2], s[8 * c + 3]);
+            v.z = pack_bf16(s[8 * c + 4], s[8 * c + 5]);
+            v.w = pack_bf16(s[8 * c + 6], s[8 * c + 7]);
+            const int region = c >> 3, cc = c & 7;
+            *reinterpret_cast<uint4*>(prow + region * 16384 + ((cc ^ (row & 7)) << 4)) = v;
+          }
+          fence_async_smem();
+        }
+        tc_fence_before();
+        if (row == 0) {
+          ctl->skip_flag[gb] = skip ? 1u : 0u;
+          if (p.skip_log && p.row_ptr) p.skip_log[u.lo + t] = skip ? 1 : 0;
+        }
+        mbar_arrive(&ctl->p_full[gb]);
+      }
+      // Epilogue: O / l from TMEM once the unit's last PV has landed.
+      const uint32_t gl = g + (uint32_t)u.n - 1;
+      mbar_wait(&ctl->pv_done[gl & 1], (gl >> 1) & 1, ctl, p.status);
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      uint16_t* orow = p.out + (u.bh * p.N + row_g) * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(tmem + lane_off + c * 32, o);
+        tmem_wait_ld();
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v;
+            v.x = pack_bf16(o[8 * q4 + 0] * inv_l, o[8 * q4 + 1] * inv_l);
+            v.y = pack_bf16(o[8 * q4 + 2] * inv_l, o[8 * q4 + 3] * inv_l);
+            v.z = pack_bf16(o[8 * q4 + 4] * inv_l, o[8 * q4 + 5] * inv_l);
+            v.w = pack_bf16(o[8 * q4 + 6] * inv_l, o[8 * q4 + 7] * inv_l);
+            dst[q4] = v;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->o_free);
+      if (row_valid) {
+        if (!(l > 0.f)) raise_status(p.status, SA_ERR_EMPTY_ROW);
+        if (p.lse) p.lse[u.bh * p.N + row_g] = (m_ref + __log2f(l)) * kLn2;
+      }
+      g += (uint32_t)u.n;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMMA) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D map over [heads][N][128] bf16, box [1][rows][64], 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t heads, int64_t N, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)N, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)N * 128 * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BK>
+sa_status launch_bk(const AttnArgs& a, cudaStream_t st) {
+  using C = Cfg<BK>;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, a.B * a.Hq, a.N, 128) || !make_map(&mk, a.k, a.B * a.Hkv, a.N, BK) ||
+      !make_map(&mv, a.v, a.B * a.Hkv, a.N, BK))
+    return set_error(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable or bad map)");
+  TcParams p;
+  p.row_ptr = a.row_ptr;
+  p.col_idx = a.col_idx;
+  p.order = a.order;
+  p.out = static_cast<uint16_t*>(a.out);
+  p.lse = a.lse;
+  p.skip_log = a.skip_log;
+  p.status = a.status;
+  p.N = a.N;
+  p.nqb = a.nqb;
+  p.nkb = a.nkb;
+  p.Hq = (int32_t)a.Hq;
+  p.Hkv = (int32_t)a.Hkv;
+  p.num_units = (int32_t)(a.B * a.Hq * a.nqb);
+  p.causal = a.causal;
+  p.scale_log2 = a.scale * kLog2e;
+  p.lam_log2 = a.lambda * kLog2e;
+  if (p.num_units == 0) return SA_OK;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaFuncSetAttribute(attn_tc_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+    return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(attn_tc_kernel) failed");
+  const int grid = p.num_units < sms ? p.num_units : sms;
+  attn_tc_kernel<BK><<<grid, kThreadsTC, C::SMEM, st>>>(mq, mk, mv, p);
+  return check_launch("attn_tc_kernel");
+}
+
+}  // namespace
+
+bool attn_tc_supported(const sa_shape& s, int bq, int bk) {
+  return s.dtype == SA_BF16 && s.d == 128 && s.dv == 128 && bq == 128 && (bk == 64 || bk == 128);
+}
+
+sa_status launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
+  if ((uintptr_t)a.q % 16 || (uintptr_t)a.k % 16 || (uintptr_t)a.v % 16 || (uintptr_t)a.out % 16)
+    return set_error(SA_ERR_INVALID_ARG, "tensor-core path needs 16-byte aligned q, k, v, out");
+  return a.bk == 64 ? launch_bk<64>(a, st) : launch_bk<128>(a, st);
+}
+
+}  // namespace sa

@@ -1,0 +1,574 @@
+// Mask prediction: block pooling with the intra-block similarity guard, the
+// compressed softmax with TopCdf selection, forced rows/columns, and the
+// compaction of the block mask into CSR lists and a work order.
+//
+// [P3] SpargeAttention notes, 2.2 "selective token compression": block means
+// q_hat, k_hat; a block-similarity guard theta; S_hat = q_hat k_hat^T with
+// low-similarity key columns at -inf, softmax, TopCdf(tau) per row; rows of
+// low-similarity query blocks and columns of low-similarity key blocks
+// forced to 1.  [P2] MindIE-SD "稀疏": first-frame sink forced into full
+// attention; text tokens.  [P4]/[P5]: local window and anchor keys.
+//
+// Readings: the similarity is the mean pairwise cosine of the block's tokens
+// (diagonal included), which equals |sum_i x_i/|x_i||^2 / n^2 and is computed
+// in one pass; S_hat carries 1/sqrt(d); TopCdf keeps an entry iff the mass
+// sorted before it is < tau * total (ties: lower block index first); a row
+// with no eligible entry selects nothing; causal: key block kb is future for
+// query block qb iff kb*bk > last row of qb.
+#include "sa_internal.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kPoolThreads = 128;
+constexpr int kPoolWarps = kPoolThreads / 32;
+
+// ---------------------------------------------------------------------------
+// a2: one CTA per (head, block): block mean and mean pairwise cosine.  A warp
+// covers 32/chunks tokens per step (chunks = 16-byte pieces of a token),
+// two steps in flight; token norms reduce inside each token's lane group.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
+    const T* __restrict__ x, int64_t N, int d, int b, int nB, float* __restrict__ mean_out,
+    float* __restrict__ s_out) {
+  constexpr int EPL = 16 / sizeof(T);
+  const int blk = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int64_t t0 = (int64_t)blk * b;
+  const int cnt = (int)min64(b, N - t0);
+  const int chunks = d / EPL;
+  const int tpw = 32 / chunks;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane / chunks, c = lane % chunks;
+  float ax[EPL], au[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) ax[e] = au[e] = 0.f;
+  const uint4* base = reinterpret_cast<const uint4*>(x + (bh * N + t0) * (int64_t)d);
+  const int step = kPoolWarps * tpw;
+  for (int tb = warp * tpw; tb < cnt; tb += 2 * step) {
+    uint4 raw[2];
+    bool ok[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int tok = tb + u * step + sub;
+      ok[u] = tok < cnt;
+      raw[u] = ok[u] ? __ldg(base + (int64_t)tok * chunks + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float v[EPL];
+      unpack16(raw[u], T(), v);
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) ss = fmaf(v[e], v[e], ss);
+      for (int off = chunks >> 1; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      const float inv = (ok[u] && ss > 0.f) ? 1.0f / sqrtf(ss) : 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        ax[e] += v[e];
+        au[e] = fmaf(v[e], inv, au[e]);
+      }
+    }
+  }
+  for (int off = chunks; off < 32; off <<= 1) {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      ax[e] += __shfl_xor_sync(0xffffffffu, ax[e], off);
+      au[e] += __shfl_xor_sync(0xffffffffu, au[e], off);
+    }
+  }
+  __shared__ float sx[kPoolWarps][256];
+  __shared__ float su[kPoolWarps][256];
+  __shared__ float red[kPoolWarps];
+  if (lane < chunks) {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      sx[warp][c * EPL + e] = ax[e];
+      su[warp][c * EPL + e] = au[e];
+    }
+  }
+  __syncthreads();
+  float part = 0.f;
+  for (int i = threadIdx.x; i < d; i += kPoolThreads) {
+    float X = 0.f, U = 0.f;
+#pragma unroll
+    for (int w = 0; w < kPoolWarps; ++w) {
+      X += sx[w][i];
+      U += su[w][i];
+    }
+    mean_out[(bh * nB + blk) * (int64_t)d + i] = X / (float)cnt;
+    part = fmaf(U, U, part);
+  }
+  for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+  if (lane == 0) red[warp] = part;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int w = 0; w < kPoolWarps; ++w) tot += red[w];
+    s_out[bh * nB + blk] = tot / ((float)cnt * (float)cnt);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Shared row rules (structure-forced rows/columns, window, causal validity).
+// ---------------------------------------------------------------------------
+struct RowRules {
+  int64_t N, sink, txt, window, anchor;
+  int bq, bk, causal;
+  __device__ bool struct_row(int64_t qb) const {
+    const int64_t i0 = qb * bq, i1 = min(N, (qb + 1) * bq);
+    return i0 < sink || (txt > 0 && i1 - 1 >= N - txt);
+  }
+  __device__ bool struct_col(int64_t kb) const {
+    const int64_t j0 = kb * bk, j1 = min(N, (kb + 1) * bk);
+    return j0 < sink || j0 < anchor || (txt > 0 && j1 - 1 >= N - txt);
+  }
+  __device__ bool in_window(int64_t qb, int64_t kb) const {
+    if (window <= 0) return false;
+    const int64_t i0 = qb * bq, i1 = min(N, (qb + 1) * bq);
+    const int64_t j0 = kb * bk, j1 = min(N, (kb + 1) * bk);
+    return (i1 - 1 >= j0) && (i0 - (j1 - 1) < window);
+  }
+  __device__ bool valid(int64_t qb, int64_t kb) const {
+    if (!causal) return true;
+    return kb * bk <= min(N, (qb + 1) * bq) - 1;
+  }
+};
+
+constexpr int kRowThreads = 256;
+
+__device__ __forceinline__ float block_reduce_max(float v, float* sh) {
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  float r = -INFINITY;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, sh[w]);
+  return r;
+}
+
+__device__ __forceinline__ float block_reduce_sum(float v, float* sh) {
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  float r = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += sh[w];
+  return r;
+}
+
+__device__ __forceinline__ int block_reduce_sum_int(int v, int* sh) {
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  int r = 0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += sh[w];
+  return r;
+}
+
+__device__ __forceinline__ int block_reduce_min_int(int v, int* sh) {
+  for (int off = 16; off > 0; off >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, off));
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  int r = 0x7fffffff;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = min(r, sh[w]);
+  return r;
+}
+
+// Finishes one mask row: writes the bytes, the row count, and raises
+// SA_ERR_EMPTY_ROW when the block's first query row would see no key
+// (causal: some kept kb with kb*bk <= first row; else any kept kb).
+__device__ void finish_row(const uint8_t* flags, int64_t u, int64_t qb, int64_t nkb,
+                           const RowRules& r, uint8_t* mask_row_out, int32_t* counts,
+                           int32_t* status, int* sh_int) {
+  int cnt = 0, first = 0x7fffffff;
+  for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) {
+    const uint8_t f = flags[kb];
+    mask_row_out[kb] = f;
+    if (f) {
+      ++cnt;
+      first = min(first, (int)kb);
+    }
+  }
+  cnt = block_reduce_sum_int(cnt, sh_int);
+  first = block_reduce_min_int(first, sh_int);
+  if (threadIdx.x == 0) {
+    counts[u] = cnt;
+    const bool empty = r.causal ? (cnt == 0 || (int64_t)first * r.bk > qb * r.bq) : cnt == 0;
+    if (empty) raise_status(status, SA_ERR_EMPTY_ROW);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a3 + a4: one CTA per mask row (b, h, qb).  Scores, softmax, bitonic sort of
+// (p, kb) keys descending (ties: lower kb first), scan, TopCdf, then the
+// union with the forced parts and the causal AND.
+// Dynamic shared memory: keys[P2] (u64) | flags[nkb] (u8) | q_hat[d] (f32).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
+    const float* __restrict__ qhat, const float* __restrict__ khat, const float* __restrict__ sq,
+    const float* __restrict__ sk, int64_t Hq, int64_t Hkv, int64_t nqb, int64_t nkb, int d,
+    int P2, float tau, float theta, RowRules rules, uint8_t* __restrict__ mask,
+    int32_t* __restrict__ counts, int32_t* status) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
+  uint8_t* flags = smem + (size_t)P2 * 8;
+  float* qv = reinterpret_cast<float*>(smem + (size_t)P2 * 8 + ((nkb + 15) / 16) * 16);
+  __shared__ float shf[32];
+  __shared__ int shi[32];
+  __shared__ float scan_part[kRowThreads];
+
+  const int64_t u = blockIdx.x;
+  const int64_t bh = u / nqb, qb = u % nqb;
+  const int64_t b = bh / Hq, h = bh % Hq;
+  const int64_t g = b * Hkv + h / (Hq / Hkv);
+  const bool guard = theta > 0.f;
+  const bool row_forced = rules.struct_row(qb) || (guard && sq[u] < theta);
+
+  for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) flags[kb] = 0;
+  if (!row_forced) {
+    for (int i = threadIdx.x; i < d; i += blockDim.x) qv[i] = qhat[u * (int64_t)d + i];
+    __syncthreads();
+    const float scale = rsqrtf((float)d);
+    float mx = -INFINITY;
+    for (int64_t kb = threadIdx.x; kb < P2; kb += blockDim.x) {
+      float s = -INFINITY;
+      if (kb < nkb && rules.valid(qb, kb) && !(guard && sk[g * nkb + kb] < theta)) {
+        const float4* kr = reinterpret_cast<const float4*>(khat + (g * nkb + kb) * (int64_t)d);
+        const float4* qr = reinterpret_cast<const float4*>(qv);
+        float acc = 0.f;
+        for (int i = 0; i < d / 4; ++i) {
+          const float4 a = qr[i], bb = __ldg(kr + i);
+          acc = fmaf(a.x, bb.x, acc);
+          acc = fmaf(a.y, bb.y, acc);
+          acc = fmaf(a.z, bb.z, acc);
+          acc = fmaf(a.w, bb.w, acc);
+        }
+        s = acc * scale;
+      }
+      keys[kb] = (uint64_t)__float_as_uint(s);   // stash raw score bits for now
+      mx = fmaxf(mx, s);
+    }
+    mx = block_reduce_max(mx, shf);
+    if (mx > -INFINITY) {
+      float sum = 0.f;
+      for (int64_t kb = threadIdx.x; kb < P2; kb += blockDim.x) {
+        const float s = __uint_as_float((uint32_t)keys[kb]);
+        const float p = (s == -INFINITY) ? 0.f : expf(s - mx);
+        // key = p bits (p >= 0: integer order = float order) | ~kb
+        keys[kb] = (kb < nkb) ? (((uint64_t)__float_as_uint(p) << 32) | (uint32_t)(~(uint32_t)kb))
+                              : 0ull;
+        sum += p;
+      }
+      __syncthreads();
+      // Bitonic sort, descending.
+      for (int k = 2; k <= P2; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+          for (int i = threadIdx.x; i < P2; i += blockDim.x) {
+            const int ixj = i ^ j;
+            if (ixj > i) {
+              const uint64_t a = keys[i], c = keys[ixj];
+              const bool desc = (i & k) == 0;
+              if (desc ? (a < c) : (a > c)) {
+                keys[i] = c;
+                keys[ixj] = a;
+              }
+            }
+          }
+          __syncthreads();
+        }
+      }
+      // Inclusive scan of the sorted probabilities: each thread a contiguous
+      // run, then a block scan of the run totals.
+      const int per = P2 / blockDim.x > 0 ? P2 / blockDim.x : 1;
+      const int beg = threadIdx.x * per;
+      float run = 0.f;
+      for (int i = beg; i < beg + per && i < P2; ++i) run += __uint_as_float((uint32_t)(keys[i] >> 32));
+      scan_part[threadIdx.x] = run;
+      __syncthreads();
+      for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+        const float v = threadIdx.x >= (unsigned)off ? scan_part[threadIdx.x - off] : 0.f;
+        __syncthreads();
+        scan_part[threadIdx.x] += v;
+        __syncthreads();
+      }
+      const float total = scan_part[blockDim.x - 1];
+      const float limit = tau * total;
+      float excl = scan_part[threadIdx.x] - run;
+      for (int i = beg; i < beg + per && i < P2; ++i) {
+        const float p = __uint_as_float((uint32_t)(keys[i] >> 32));
+        const uint32_t kb = ~(uint32_t)keys[i];
+        if (p > 0.f && excl < limit) flags[kb] = 1;
+        excl += p;
+      }
+      (void)sum;
+    }
+  }
+  __syncthreads();
+  for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) {
+    const bool col = rules.struct_col(kb) || (guard && sk[g * nkb + kb] < theta);
+    const bool keep = rules.valid(qb, kb) &&
+                      (row_forced || flags[kb] || col || rules.in_window(qb, kb));
+    flags[kb] = keep ? 1 : 0;
+  }
+  __syncthreads();
+  finish_row(flags, u, qb, nkb, rules, mask + u * nkb, counts, status, shi);
+}
+
+// A caller-supplied mask row: AND causal validity, copy, count, check.
+__global__ void __launch_bounds__(kRowThreads) mask_copy_kernel(
+    const uint8_t* __restrict__ in, int64_t nqb, int64_t nkb, RowRules rules,
+    uint8_t* __restrict__ out, int32_t* __restrict__ counts, int32_t* status) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint8_t* flags = smem;
+  __shared__ int shi[32];
+  const int64_t u = blockIdx.x;
+  const int64_t qb = u % nqb;
+  for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x)
+    flags[kb] = (in[u * nkb + kb] != 0 && rules.valid(qb, kb)) ? 1 : 0;
+  __syncthreads();
+  finish_row(flags, u, qb, nkb, rules, out + u * nkb, counts, status, shi);
+}
+
+// ---------------------------------------------------------------------------
+// CSR: one CTA scans the row counts into row_ptr and checks capacity.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) rows_scan_kernel(const int32_t* __restrict__ counts,
+                                                         int64_t R, int64_t capacity,
+                                                         int32_t* __restrict__ row_ptr,
+                                                         int64_t* kept_total, int32_t* status) {
+  __shared__ int64_t part[1024];
+  const int64_t per = (R + blockDim.x - 1) / blockDim.x;
+  const int64_t beg = threadIdx.x * per, end = min(R, beg + per);
+  int64_t s = 0;
+  for (int64_t i = beg; i < end; ++i) s += counts[i];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+    const int64_t v = threadIdx.x >= (unsigned)off ? part[threadIdx.x - off] : 0;
+    __syncthreads();
+    part[threadIdx.x] += v;
+    __syncthreads();
+  }
+  int64_t run = part[threadIdx.x] - s;
+  for (int64_t i = beg; i < end; ++i) {
+    row_ptr[i] = (int32_t)min64(run, INT32_MAX);
+    run += counts[i];
+  }
+  if (threadIdx.x == blockDim.x - 1) {
+    const int64_t tot = part[blockDim.x - 1];
+    row_ptr[R] = (int32_t)min64(tot, INT32_MAX);
+    *kept_total = tot;
+    if (tot > capacity || tot > INT32_MAX) raise_status(status, SA_ERR_CAPACITY);
+  }
+}
+
+// One warp per row: ascending kept block indices by ballot compaction.
+__global__ void fill_cols_kernel(const uint8_t* __restrict__ mask, int64_t R, int64_t nkb,
+                                 const int32_t* __restrict__ row_ptr, int64_t capacity,
+                                 int32_t* __restrict__ col_idx) {
+  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= R) return;
+  const int64_t lo = row_ptr[warp];
+  const int64_t hi = row_ptr[warp + 1];
+  if (hi > capacity) return;  // capacity error already raised
+  int64_t pos = lo;
+  for (int64_t kb0 = 0; kb0 < nkb; kb0 += 32) {
+    const int64_t kb = kb0 + lane;
+    const bool f = kb < nkb && mask[warp * nkb + kb] != 0;
+    const uint32_t bal = __ballot_sync(0xffffffffu, f);
+    if (f) col_idx[pos + __popc(bal & ((1u << lane) - 1u))] = (int32_t)kb;
+    pos += __popc(bal);
+  }
+}
+
+// Work order: stable LSD radix sort of rows by key = 4095 - count (3 passes
+// of 4 bits), i.e. descending count, ties by ascending row index.  One CTA;
+// each thread owns a contiguous range of the current sequence; the digit
+// histogram is kept per (digit, thread) so the scatter stays stable.
+constexpr int kOrderThreads = 1024;
+__global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __restrict__ counts,
+                                                              int64_t R, int32_t* __restrict__ tmp,
+                                                              int32_t* __restrict__ order) {
+  extern __shared__ uint32_t hist[];  // [16][kOrderThreads]
+  __shared__ uint32_t part[kOrderThreads];
+  const int tid = threadIdx.x;
+  const int64_t per = (R + kOrderThreads - 1) / kOrderThreads;
+  const int64_t beg = tid * per, end = min(R, beg + per);
+  for (int pass = 0; pass < 3; ++pass) {
+    const int32_t* src = pass == 0 ? nullptr : (pass == 1 ? order : tmp);
+    int32_t* dst = pass == 1 ? tmp : order;
+    const int shift = 4 * pass;
+    for (int dgt = 0; dgt < 16; ++dgt) hist[dgt * kOrderThreads + tid] = 0;
+    __syncthreads();
+    for (int64_t i = beg; i < end; ++i) {
+      const int32_t row = src ? src[i] : (int32_t)i;
+      const uint32_t key = 4095u - (uint32_t)counts[row];
+      hist[((key >> shift) & 15u) * kOrderThreads + tid] += 1;
+    }
+    __syncthreads();
+    // Exclusive scan over the 16*1024 entries in (digit, thread) order:
+    // thread j owns entries [16j, 16j+16).
+    uint32_t s = 0;
+    for (int e = 0; e < 16; ++e) s += hist[tid * 16 + e];
+    part[tid] = s;
+    __syncthreads();
+    for (int off = 1; off < kOrderThreads; off <<= 1) {
+      const uint32_t v = tid >= off ? part[tid - off] : 0;
+      __syncthreads();
+      part[tid] += v;
+      __syncthreads();
+    }
+    uint32_t run = part[tid] - s;
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t c = hist[tid * 16 + e];
+      hist[tid * 16 + e] = run;
+      run += c;
+    }
+    __syncthreads();
+    for (int64_t i = beg; i < end; ++i) {
+      const int32_t row = src ? src[i] : (int32_t)i;
+      const uint32_t key = 4095u - (uint32_t)counts[row];
+      uint32_t& slot = hist[((key >> shift) & 15u) * kOrderThreads + tid];
+      dst[slot] = row;
+      slot += 1;
+    }
+    __syncthreads();
+  }
+}
+
+sa_status launch_lists(const sa_shape& s, int bq, int bk, int32_t* counts, int32_t* tmp,
+                       sa_mask& out, cudaStream_t st) {
+  const int64_t R = s.B * s.Hq * out.nqb;
+  rows_scan_kernel<<<1, 1024, 0, st>>>(counts, R, out.col_capacity, out.row_ptr, out.kept_total,
+                                       out.status);
+  if (sa_status e = check_launch("rows_scan_kernel")) return e;
+  const int64_t warps_per_block = 8;
+  fill_cols_kernel<<<(unsigned)ceil_div(R, warps_per_block), 32 * warps_per_block, 0, st>>>(
+      out.block_mask, R, out.nkb, out.row_ptr, out.col_capacity, out.col_idx);
+  if (sa_status e = check_launch("fill_cols_kernel")) return e;
+  const size_t hist_bytes = 16 * kOrderThreads * sizeof(uint32_t);
+  if (cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)hist_bytes) != cudaSuccess)
+    return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(order_kernel) failed");
+  order_kernel<<<1, kOrderThreads, hist_bytes, st>>>(counts, R, tmp, out.order);
+  return check_launch("order_kernel");
+}
+
+RowRules make_rules(const sa_shape& s, const sa_mask_params& p) {
+  RowRules r;
+  r.N = s.N;
+  r.sink = p.sink_tokens;
+  r.txt = p.txt_len;
+  r.window = p.local_window;
+  r.anchor = p.anchor_tokens;
+  r.bq = p.bq;
+  r.bk = p.bk;
+  r.causal = p.causal;
+  return r;
+}
+
+template <typename T>
+sa_status launch_pool(const void* x, int64_t BH, int64_t N, int d, int b, int64_t nB, float* mean,
+                      float* sim, cudaStream_t st) {
+  dim3 grid((unsigned)nB, (unsigned)BH);
+  pool_cossim_kernel<T><<<grid, kPoolThreads, 0, st>>>(static_cast<const T*>(x), N, d, b, (int)nB,
+                                                       mean, sim);
+  return check_launch("pool_cossim_kernel");
+}
+
+}  // namespace
+
+size_t predict_ws_bytes(const sa_shape& s, int bq, int bk, size_t off[6]) {
+  const int64_t nqb = ceil_div(s.N, bq), nkb = ceil_div(s.N, bk);
+  const int64_t R = s.B * s.Hq * nqb;
+  size_t o = 0;
+  const size_t sizes[6] = {(size_t)(s.B * s.Hq * nqb * s.d) * 4, (size_t)(s.B * s.Hkv * nkb * s.d) * 4,
+                           (size_t)(s.B * s.Hq * nqb) * 4,      (size_t)(s.B * s.Hkv * nkb) * 4,
+                           (size_t)R * 4,                        (size_t)R * 4};
+  for (int i = 0; i < 6; ++i) {
+    off[i] = o;
+    o += align_up(sizes[i], 256);
+  }
+  return o;
+}
+
+PredictWs predict_ws_carve(void* ws, const sa_shape& s, int bq, int bk) {
+  size_t off[6];
+  predict_ws_bytes(s, bq, bk, off);
+  char* p = static_cast<char*>(ws);
+  PredictWs w;
+  w.qhat = reinterpret_cast<float*>(p + off[0]);
+  w.khat = reinterpret_cast<float*>(p + off[1]);
+  w.sq = reinterpret_cast<float*>(p + off[2]);
+  w.sk = reinterpret_cast<float*>(p + off[3]);
+  w.counts = reinterpret_cast<int32_t*>(p + off[4]);
+  w.tmp = reinterpret_cast<int32_t*>(p + off[5]);
+  return w;
+}
+
+size_t lists_ws_bytes(const sa_shape& s, int bq, int) {
+  const int64_t R = s.B * s.Hq * ceil_div(s.N, bq);
+  return align_up((size_t)R * 4, 256) * 2;
+}
+
+sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
+                         const sa_mask_params& p, const PredictWs& w, sa_mask& out,
+                         cudaStream_t st) {
+  const int64_t nqb = out.nqb, nkb = out.nkb;
+  if (cudaMemsetAsync(out.status, 0, sizeof(int32_t), st) != cudaSuccess)
+    return set_error(SA_ERR_CUDA, "cudaMemsetAsync(status) failed");
+  sa_status e;
+  if (s.dtype == SA_BF16) {
+    if ((e = launch_pool<uint16_t>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, st))) return e;
+    if ((e = launch_pool<uint16_t>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, w.sk, st))) return e;
+  } else {
+    if ((e = launch_pool<float>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, st))) return e;
+    if ((e = launch_pool<float>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, w.sk, st))) return e;
+  }
+  int P2 = 1;
+  while (P2 < nkb) P2 <<= 1;
+  const size_t smem = (size_t)P2 * 8 + ((nkb + 15) / 16) * 16 + (size_t)s.d * 4;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(score_topcdf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(score_topcdf_kernel) failed");
+  }
+  const int64_t R = s.B * s.Hq * nqb;
+  score_topcdf_kernel<<<(unsigned)R, kRowThreads, smem, st>>>(
+      w.qhat, w.khat, w.sq, w.sk, s.Hq, s.Hkv, nqb, nkb, (int)s.d, P2, p.tau, p.theta,
+      make_rules(s, p), out.block_mask, w.counts, out.status);
+  if ((e = check_launch("score_topcdf_kernel"))) return e;
+  return launch_lists(s, p.bq, p.bk, w.counts, w.tmp, out, st);
+}
+
+sa_status launch_mask_from_blocks(const uint8_t* in, const sa_shape& s, int bq, int bk, int causal,
+                                  int32_t* counts, int32_t* tmp, sa_mask& out, cudaStream_t st) {
+  if (cudaMemsetAsync(out.status, 0, sizeof(int32_t), st) != cudaSuccess)
+    return set_error(SA_ERR_CUDA, "cudaMemsetAsync(status) failed");
+  sa_mask_params p{};
+  p.bq = bq;
+  p.bk = bk;
+  p.causal = causal;
+  const int64_t R = s.B * s.Hq * out.nqb;
+  const size_t smem = align_up((size_t)out.nkb, 16);
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(mask_copy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(mask_copy_kernel) failed");
+  }
+  mask_copy_kernel<<<(unsigned)R, kRowThreads, smem, st>>>(in, out.nqb, out.nkb, make_rules(s, p),
+                                                          out.block_mask, counts, out.status);
+  if (sa_status e = check_launch("mask_copy_kernel")) return e;
+  return launch_lists(s, bq, bk, counts, tmp, out, st);
+}
+
+}  // namespace sa

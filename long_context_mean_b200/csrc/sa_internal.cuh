@@ -1,0 +1,118 @@
+// Internal declarations shared by the CUDA translation units of
+// libsparseattn.so.  Nothing here is part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "sparse_attn.h"
+
+namespace sa {
+
+// ---------------------------------------------------------------------------
+// Host-side error reporting (thread-local message, see abi.cu)
+// ---------------------------------------------------------------------------
+sa_status set_error(sa_status code, const char* fmt, ...);
+sa_status check_launch(const char* what);
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void raise_status(int32_t* status, int32_t code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float load(const float* p) { return __ldg(p); }
+  static __device__ __forceinline__ void store(float* p, float v) { *p = v; }
+};
+template <> struct Elem<uint16_t> {
+  static __device__ __forceinline__ float load(const uint16_t* p) { return bf16_to_f32(__ldg(p)); }
+  static __device__ __forceinline__ void store(uint16_t* p, float v) { *p = f32_to_bf16_rne(v); }
+};
+
+// Unpack a 16-byte vector of elements into floats (8 bf16 or 4 fp32).
+__device__ __forceinline__ void unpack16(const uint4& u, uint16_t, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void unpack16(const uint4& u, float, float* f) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+// ---------------------------------------------------------------------------
+// Launch entry points implemented in the .cu files (called from abi.cu after
+// argument validation).
+// ---------------------------------------------------------------------------
+sa_status launch_layout(const sa_layout_desc& d, int32_t* perm, int32_t* inv, void* ws,
+                        cudaStream_t st);
+size_t layout_ws_bytes(const sa_layout_desc& d);
+
+sa_status launch_reorder(const int32_t* perm, const void* src, void* dst, int64_t outer,
+                         int64_t N, int64_t row_bytes, bool scatter, cudaStream_t st);
+
+struct PredictWs {
+  float* qhat;     // [B*Hq, nqb, d]
+  float* khat;     // [B*Hkv, nkb, d]
+  float* sq;       // [B*Hq, nqb]
+  float* sk;       // [B*Hkv, nkb]
+  int32_t* counts; // [B*Hq*nqb]
+  int32_t* tmp;    // [B*Hq*nqb] radix-sort scratch
+};
+size_t predict_ws_bytes(const sa_shape& s, int bq, int bk, size_t offsets[6]);
+PredictWs predict_ws_carve(void* ws, const sa_shape& s, int bq, int bk);
+size_t lists_ws_bytes(const sa_shape& s, int bq, int bk);
+
+sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
+                         const sa_mask_params& p, const PredictWs& w, sa_mask& out,
+                         cudaStream_t st);
+sa_status launch_mask_from_blocks(const uint8_t* in, const sa_shape& s, int bq, int bk,
+                                  int causal, int32_t* counts, int32_t* tmp, sa_mask& out,
+                                  cudaStream_t st);
+
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;
+  uint8_t* skip_log;
+  const int32_t* row_ptr;   // nullptr = dense (every causally valid block)
+  const int32_t* col_idx;
+  const int32_t* order;     // nullptr = natural row order
+  int32_t* status;
+  int64_t B, Hq, Hkv, N, d, dv;
+  int32_t dtype;
+  int32_t bq, bk, causal;
+  int64_t nqb, nkb;
+  float scale;
+  float lambda;
+};
+sa_status launch_attn_simt(const AttnArgs& a, cudaStream_t st);
+sa_status launch_attn_tc(const AttnArgs& a, cudaStream_t st);
+bool attn_tc_supported(const sa_shape& s, int bq, int bk);
+
+}  // namespace sa

@@ -1,0 +1,333 @@
+"""ctypes binding of libsparseattn.so (C ABI in include/sparse_attn.h).
+
+Argument marshalling only: every function below packs its arguments into the
+C structs and calls the entry point of the same name; all computation runs in
+the library's CUDA kernels.  Tensors are torch CUDA tensors (PyTorch provides
+device memory and streams).  If the library is missing, loading fails with
+an error that says how to build it: there is no other implementation.
+
+``Pipeline`` strings the calls of one forward pass together (layout ->
+reorder -> mask prediction -> block-sparse attention -> inverse reorder) and
+owns the buffers it allocates through torch.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsparseattn.so")
+
+SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE = 0, 1, 2, 3
+SA_ERR_EMPTY_ROW, SA_ERR_TIMEOUT, SA_ERR_CUDA, SA_ERR_CAPACITY = 4, 5, 6, 7
+SA_BF16, SA_FP32 = 0, 1
+SA_ORDER = {"identity": 0, "window": 1, "hilbert": 2}
+SA_FLAG_FORCE_SIMT = 1
+
+STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_WORKSPACE",
+                4: "SA_ERR_EMPTY_ROW", 5: "SA_ERR_TIMEOUT", 6: "SA_ERR_CUDA", 7: "SA_ERR_CAPACITY"}
+
+EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_layout_workspace",
+           "sa_layout_build", "sa_reorder", "sa_unreorder", "sa_predict_mask_workspace",
+           "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_mask_from_blocks_workspace",
+           "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status"]
+
+
+class SAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("Hq", ctypes.c_int64), ("Hkv", ctypes.c_int64),
+                ("N", ctypes.c_int64), ("d", ctypes.c_int64), ("dv", ctypes.c_int64),
+                ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class LayoutDesc(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int64), ("W", ctypes.c_int64),
+                ("txt_len", ctypes.c_int64), ("sink_frames", ctypes.c_int64),
+                ("win", ctypes.c_int64 * 3), ("mode", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class MaskParams(ctypes.Structure):
+    _fields_ = [("bq", ctypes.c_int32), ("bk", ctypes.c_int32), ("tau", ctypes.c_float),
+                ("theta", ctypes.c_float), ("sink_tokens", ctypes.c_int64),
+                ("txt_len", ctypes.c_int64), ("local_window", ctypes.c_int64),
+                ("anchor_tokens", ctypes.c_int64), ("causal", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+class Mask(ctypes.Structure):
+    _fields_ = [("block_mask", ctypes.c_void_p), ("row_ptr", ctypes.c_void_p),
+                ("col_idx", ctypes.c_void_p), ("order", ctypes.c_void_p),
+                ("kept_total", ctypes.c_void_p), ("status", ctypes.c_void_p),
+                ("col_capacity", ctypes.c_int64), ("nqb", ctypes.c_int64), ("nkb", ctypes.c_int64),
+                ("bq", ctypes.c_int32), ("bk", ctypes.c_int32), ("causal", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} not found: build it with `python -m long_context_mean_b200.build` "
+                           "(there is no fallback implementation)")
+    lib = ctypes.CDLL(path)
+    P, I32, I64, SZ, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+    sig = {
+        "sa_version": (ctypes.c_char_p, []),
+        "sa_last_error": (ctypes.c_char_p, []),
+        "sa_attn_kernel_path": (I32, [ctypes.POINTER(Shape), I32, I32, I32]),
+        "sa_layout_workspace": (SZ, [ctypes.POINTER(LayoutDesc)]),
+        "sa_layout_build": (I32, [ctypes.POINTER(LayoutDesc), P, P, P, SZ, P]),
+        "sa_reorder": (I32, [P, P, P, I64, I64, I64, I32, P]),
+        "sa_unreorder": (I32, [P, P, P, I64, I64, I64, I32, P]),
+        "sa_predict_mask_workspace": (SZ, [ctypes.POINTER(Shape), ctypes.POINTER(MaskParams)]),
+        "sa_predict_mask_ws_layout": (I32, [ctypes.POINTER(Shape), ctypes.POINTER(MaskParams),
+                                            ctypes.POINTER(SZ * 6)]),
+        "sa_predict_mask": (I32, [P, P, ctypes.POINTER(Shape), ctypes.POINTER(MaskParams), P, SZ,
+                                  ctypes.POINTER(Mask), P]),
+        "sa_mask_from_blocks_workspace": (SZ, [ctypes.POINTER(Shape), I32, I32]),
+        "sa_mask_from_blocks": (I32, [P, ctypes.POINTER(Shape), I32, I32, I32, P, SZ,
+                                      ctypes.POINTER(Mask), P]),
+        "sa_block_sparse_attn": (I32, [P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F, F,
+                                       P, P, P, I32, P]),
+        "sa_dense_attn": (I32, [P, P, P, ctypes.POINTER(Shape), I32, F, P, P, P, I32, P]),
+        "sa_read_status": (I32, [P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(code: int):
+    if code != SA_OK:
+        raise SAError(code, load().sa_last_error().decode(errors="replace"))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return SA_BF16
+    if t.dtype == torch.float32:
+        return SA_FP32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def make_shape(q, k, v) -> Shape:
+    B, Hq, N, d = q.shape
+    return Shape(B, Hq, k.shape[1], N, d, v.shape[3], dtype_code(q), 0)
+
+
+def make_layout(T, H, W, txt_len=0, sink_frames=0, mode="identity", win=(1, 1, 1)) -> LayoutDesc:
+    w = (ctypes.c_int64 * 3)(*[int(x) for x in win])
+    return LayoutDesc(int(T), int(H), int(W), int(txt_len), int(sink_frames), w, SA_ORDER[mode], 0)
+
+
+def make_params(bq, bk, tau, theta=0.0, sink_tokens=0, txt_len=0, local_window=0,
+                anchor_tokens=0, causal=False) -> MaskParams:
+    return MaskParams(int(bq), int(bk), float(tau), float(theta), int(sink_tokens), int(txt_len),
+                      int(local_window), int(anchor_tokens), int(bool(causal)), 0)
+
+
+# ---------------------------------------------------------------------------
+# Thin wrappers (one per entry point)
+# ---------------------------------------------------------------------------
+
+def version() -> str:
+    return load().sa_version().decode()
+
+
+def attn_kernel_path(shape: Shape, bq: int, bk: int, flags: int = 0) -> int:
+    return int(load().sa_attn_kernel_path(ctypes.byref(shape), bq, bk, flags))
+
+
+def layout_workspace(desc: LayoutDesc) -> int:
+    return int(load().sa_layout_workspace(ctypes.byref(desc)))
+
+
+def layout_build(desc: LayoutDesc, perm, inv, ws=None, stream=None):
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(load().sa_layout_build(ctypes.byref(desc), _ptr(perm), _ptr(inv), _ptr(ws), nbytes,
+                                  _stream(stream)))
+
+
+def reorder(perm, x, y, stream=None):
+    """y[..., n, :] = x[..., perm[n], :] for x of shape [..., N, row]."""
+    N, row = x.shape[-2], x.shape[-1]
+    outer = x.numel() // (N * row)
+    _check(load().sa_reorder(_ptr(perm), _ptr(x), _ptr(y), outer, N, row, dtype_code(x), _stream(stream)))
+
+
+def unreorder(perm, y, x, stream=None):
+    """x[..., perm[n], :] = y[..., n, :]."""
+    N, row = y.shape[-2], y.shape[-1]
+    outer = y.numel() // (N * row)
+    _check(load().sa_unreorder(_ptr(perm), _ptr(y), _ptr(x), outer, N, row, dtype_code(y), _stream(stream)))
+
+
+def predict_mask_workspace(shape: Shape, params: MaskParams) -> int:
+    return int(load().sa_predict_mask_workspace(ctypes.byref(shape), ctypes.byref(params)))
+
+
+def predict_mask_ws_layout(shape: Shape, params: MaskParams):
+    off = (ctypes.c_size_t * 6)()
+    _check(load().sa_predict_mask_ws_layout(ctypes.byref(shape), ctypes.byref(params), ctypes.byref(off)))
+    return list(off)
+
+
+def predict_mask(q, k, shape: Shape, params: MaskParams, ws, mask: Mask, stream=None):
+    _check(load().sa_predict_mask(_ptr(q), _ptr(k), ctypes.byref(shape), ctypes.byref(params), _ptr(ws),
+                                  ws.numel() * ws.element_size(), ctypes.byref(mask), _stream(stream)))
+
+
+def mask_from_blocks_workspace(shape: Shape, bq: int, bk: int) -> int:
+    return int(load().sa_mask_from_blocks_workspace(ctypes.byref(shape), bq, bk))
+
+
+def mask_from_blocks(block_mask, shape: Shape, bq, bk, causal, ws, mask: Mask, stream=None):
+    _check(load().sa_mask_from_blocks(_ptr(block_mask), ctypes.byref(shape), bq, bk, int(bool(causal)),
+                                      _ptr(ws), ws.numel() * ws.element_size(), ctypes.byref(mask),
+                                      _stream(stream)))
+
+
+def block_sparse_attn(q, k, v, shape: Shape, mask: Mask, lam, scale, out, lse=None, skip_log=None,
+                      flags=0, stream=None):
+    _check(load().sa_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), ctypes.byref(mask),
+                                       float(lam), float(scale), _ptr(out), _ptr(lse), _ptr(skip_log),
+                                       int(flags), _stream(stream)))
+
+
+def dense_attn(q, k, v, shape: Shape, causal, scale, out, lse=None, status=None, flags=0, stream=None):
+    _check(load().sa_dense_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), int(bool(causal)),
+                                float(scale), _ptr(out), _ptr(lse), _ptr(status), int(flags),
+                                _stream(stream)))
+
+
+def read_status(status, stream=None) -> int:
+    """Synchronises the stream and returns the device status code (no raise)."""
+    return int(load().sa_read_status(_ptr(status), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# Buffers and the whole forward path
+# ---------------------------------------------------------------------------
+
+@dataclass
+class MaskBuffers:
+    block_mask: object
+    row_ptr: object
+    col_idx: object
+    order: object
+    kept_total: object
+    status: object
+    struct: Mask
+
+    @classmethod
+    def allocate(cls, B, Hq, N, bq, bk, device, capacity=None):
+        import torch
+        nqb, nkb = -(-N // bq), -(-N // bk)
+        R = B * Hq * nqb
+        cap = capacity if capacity is not None else R * nkb
+        bm = torch.zeros(R * nkb, dtype=torch.uint8, device=device)
+        rp = torch.zeros(R + 1, dtype=torch.int32, device=device)
+        ci = torch.zeros(max(1, cap), dtype=torch.int32, device=device)
+        od = torch.zeros(R, dtype=torch.int32, device=device)
+        kt = torch.zeros(1, dtype=torch.int64, device=device)
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        m = Mask(bm.data_ptr(), rp.data_ptr(), ci.data_ptr(), od.data_ptr(), kt.data_ptr(), st.data_ptr(),
+                 max(1, cap), nqb, nkb, bq, bk, 0, 0)
+        return cls(bm, rp, ci, od, kt, st, m)
+
+
+def workspace(nbytes, device):
+    """A 256-byte aligned byte buffer (torch allocations are 512-byte aligned)."""
+    import torch
+    return torch.empty(max(256, int(nbytes)), dtype=torch.uint8, device=device)
+
+
+class Pipeline:
+    """One forward pass of the block-sparse path for a fixed problem.
+
+    Allocates (through torch) the layout, reordered copies, workspace, mask
+    lists and outputs once; ``run(q, k, v)`` then enqueues, on the current
+    stream: layout build, reorder of Q, K, V, mask prediction, block-sparse
+    attention and inverse reorder of O and LSE.  Inputs are BNSD in the
+    original token order; ``out``/``lse`` come back in that order too.
+    """
+
+    def __init__(self, B, Hq, Hkv, N, d, dv, dtype, *, layout: LayoutDesc, params: MaskParams,
+                 lam=-math.inf, scale=0.0, flags=0, device="cuda", log_skips=False):
+        import torch
+        tdt = torch.bfloat16 if dtype in ("bf16", SA_BF16) else torch.float32
+        self.shape = Shape(B, Hq, Hkv, N, d, dv, SA_BF16 if tdt == torch.bfloat16 else SA_FP32, 0)
+        self.layout, self.params = layout, params
+        self.lam, self.scale, self.flags = lam, scale, flags
+        self.identity = layout.mode == SA_ORDER["identity"]
+        self.perm = torch.empty(N, dtype=torch.int32, device=device)
+        self.inv = torch.empty(N, dtype=torch.int32, device=device)
+        self.layout_ws = workspace(layout_workspace(layout), device)
+        if not self.identity:
+            self.qr = torch.empty(B, Hq, N, d, dtype=tdt, device=device)
+            self.kr = torch.empty(B, Hkv, N, d, dtype=tdt, device=device)
+            self.vr = torch.empty(B, Hkv, N, dv, dtype=tdt, device=device)
+            self.out_r = torch.empty(B, Hq, N, dv, dtype=tdt, device=device)
+            self.lse_r = torch.empty(B, Hq, N, 1, dtype=torch.float32, device=device)
+        self.out = torch.empty(B, Hq, N, dv, dtype=tdt, device=device)
+        self.lse = torch.empty(B, Hq, N, 1, dtype=torch.float32, device=device)
+        self.ws = workspace(predict_mask_workspace(self.shape, params), device)
+        self.mask = MaskBuffers.allocate(B, Hq, N, params.bq, params.bk, device)
+        self.skip_log = (torch.zeros(self.mask.col_idx.numel(), dtype=torch.uint8, device=device)
+                         if log_skips else None)
+
+    def run(self, q, k, v, stream=None):
+        if self.identity:
+            qr, kr, vr, out_r, lse_r = q, k, v, self.out, self.lse
+        else:
+            layout_build(self.layout, self.perm, self.inv, self.layout_ws, stream)
+            reorder(self.perm, q, self.qr, stream)
+            reorder(self.perm, k, self.kr, stream)
+            reorder(self.perm, v, self.vr, stream)
+            qr, kr, vr, out_r, lse_r = self.qr, self.kr, self.vr, self.out_r, self.lse_r
+        predict_mask(qr, kr, self.shape, self.params, self.ws, self.mask.struct, stream)
+        block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, out_r, lse_r,
+                          self.skip_log, self.flags, stream)
+        if not self.identity:
+            unreorder(self.perm, out_r, self.out, stream)
+            unreorder(self.perm, lse_r, self.lse, stream)
+        return self.out, self.lse
+
+    def status(self, stream=None) -> int:
+        return read_status(self.mask.status, stream)
+
+
+def pipeline_for(w, device="cuda", **kw) -> Pipeline:
+    """Pipeline for a workload description from ``inputs.WORKLOADS``."""
+    lay = make_layout(w.T, w.H, w.W, w.txt_len, w.sink_frames, w.order, w.win)
+    prm = make_params(w.bq, w.bk, w.tau, w.theta, w.sink_tokens, w.txt_len, w.local_window,
+                      w.anchor_tokens, w.causal)
+    return Pipeline(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, w.dtype, layout=lay, params=prm, lam=w.lam,
+                    device=device, **kw)

@@ -1,0 +1,126 @@
+"""The C ABI library loads, exports every declared entry point, and rejects
+bad arguments on the host (no GPU needed; no compute is launched)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_mean_b200 import sa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparse_attn.h")
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(sa.LIB_PATH):
+        from long_context_mean_b200 import build
+        build.build()
+    return sa.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_entry_points()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(sa.EXPORTS)
+
+
+def test_version(lib):
+    assert "sm_100a" in sa.version()
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = sa._lib
+    try:
+        sa._lib = None
+        with pytest.raises(RuntimeError, match="no fallback"):
+            sa.load(str(tmp_path / "nope.so"))
+    finally:
+        sa._lib = saved
+
+
+FAKE = ctypes.c_void_p(4096)
+
+
+def _shape(**kw):
+    base = dict(B=1, Hq=2, Hkv=2, N=300, d=128, dv=128, dtype=sa.SA_BF16)
+    base.update(kw)
+    return sa.Shape(base["B"], base["Hq"], base["Hkv"], base["N"], base["d"], base["dv"], base["dtype"], 0)
+
+
+def _mask():
+    return sa.Mask(4096, 4096, 4096, 4096, 4096, 4096, 100, 0, 0, 0, 0, 0, 0)
+
+
+def test_host_validation_codes(lib):
+    s = _shape()
+    p = sa.make_params(128, 64, 0.5)
+    null = ctypes.c_void_p(None)
+    m = _mask()
+    # layout
+    bad = sa.make_layout(0, 4, 4)
+    assert lib.sa_layout_build(ctypes.byref(bad), FAKE, FAKE, null, 0, null) == sa.SA_ERR_INVALID_ARG
+    big = sa.make_layout(3, 1000, 4, mode="hilbert")
+    assert lib.sa_layout_build(ctypes.byref(big), FAKE, FAKE, null, 0, null) == sa.SA_ERR_UNSUPPORTED
+    hil = sa.make_layout(5, 8, 8, mode="hilbert")
+    assert lib.sa_layout_build(ctypes.byref(hil), FAKE, FAKE, null, 0, null) == sa.SA_ERR_WORKSPACE
+    # reorder
+    assert lib.sa_reorder(FAKE, FAKE, FAKE, 1, 10, 128, 0, null) == sa.SA_ERR_INVALID_ARG  # in place
+    assert lib.sa_reorder(null, FAKE, ctypes.c_void_p(8192), 1, 10, 128, 0, null) == sa.SA_ERR_INVALID_ARG
+    # predict
+    p_bad = sa.make_params(128, 64, 0.0)
+    assert lib.sa_predict_mask(FAKE, FAKE, ctypes.byref(s), ctypes.byref(p_bad), FAKE, 1 << 30,
+                               ctypes.byref(m), null) == sa.SA_ERR_INVALID_ARG
+    p_blk = sa.make_params(256, 64, 0.5)
+    assert lib.sa_predict_mask(FAKE, FAKE, ctypes.byref(s), ctypes.byref(p_blk), FAKE, 1 << 30,
+                               ctypes.byref(m), null) == sa.SA_ERR_INVALID_ARG
+    s_d = _shape(d=96)
+    assert lib.sa_predict_mask(FAKE, FAKE, ctypes.byref(s_d), ctypes.byref(p), FAKE, 1 << 30,
+                               ctypes.byref(m), null) == sa.SA_ERR_UNSUPPORTED
+    assert lib.sa_predict_mask(FAKE, FAKE, ctypes.byref(s), ctypes.byref(p), FAKE, 16,
+                               ctypes.byref(m), null) == sa.SA_ERR_WORKSPACE
+    s_g = _shape(Hq=3, Hkv=2)
+    assert lib.sa_predict_mask(FAKE, FAKE, ctypes.byref(s_g), ctypes.byref(p), FAKE, 1 << 30,
+                               ctypes.byref(m), null) == sa.SA_ERR_INVALID_ARG
+    # attention
+    m2 = _mask()
+    m2.bq, m2.bk, m2.nqb, m2.nkb = 128, 64, 3, 5
+    assert lib.sa_block_sparse_attn(FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m2), ctypes.c_float(0.5),
+                                    ctypes.c_float(0), FAKE, null, null, 0, null) == sa.SA_ERR_INVALID_ARG
+    m2.nqb = 4   # wrong for N=300, bq=128
+    assert lib.sa_block_sparse_attn(FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m2), ctypes.c_float(-1),
+                                    ctypes.c_float(0), FAKE, null, null, 0, null) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_dense_attn(FAKE, FAKE, FAKE, ctypes.byref(s), 2, ctypes.c_float(0), FAKE, null, null, 0,
+                             null) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_read_status(null, null) == sa.SA_ERR_INVALID_ARG
+    assert b"status" in lib.sa_last_error()
+
+
+def test_workspace_queries_are_host_only(lib):
+    s = _shape(N=20506, Hq=24, Hkv=24)
+    p = sa.make_params(128, 64, 0.5)
+    off = sa.predict_mask_ws_layout(s, p)
+    nqb, nkb = -(-20506 // 128), -(-20506 // 64)
+    assert off[0] == 0 and off[1] >= 24 * nqb * 128 * 4
+    assert sa.predict_mask_workspace(s, p) >= off[5] + 24 * nqb * 4
+    assert all(o % 256 == 0 for o in off)
+    assert sa.layout_workspace(sa.make_layout(21, 45, 80, 0, 1, "hilbert")) >= 2 * (1 << 21) // 8
+    assert sa.layout_workspace(sa.make_layout(13, 30, 52, 226, 1, "window", (2, 8, 8))) == 0
+
+
+def test_kernel_path_selection(lib):
+    s = _shape()
+    assert sa.attn_kernel_path(s, 128, 64, sa.SA_FLAG_FORCE_SIMT) == 0
+    s32 = _shape(dtype=sa.SA_FP32, d=16, dv=16)
+    assert sa.attn_kernel_path(s32, 16, 16) == 0
+    assert sa.attn_kernel_path(s, 129, 64) == -1

@@ -1,0 +1,105 @@
+"""GPU parity of the whole forward path (layout -> reorder -> predict ->
+attention -> inverse reorder) against the oracle, on the toy ledger and on
+sampled rows of the image and video workloads at full size."""
+
+import math
+
+import numpy as np
+import pytest
+
+from long_context_mean_b200 import inputs as I
+from oracle import attention as A
+from oracle import layout as Y
+from oracle import predict as Pr
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def run_pipeline(w, g, flags=0):
+    from long_context_mean_b200 import sa
+    q, k, v = P.qkv_dev(g, w.dtype)
+    pipe = sa.pipeline_for(w, flags=flags, log_skips=True)
+    out, lse = pipe.run(q, k, v)
+    st = pipe.status()
+    return pipe, out.float().cpu().numpy(), lse.cpu().numpy()[..., 0], st
+
+
+def oracle_check(w, g, pipe, out, lse, heads, qblocks):
+    """Oracle on the permuted inputs with the GPU's mask (validated against
+    the oracle's own mask up to the boundary bands first)."""
+    perm, inv = Y.build_layout(w.order, w.T, w.H, w.W, w.win, w.sink_frames, w.txt_len)
+    q, k, v = (Y.reorder(g[n], perm) for n in "qkv")
+    B, Hq = w.B, w.Hq
+    nqb, nkb = pipe.mask.struct.nqb, pipe.mask.struct.nkb
+    gmask = pipe.mask.block_mask.cpu().numpy().reshape(B, Hq, nqb, nkb).astype(bool)
+    orc = Pr.predict_mask(q, k, w.bq, w.bk, w.tau, w.theta, w.causal, w.sink_tokens, w.txt_len,
+                          w.local_window, w.anchor_tokens)
+    P.compare_masks(gmask, orc, w.tau, w.theta, w.Hq // w.Hkv)
+    ref = A.block_sparse_attention_heads(q, k, v, gmask, w.bq, w.bk, w.causal, w.lam, heads=heads,
+                                         qblocks=qblocks)
+    if w.lam > -math.inf:
+        rp = pipe.mask.row_ptr.cpu().numpy()
+        ci = pipe.mask.col_idx.cpu().numpy()
+        over = P.skip_override_from_gpu(pipe.skip_log.cpu().numpy(), rp, ci, nqb, B, Hq)
+        if P.check_skip_decisions(over, ref["skips"], ref["gaps"], w.lam):
+            ref = A.block_sparse_attention_heads(q, k, v, gmask, w.bq, w.bk, w.causal, w.lam, heads=heads,
+                                                 qblocks=qblocks, skip_override=over, band=P.LAMBDA_BAND)
+    # back to the original token order
+    ref_out = Y.unreorder(ref["out"], perm, axis=2)
+    ref_lse = Y.unreorder(ref["lse"], perm, axis=2)
+    return P.attention_check(out, lse, {"out": ref_out, "lse": ref_lse})
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+def test_toy_pipeline(flags):
+    w = I.WORKLOADS["toy"]
+    g = I.gen_qkv(w)
+    pipe, out, lse, st = run_pipeline(w, g, flags)
+    assert st == 0
+    oracle_check(w, g, pipe, out, lse, None, None)
+
+
+def test_toy_full_and_same_frame_masks():
+    """The worked example's fixed masks on the toy grid: full and same-frame
+    (block-diagonal 16-token blocks) through sa_mask_from_blocks."""
+    import torch
+    from long_context_mean_b200 import sa
+    w = I.WORKLOADS["toy"]
+    g = I.gen_qkv(w)
+    q, k, v = P.qkv_dev(g, "fp32")
+    shape = sa.make_shape(q, k, v)
+    for name, blocks in (("full", np.ones((4, 4), bool)), ("spatial", np.eye(4, dtype=bool))):
+        mb = sa.MaskBuffers.allocate(1, 1, 64, 16, 16, "cuda")
+        ws = sa.workspace(sa.mask_from_blocks_workspace(shape, 16, 16), "cuda")
+        sa.mask_from_blocks(torch.from_numpy(blocks.astype(np.uint8).ravel()).cuda(), shape, 16, 16, False,
+                            ws, mb.struct)
+        out = torch.empty_like(q)
+        lse = torch.empty(1, 1, 64, dtype=torch.float32, device="cuda")
+        sa.block_sparse_attn(q, k, v, shape, mb.struct, -math.inf, 0.0, out, lse)
+        assert sa.read_status(mb.status) == 0
+        tok = A.kept_blocks_to_token_mask(blocks, 64, 16, 16)
+        y, _, l = A.masked_attention(g["q"][0, 0], g["k"][0, 0], g["v"][0, 0], tok)
+        assert np.abs(out.cpu().numpy()[0, 0] - y).max() < 1e-5
+        assert np.abs(lse.cpu().numpy()[0, 0] - l).max() < 1e-5
+
+
+@pytest.mark.parametrize("name", ["video", "image"])
+def test_full_size_pipeline_sampled(name):
+    w = I.WORKLOADS[name]
+    g = I.gen_qkv(w)
+    pipe, out, lse, st = run_pipeline(w, g)
+    assert st == 0
+    nqb = pipe.mask.struct.nqb
+    heads = [(0, 0), (0, w.Hq - 1)] + ([(1, 5)] if w.B > 1 else [(0, 7)])
+    qblocks = sorted({0, 1, nqb // 2, nqb - 2, nqb - 1})
+    perm, _ = Y.build_layout(w.order, w.T, w.H, w.W, w.win, w.sink_frames, w.txt_len)
+    rows = np.zeros(w.N, bool)
+    for qb in qblocks:
+        rows[qb * w.bq:(qb + 1) * w.bq] = True
+    rows_orig = np.zeros(w.N, bool)
+    rows_orig[perm[rows]] = True
+    sel = np.zeros((w.B, w.Hq, w.N), bool)
+    for b, h in heads:
+        sel[b, h] = rows_orig
+    oracle_check(w, g, pipe, out, lse, heads, qblocks)

@@ -1,0 +1,191 @@
+"""GPU parity: mask prediction (pooling, similarity guard, TopCdf, forced
+blocks) and the CSR lists / work order, against the fp64 oracle."""
+
+import math
+
+import numpy as np
+import pytest
+
+from long_context_mean_b200 import inputs as I
+from oracle import layout as Y
+from oracle import predict as Pr
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu_predict(q_dev, k_dev, w, params, capacity=None):
+    import torch
+    from long_context_mean_b200 import sa
+    shape = sa.Shape(q_dev.shape[0], q_dev.shape[1], k_dev.shape[1], q_dev.shape[2], q_dev.shape[3],
+                     q_dev.shape[3], sa.dtype_code(q_dev), 0)
+    ws = sa.workspace(sa.predict_mask_workspace(shape, params), "cuda")
+    ws.fill_(0xFF)          # poison: every output must be written
+    mb = sa.MaskBuffers.allocate(shape.B, shape.Hq, shape.N, params.bq, params.bk, "cuda", capacity)
+    mb.row_ptr.fill_(-7)
+    mb.order.fill_(-7)
+    sa.predict_mask(q_dev, k_dev, shape, params, ws, mb.struct)
+    status = sa.read_status(mb.status)
+    off = sa.predict_mask_ws_layout(shape, params)
+    nqb, nkb = mb.struct.nqb, mb.struct.nkb
+    B, Hq, Hkv, d = shape.B, shape.Hq, shape.Hkv, shape.d
+
+    def view(i, n):
+        return ws[off[i]:off[i] + n * 4].view(torch.float32).cpu().numpy()
+    out = {
+        "status": status,
+        "qhat": view(0, B * Hq * nqb * d).reshape(B, Hq, nqb, d),
+        "khat": view(1, B * Hkv * nkb * d).reshape(B, Hkv, nkb, d),
+        "s_q": view(2, B * Hq * nqb).reshape(B, Hq, nqb),
+        "s_k": view(3, B * Hkv * nkb).reshape(B, Hkv, nkb),
+        "mask": mb.block_mask.cpu().numpy().reshape(B, Hq, nqb, nkb).astype(bool),
+        "row_ptr": mb.row_ptr.cpu().numpy(),
+        "col_idx": mb.col_idx.cpu().numpy(),
+        "order": mb.order.cpu().numpy(),
+        "kept_total": int(mb.kept_total.item()),
+    }
+    return out
+
+
+def oracle_predict(q, k, w):
+    return Pr.predict_mask(q, k, w.bq, w.bk, w.tau, w.theta, w.causal, w.sink_tokens, w.txt_len,
+                           w.local_window, w.anchor_tokens)
+
+
+def check_lists(g, mask):
+    c = Pr.mask_to_csr(mask)
+    assert g["kept_total"] == c["kept_total"]
+    assert np.array_equal(g["row_ptr"], c["row_ptr"])
+    assert np.array_equal(g["col_idx"][:c["kept_total"]], c["col_idx"])
+    assert np.array_equal(g["order"], c["order"])
+
+
+def check_predict(w, q_np, k_np, q_dev, k_dev):
+    from long_context_mean_b200 import sa
+    prm = sa.make_params(w.bq, w.bk, w.tau, w.theta, w.sink_tokens, w.txt_len, w.local_window,
+                         w.anchor_tokens, w.causal)
+    g = run_gpu_predict(q_dev, k_dev, w, prm)
+    assert g["status"] == sa.SA_OK
+    orc = oracle_predict(q_np, k_np, w)
+    np.testing.assert_allclose(g["qhat"], orc["qhat"], rtol=0, atol=2e-6 * max(1, np.abs(orc["qhat"]).max()))
+    np.testing.assert_allclose(g["khat"], orc["khat"], rtol=0, atol=2e-6 * max(1, np.abs(orc["khat"]).max()))
+    np.testing.assert_allclose(g["s_q"], orc["s_q"], rtol=0, atol=2e-6)
+    np.testing.assert_allclose(g["s_k"], orc["s_k"], rtol=0, atol=2e-6)
+    ndiff = P.compare_masks(g["mask"], orc, w.tau, w.theta, w.Hq // w.Hkv)
+    # The lists are a function of the mask: bit-exact against the oracle's
+    # compaction of the GPU's mask (identical to the oracle's own mask when
+    # no boundary block differs).
+    check_lists(g, g["mask"])
+    if ndiff == 0:
+        check_lists(g, orc["mask"])
+    return g, orc, ndiff
+
+
+SMALL = [
+    # name, B, Hq, Hkv, N, d, bq, bk, tau, theta, causal, sink, txt, window, anchors, dtype
+    ("plain", 1, 2, 2, 700, 64, 64, 32, 0.6, 0.0, False, 0, 0, 0, 0, "bf16"),
+    ("guard", 2, 3, 3, 513, 128, 128, 64, 0.5, 0.25, False, 0, 0, 0, 0, "bf16"),
+    ("sink_text", 1, 2, 2, 1000, 128, 128, 64, 0.3, 0.0, False, 130, 77, 0, 0, "bf16"),
+    ("causal_gqa", 1, 4, 2, 1500, 128, 128, 64, 0.8, 0.0, True, 0, 0, 300, 128, "bf16"),
+    ("causal_small_blocks", 1, 2, 1, 333, 32, 16, 8, 0.9, 0.0, True, 0, 0, 40, 5, "fp32"),
+    ("toy", 1, 1, 1, 64, 16, 16, 16, 0.9, 0.5, False, 0, 0, 0, 0, "fp32"),
+    ("tau_one", 1, 2, 2, 640, 128, 128, 64, 1.0, 0.0, False, 0, 0, 0, 0, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_predict_small(case):
+    name, B, Hq, Hkv, N, d, bq, bk, tau, theta, causal, sink, txt, win, anch, dt = case
+    w = I.Workload(name, 77 + len(name), B, Hq, Hkv, 1, 1, N - txt, txt, d, d, dt, "field" if Hq == Hkv else "lowrank",
+                   bq=bq, bk=bk, tau=tau, theta=theta, causal=causal, local_window=win,
+                   anchor_tokens=anch, sigma=(0.0, 0.0, 6.0), sigma_pos=20.0)
+    g = I.gen_qkv(w)
+    q_dev, k_dev, _ = P.qkv_dev(g, dt)
+    # sink tokens are given directly for these synthetic cases
+    from long_context_mean_b200 import sa
+    prm = sa.make_params(bq, bk, tau, theta, sink, txt, win, anch, causal)
+    gres = run_gpu_predict(q_dev, k_dev, w, prm)
+    assert gres["status"] == sa.SA_OK
+    orc = Pr.predict_mask(g["q"], g["k"], bq, bk, tau, theta, causal, sink, txt, win, anch)
+    np.testing.assert_allclose(gres["s_q"], orc["s_q"], rtol=0, atol=2e-6)
+    np.testing.assert_allclose(gres["s_k"], orc["s_k"], rtol=0, atol=2e-6)
+    np.testing.assert_allclose(gres["qhat"], orc["qhat"], rtol=0, atol=1e-5)
+    P.compare_masks(gres["mask"], orc, tau, theta, Hq // Hkv)
+    check_lists(gres, gres["mask"])
+    assert gres["mask"].any()
+
+
+@pytest.mark.parametrize("name", ["video", "image"])
+def test_predict_full_size(name):
+    w = I.WORKLOADS[name]
+    g = I.gen_qkv(w)
+    perm, _ = Y.build_layout(w.order, w.T, w.H, w.W, w.win, w.sink_frames, w.txt_len)
+    qn, kn = Y.reorder(g["q"], perm), Y.reorder(g["k"], perm)
+    import torch
+    q_dev = P.bf16_dev(Y.reorder(g["q_bits"], perm))
+    k_dev = P.bf16_dev(Y.reorder(g["k_bits"], perm))
+    gres, orc, ndiff = check_predict(w, qn, kn, q_dev, k_dev)
+    valid = np.broadcast_to(orc["valid"][:, None], gres["mask"].shape)
+    sp = Pr.block_sparsity(gres["mask"], valid)
+    if name == "video":
+        assert abs(sp - w.target_sparsity) < 0.01
+    else:
+        assert sp == 0.0     # theta = 0.6 forces every block of this generator
+
+
+def test_empty_row_status():
+    import torch
+    from long_context_mean_b200 import sa
+    B, Hq, N, bq, bk = 1, 2, 256, 128, 64
+    shape = sa.Shape(B, Hq, Hq, N, 128, 128, sa.SA_BF16, 0)
+    nqb, nkb = 2, 4
+    blocks = torch.ones(B * Hq * nqb * nkb, dtype=torch.uint8, device="cuda")
+    blocks.view(B * Hq, nqb, nkb)[1, 1, :] = 0          # head 1, q-block 1: nothing kept
+    mb = sa.MaskBuffers.allocate(B, Hq, N, bq, bk, "cuda")
+    ws = sa.workspace(sa.mask_from_blocks_workspace(shape, bq, bk), "cuda")
+    sa.mask_from_blocks(blocks, shape, bq, bk, False, ws, mb.struct)
+    assert sa.read_status(mb.status) == sa.SA_ERR_EMPTY_ROW
+    # causal: q-block 1 (rows 128..255) keeping only k-block 3 (keys 192..255)
+    blocks.fill_(0)
+    blocks.view(B * Hq, nqb, nkb)[:, 0, 0] = 1
+    blocks.view(B * Hq, nqb, nkb)[:, 1, 3] = 1
+    sa.mask_from_blocks(blocks, shape, bq, bk, True, ws, mb.struct)
+    assert sa.read_status(mb.status) == sa.SA_ERR_EMPTY_ROW
+    blocks.view(B * Hq, nqb, nkb)[:, 1, 2] = 1
+    sa.mask_from_blocks(blocks, shape, bq, bk, True, ws, mb.struct)
+    assert sa.read_status(mb.status) == sa.SA_OK
+
+
+def test_capacity_status():
+    import torch
+    from long_context_mean_b200 import sa
+    shape = sa.Shape(1, 1, 1, 512, 128, 128, sa.SA_BF16, 0)
+    blocks = torch.ones(4 * 8, dtype=torch.uint8, device="cuda")
+    mb = sa.MaskBuffers.allocate(1, 1, 512, 128, 64, "cuda", capacity=31)
+    ws = sa.workspace(sa.mask_from_blocks_workspace(shape, 128, 64), "cuda")
+    sa.mask_from_blocks(blocks, shape, 128, 64, False, ws, mb.struct)
+    assert sa.read_status(mb.status) == sa.SA_ERR_CAPACITY
+
+
+def test_mask_from_blocks_lists_and_causal_and():
+    import torch
+    from long_context_mean_b200 import sa
+    rng = np.random.default_rng(3)
+    B, Hq, N, bq, bk = 2, 3, 1000, 128, 64
+    nqb, nkb = 8, 16
+    m = rng.random((B, Hq, nqb, nkb)) < 0.3
+    m[..., 0] = True
+    shape = sa.Shape(B, Hq, Hq, N, 128, 128, sa.SA_BF16, 0)
+    blocks = torch.from_numpy(m.astype(np.uint8).ravel()).to("cuda")
+    mb = sa.MaskBuffers.allocate(B, Hq, N, bq, bk, "cuda")
+    ws = sa.workspace(sa.mask_from_blocks_workspace(shape, bq, bk), "cuda")
+    sa.mask_from_blocks(blocks, shape, bq, bk, True, ws, mb.struct)
+    assert sa.read_status(mb.status) == sa.SA_OK
+    valid = np.array([[not Pr.causal_future(qb, kb, N, bq, bk) for kb in range(nkb)] for qb in range(nqb)])
+    want = m & valid
+    got = mb.block_mask.cpu().numpy().reshape(B, Hq, nqb, nkb).astype(bool)
+    assert np.array_equal(got, want)
+    c = Pr.mask_to_csr(want)
+    assert np.array_equal(mb.row_ptr.cpu().numpy(), c["row_ptr"])
+    assert np.array_equal(mb.col_idx.cpu().numpy()[:c["kept_total"]], c["col_idx"])
+    assert np.array_equal(mb.order.cpu().numpy(), c["order"])
