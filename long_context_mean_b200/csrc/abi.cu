@@ -265,9 +265,9 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
   }
   const bool tc_ok = !(flags & SA_FLAG_FORCE_SIMT) && is_sm100();
   if (!mask) {
-    if (tc_ok && attn_tc_supported(*shape, 128, 128)) {
+    if (tc_ok && attn_tc_supported(*shape, 128, 64)) {
       a.bq = 128;
-      a.bk = 128;
+      a.bk = 64;
     } else {
       a.bq = 64;
       a.bk = 64;

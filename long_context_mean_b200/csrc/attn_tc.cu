@@ -6,25 +6,29 @@
 // (rowmax S - running max) < lambda, l still counting the tile.
 //
 // Design (bf16, d = dv = 128, bq = 128, bk = 64 or 128):
-//   * persistent grid, one CTA per SM, work units (b, h, q-block) taken in
-//     the work order of the mask (rows by descending kept count);
-//   * warp 0 (one lane): TMA producer -- Q tile once per unit, K and V tiles
-//     of the unit's kept key blocks through a STAGES-deep ring;
-//   * warp 1 (one lane): tcgen05.mma issuer -- S = Q K^T into one of two
-//     TMEM S buffers, then O += P V into the TMEM O accumulator, one tile
-//     behind, so the tensor core works on S(t+1) and PV(t) while the softmax
-//     warps work on S(t+1)'s predecessor;
-//   * warps 4..7 (one thread per query row, TMEM lanes 0..127): load S from
-//     TMEM, mask, running max, the lambda decision for the whole block (a
-//     named barrier across the four warps), exp2, P to shared memory in the
-//     SW128 K-major layout the MMA reads, O rescale in TMEM when the reference
-//     maximum moves, and the epilogue O / l, LSE.
+//   * persistent grid, one CTA per SM.  A CTA runs PIPES independent
+//     pipelines (2 for bk = 64, 1 for bk = 128), each on its own stream of
+//     work units (b, h, q-block) taken in the mask's work order, so every
+//     SM sub-partition holds PIPES softmax warps;
+//   * per pipeline, warp p (one lane) is the TMA producer (Q tile once per
+//     unit, K and V tiles of the kept key blocks through a STAGES ring) and
+//     warp 2+p (one lane) issues tcgen05.mma: S = Q K^T into one of two TMEM
+//     S buffers, and O += P V one tile behind with P read from TMEM (the
+//     softmax overwrites S with P in place), so the tensor core runs S(t+1)
+//     and PV(t-1) while the softmax warps work on S(t);
+//   * per pipeline, four softmax warps (one thread per query row = TMEM
+//     lane): S from TMEM, masks, running max, exp2, P back to TMEM, O rescale
+//     in TMEM when the reference maximum moves, the epilogue O / l and LSE.
+//     Each warp publishes the largest (tile max - running max) of its rows;
+//     the MMA warp combines the four and takes the lambda decision, so the
+//     softmax warps never wait for one another.
 //   The exact running max drives the lambda test; O and l use a reference
-//   maximum that is only moved when the running max exceeds it by more than
-//   2^8 (the final O / l is the same quotient).
+//   maximum that only moves when the running max exceeds it by more than
+//   2^8 (O / l is the same quotient).  A row whose maximum moves has a gap of
+//   0, so a tile that needs a rescale is never skipped.
 // Every mbarrier wait is bounded (2 s); on expiry the kernel raises
-// SA_ERR_TIMEOUT, every later wait returns at once, the producer drains its
-// own loads (bounded) and the TMEM allocation is released.
+// SA_ERR_TIMEOUT, every later wait returns at once, the producers drain
+// their own loads (bounded) and the TMEM allocation is released.
 #include <cuda.h>
 
 #include "sa_internal.cuh"
@@ -32,10 +36,6 @@
 namespace sa {
 namespace {
 
-constexpr int kThreadsTC = 256;
-constexpr int kWarpTMA = 0;
-constexpr int kWarpMMA = 1;
-constexpr int kWarpSoftmax0 = 4;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
@@ -43,30 +43,31 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 template <int BK>
 struct Cfg {
-  static constexpr int STAGES = BK == 64 ? 3 : 2;
+  static constexpr int PIPES = BK == 64 ? 2 : 1;
+  static constexpr int STAGES = BK == 64 ? 2 : 3;
+  static constexpr int THREADS = 128 + 128 * PIPES;
   static constexpr int Q_BYTES = 128 * 128 * 2;
   static constexpr int KV_BYTES = BK * 128 * 2;
   static constexpr int KV_CHUNK = BK * 128;          // one 64-column chunk: BK rows x 128 B
-  static constexpr int P_BYTES = 128 * BK * 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;
-  static constexpr int OFF_CTL = OFF_P + 2 * P_BYTES;
+  static constexpr int PIPE_BYTES = Q_BYTES + 2 * STAGES * KV_BYTES;
+  static constexpr int OFF_CTL = PIPES * PIPE_BYTES;
   static constexpr int CTL_BYTES = 1024;
-  static constexpr int SMEM = OFF_CTL + CTL_BYTES + 1024;   // + alignment slack
-  static constexpr int TMEM_COLS = (128 + 2 * BK) <= 256 ? 256 : 512;
-  static constexpr int S_COL = 128;                          // O occupies columns 0..127
+  static constexpr int SMEM = OFF_CTL + PIPES * CTL_BYTES + 1024;   // + alignment slack
+  static constexpr int TMEM_PIPE = (128 + 2 * BK) <= 256 ? 256 : 512;
+  static constexpr int TMEM_COLS = PIPES * TMEM_PIPE;
+  static constexpr int S_COL = 128;                  // O occupies columns 0..127 of a pipe
+  static __host__ __device__ constexpr int off_q(int p) { return p * PIPE_BYTES; }
+  static __host__ __device__ constexpr int off_k(int p) { return p * PIPE_BYTES + Q_BYTES; }
+  static __host__ __device__ constexpr int off_v(int p) { return p * PIPE_BYTES + Q_BYTES + STAGES * KV_BYTES; }
 };
 
-// Control block at OFF_CTL (8-byte mbarriers first).
+// Per-pipeline control block (8-byte mbarriers first).
 struct Ctl {
   uint64_t q_full, q_empty, o_free;
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
-  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
+  uint64_t s_full[2], p_full[2], pv_done[2];
   uint32_t tmem_base;
   volatile uint32_t abort;
-  volatile uint32_t skip_flag[2];
   float gapw[2][4];
 };
 
@@ -120,15 +121,15 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
 }
 // Bounded wait.  Returns false when the CTA is aborting (a wait elsewhere
 // expired) or this wait expired (then it raises the abort itself).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl* ctl, int32_t* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl* g, int32_t* status) {
   if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 63) == 0) {
-      if (ctl->abort) return false;
+      if (g->abort) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {
-        ctl->abort = 1;
+        g->abort = 1;
         raise_status(status, SA_ERR_TIMEOUT);
         return false;
       }
@@ -152,16 +153,22 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void named_bar(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// D (TMEM) = A (SMEM desc) x B (SMEM desc) [+ D]
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// D (TMEM) = A (TMEM) x B (SMEM desc) [+ D]
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -182,8 +189,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
-  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -244,40 +250,285 @@ __device__ __forceinline__ int64_t kblock_at(const TcParams& p, const Unit& u, i
   return p.row_ptr ? p.col_idx[u.lo + t] : t;
 }
 
+// ---------------------------------------------------------------------------
+// Roles
+// ---------------------------------------------------------------------------
 template <int BK>
-__global__ void __launch_bounds__(kThreadsTC, 1)
+__device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                         const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, int pipe) {
+  using C = Cfg<BK>;
+  uint32_t kv_it = 0, nq = 0;
+  for (int i = blockIdx.x * C::PIPES + pipe; i < p.num_units; i += gridDim.x * C::PIPES) {
+    const Unit u = unit_at(p, i, BK);
+    if (u.n <= 0) continue;
+    mbar_wait(&c->q_empty, (nq & 1) ^ 1, g, p.status);
+    ++nq;
+    mbar_expect_tx(&c->q_full, C::Q_BYTES);
+    tma_load_3d(sb + C::off_q(pipe), tmQ, 0, (int)(u.qb * 128), (int)u.bh, &c->q_full);
+    tma_load_3d(sb + C::off_q(pipe) + C::Q_BYTES / 2, tmQ, 64, (int)(u.qb * 128), (int)u.bh, &c->q_full);
+    for (int64_t t = 0; t < u.n; ++t, ++kv_it) {
+      const int kb = (int)kblock_at(p, u, t);
+      const int s = kv_it % C::STAGES;
+      const uint32_t ph = (kv_it / C::STAGES) & 1;
+      const uint32_t kdst = sb + C::off_k(pipe) + s * C::KV_BYTES;
+      const uint32_t vdst = sb + C::off_v(pipe) + s * C::KV_BYTES;
+      mbar_wait(&c->k_empty[s], ph ^ 1, g, p.status);
+      mbar_expect_tx(&c->k_full[s], C::KV_BYTES);
+      tma_load_3d(kdst, tmK, 0, kb * BK, (int)u.kvh, &c->k_full[s]);
+      tma_load_3d(kdst + C::KV_CHUNK, tmK, 64, kb * BK, (int)u.kvh, &c->k_full[s]);
+      mbar_wait(&c->v_empty[s], ph ^ 1, g, p.status);
+      mbar_expect_tx(&c->v_full[s], C::KV_BYTES);
+      tma_load_3d(vdst, tmV, 0, kb * BK, (int)u.kvh, &c->v_full[s]);
+      tma_load_3d(vdst + C::KV_CHUNK, tmV, 64, kb * BK, (int)u.kvh, &c->v_full[s]);
+    }
+  }
+  // Drain: the last loads of every stage (and the last Q) have landed.
+  if (nq > 0) mbar_drain(&c->q_full, (nq - 1) & 1);
+  for (uint32_t j = kv_it > (uint32_t)C::STAGES ? kv_it - C::STAGES : 0; j < kv_it; ++j) {
+    mbar_drain(&c->k_full[j % C::STAGES], (j / C::STAGES) & 1);
+    mbar_drain(&c->v_full[j % C::STAGES], (j / C::STAGES) & 1);
+  }
+}
+
+template <int BK>
+__device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint32_t tm, int pipe) {
+  using C = Cfg<BK>;
+  constexpr uint32_t idesc_s = make_idesc(128, BK, 0);
+  constexpr uint32_t idesc_pv = make_idesc(128, 128, 1);
+  uint32_t kv_it = 0, gt0 = 0, unit_it = 0;   // unit_it counts units with work
+  for (int i = blockIdx.x * C::PIPES + pipe; i < p.num_units; i += gridDim.x * C::PIPES) {
+    const Unit u = unit_at(p, i, BK);
+    if (u.n <= 0) continue;
+    mbar_wait(&c->q_full, unit_it & 1, g, p.status);
+    tc_fence_after();
+    bool first_pv = true;
+    auto do_pv = [&](int64_t tt) {
+      const uint32_t it = kv_it + (uint32_t)tt, gt = gt0 + (uint32_t)tt;
+      const int s = it % C::STAGES;
+      const uint32_t ph = (it / C::STAGES) & 1;
+      const int gb = gt & 1;
+      mbar_wait(&c->p_full[gb], (gt >> 1) & 1, g, p.status);
+      tc_fence_after();
+      const float gap = fmaxf(fmaxf(c->gapw[gb][0], c->gapw[gb][1]), fmaxf(c->gapw[gb][2], c->gapw[gb][3]));
+      const bool skip = gap < p.lam_log2;
+      if (p.skip_log && p.row_ptr) p.skip_log[u.lo + tt] = skip ? 1 : 0;
+      if (tt == 0) {
+        mbar_wait(&c->o_free, (unit_it & 1) ^ 1, g, p.status);
+        tc_fence_after();
+      }
+      mbar_wait(&c->v_full[s], ph, g, p.status);
+      tc_fence_after();
+      if (!skip) {
+        const uint32_t vbase = sb + C::off_v(pipe) + s * C::KV_BYTES;
+        const uint32_t pcol = tm + C::S_COL + gb * BK;   // P (bf16 pairs) over the S buffer
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t b = desc_sw128(vbase + kk * 2048, C::KV_CHUNK, 1024);
+          umma_ts(tm, pcol + kk * 8, b, idesc_pv, (first_pv && kk == 0) ? 0u : 1u);
+        }
+        first_pv = false;
+      }
+      umma_commit(&c->v_empty[s]);
+      umma_commit(&c->pv_done[gb]);
+    };
+    for (int64_t t = 0; t < u.n; ++t) {
+      const uint32_t it = kv_it + (uint32_t)t, gt = gt0 + (uint32_t)t;
+      const int s = it % C::STAGES;
+      const uint32_t ph = (it / C::STAGES) & 1;
+      const int gb = gt & 1;
+      mbar_wait(&c->k_full[s], ph, g, p.status);
+      tc_fence_after();
+      const uint32_t kbase = sb + C::off_k(pipe) + s * C::KV_BYTES;
+      const uint32_t qbase = sb + C::off_q(pipe);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t a = desc_sw128(qbase + (kk >> 2) * (C::Q_BYTES / 2) + (kk & 3) * 32, 16, 1024);
+        const uint64_t b = desc_sw128(kbase + (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32, 16, 1024);
+        umma_ss(tm + C::S_COL + gb * BK, a, b, idesc_s, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(&c->s_full[gb]);
+      umma_commit(&c->k_empty[s]);
+      if (t == u.n - 1) umma_commit(&c->q_empty);
+      if (t >= 1) do_pv(t - 1);
+    }
+    do_pv(u.n - 1);
+    kv_it += (uint32_t)u.n;
+    gt0 += (uint32_t)u.n;
+    ++unit_it;
+  }
+}
+
+template <int BK>
+__device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int pipe, int wq, int lane) {
+  using C = Cfg<BK>;
+  const int row = wq * 32 + lane;
+  const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+  const float sc = p.scale_log2;
+  uint32_t gt0 = 0;
+  for (int i = blockIdx.x * C::PIPES + pipe; i < p.num_units; i += gridDim.x * C::PIPES) {
+    const Unit u = unit_at(p, i, BK);
+    const int64_t row_g = u.qb * 128 + row;
+    const bool row_valid = row_g < p.N;
+    if (u.n <= 0) {
+      if (row_valid) raise_status(p.status, SA_ERR_EMPTY_ROW);
+      continue;
+    }
+    float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
+    for (int64_t t = 0; t < u.n; ++t) {
+      const uint32_t gt = gt0 + (uint32_t)t;
+      const int gb = gt & 1;
+      const uint32_t scol = tm + lane_off + C::S_COL + gb * BK;
+      mbar_wait(&c->s_full[gb], (gt >> 1) & 1, g, p.status);
+      tc_fence_after();
+      float s[BK];
+#pragma unroll
+      for (int cc = 0; cc < BK / 32; ++cc) tmem_ld32(scol + cc * 32, s + cc * 32);
+      tmem_wait_ld();
+
+      const int64_t k0 = kblock_at(p, u, t) * BK;
+      if ((k0 + BK > p.N) || (p.causal && k0 + BK - 1 > u.qb * 128)) {
+#pragma unroll
+        for (int j = 0; j < BK; ++j) {
+          const int64_t key = k0 + j;
+          if (key >= p.N || (p.causal && key > row_g)) s[j] = -INFINITY;
+        }
+      }
+      // Row max as a tree (independent chains), in raw score units.
+      float mx[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) mx[j] = s[j];
+#pragma unroll
+      for (int j = 16; j < BK; ++j) mx[j & 15] = fmaxf(mx[j & 15], s[j]);
+#pragma unroll
+      for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
+      const float mloc = mx[0] * sc;                    // scale > 0: max commutes
+      const float m_new = fmaxf(m_run, mloc);
+      float gap = (row_valid && mloc > -INFINITY) ? mloc - m_new : -INFINITY;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) gap = fmaxf(gap, __shfl_xor_sync(0xffffffffu, gap, off));
+      if (lane == 0) c->gapw[gb][wq] = gap;
+      m_run = m_new;
+      float corr = 1.f;
+      bool resc = false;
+      if (m_new > -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kRescaleThreshold)) {
+        corr = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
+        m_ref = m_new;
+        resc = (t > 0);
+      }
+      // P = exp2(s * scale_log2 - m_ref), packed to bf16 pairs; row sum.
+      uint32_t pk[BK / 2];
+      float rs[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) rs[j] = 0.f;
+      const float neg = (m_ref > -INFINITY) ? -m_ref : 0.f;
+      const bool live = m_ref > -INFINITY;
+#pragma unroll
+      for (int j = 0; j < BK; j += 2) {
+        const float p0 = live ? ex2(fmaf(s[j], sc, neg)) : 0.f;
+        const float p1 = live ? ex2(fmaf(s[j + 1], sc, neg)) : 0.f;
+        rs[(j >> 1) & 7] += p0 + p1;
+        pk[j >> 1] = pack_bf16(p0, p1);
+      }
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j) rs[j] += rs[j + w];
+      l = l * corr + rs[0];
+      // tcgen05.ld/st are warp-collective: a warp rescales when any of its
+      // rows needs it (corr is 1 for the others).  A rescale implies the
+      // tile is not skipped, so PV(t-1) is the last product to wait for.
+      if (__any_sync(0xffffffffu, resc)) {
+        const uint32_t gp = gt - 1;
+        mbar_wait(&c->pv_done[gp & 1], (gp >> 1) & 1, g, p.status);
+        tc_fence_after();
+        const float f = resc ? corr : 1.f;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          float o[32];
+          tmem_ld32(tm + lane_off + cc * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] *= f;
+          tmem_st32(tm + lane_off + cc * 32, reinterpret_cast<const uint32_t*>(o));
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < BK / 64; ++cc) tmem_st32(scol + cc * 32, pk + cc * 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&c->p_full[gb]);
+    }
+    // Epilogue: O / l from TMEM once the unit's last PV has landed.
+    const uint32_t gl = gt0 + (uint32_t)u.n - 1;
+    mbar_wait(&c->pv_done[gl & 1], (gl >> 1) & 1, g, p.status);
+    tc_fence_after();
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    uint16_t* orow = p.out + (u.bh * p.N + row_g) * 128;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      float o[32];
+      tmem_ld32(tm + lane_off + cc * 32, o);
+      tmem_wait_ld();
+      if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 v;
+          v.x = pack_bf16(o[8 * q4 + 0] * inv_l, o[8 * q4 + 1] * inv_l);
+          v.y = pack_bf16(o[8 * q4 + 2] * inv_l, o[8 * q4 + 3] * inv_l);
+          v.z = pack_bf16(o[8 * q4 + 4] * inv_l, o[8 * q4 + 5] * inv_l);
+          v.w = pack_bf16(o[8 * q4 + 6] * inv_l, o[8 * q4 + 7] * inv_l);
+          dst[q4] = v;
+        }
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(&c->o_free);
+    if (row_valid) {
+      if (!(l > 0.f)) raise_status(p.status, SA_ERR_EMPTY_ROW);
+      if (p.lse) p.lse[u.bh * p.N + row_g] = (m_ref + __log2f(l)) * kLn2;
+    }
+    gt0 += (uint32_t)u.n;
+  }
+}
+
+template <int BK>
+__global__ void __launch_bounds__(Cfg<BK>::THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, TcParams p) {
   using C = Cfg<BK>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-  Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::OFF_CTL);
+  Ctl* ctl0 = reinterpret_cast<Ctl*>(smem + C::OFF_CTL);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&ctl->q_full, 1);
-    mbar_init(&ctl->q_empty, 1);
-    mbar_init(&ctl->o_free, 128);
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&ctl->k_full[s], 1);
-      mbar_init(&ctl->k_empty[s], 1);
-      mbar_init(&ctl->v_full[s], 1);
-      mbar_init(&ctl->v_empty[s], 1);
+    for (int q = 0; q < C::PIPES; ++q) {
+      Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + q * C::CTL_BYTES);
+      mbar_init(&c->q_full, 1);
+      mbar_init(&c->q_empty, 1);
+      mbar_init(&c->o_free, 128);
+      for (int s = 0; s < C::STAGES; ++s) {
+        mbar_init(&c->k_full[s], 1);
+        mbar_init(&c->k_empty[s], 1);
+        mbar_init(&c->v_full[s], 1);
+        mbar_init(&c->v_empty[s], 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&c->s_full[b], 1);
+        mbar_init(&c->p_full[b], 128);
+        mbar_init(&c->pv_done[b], 1);
+      }
+      c->abort = 0;
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&ctl->s_full[b], 1);
-      mbar_init(&ctl->s_empty[b], 128);
-      mbar_init(&ctl->p_full[b], 128);
-      mbar_init(&ctl->pv_done[b], 1);
-      ctl->skip_flag[b] = 0;
-    }
-    ctl->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == kWarpMMA) {
+  if (warp == 2) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&ctl->tmem_base)),
+                     smem_u32(&ctl0->tmem_base)),
                  "r"((uint32_t)C::TMEM_COLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -285,255 +536,29 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = ctl->tmem_base;
+  const uint32_t tmem = ctl0->tmem_base;
 
-  if (warp == kWarpTMA) {
-    if (lane == 0) {
-      // ------------------------------------------------------------- producer
-      uint32_t kv_it = 0, nq = 0;   // tiles and Q tiles loaded so far
-      for (int i = blockIdx.x; i < p.num_units; i += gridDim.x) {
-        const Unit u = unit_at(p, i, BK);
-        if (u.n <= 0) continue;
-        mbar_wait(&ctl->q_empty, (nq & 1) ^ 1, ctl, p.status);
-        ++nq;
-        mbar_expect_tx(&ctl->q_full, C::Q_BYTES);
-        tma_load_3d(sb + C::OFF_Q, &tmQ, 0, (int)(u.qb * 128), (int)u.bh, &ctl->q_full);
-        tma_load_3d(sb + C::OFF_Q + C::Q_BYTES / 2, &tmQ, 64, (int)(u.qb * 128), (int)u.bh, &ctl->q_full);
-        for (int64_t t = 0; t < u.n; ++t, ++kv_it) {
-          const int kb = (int)kblock_at(p, u, t);
-          const int s = kv_it % C::STAGES;
-          const uint32_t ph = (kv_it / C::STAGES) & 1;
-          const uint32_t kdst = sb + C::OFF_K + s * C::KV_BYTES;
-          const uint32_t vdst = sb + C::OFF_V + s * C::KV_BYTES;
-          mbar_wait(&ctl->k_empty[s], ph ^ 1, ctl, p.status);
-          mbar_expect_tx(&ctl->k_full[s], C::KV_BYTES);
-          tma_load_3d(kdst, &tmK, 0, kb * BK, (int)u.kvh, &ctl->k_full[s]);
-          tma_load_3d(kdst + C::KV_CHUNK, &tmK, 64, kb * BK, (int)u.kvh, &ctl->k_full[s]);
-          mbar_wait(&ctl->v_empty[s], ph ^ 1, ctl, p.status);
-          mbar_expect_tx(&ctl->v_full[s], C::KV_BYTES);
-          tma_load_3d(vdst, &tmV, 0, kb * BK, (int)u.kvh, &ctl->v_full[s]);
-          tma_load_3d(vdst + C::KV_CHUNK, &tmV, 64, kb * BK, (int)u.kvh, &ctl->v_full[s]);
-        }
-      }
-      // Drain: the last loads of every stage (and the last Q) have landed.
-      if (nq > 0) mbar_drain(&ctl->q_full, (nq - 1) & 1);  // no-op unless a wait was abandoned
-      for (uint32_t j = kv_it > (uint32_t)C::STAGES ? kv_it - C::STAGES : 0; j < kv_it; ++j) {
-        mbar_drain(&ctl->k_full[j % C::STAGES], (j / C::STAGES) & 1);
-        mbar_drain(&ctl->v_full[j % C::STAGES], (j / C::STAGES) & 1);
-      }
+  if (warp < 2) {
+    if (warp < C::PIPES && lane == 0) {
+      Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + warp * C::CTL_BYTES);
+      producer<BK>(&tmQ, &tmK, &tmV, p, c, ctl0, sb, warp);
     }
-  } else if (warp == kWarpMMA) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc_s = make_idesc(128, BK, 0);
-      constexpr uint32_t idesc_pv = make_idesc(128, 128, 1);
-      uint32_t kv_it = 0, g = 0, unit_it = 0;   // unit_it counts units with work
-      for (int i = blockIdx.x; i < p.num_units; i += gridDim.x) {
-        const Unit u = unit_at(p, i, BK);
-        if (u.n <= 0) continue;
-        mbar_wait(&ctl->q_full, unit_it & 1, ctl, p.status);
-        tc_fence_after();
-        bool first_pv = true;
-        auto do_pv = [&](int64_t tt) {
-          const uint32_t it = kv_it + (uint32_t)tt, gt = g + (uint32_t)tt;
-          const int s = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1;
-          const int gb = gt & 1;
-          mbar_wait(&ctl->p_full[gb], (gt >> 1) & 1, ctl, p.status);
-          tc_fence_after();
-          const uint32_t skip = ctl->skip_flag[gb];
-          if (tt == 0) {
-            mbar_wait(&ctl->o_free, (unit_it & 1) ^ 1, ctl, p.status);
-            tc_fence_after();
-          }
-          mbar_wait(&ctl->v_full[s], ph, ctl, p.status);
-          tc_fence_after();
-          if (!skip) {
-            const uint32_t pbase = sb + C::OFF_P + gb * C::P_BYTES;
-            const uint32_t vbase = sb + C::OFF_V + s * C::KV_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t a = desc_sw128(pbase + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-              const uint64_t b = desc_sw128(vbase + kk * 2048, C::KV_CHUNK, 1024);
-              umma_f16(tmem, a, b, idesc_pv, (first_pv && kk == 0) ? 0u : 1u);
-            }
-            first_pv = false;
-          }
-          umma_commit(&ctl->v_empty[s]);
-          umma_commit(&ctl->pv_done[gb]);
-        };
-        for (int64_t t = 0; t < u.n; ++t) {
-          const uint32_t it = kv_it + (uint32_t)t, gt = g + (uint32_t)t;
-          const int s = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1;
-          const int gb = gt & 1;
-          mbar_wait(&ctl->k_full[s], ph, ctl, p.status);
-          mbar_wait(&ctl->s_empty[gb], ((gt >> 1) & 1) ^ 1, ctl, p.status);
-          tc_fence_after();
-          const uint32_t kbase = sb + C::OFF_K + s * C::KV_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = desc_sw128(sb + C::OFF_Q + (kk >> 2) * (C::Q_BYTES / 2) + (kk & 3) * 32, 16, 1024);
-            const uint64_t b = desc_sw128(kbase + (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32, 16, 1024);
-            umma_f16(tmem + C::S_COL + gb * BK, a, b, idesc_s, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&ctl->s_full[gb]);
-          umma_commit(&ctl->k_empty[s]);
-          if (t == u.n - 1) umma_commit(&ctl->q_empty);
-          if (t >= 1) do_pv(t - 1);
-        }
-        do_pv(u.n - 1);
-        kv_it += (uint32_t)u.n;
-        g += (uint32_t)u.n;
-        ++unit_it;
-      }
+  } else if (warp < 4) {
+    const int pipe = warp - 2;
+    if (pipe < C::PIPES && lane == 0) {
+      Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + pipe * C::CTL_BYTES);
+      mma_issuer<BK>(p, c, ctl0, sb, tmem + pipe * C::TMEM_PIPE, pipe);
     }
     __syncwarp();
-  } else if (warp >= kWarpSoftmax0) {
-    // ------------------------------------------------------------- softmax
-    const int wq = warp - kWarpSoftmax0;        // == warp % 4: TMEM lanes 32*wq ..
-    const int row = wq * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    uint32_t g = 0;
-    for (int i = blockIdx.x; i < p.num_units; i += gridDim.x) {
-      const Unit u = unit_at(p, i, BK);
-      const int64_t row_g = u.qb * 128 + row;
-      const bool row_valid = row_g < p.N;
-      if (u.n <= 0) {
-        if (row_valid) raise_status(p.status, SA_ERR_EMPTY_ROW);
-        continue;
-      }
-      float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
-      for (int64_t t = 0; t < u.n; ++t) {
-        const uint32_t gt = g + (uint32_t)t;
-        const int gb = gt & 1;
-        const int64_t kb = kblock_at(p, u, t);
-        mbar_wait(&ctl->s_full[gb], (gt >> 1) & 1, ctl, p.status);
-        tc_fence_after();
-        float s[BK];
-#pragma unroll
-        for (int c = 0; c < BK / 32; ++c) tmem_ld32(tmem + lane_off + C::S_COL + gb * BK + c * 32, s + c * 32);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&ctl->s_empty[gb]);
-
-        const int64_t k0 = kb * BK;
-        const bool need_mask = (k0 + BK > p.N) || (p.causal && k0 + BK - 1 > u.qb * 128);
-        float mloc = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < BK; ++j) {
-          float x = s[j] * p.scale_log2;
-          if (need_mask) {
-            const int64_t key = k0 + j;
-            if (key >= p.N || (p.causal && key > row_g)) x = -INFINITY;
-          }
-          s[j] = x;
-          mloc = fmaxf(mloc, x);
-        }
-        const float m_new = fmaxf(m_run, mloc);
-        float gap = (row_valid && mloc > -INFINITY) ? mloc - m_new : -INFINITY;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) gap = fmaxf(gap, __shfl_xor_sync(0xffffffffu, gap, off));
-        if (lane == 0) ctl->gapw[gb][wq] = gap;
-        named_bar(1, 128);
-        const float G = fmaxf(fmaxf(ctl->gapw[gb][0], ctl->gapw[gb][1]), fmaxf(ctl->gapw[gb][2], ctl->gapw[gb][3]));
-        const bool skip = G < p.lam_log2;
-        m_run = m_new;
-        float corr = 1.f;
-        bool resc = false;
-        if (m_new > -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kRescaleThreshold)) {
-          corr = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
-          m_ref = m_new;
-          resc = (t > 0);
-        }
-        float rs = 0.f;
-        if (m_ref > -INFINITY) {
-#pragma unroll
-          for (int j = 0; j < BK; ++j) {
-            s[j] = ex2(s[j] - m_ref);
-            rs += s[j];
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < BK; ++j) s[j] = 0.f;
-        }
-        l = l * corr + rs;
-        if (!skip) {
-          if (gt >= 2) mbar_wait(&ctl->pv_done[gb], ((gt - 2) >> 1) & 1, ctl, p.status);
-          // tcgen05.ld/st are warp-collective: a warp rescales when any of
-          // its rows needs it (corr is 1 for the others).
-          if (__any_sync(0xffffffffu, resc)) {
-            const uint32_t gp = gt - 1;
-            mbar_wait(&ctl->pv_done[gp & 1], (gp >> 1) & 1, ctl, p.status);
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              float o[32];
-              tmem_ld32(tmem + lane_off + c * 32, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] *= corr;
-              tmem_st32(tmem + lane_off + c * 32, o);
-            }
-            tmem_wait_st();
-          }
-          uint8_t* prow = smem + C::OFF_P + gb * C::P_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-          for (int c = 0; c < BK / 8; ++c) {
-            uint4 v;
-            v.x = pack_bf16(s[8 * c + 0], s[8 * c + 1]);
-            v.y = pack_bf16(s[8 * c + 2], s[8 * c + 3]);
-            v.z = pack_bf16(s[8 * c + 4], s[8 * c + 5]);
-            v.w = pack_bf16(s[8 * c + 6], s[8 * c + 7]);
-            const int region = c >> 3, cc = c & 7;
-            *reinterpret_cast<uint4*>(prow + region * 16384 + ((cc ^ (row & 7)) << 4)) = v;
-          }
-          fence_async_smem();
-        }
-        tc_fence_before();
-        if (row == 0) {
-          ctl->skip_flag[gb] = skip ? 1u : 0u;
-          if (p.skip_log && p.row_ptr) p.skip_log[u.lo + t] = skip ? 1 : 0;
-        }
-        mbar_arrive(&ctl->p_full[gb]);
-      }
-      // Epilogue: O / l from TMEM once the unit's last PV has landed.
-      const uint32_t gl = g + (uint32_t)u.n - 1;
-      mbar_wait(&ctl->pv_done[gl & 1], (gl >> 1) & 1, ctl, p.status);
-      tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      uint16_t* orow = p.out + (u.bh * p.N + row_g) * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float o[32];
-        tmem_ld32(tmem + lane_off + c * 32, o);
-        tmem_wait_ld();
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 v;
-            v.x = pack_bf16(o[8 * q4 + 0] * inv_l, o[8 * q4 + 1] * inv_l);
-            v.y = pack_bf16(o[8 * q4 + 2] * inv_l, o[8 * q4 + 3] * inv_l);
-            v.z = pack_bf16(o[8 * q4 + 4] * inv_l, o[8 * q4 + 5] * inv_l);
-            v.w = pack_bf16(o[8 * q4 + 6] * inv_l, o[8 * q4 + 7] * inv_l);
-            dst[q4] = v;
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&ctl->o_free);
-      if (row_valid) {
-        if (!(l > 0.f)) raise_status(p.status, SA_ERR_EMPTY_ROW);
-        if (p.lse) p.lse[u.bh * p.N + row_g] = (m_ref + __log2f(l)) * kLn2;
-      }
-      g += (uint32_t)u.n;
-    }
+  } else {
+    const int pipe = (warp - 4) >> 2;
+    Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + pipe * C::CTL_BYTES);
+    softmax_rows<BK>(p, c, ctl0, tmem + pipe * C::TMEM_PIPE, pipe, warp & 3, lane);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMMA) {
+  if (warp == 2) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::TMEM_COLS)
                  : "memory");
@@ -602,8 +627,9 @@ sa_status launch_bk(const AttnArgs& a, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (cudaFuncSetAttribute(attn_tc_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(attn_tc_kernel) failed");
-  const int grid = p.num_units < sms ? p.num_units : sms;
-  attn_tc_kernel<BK><<<grid, kThreadsTC, C::SMEM, st>>>(mq, mk, mv, p);
+  const int want = (p.num_units + C::PIPES - 1) / C::PIPES;
+  const int grid = want < sms ? want : sms;
+  attn_tc_kernel<BK><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, p);
   return check_launch("attn_tc_kernel");
 }
 
