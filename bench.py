@@ -212,7 +212,8 @@ def run_ours(args, rank, world, local_rank):
             qr, kr, vr, out_r, lse_r = q, k, v, pipe.out, pipe.lse
         sa.predict_mask(qr, kr, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
         e[1].record(stream)
-        sa.block_sparse_attn(qr, kr, vr, pipe.shape, pipe.mask.struct, pipe.lam, pipe.scale, out_r, lse_r)
+        sa.block_sparse_attn(qr, kr, vr, pipe.shape, pipe.mask.struct, pipe.lam, pipe.scale, out_r, lse_r,
+                             ws=pipe.attn_ws)
         e[2].record(stream)
         if not pipe.identity:
             sa.unreorder(pipe.perm, out_r, pipe.out)
@@ -263,7 +264,7 @@ def run_ours(args, rank, world, local_rank):
         l2_flush()
         a, b = ev(), ev()
         a.record(stream)
-        sa.dense_attn(qr, kr, vr, pipe.shape, w.causal, 0.0, od, ld, dst)
+        sa.dense_attn(qr, kr, vr, pipe.shape, w.causal, 0.0, od, ld, dst, ws=pipe.attn_ws)
         b.record(stream)
         if i >= args.warmup:
             dense.append((a, b))

@@ -195,6 +195,12 @@ sa_status sa_mask_from_blocks(const uint8_t* block_mask, const sa_shape* shape, 
                               int32_t bk, int32_t causal, void* ws, size_t ws_bytes,
                               sa_mask* out, void* stream);
 
+/* Scratch of the attention entry points (a work counter the kernel zeroes
+ * with an asynchronous memset before each launch): sa_attn_workspace() bytes,
+ * 256-byte aligned.  Calls that share one workspace must not overlap on the
+ * GPU. */
+size_t sa_attn_workspace(void);
+
 /* ---- a5/a6: block-sparse attention ([P3] 2.1, 2.3) -----------------------
  * For every query block, visits its kept key blocks in ascending order with
  * the online-softmax recurrence; skips P~V of a tile when the largest
@@ -207,7 +213,7 @@ sa_status sa_mask_from_blocks(const uint8_t* block_mask, const sa_shape* shape, 
 sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v,
                                const sa_shape* shape, const sa_mask* mask, float lambda,
                                float scale, void* out, float* lse, uint8_t* pv_skip_log,
-                               int32_t flags, void* stream);
+                               void* ws, size_t ws_bytes, int32_t flags, void* stream);
 
 /* ---- a8: dense reference --------------------------------------------------
  * The same recurrence with every (causally valid) key visible and no lists
@@ -215,7 +221,7 @@ sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v,
  * nullable) receives kernel errors. */
 sa_status sa_dense_attn(const void* q, const void* k, const void* v, const sa_shape* shape,
                         int32_t causal, float scale, void* out, float* lse, int32_t* status,
-                        int32_t flags, void* stream);
+                        void* ws, size_t ws_bytes, int32_t flags, void* stream);
 
 /* Synchronises `stream` and returns the device status word's code (0 =
  * SA_OK).  The word is not cleared. */

@@ -102,6 +102,8 @@ int32_t sa_attn_kernel_path(const sa_shape* shape, int32_t bq, int32_t bk, int32
   return smem <= 227 * 1024 ? 0 : -1;
 }
 
+size_t sa_attn_workspace(void) { return 256; }
+
 size_t sa_layout_workspace(const sa_layout_desc* desc) {
   if (!desc) return 0;
   return layout_ws_bytes(*desc);
@@ -224,10 +226,13 @@ sa_status sa_mask_from_blocks(const uint8_t* block_mask, const sa_shape* shape, 
 
 static sa_status attn_common(const void* q, const void* k, const void* v, const sa_shape* shape,
                              const sa_mask* mask, int32_t causal, float lambda, float scale, void* out,
-                             float* lse, uint8_t* skip_log, int32_t* status, int32_t flags,
-                             void* stream) {
+                             float* lse, uint8_t* skip_log, int32_t* status, void* ws, size_t ws_bytes,
+                             int32_t flags, void* stream) {
   if (sa_status e = check_shape(shape)) return e;
   if (!q || !k || !v || !out) return set_error(SA_ERR_INVALID_ARG, "NULL tensor argument");
+  if (!ws || ws_bytes < sa_attn_workspace() || (uintptr_t)ws % 256)
+    return set_error(SA_ERR_WORKSPACE, "attention needs %zu bytes of 256-byte aligned workspace",
+                     sa_attn_workspace());
   if (std::isnan(lambda) || lambda > 0.f)
     return set_error(SA_ERR_INVALID_ARG, "lambda must be <= 0 (or -INFINITY to disable the PV skip)");
   if (!(scale >= 0.f) || std::isinf(scale)) return set_error(SA_ERR_INVALID_ARG, "scale must be finite and >= 0");
@@ -247,6 +252,7 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
   a.dtype = shape->dtype;
   a.scale = scale > 0.f ? scale : 1.0f / std::sqrt((float)shape->d);
   a.lambda = lambda;
+  a.counter = static_cast<int32_t*>(ws);
   if (mask) {
     if (sa_status e = check_mask_out(mask)) return e;
     if (mask->bq < 1 || mask->bq > 128 || mask->bk < 1 || mask->bk > 128 ||
@@ -285,17 +291,19 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
 
 sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v, const sa_shape* shape,
                                const sa_mask* mask, float lambda, float scale, void* out, float* lse,
-                               uint8_t* pv_skip_log, int32_t flags, void* stream) {
+                               uint8_t* pv_skip_log, void* ws, size_t ws_bytes, int32_t flags,
+                               void* stream) {
   if (!mask) return set_error(SA_ERR_INVALID_ARG, "mask is NULL");
-  return attn_common(q, k, v, shape, mask, 0, lambda, scale, out, lse, pv_skip_log, nullptr, flags,
-                     stream);
+  return attn_common(q, k, v, shape, mask, 0, lambda, scale, out, lse, pv_skip_log, nullptr, ws, ws_bytes,
+                     flags, stream);
 }
 
 sa_status sa_dense_attn(const void* q, const void* k, const void* v, const sa_shape* shape, int32_t causal,
-                        float scale, void* out, float* lse, int32_t* status, int32_t flags, void* stream) {
+                        float scale, void* out, float* lse, int32_t* status, void* ws, size_t ws_bytes,
+                        int32_t flags, void* stream) {
   if (causal != 0 && causal != 1) return set_error(SA_ERR_INVALID_ARG, "causal must be 0 or 1");
-  return attn_common(q, k, v, shape, nullptr, causal, -INFINITY, scale, out, lse, nullptr, status, flags,
-                     stream);
+  return attn_common(q, k, v, shape, nullptr, causal, -INFINITY, scale, out, lse, nullptr, status, ws,
+                     ws_bytes, flags, stream);
 }
 
 sa_status sa_read_status(const int32_t* status, void* stream) {

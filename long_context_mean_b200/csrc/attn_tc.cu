@@ -66,9 +66,11 @@ struct Ctl {
   uint64_t q_full, q_empty, o_free;
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
   uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t u_full[4], u_empty[4];          // unit announcement ring
   uint32_t tmem_base;
   volatile uint32_t abort;
   float gapw[2][4];
+  volatile int32_t ring[4];
 };
 
 struct TcParams {
@@ -79,6 +81,7 @@ struct TcParams {
   float* lse;
   uint8_t* skip_log;
   int32_t* status;
+  int32_t* counter;      // work counter, zero at launch
   int64_t N, nqb, nkb;
   int32_t Hq, Hkv;
   int32_t num_units;
@@ -207,6 +210,30 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+// Two fp32 values in one 64-bit register for the packed fp32x2 pipe.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -258,7 +285,16 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const C
                          const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, int pipe) {
   using C = Cfg<BK>;
   uint32_t kv_it = 0, nq = 0;
-  for (int i = blockIdx.x * C::PIPES + pipe; i < p.num_units; i += gridDim.x * C::PIPES) {
+  for (uint32_t j = 0;; ++j) {
+    // Take the next unit of the work order and announce it to the pipeline's
+    // MMA and softmax warps through a 4-slot ring.
+    const int slot = j & 3;
+    mbar_wait(&c->u_empty[slot], ((j >> 2) & 1) ^ 1, g, p.status);
+    int i = atomicAdd(p.counter, 1);
+    if (i >= p.num_units) i = -1;
+    c->ring[slot] = i;
+    mbar_arrive(&c->u_full[slot]);
+    if (i < 0) break;
     const Unit u = unit_at(p, i, BK);
     if (u.n <= 0) continue;
     mbar_wait(&c->q_empty, (nq & 1) ^ 1, g, p.status);
@@ -296,7 +332,12 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
   constexpr uint32_t idesc_s = make_idesc(128, BK, 0);
   constexpr uint32_t idesc_pv = make_idesc(128, 128, 1);
   uint32_t kv_it = 0, gt0 = 0, unit_it = 0;   // unit_it counts units with work
-  for (int i = blockIdx.x * C::PIPES + pipe; i < p.num_units; i += gridDim.x * C::PIPES) {
+  for (uint32_t j = 0;; ++j) {
+    const int slot = j & 3;
+    mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status);
+    const int i = c->ring[slot];
+    mbar_arrive(&c->u_empty[slot]);
+    if (i < 0) break;
     const Unit u = unit_at(p, i, BK);
     if (u.n <= 0) continue;
     mbar_wait(&c->q_full, unit_it & 1, g, p.status);
@@ -365,7 +406,13 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
   const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
   const float sc = p.scale_log2;
   uint32_t gt0 = 0;
-  for (int i = blockIdx.x * C::PIPES + pipe; i < p.num_units; i += gridDim.x * C::PIPES) {
+  for (uint32_t j = 0;; ++j) {
+    const int slot = j & 3;
+    mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status);
+    const int i = c->ring[slot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&c->u_empty[slot]);
+    if (i < 0) break;
     const Unit u = unit_at(p, i, BK);
     const int64_t row_g = u.qb * 128 + row;
     const bool row_valid = row_g < p.N;
@@ -374,10 +421,12 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
       continue;
     }
     float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
+    int64_t kb_cur = kblock_at(p, u, 0);
     for (int64_t t = 0; t < u.n; ++t) {
       const uint32_t gt = gt0 + (uint32_t)t;
       const int gb = gt & 1;
       const uint32_t scol = tm + lane_off + C::S_COL + gb * BK;
+      const int64_t kb_next = (t + 1 < u.n) ? kblock_at(p, u, t + 1) : 0;   // load ahead
       mbar_wait(&c->s_full[gb], (gt >> 1) & 1, g, p.status);
       tc_fence_after();
       float s[BK];
@@ -385,7 +434,8 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
       for (int cc = 0; cc < BK / 32; ++cc) tmem_ld32(scol + cc * 32, s + cc * 32);
       tmem_wait_ld();
 
-      const int64_t k0 = kblock_at(p, u, t) * BK;
+      const int64_t k0 = kb_cur * BK;
+      kb_cur = kb_next;
       if ((k0 + BK > p.N) || (p.causal && k0 + BK - 1 > u.qb * 128)) {
 #pragma unroll
         for (int j = 0; j < BK; ++j) {
@@ -393,16 +443,20 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
           if (key >= p.N || (p.causal && key > row_g)) s[j] = -INFINITY;
         }
       }
-      // Row max as a tree (independent chains), in raw score units.
-      float mx[16];
+      // Row max as a tree of 3-input maxima (independent chains), raw units.
+      float mx[BK / 4];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) mx[j] = s[j];
+      for (int j = 0; j < BK / 4; ++j) mx[j] = max3(fmaxf(s[4 * j], s[4 * j + 1]), s[4 * j + 2], s[4 * j + 3]);
 #pragma unroll
-      for (int j = 16; j < BK; ++j) mx[j & 15] = fmaxf(mx[j & 15], s[j]);
+      for (int w = BK / 4; w > 1; w = (w + 2) / 3) {
 #pragma unroll
-      for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-        for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
+        for (int j = 0; j < (w + 2) / 3; ++j) {
+          const float a = mx[3 * j];
+          const float b = 3 * j + 1 < w ? mx[3 * j + 1] : a;
+          const float d = 3 * j + 2 < w ? mx[3 * j + 2] : a;
+          mx[j] = max3(a, b, d);
+        }
+      }
       const float mloc = mx[0] * sc;                    // scale > 0: max commutes
       const float m_new = fmaxf(m_run, mloc);
       float gap = (row_valid && mloc > -INFINITY) ? mloc - m_new : -INFINITY;
@@ -419,23 +473,31 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
       }
       // P = exp2(s * scale_log2 - m_ref), packed to bf16 pairs; row sum.
       uint32_t pk[BK / 2];
-      float rs[8];
+      float row_sum = 0.f;
+      if (m_ref > -INFINITY) {
+        // Pairs of columns on the packed fp32x2 pipe: x = s * scale - m_ref.
+        const uint64_t sc2 = pack2(sc, sc), neg2 = pack2(-m_ref, -m_ref);
+        uint64_t acc[4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) rs[j] = 0.f;
-      const float neg = (m_ref > -INFINITY) ? -m_ref : 0.f;
-      const bool live = m_ref > -INFINITY;
+        for (int j = 0; j < 4; ++j) acc[j] = pack2(0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < BK; j += 2) {
-        const float p0 = live ? ex2(fmaf(s[j], sc, neg)) : 0.f;
-        const float p1 = live ? ex2(fmaf(s[j + 1], sc, neg)) : 0.f;
-        rs[(j >> 1) & 7] += p0 + p1;
-        pk[j >> 1] = pack_bf16(p0, p1);
+        for (int j = 0; j < BK; j += 2) {
+          const uint64_t x = ffma2(pack2(s[j], s[j + 1]), sc2, neg2);
+          float x0, x1;
+          unpack2(x, x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          acc[(j >> 1) & 3] = fadd2(acc[(j >> 1) & 3], pack2(p0, p1));
+          pk[j >> 1] = pack_bf16(p0, p1);
+        }
+        const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+        float lo, hi;
+        unpack2(a2, lo, hi);
+        row_sum = lo + hi;
+      } else {
+#pragma unroll
+        for (int j = 0; j < BK / 2; ++j) pk[j] = 0u;
       }
-#pragma unroll
-      for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-        for (int j = 0; j < w; ++j) rs[j] += rs[j + w];
-      l = l * corr + rs[0];
+      l = l * corr + row_sum;
       // tcgen05.ld/st are warp-collective: a warp rescales when any of its
       // rows needs it (corr is 1 for the others).  A rescale implies the
       // tile is not skipped, so PV(t-1) is the last product to wait for.
@@ -521,6 +583,10 @@ __global__ void __launch_bounds__(Cfg<BK>::THREADS, 1)
         mbar_init(&c->s_full[b], 1);
         mbar_init(&c->p_full[b], 128);
         mbar_init(&c->pv_done[b], 1);
+      }
+      for (int r = 0; r < 4; ++r) {
+        mbar_init(&c->u_full[r], 1);
+        mbar_init(&c->u_empty[r], 1 + 4);   // the MMA lane + one lane per softmax warp
       }
       c->abort = 0;
     }
@@ -612,6 +678,7 @@ sa_status launch_bk(const AttnArgs& a, cudaStream_t st) {
   p.lse = a.lse;
   p.skip_log = a.skip_log;
   p.status = a.status;
+  p.counter = a.counter;
   p.N = a.N;
   p.nqb = a.nqb;
   p.nkb = a.nkb;
@@ -622,6 +689,8 @@ sa_status launch_bk(const AttnArgs& a, cudaStream_t st) {
   p.scale_log2 = a.scale * kLog2e;
   p.lam_log2 = a.lambda * kLog2e;
   if (p.num_units == 0) return SA_OK;
+  if (cudaMemsetAsync(p.counter, 0, sizeof(int32_t), st) != cudaSuccess)
+    return set_error(SA_ERR_CUDA, "cudaMemsetAsync(work counter) failed");
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

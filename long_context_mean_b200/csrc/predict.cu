@@ -207,119 +207,164 @@ __device__ void finish_row(const uint8_t* flags, int64_t u, int64_t qb, int64_t 
 }
 
 // ---------------------------------------------------------------------------
-// a3 + a4: one CTA per mask row (b, h, qb).  Scores, softmax, bitonic sort of
-// (p, kb) keys descending (ties: lower kb first), scan, TopCdf, then the
-// union with the forced parts and the causal AND.
-// Dynamic shared memory: keys[P2] (u64) | flags[nkb] (u8) | q_hat[d] (f32).
+// a3 + a4: one CTA per (head, group of kRowsPerCta query blocks).  The
+// group's q_hat rows and 32-row chunks of the kv head's k_hat are staged in
+// shared memory (padded rows, conflict-free) so every k_hat element is read
+// once per group; then, row by row: softmax, bitonic sort of (p, kb) keys
+// descending (ties: lower kb first), scan, TopCdf, and the union with the
+// forced parts and the causal AND.
+// Dynamic shared memory: q_hat [G][d] | k_hat chunk [32][d+1] |
+// scores [G][nkb] | keys [P2] (u64) | flags [nkb] (u8).
 // ---------------------------------------------------------------------------
+constexpr int kRowsPerCta = 8;
+constexpr int kChunk = 32;
+
+size_t score_smem_bytes(int d, int64_t nkb, int P2) {
+  return (size_t)kRowsPerCta * d * 4 + (size_t)kChunk * (d + 1) * 4 + (size_t)kRowsPerCta * nkb * 4 +
+         (size_t)P2 * 8 + (size_t)((nkb + 15) / 16) * 16;
+}
+
 __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
     const float* __restrict__ qhat, const float* __restrict__ khat, const float* __restrict__ sq,
     const float* __restrict__ sk, int64_t Hq, int64_t Hkv, int64_t nqb, int64_t nkb, int d,
     int P2, float tau, float theta, RowRules rules, uint8_t* __restrict__ mask,
     int32_t* __restrict__ counts, int32_t* status) {
   extern __shared__ __align__(16) unsigned char smem[];
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
-  uint8_t* flags = smem + (size_t)P2 * 8;
-  float* qv = reinterpret_cast<float*>(smem + (size_t)P2 * 8 + ((nkb + 15) / 16) * 16);
+  float* qs = reinterpret_cast<float*>(smem);
+  float* ks = qs + kRowsPerCta * d;
+  float* sc = ks + kChunk * (d + 1);
+  // 8-byte aligned: the float offset 8d + 32(d+1) + 8 nkb is even.
+  uint64_t* keys = reinterpret_cast<uint64_t*>(sc + kRowsPerCta * nkb);
+  uint8_t* flags = reinterpret_cast<uint8_t*>(keys + P2);
   __shared__ float shf[32];
   __shared__ int shi[32];
   __shared__ float scan_part[kRowThreads];
+  __shared__ int s_forced[kRowsPerCta];
 
-  const int64_t u = blockIdx.x;
-  const int64_t bh = u / nqb, qb = u % nqb;
+  const int64_t bh = blockIdx.y;
+  const int64_t qb0 = (int64_t)blockIdx.x * kRowsPerCta;
+  const int rows = (int)min64(kRowsPerCta, nqb - qb0);
   const int64_t b = bh / Hq, h = bh % Hq;
   const int64_t g = b * Hkv + h / (Hq / Hkv);
   const bool guard = theta > 0.f;
-  const bool row_forced = rules.struct_row(qb) || (guard && sq[u] < theta);
+  const float scale = rsqrtf((float)d);
 
-  for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) flags[kb] = 0;
-  if (!row_forced) {
-    for (int i = threadIdx.x; i < d; i += blockDim.x) qv[i] = qhat[u * (int64_t)d + i];
-    __syncthreads();
-    const float scale = rsqrtf((float)d);
-    float mx = -INFINITY;
-    for (int64_t kb = threadIdx.x; kb < P2; kb += blockDim.x) {
-      float s = -INFINITY;
-      if (kb < nkb && rules.valid(qb, kb) && !(guard && sk[g * nkb + kb] < theta)) {
-        const float4* kr = reinterpret_cast<const float4*>(khat + (g * nkb + kb) * (int64_t)d);
-        const float4* qr = reinterpret_cast<const float4*>(qv);
-        float acc = 0.f;
-        for (int i = 0; i < d / 4; ++i) {
-          const float4 a = qr[i], bb = __ldg(kr + i);
-          acc = fmaf(a.x, bb.x, acc);
-          acc = fmaf(a.y, bb.y, acc);
-          acc = fmaf(a.z, bb.z, acc);
-          acc = fmaf(a.w, bb.w, acc);
-        }
-        s = acc * scale;
-      }
-      keys[kb] = (uint64_t)__float_as_uint(s);   // stash raw score bits for now
-      mx = fmaxf(mx, s);
-    }
-    mx = block_reduce_max(mx, shf);
-    if (mx > -INFINITY) {
-      float sum = 0.f;
-      for (int64_t kb = threadIdx.x; kb < P2; kb += blockDim.x) {
-        const float s = __uint_as_float((uint32_t)keys[kb]);
-        const float p = (s == -INFINITY) ? 0.f : expf(s - mx);
-        // key = p bits (p >= 0: integer order = float order) | ~kb
-        keys[kb] = (kb < nkb) ? (((uint64_t)__float_as_uint(p) << 32) | (uint32_t)(~(uint32_t)kb))
-                              : 0ull;
-        sum += p;
+  if (threadIdx.x < kRowsPerCta) {
+    const int r = threadIdx.x;
+    const int64_t u = bh * nqb + qb0 + r;
+    s_forced[r] = (r >= rows) ? 1 : ((rules.struct_row(qb0 + r) || (guard && sq[u] < theta)) ? 1 : 0);
+  }
+  for (int i = threadIdx.x; i < rows * d; i += blockDim.x) qs[i] = qhat[(bh * nqb + qb0) * (int64_t)d + i];
+  __syncthreads();
+  int any_scored = 0;
+  for (int r = 0; r < rows; ++r) any_scored |= !s_forced[r];
+
+  if (any_scored) {
+    // Scores of the whole group, one k_hat chunk at a time.
+    const float* kg = khat + g * nkb * (int64_t)d;
+    const int r = threadIdx.x / kChunk, j = threadIdx.x % kChunk;
+    for (int64_t c0 = 0; c0 < nkb; c0 += kChunk) {
+      const int cn = (int)min64(kChunk, nkb - c0);
+      for (int i = threadIdx.x; i < cn * d; i += blockDim.x) {
+        const int jj = i / d, e = i % d;
+        ks[jj * (d + 1) + e] = kg[(c0 + jj) * d + e];
       }
       __syncthreads();
-      // Bitonic sort, descending.
-      for (int k = 2; k <= P2; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-          for (int i = threadIdx.x; i < P2; i += blockDim.x) {
-            const int ixj = i ^ j;
-            if (ixj > i) {
-              const uint64_t a = keys[i], c = keys[ixj];
-              const bool desc = (i & k) == 0;
-              if (desc ? (a < c) : (a > c)) {
-                keys[i] = c;
-                keys[ixj] = a;
+      const int64_t kb = c0 + j;
+      if (r < rows && j < cn) {
+        float s = -INFINITY;
+        if (!s_forced[r] && rules.valid(qb0 + r, kb) && !(guard && sk[g * nkb + kb] < theta)) {
+          const float* qr = qs + r * d;
+          const float* kr = ks + j * (d + 1);
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          for (int e = 0; e < d; e += 4) {
+            a0 = fmaf(qr[e], kr[e], a0);
+            a1 = fmaf(qr[e + 1], kr[e + 1], a1);
+            a2 = fmaf(qr[e + 2], kr[e + 2], a2);
+            a3 = fmaf(qr[e + 3], kr[e + 3], a3);
+          }
+          s = ((a0 + a1) + (a2 + a3)) * scale;
+        }
+        sc[r * nkb + kb] = s;
+      }
+      __syncthreads();
+    }
+  }
+
+  for (int r = 0; r < rows; ++r) {
+    const int64_t qb = qb0 + r;
+    const int64_t u = bh * nqb + qb;
+    const bool row_forced = s_forced[r] != 0;
+    for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) flags[kb] = 0;
+    if (!row_forced) {
+      const float* srow = sc + r * nkb;
+      float mx = -INFINITY;
+      for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) mx = fmaxf(mx, srow[kb]);
+      mx = block_reduce_max(mx, shf);
+      if (mx > -INFINITY) {
+        for (int64_t kb = threadIdx.x; kb < P2; kb += blockDim.x) {
+          uint64_t key = 0ull;
+          if (kb < nkb) {
+            const float s = srow[kb];
+            const float p = (s == -INFINITY) ? 0.f : expf(s - mx);
+            // key = p bits (p >= 0: integer order = float order) | ~kb
+            key = ((uint64_t)__float_as_uint(p) << 32) | (uint32_t)(~(uint32_t)kb);
+          }
+          keys[kb] = key;
+        }
+        __syncthreads();
+        // Bitonic sort, descending.
+        for (int k = 2; k <= P2; k <<= 1) {
+          for (int jj = k >> 1; jj > 0; jj >>= 1) {
+            for (int i = threadIdx.x; i < P2; i += blockDim.x) {
+              const int ixj = i ^ jj;
+              if (ixj > i) {
+                const uint64_t a = keys[i], c = keys[ixj];
+                const bool desc = (i & k) == 0;
+                if (desc ? (a < c) : (a > c)) {
+                  keys[i] = c;
+                  keys[ixj] = a;
+                }
               }
             }
+            __syncthreads();
           }
+        }
+        // Inclusive scan of the sorted probabilities: each thread a contiguous
+        // run, then a block scan of the run totals.
+        const int per = P2 / (int)blockDim.x > 0 ? P2 / (int)blockDim.x : 1;
+        const int beg = threadIdx.x * per;
+        float run = 0.f;
+        for (int i = beg; i < beg + per && i < P2; ++i) run += __uint_as_float((uint32_t)(keys[i] >> 32));
+        scan_part[threadIdx.x] = run;
+        __syncthreads();
+        for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+          const float v = threadIdx.x >= (unsigned)off ? scan_part[threadIdx.x - off] : 0.f;
+          __syncthreads();
+          scan_part[threadIdx.x] += v;
           __syncthreads();
         }
+        const float total = scan_part[blockDim.x - 1];
+        const float limit = tau * total;
+        float excl = scan_part[threadIdx.x] - run;
+        for (int i = beg; i < beg + per && i < P2; ++i) {
+          const float p = __uint_as_float((uint32_t)(keys[i] >> 32));
+          const uint32_t kb = ~(uint32_t)keys[i];
+          if (p > 0.f && excl < limit) flags[kb] = 1;
+          excl += p;
+        }
       }
-      // Inclusive scan of the sorted probabilities: each thread a contiguous
-      // run, then a block scan of the run totals.
-      const int per = P2 / blockDim.x > 0 ? P2 / blockDim.x : 1;
-      const int beg = threadIdx.x * per;
-      float run = 0.f;
-      for (int i = beg; i < beg + per && i < P2; ++i) run += __uint_as_float((uint32_t)(keys[i] >> 32));
-      scan_part[threadIdx.x] = run;
-      __syncthreads();
-      for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-        const float v = threadIdx.x >= (unsigned)off ? scan_part[threadIdx.x - off] : 0.f;
-        __syncthreads();
-        scan_part[threadIdx.x] += v;
-        __syncthreads();
-      }
-      const float total = scan_part[blockDim.x - 1];
-      const float limit = tau * total;
-      float excl = scan_part[threadIdx.x] - run;
-      for (int i = beg; i < beg + per && i < P2; ++i) {
-        const float p = __uint_as_float((uint32_t)(keys[i] >> 32));
-        const uint32_t kb = ~(uint32_t)keys[i];
-        if (p > 0.f && excl < limit) flags[kb] = 1;
-        excl += p;
-      }
-      (void)sum;
     }
+    __syncthreads();
+    for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) {
+      const bool col = rules.struct_col(kb) || (guard && sk[g * nkb + kb] < theta);
+      const bool keep = rules.valid(qb, kb) && (row_forced || flags[kb] || col || rules.in_window(qb, kb));
+      flags[kb] = keep ? 1 : 0;
+    }
+    __syncthreads();
+    finish_row(flags, u, qb, nkb, rules, mask + u * nkb, counts, status, shi);
+    __syncthreads();
   }
-  __syncthreads();
-  for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) {
-    const bool col = rules.struct_col(kb) || (guard && sk[g * nkb + kb] < theta);
-    const bool keep = rules.valid(qb, kb) &&
-                      (row_forced || flags[kb] || col || rules.in_window(qb, kb));
-    flags[kb] = keep ? 1 : 0;
-  }
-  __syncthreads();
-  finish_row(flags, u, qb, nkb, rules, mask + u * nkb, counts, status, shi);
 }
 
 // A caller-supplied mask row: AND causal validity, copy, count, check.
@@ -536,14 +581,14 @@ sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
   }
   int P2 = 1;
   while (P2 < nkb) P2 <<= 1;
-  const size_t smem = (size_t)P2 * 8 + ((nkb + 15) / 16) * 16 + (size_t)s.d * 4;
+  const size_t smem = score_smem_bytes((int)s.d, nkb, P2) + 16;
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(score_topcdf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(score_topcdf_kernel) failed");
   }
-  const int64_t R = s.B * s.Hq * nqb;
-  score_topcdf_kernel<<<(unsigned)R, kRowThreads, smem, st>>>(
+  dim3 grid((unsigned)ceil_div(nqb, kRowsPerCta), (unsigned)(s.B * s.Hq));
+  score_topcdf_kernel<<<grid, kRowThreads, smem, st>>>(
       w.qhat, w.khat, w.sq, w.sk, s.Hq, s.Hkv, nqb, nkb, (int)s.d, P2, p.tau, p.theta,
       make_rules(s, p), out.block_mask, w.counts, out.status);
   if ((e = check_launch("score_topcdf_kernel"))) return e;

@@ -104,6 +104,7 @@ struct AttnArgs {
   const int32_t* col_idx;
   const int32_t* order;     // nullptr = natural row order
   int32_t* status;
+  int32_t* counter;         // attention workspace: the work counter
   int64_t B, Hq, Hkv, N, d, dv;
   int32_t dtype;
   int32_t bq, bk, causal;

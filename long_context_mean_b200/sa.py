@@ -30,7 +30,7 @@ SA_FLAG_FORCE_SIMT = 1
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_WORKSPACE",
                 4: "SA_ERR_EMPTY_ROW", 5: "SA_ERR_TIMEOUT", 6: "SA_ERR_CUDA", 7: "SA_ERR_CAPACITY"}
 
-EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_layout_workspace",
+EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_attn_workspace", "sa_layout_workspace",
            "sa_layout_build", "sa_reorder", "sa_unreorder", "sa_predict_mask_workspace",
            "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_mask_from_blocks_workspace",
            "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status"]
@@ -100,9 +100,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sa_mask_from_blocks_workspace": (SZ, [ctypes.POINTER(Shape), I32, I32]),
         "sa_mask_from_blocks": (I32, [P, ctypes.POINTER(Shape), I32, I32, I32, P, SZ,
                                       ctypes.POINTER(Mask), P]),
+        "sa_attn_workspace": (SZ, []),
         "sa_block_sparse_attn": (I32, [P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F, F,
-                                       P, P, P, I32, P]),
-        "sa_dense_attn": (I32, [P, P, P, ctypes.POINTER(Shape), I32, F, P, P, P, I32, P]),
+                                       P, P, P, P, SZ, I32, P]),
+        "sa_dense_attn": (I32, [P, P, P, ctypes.POINTER(Shape), I32, F, P, P, P, P, SZ, I32, P]),
         "sa_read_status": (I32, [P, P]),
     }
     for name, (res, args) in sig.items():
@@ -214,17 +215,38 @@ def mask_from_blocks(block_mask, shape: Shape, bq, bk, causal, ws, mask: Mask, s
                                       _stream(stream)))
 
 
+def attn_workspace() -> int:
+    return int(load().sa_attn_workspace())
+
+
+_attn_ws = {}
+
+
+def _default_attn_ws(device):
+    """A per-device attention workspace for callers that pass none (calls on
+    one device then share it, so they must not overlap on the GPU)."""
+    import torch
+    key = str(device)
+    if key not in _attn_ws:
+        _attn_ws[key] = workspace(attn_workspace(), device)
+    return _attn_ws[key]
+
+
 def block_sparse_attn(q, k, v, shape: Shape, mask: Mask, lam, scale, out, lse=None, skip_log=None,
-                      flags=0, stream=None):
+                      flags=0, stream=None, ws=None):
+    ws = ws if ws is not None else _default_attn_ws(q.device)
     _check(load().sa_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), ctypes.byref(mask),
                                        float(lam), float(scale), _ptr(out), _ptr(lse), _ptr(skip_log),
-                                       int(flags), _stream(stream)))
+                                       _ptr(ws), ws.numel() * ws.element_size(), int(flags),
+                                       _stream(stream)))
 
 
-def dense_attn(q, k, v, shape: Shape, causal, scale, out, lse=None, status=None, flags=0, stream=None):
+def dense_attn(q, k, v, shape: Shape, causal, scale, out, lse=None, status=None, flags=0, stream=None,
+               ws=None):
+    ws = ws if ws is not None else _default_attn_ws(q.device)
     _check(load().sa_dense_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), int(bool(causal)),
-                                float(scale), _ptr(out), _ptr(lse), _ptr(status), int(flags),
-                                _stream(stream)))
+                                float(scale), _ptr(out), _ptr(lse), _ptr(status), _ptr(ws),
+                                ws.numel() * ws.element_size(), int(flags), _stream(stream)))
 
 
 def read_status(status, stream=None) -> int:
@@ -299,6 +321,7 @@ class Pipeline:
         self.out = torch.empty(B, Hq, N, dv, dtype=tdt, device=device)
         self.lse = torch.empty(B, Hq, N, 1, dtype=torch.float32, device=device)
         self.ws = workspace(predict_mask_workspace(self.shape, params), device)
+        self.attn_ws = workspace(attn_workspace(), device)
         self.mask = MaskBuffers.allocate(B, Hq, N, params.bq, params.bk, device)
         self.skip_log = (torch.zeros(self.mask.col_idx.numel(), dtype=torch.uint8, device=device)
                          if log_skips else None)
@@ -314,7 +337,7 @@ class Pipeline:
             qr, kr, vr, out_r, lse_r = self.qr, self.kr, self.vr, self.out_r, self.lse_r
         predict_mask(qr, kr, self.shape, self.params, self.ws, self.mask.struct, stream)
         block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, out_r, lse_r,
-                          self.skip_log, self.flags, stream)
+                          self.skip_log, self.flags, stream, ws=self.attn_ws)
         if not self.identity:
             unreorder(self.perm, out_r, self.out, stream)
             unreorder(self.perm, lse_r, self.lse, stream)
