@@ -207,13 +207,17 @@ size_t sa_attn_workspace(void);
  * (tile row max - running row max) over the block's rows is < lambda
  * (lambda = -INFINITY disables the skip; the normaliser l still counts the
  * tile).  scale = 0 means 1/sqrt(d).  out gets O / l in the input dtype,
- * lse (nullable) gets m + ln l.  pv_skip_log (nullable) gets one byte per
- * kept tile in CSR order, 1 = PV skipped.  The mask's status word also
- * receives kernel errors. */
+ * lse (nullable) gets m + ln l.  out_perm (nullable, int32 [N]) fuses the
+ * inverse reorder into the store: row n of the problem is written to row
+ * out_perm[n] of out and lse (pass the layout's perm to get the original
+ * token order back; out must not alias q).  pv_skip_log (nullable) gets one
+ * byte per kept tile in CSR order, 1 = PV skipped.  The mask's status word
+ * also receives kernel errors. */
 sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v,
                                const sa_shape* shape, const sa_mask* mask, float lambda,
-                               float scale, void* out, float* lse, uint8_t* pv_skip_log,
-                               void* ws, size_t ws_bytes, int32_t flags, void* stream);
+                               float scale, void* out, float* lse, const int32_t* out_perm,
+                               uint8_t* pv_skip_log, void* ws, size_t ws_bytes, int32_t flags,
+                               void* stream);
 
 /* ---- a8: dense reference --------------------------------------------------
  * The same recurrence with every (causally valid) key visible and no lists

@@ -226,7 +226,8 @@ sa_status sa_mask_from_blocks(const uint8_t* block_mask, const sa_shape* shape, 
 
 static sa_status attn_common(const void* q, const void* k, const void* v, const sa_shape* shape,
                              const sa_mask* mask, int32_t causal, float lambda, float scale, void* out,
-                             float* lse, uint8_t* skip_log, int32_t* status, void* ws, size_t ws_bytes,
+                             float* lse, const int32_t* out_perm, uint8_t* skip_log, int32_t* status,
+                             void* ws, size_t ws_bytes,
                              int32_t flags, void* stream) {
   if (sa_status e = check_shape(shape)) return e;
   if (!q || !k || !v || !out) return set_error(SA_ERR_INVALID_ARG, "NULL tensor argument");
@@ -242,6 +243,9 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
   a.v = v;
   a.out = out;
   a.lse = lse;
+  a.out_perm = out_perm;
+  if (out_perm && (out == q || out == k || out == v))
+    return set_error(SA_ERR_INVALID_ARG, "out must not alias an input when out_perm is given");
   a.skip_log = skip_log;
   a.B = shape->B;
   a.Hq = shape->Hq;
@@ -291,19 +295,19 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
 
 sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v, const sa_shape* shape,
                                const sa_mask* mask, float lambda, float scale, void* out, float* lse,
-                               uint8_t* pv_skip_log, void* ws, size_t ws_bytes, int32_t flags,
-                               void* stream) {
+                               const int32_t* out_perm, uint8_t* pv_skip_log, void* ws, size_t ws_bytes,
+                               int32_t flags, void* stream) {
   if (!mask) return set_error(SA_ERR_INVALID_ARG, "mask is NULL");
-  return attn_common(q, k, v, shape, mask, 0, lambda, scale, out, lse, pv_skip_log, nullptr, ws, ws_bytes,
-                     flags, stream);
+  return attn_common(q, k, v, shape, mask, 0, lambda, scale, out, lse, out_perm, pv_skip_log, nullptr, ws,
+                     ws_bytes, flags, stream);
 }
 
 sa_status sa_dense_attn(const void* q, const void* k, const void* v, const sa_shape* shape, int32_t causal,
                         float scale, void* out, float* lse, int32_t* status, void* ws, size_t ws_bytes,
                         int32_t flags, void* stream) {
   if (causal != 0 && causal != 1) return set_error(SA_ERR_INVALID_ARG, "causal must be 0 or 1");
-  return attn_common(q, k, v, shape, nullptr, causal, -INFINITY, scale, out, lse, nullptr, status, ws,
-                     ws_bytes, flags, stream);
+  return attn_common(q, k, v, shape, nullptr, causal, -INFINITY, scale, out, lse, nullptr, nullptr, status,
+                     ws, ws_bytes, flags, stream);
 }
 
 sa_status sa_read_status(const int32_t* status, void* stream) {

@@ -121,11 +121,13 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
   for (int idx = threadIdx.x; idx < nr * dv; idx += kThreads) {
     const int r = idx / dv, c = idx % dv;
     const float lr = l[r];
-    Elem<T>::store(out + (i0 + r) * dv + c, lr > 0.f ? O[idx] / lr : 0.f);
+    const int64_t orow = a.out_perm ? a.out_perm[i0 + r] : i0 + r;
+    Elem<T>::store(out + orow * dv + c, lr > 0.f ? O[idx] / lr : 0.f);
   }
   for (int r = threadIdx.x; r < nr; r += kThreads) {
     if (!(l[r] > 0.f)) raise_status(a.status, SA_ERR_EMPTY_ROW);
-    if (a.lse) a.lse[bh * a.N + i0 + r] = m[r] + logf(l[r]);
+    const int64_t orow = a.out_perm ? a.out_perm[i0 + r] : i0 + r;
+    if (a.lse) a.lse[bh * a.N + orow] = m[r] + logf(l[r]);
   }
 }
 

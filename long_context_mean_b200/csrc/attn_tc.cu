@@ -6,22 +6,29 @@
 // (rowmax S - running max) < lambda, l still counting the tile.
 //
 // Design (bf16, d = dv = 128, bq = 128, bk = 64 or 128):
-//   * persistent grid, one CTA per SM.  A CTA runs PIPES independent
-//     pipelines (2 for bk = 64, 1 for bk = 128), each on its own stream of
-//     work units (b, h, q-block) taken in the mask's work order, so every
-//     SM sub-partition holds PIPES softmax warps;
+//   * persistent grid, one CTA per SM, PIPES independent pipelines per CTA
+//     (2 for bk = 64, 1 for bk = 128) so every SM sub-partition holds PIPES
+//     softmax warps.  Units (b, h, q-block) are taken dynamically, in the
+//     mask's work order (descending kept count), from a global counter by
+//     each pipeline's producer and announced to its MMA and softmax warps
+//     through a 4-slot ring.
 //   * per pipeline, warp p (one lane) is the TMA producer (Q tile once per
 //     unit, K and V tiles of the kept key blocks through a STAGES ring) and
 //     warp 2+p (one lane) issues tcgen05.mma: S = Q K^T into one of two TMEM
-//     S buffers, and O += P V one tile behind with P read from TMEM (the
-//     softmax overwrites S with P in place), so the tensor core runs S(t+1)
-//     and PV(t-1) while the softmax warps work on S(t);
+//     S buffers and O += P V into the TMEM O accumulator.
+//       bk = 64:  the softmax releases an S buffer as soon as it has loaded
+//                 it and writes P (bf16) to a shared-memory buffer in the
+//                 128-byte-swizzled K-major layout, so S runs two tiles
+//                 ahead of PV (S(t+2) and PV(t) overlap the softmax of t+1);
+//       bk = 128: P overwrites S in TMEM and PV reads it from there, S runs
+//                 one tile ahead.
 //   * per pipeline, four softmax warps (one thread per query row = TMEM
-//     lane): S from TMEM, masks, running max, exp2, P back to TMEM, O rescale
-//     in TMEM when the reference maximum moves, the epilogue O / l and LSE.
-//     Each warp publishes the largest (tile max - running max) of its rows;
-//     the MMA warp combines the four and takes the lambda decision, so the
-//     softmax warps never wait for one another.
+//     lane): S from TMEM, masks, running max, exp2 (scale folded into one
+//     packed fp32x2 FMA), P, O rescale in TMEM when the reference maximum
+//     moves, the epilogue O / l and LSE (stored through an optional row
+//     permutation).  Each warp publishes the largest (tile max - running
+//     max) of its rows; the MMA warp combines the four and takes the lambda
+//     decision, so the softmax warps never wait for one another.
 //   The exact running max drives the lambda test; O and l use a reference
 //   maximum that only moves when the running max exceeds it by more than
 //   2^8 (O / l is the same quotient).  A row whose maximum moves has a gap of
@@ -43,15 +50,22 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 template <int BK>
 struct Cfg {
+  // P in shared memory (SS MMA, S two tiles ahead of PV) or over S in TMEM
+  // (TS MMA, S one tile ahead).  Measured on B200 at bk = 64 the TMEM form
+  // is faster (the SS form adds 16 KB of operand reads per tile), so both
+  // block sizes use it; the shared-memory form stays for other shapes.
+  static constexpr bool P_SMEM = false;
   static constexpr int PIPES = BK == 64 ? 2 : 1;
   static constexpr int STAGES = BK == 64 ? 2 : 3;
+  static constexpr int LOOKAHEAD = P_SMEM ? 2 : 1;    // S tiles issued ahead of PV
   static constexpr int THREADS = 128 + 128 * PIPES;
   static constexpr int Q_BYTES = 128 * 128 * 2;
   static constexpr int KV_BYTES = BK * 128 * 2;
   static constexpr int KV_CHUNK = BK * 128;          // one 64-column chunk: BK rows x 128 B
-  static constexpr int PIPE_BYTES = Q_BYTES + 2 * STAGES * KV_BYTES;
+  static constexpr int P_BYTES = P_SMEM ? 128 * BK * 2 : 0;
+  static constexpr int PIPE_BYTES = Q_BYTES + 2 * STAGES * KV_BYTES + P_BYTES;
   static constexpr int OFF_CTL = PIPES * PIPE_BYTES;
-  static constexpr int CTL_BYTES = 1024;
+  static constexpr int CTL_BYTES = 512;
   static constexpr int SMEM = OFF_CTL + PIPES * CTL_BYTES + 1024;   // + alignment slack
   static constexpr int TMEM_PIPE = (128 + 2 * BK) <= 256 ? 256 : 512;
   static constexpr int TMEM_COLS = PIPES * TMEM_PIPE;
@@ -59,19 +73,21 @@ struct Cfg {
   static __host__ __device__ constexpr int off_q(int p) { return p * PIPE_BYTES; }
   static __host__ __device__ constexpr int off_k(int p) { return p * PIPE_BYTES + Q_BYTES; }
   static __host__ __device__ constexpr int off_v(int p) { return p * PIPE_BYTES + Q_BYTES + STAGES * KV_BYTES; }
+  static __host__ __device__ constexpr int off_p(int p) { return p * PIPE_BYTES + Q_BYTES + 2 * STAGES * KV_BYTES; }
 };
 
 // Per-pipeline control block (8-byte mbarriers first).
 struct Ctl {
   uint64_t q_full, q_empty, o_free;
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
-  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
   uint64_t u_full[4], u_empty[4];          // unit announcement ring
   uint32_t tmem_base;
   volatile uint32_t abort;
-  float gapw[2][4];
+  float gapw[4][4];                        // [tile & 3][softmax warp]
   volatile int32_t ring[4];
 };
+static_assert(sizeof(Ctl) <= 512, "control block too large");
 
 struct TcParams {
   const int32_t* row_ptr;
@@ -79,6 +95,7 @@ struct TcParams {
   const int32_t* order;
   uint16_t* out;
   float* lse;
+  const int32_t* out_perm;
   uint8_t* skip_log;
   int32_t* status;
   int32_t* counter;      // work counter, zero at launch
@@ -111,14 +128,16 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
+// One try_wait; the thread may be suspended (up to the hint, in ns) until
+// the phase completes, so waiting warps do not take issue slots.
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
@@ -127,15 +146,13 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl* g, int32_t* status) {
   if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try(bar, parity)) return true;
-    if ((it & 63) == 0) {
-      if (g->abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        g->abort = 1;
-        raise_status(status, SA_ERR_TIMEOUT);
-        return false;
-      }
+    if (g->abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      g->abort = 1;
+      raise_status(status, SA_ERR_TIMEOUT);
+      return false;
     }
   }
 }
@@ -156,6 +173,8 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Generic-proxy shared-memory writes become visible to the tensor core.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // D (TMEM) = A (SMEM desc) x B (SMEM desc) [+ D]
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -233,6 +252,33 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
+}
+// 2^x for a pair of arguments on the FMA pipe.  Cody-Waite range reduction
+// (n = round(x) by the 1.5 * 2^23 addition, f = x - n in [-1/2, 1/2]), a cubic
+// for 2^f fitted for minimax relative error by csrc/fit_exp2.py (max relative
+// error 1.5e-4 in float32, below the bf16 rounding of P), and n added to the
+// exponent field.  x is clamped at -125 so the result stays a normal number;
+// the caller never passes masked (-inf) scores.
+constexpr float kExpC0 = 9.999280572e-01f, kExpC1 = 6.932609677e-01f;
+constexpr float kExpC2 = 2.426109314e-01f, kExpC3 = 5.517149344e-02f;
+constexpr int kEmuPairs = 0;   // of every 8 column pairs, this many use the FMA pipe
+                               // (0: measured slower on B200 at bk = 64 -- the
+                               // softmax is latency-bound, not MUFU-bound)
+__device__ __forceinline__ void exp2_fma_pair(uint64_t x2, float& r0, float& r1) {
+  float x0, x1;
+  unpack2(x2, x0, x1);
+  x2 = pack2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t magic = pack2(12582912.f, 12582912.f);
+  const uint64_t t = fadd2(x2, magic);
+  const uint64_t f = ffma2(fadd2(t, pack2(-12582912.f, -12582912.f)), pack2(-1.f, -1.f), x2);
+  uint64_t q = ffma2(pack2(kExpC3, kExpC3), f, pack2(kExpC2, kExpC2));
+  q = ffma2(q, f, pack2(kExpC1, kExpC1));
+  q = ffma2(q, f, pack2(kExpC0, kExpC0));
+  float q0, q1, t0, t1;
+  unpack2(q, q0, q1);
+  unpack2(t, t0, t1);
+  r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -350,8 +396,8 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
       const int gb = gt & 1;
       mbar_wait(&c->p_full[gb], (gt >> 1) & 1, g, p.status);
       tc_fence_after();
-      const float gap = fmaxf(fmaxf(c->gapw[gb][0], c->gapw[gb][1]), fmaxf(c->gapw[gb][2], c->gapw[gb][3]));
-      const bool skip = gap < p.lam_log2;
+      const float* gw = c->gapw[gt & 3];
+      const bool skip = fmaxf(fmaxf(gw[0], gw[1]), fmaxf(gw[2], gw[3])) < p.lam_log2;
       if (p.skip_log && p.row_ptr) p.skip_log[u.lo + tt] = skip ? 1 : 0;
       if (tt == 0) {
         mbar_wait(&c->o_free, (unit_it & 1) ^ 1, g, p.status);
@@ -361,11 +407,16 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
       tc_fence_after();
       if (!skip) {
         const uint32_t vbase = sb + C::off_v(pipe) + s * C::KV_BYTES;
-        const uint32_t pcol = tm + C::S_COL + gb * BK;   // P (bf16 pairs) over the S buffer
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t b = desc_sw128(vbase + kk * 2048, C::KV_CHUNK, 1024);
-          umma_ts(tm, pcol + kk * 8, b, idesc_pv, (first_pv && kk == 0) ? 0u : 1u);
+          const uint32_t acc = (first_pv && kk == 0) ? 0u : 1u;
+          if constexpr (C::P_SMEM) {
+            const uint64_t a = desc_sw128(sb + C::off_p(pipe) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            umma_ss(tm, a, b, idesc_pv, acc);
+          } else {
+            umma_ts(tm, tm + C::S_COL + gb * BK + kk * 8, b, idesc_pv, acc);   // P over the S buffer
+          }
         }
         first_pv = false;
       }
@@ -378,6 +429,7 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
       const uint32_t ph = (it / C::STAGES) & 1;
       const int gb = gt & 1;
       mbar_wait(&c->k_full[s], ph, g, p.status);
+      if constexpr (C::P_SMEM) mbar_wait(&c->s_empty[gb], ((gt >> 1) & 1) ^ 1, g, p.status);
       tc_fence_after();
       const uint32_t kbase = sb + C::off_k(pipe) + s * C::KV_BYTES;
       const uint32_t qbase = sb + C::off_q(pipe);
@@ -390,21 +442,31 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
       umma_commit(&c->s_full[gb]);
       umma_commit(&c->k_empty[s]);
       if (t == u.n - 1) umma_commit(&c->q_empty);
-      if (t >= 1) do_pv(t - 1);
+      if (t >= C::LOOKAHEAD) do_pv(t - C::LOOKAHEAD);
     }
-    do_pv(u.n - 1);
+    for (int64_t tt = u.n > C::LOOKAHEAD ? u.n - C::LOOKAHEAD : 0; tt < u.n; ++tt) do_pv(tt);
     kv_it += (uint32_t)u.n;
     gt0 += (uint32_t)u.n;
     ++unit_it;
   }
 }
 
+// Largest value of a float over the warp (order-preserving int key).
+__device__ __forceinline__ float warp_fmax(float v) {
+  int k = __float_as_int(v);
+  k = k >= 0 ? k : k ^ 0x7FFFFFFF;
+  const int m = __reduce_max_sync(0xffffffffu, k);
+  return __int_as_float(m >= 0 ? m : m ^ 0x7FFFFFFF);
+}
+
 template <int BK>
-__device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int pipe, int wq, int lane) {
+__device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, uint32_t tm, int pipe, int wq,
+                             int lane) {
   using C = Cfg<BK>;
   const int row = wq * 32 + lane;
   const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
   const float sc = p.scale_log2;
+  uint8_t* prow = smem + C::off_p(pipe) + (row >> 3) * 1024 + (row & 7) * 128;
   uint32_t gt0 = 0;
   for (uint32_t j = 0;; ++j) {
     const int slot = j & 3;
@@ -433,36 +495,39 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
 #pragma unroll
       for (int cc = 0; cc < BK / 32; ++cc) tmem_ld32(scol + cc * 32, s + cc * 32);
       tmem_wait_ld();
+      if constexpr (C::P_SMEM) {
+        tc_fence_before();
+        mbar_arrive(&c->s_empty[gb]);          // S buffer free for S(t+2)
+      }
 
       const int64_t k0 = kb_cur * BK;
       kb_cur = kb_next;
-      if ((k0 + BK > p.N) || (p.causal && k0 + BK - 1 > u.qb * 128)) {
+      const bool need_mask = (k0 + BK > p.N) || (p.causal && k0 + BK - 1 > u.qb * 128);
+      if (need_mask) {
 #pragma unroll
-        for (int j = 0; j < BK; ++j) {
-          const int64_t key = k0 + j;
-          if (key >= p.N || (p.causal && key > row_g)) s[j] = -INFINITY;
+        for (int jj = 0; jj < BK; ++jj) {
+          const int64_t key = k0 + jj;
+          if (key >= p.N || (p.causal && key > row_g)) s[jj] = -INFINITY;
         }
       }
       // Row max as a tree of 3-input maxima (independent chains), raw units.
       float mx[BK / 4];
 #pragma unroll
-      for (int j = 0; j < BK / 4; ++j) mx[j] = max3(fmaxf(s[4 * j], s[4 * j + 1]), s[4 * j + 2], s[4 * j + 3]);
+      for (int jj = 0; jj < BK / 4; ++jj) mx[jj] = max3(fmaxf(s[4 * jj], s[4 * jj + 1]), s[4 * jj + 2], s[4 * jj + 3]);
 #pragma unroll
       for (int w = BK / 4; w > 1; w = (w + 2) / 3) {
 #pragma unroll
-        for (int j = 0; j < (w + 2) / 3; ++j) {
-          const float a = mx[3 * j];
-          const float b = 3 * j + 1 < w ? mx[3 * j + 1] : a;
-          const float d = 3 * j + 2 < w ? mx[3 * j + 2] : a;
-          mx[j] = max3(a, b, d);
+        for (int jj = 0; jj < (w + 2) / 3; ++jj) {
+          const float a = mx[3 * jj];
+          const float b = 3 * jj + 1 < w ? mx[3 * jj + 1] : a;
+          const float d = 3 * jj + 2 < w ? mx[3 * jj + 2] : a;
+          mx[jj] = max3(a, b, d);
         }
       }
       const float mloc = mx[0] * sc;                    // scale > 0: max commutes
       const float m_new = fmaxf(m_run, mloc);
-      float gap = (row_valid && mloc > -INFINITY) ? mloc - m_new : -INFINITY;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) gap = fmaxf(gap, __shfl_xor_sync(0xffffffffu, gap, off));
-      if (lane == 0) c->gapw[gb][wq] = gap;
+      const float gap = warp_fmax((row_valid && mloc > -INFINITY) ? mloc - m_new : -INFINITY);
+      if (lane == 0) c->gapw[gt & 3][wq] = gap;
       m_run = m_new;
       float corr = 1.f;
       bool resc = false;
@@ -479,15 +544,21 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
         const uint64_t sc2 = pack2(sc, sc), neg2 = pack2(-m_ref, -m_ref);
         uint64_t acc[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j] = pack2(0.f, 0.f);
+        for (int jj = 0; jj < 4; ++jj) acc[jj] = pack2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < BK; j += 2) {
-          const uint64_t x = ffma2(pack2(s[j], s[j + 1]), sc2, neg2);
-          float x0, x1;
-          unpack2(x, x0, x1);
-          const float p0 = ex2(x0), p1 = ex2(x1);
-          acc[(j >> 1) & 3] = fadd2(acc[(j >> 1) & 3], pack2(p0, p1));
-          pk[j >> 1] = pack_bf16(p0, p1);
+        for (int jj = 0; jj < BK; jj += 2) {
+          const uint64_t x = ffma2(pack2(s[jj], s[jj + 1]), sc2, neg2);
+          float p0, p1;
+          if (((jj >> 1) & 7) < kEmuPairs && !need_mask) {
+            exp2_fma_pair(x, p0, p1);          // FMA pipe, relieves the MUFU
+          } else {
+            float x0, x1;
+            unpack2(x, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          acc[(jj >> 1) & 3] = fadd2(acc[(jj >> 1) & 3], pack2(p0, p1));
+          pk[jj >> 1] = pack_bf16(p0, p1);
         }
         const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
         float lo, hi;
@@ -495,15 +566,17 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
         row_sum = lo + hi;
       } else {
 #pragma unroll
-        for (int j = 0; j < BK / 2; ++j) pk[j] = 0u;
+        for (int jj = 0; jj < BK / 2; ++jj) pk[jj] = 0u;
       }
       l = l * corr + row_sum;
       // tcgen05.ld/st are warp-collective: a warp rescales when any of its
       // rows needs it (corr is 1 for the others).  A rescale implies the
       // tile is not skipped, so PV(t-1) is the last product to wait for.
+      bool pv_prev_done = false;
       if (__any_sync(0xffffffffu, resc)) {
         const uint32_t gp = gt - 1;
         mbar_wait(&c->pv_done[gp & 1], (gp >> 1) & 1, g, p.status);
+        pv_prev_done = true;
         tc_fence_after();
         const float f = resc ? corr : 1.f;
 #pragma unroll
@@ -512,13 +585,28 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
           tmem_ld32(tm + lane_off + cc * 32, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] *= f;
+          for (int jj = 0; jj < 32; ++jj) o[jj] *= f;
           tmem_st32(tm + lane_off + cc * 32, reinterpret_cast<const uint32_t*>(o));
         }
+        tmem_wait_st();
       }
+      if constexpr (C::P_SMEM) {
+        // The single P buffer is free once PV of the previous tile is done.
+        if (gt >= 1 && !pv_prev_done) {
+          const uint32_t gp = gt - 1;
+          mbar_wait(&c->pv_done[gp & 1], (gp >> 1) & 1, g, p.status);
+        }
 #pragma unroll
-      for (int cc = 0; cc < BK / 64; ++cc) tmem_st32(scol + cc * 32, pk + cc * 32);
-      tmem_wait_st();
+        for (int cc = 0; cc < BK / 8; ++cc) {
+          const uint4 v4 = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+          *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) = v4;
+        }
+        fence_async_smem();
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < BK / 64; ++cc) tmem_st32(scol + cc * 32, pk + cc * 32);
+        tmem_wait_st();
+      }
       tc_fence_before();
       mbar_arrive(&c->p_full[gb]);
     }
@@ -527,7 +615,8 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
     mbar_wait(&c->pv_done[gl & 1], (gl >> 1) & 1, g, p.status);
     tc_fence_after();
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    uint16_t* orow = p.out + (u.bh * p.N + row_g) * 128;
+    const int64_t out_row = row_valid ? (p.out_perm ? (int64_t)p.out_perm[row_g] : row_g) : 0;
+    uint16_t* orow = p.out + (u.bh * p.N + out_row) * 128;
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       float o[32];
@@ -550,7 +639,7 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
     mbar_arrive(&c->o_free);
     if (row_valid) {
       if (!(l > 0.f)) raise_status(p.status, SA_ERR_EMPTY_ROW);
-      if (p.lse) p.lse[u.bh * p.N + row_g] = (m_ref + __log2f(l)) * kLn2;
+      if (p.lse) p.lse[u.bh * p.N + out_row] = (m_ref + __log2f(l)) * kLn2;
     }
     gt0 += (uint32_t)u.n;
   }
@@ -581,6 +670,7 @@ __global__ void __launch_bounds__(Cfg<BK>::THREADS, 1)
       }
       for (int b = 0; b < 2; ++b) {
         mbar_init(&c->s_full[b], 1);
+        mbar_init(&c->s_empty[b], 128);
         mbar_init(&c->p_full[b], 128);
         mbar_init(&c->pv_done[b], 1);
       }
@@ -619,7 +709,7 @@ __global__ void __launch_bounds__(Cfg<BK>::THREADS, 1)
   } else {
     const int pipe = (warp - 4) >> 2;
     Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + pipe * C::CTL_BYTES);
-    softmax_rows<BK>(p, c, ctl0, tmem + pipe * C::TMEM_PIPE, pipe, warp & 3, lane);
+    softmax_rows<BK>(p, c, ctl0, smem, tmem + pipe * C::TMEM_PIPE, pipe, warp & 3, lane);
   }
 
   tc_fence_before();
@@ -676,6 +766,7 @@ sa_status launch_bk(const AttnArgs& a, cudaStream_t st) {
   p.order = a.order;
   p.out = static_cast<uint16_t*>(a.out);
   p.lse = a.lse;
+  p.out_perm = a.out_perm;
   p.skip_log = a.skip_log;
   p.status = a.status;
   p.counter = a.counter;

@@ -26,7 +26,7 @@ constexpr int kPoolWarps = kPoolThreads / 32;
 // ---------------------------------------------------------------------------
 // a2: one CTA per (head, block): block mean and mean pairwise cosine.  A warp
 // covers 32/chunks tokens per step (chunks = 16-byte pieces of a token),
-// two steps in flight; token norms reduce inside each token's lane group.
+// four steps in flight; token norms reduce inside each token's lane group.
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
@@ -46,17 +46,18 @@ __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
   for (int e = 0; e < EPL; ++e) ax[e] = au[e] = 0.f;
   const uint4* base = reinterpret_cast<const uint4*>(x + (bh * N + t0) * (int64_t)d);
   const int step = kPoolWarps * tpw;
-  for (int tb = warp * tpw; tb < cnt; tb += 2 * step) {
-    uint4 raw[2];
-    bool ok[2];
+  constexpr int kInFlight = 4;
+  for (int tb = warp * tpw; tb < cnt; tb += kInFlight * step) {
+    uint4 raw[kInFlight];
+    bool ok[kInFlight];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kInFlight; ++u) {
       const int tok = tb + u * step + sub;
       ok[u] = tok < cnt;
       raw[u] = ok[u] ? __ldg(base + (int64_t)tok * chunks + c) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kInFlight; ++u) {
       float v[EPL];
       unpack16(raw[u], T(), v);
       float ss = 0.f;
@@ -207,49 +208,61 @@ __device__ void finish_row(const uint8_t* flags, int64_t u, int64_t qb, int64_t 
 }
 
 // ---------------------------------------------------------------------------
-// a3 + a4: one CTA per (head, group of kRowsPerCta query blocks).  The
-// group's q_hat rows and 32-row chunks of the kv head's k_hat are staged in
-// shared memory (padded rows, conflict-free) so every k_hat element is read
-// once per group; then, row by row: softmax, bitonic sort of (p, kb) keys
-// descending (ties: lower kb first), scan, TopCdf, and the union with the
-// forced parts and the causal AND.
-// Dynamic shared memory: q_hat [G][d] | k_hat chunk [32][d+1] |
-// scores [G][nkb] | keys [P2] (u64) | flags [nkb] (u8).
+// a3 + a4: one CTA per (head, group of G <= 8 query blocks).  The group's
+// q_hat rows and 32-row chunks of the kv head's k_hat are staged in shared
+// memory (padded rows, conflict-free) so every k_hat element is read once per
+// group.  Then warp r alone finishes row r: softmax, bitonic sort of
+// (p, kb) keys descending (ties: lower kb first), scan, TopCdf, the union with
+// the forced parts and the causal AND -- with warp-level synchronisation
+// only.
+// Dynamic shared memory: q_hat [8][d] | k_hat chunk [32][d+1] |
+// scores [G][nkb] | keys [G][P2] (u64) | flags [G][nkb rounded to 16] (u8).
 // ---------------------------------------------------------------------------
-constexpr int kRowsPerCta = 8;
+constexpr int kMaxRowsPerCta = 8;
 constexpr int kChunk = 32;
 
-size_t score_smem_bytes(int d, int64_t nkb, int P2) {
-  return (size_t)kRowsPerCta * d * 4 + (size_t)kChunk * (d + 1) * 4 + (size_t)kRowsPerCta * nkb * 4 +
-         (size_t)P2 * 8 + (size_t)((nkb + 15) / 16) * 16;
+int score_rows_per_cta(int P2) {
+  int g = 65536 / (P2 * 8);
+  return g < 1 ? 1 : (g > kMaxRowsPerCta ? kMaxRowsPerCta : g);
+}
+
+size_t score_smem_bytes(int d, int64_t nkb, int P2, int G) {
+  const size_t nkb16 = (size_t)((nkb + 15) / 16) * 16;
+  return (size_t)kMaxRowsPerCta * d * 4 + (size_t)kChunk * (d + 1) * 4 + (size_t)G * nkb * 4 +
+         (size_t)G * P2 * 8 + (size_t)G * nkb16;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
 }
 
 __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
     const float* __restrict__ qhat, const float* __restrict__ khat, const float* __restrict__ sq,
     const float* __restrict__ sk, int64_t Hq, int64_t Hkv, int64_t nqb, int64_t nkb, int d,
-    int P2, float tau, float theta, RowRules rules, uint8_t* __restrict__ mask,
+    int P2, int G, float tau, float theta, RowRules rules, uint8_t* __restrict__ mask,
     int32_t* __restrict__ counts, int32_t* status) {
   extern __shared__ __align__(16) unsigned char smem[];
+  const int nkb16 = (int)((nkb + 15) / 16) * 16;
   float* qs = reinterpret_cast<float*>(smem);
-  float* ks = qs + kRowsPerCta * d;
+  float* ks = qs + kMaxRowsPerCta * d;
   float* sc = ks + kChunk * (d + 1);
-  // 8-byte aligned: the float offset 8d + 32(d+1) + 8 nkb is even.
-  uint64_t* keys = reinterpret_cast<uint64_t*>(sc + kRowsPerCta * nkb);
-  uint8_t* flags = reinterpret_cast<uint8_t*>(keys + P2);
-  __shared__ float shf[32];
-  __shared__ int shi[32];
-  __shared__ float scan_part[kRowThreads];
-  __shared__ int s_forced[kRowsPerCta];
+  // 8-byte aligned: the float offset 8d + 32(d+1) + G nkb is even (G even
+  // or nkb even; see score_rows_per_cta).
+  uint64_t* keys = reinterpret_cast<uint64_t*>(sc + G * nkb);
+  uint8_t* flags = reinterpret_cast<uint8_t*>(keys + (size_t)G * P2);
+  __shared__ int s_forced[kMaxRowsPerCta];
 
   const int64_t bh = blockIdx.y;
-  const int64_t qb0 = (int64_t)blockIdx.x * kRowsPerCta;
-  const int rows = (int)min64(kRowsPerCta, nqb - qb0);
+  const int64_t qb0 = (int64_t)blockIdx.x * G;
+  const int rows = (int)min64(G, nqb - qb0);
   const int64_t b = bh / Hq, h = bh % Hq;
   const int64_t g = b * Hkv + h / (Hq / Hkv);
   const bool guard = theta > 0.f;
   const float scale = rsqrtf((float)d);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (threadIdx.x < kRowsPerCta) {
+  if (threadIdx.x < kMaxRowsPerCta) {
     const int r = threadIdx.x;
     const int64_t u = bh * nqb + qb0 + r;
     s_forced[r] = (r >= rows) ? 1 : ((rules.struct_row(qb0 + r) || (guard && sq[u] < theta)) ? 1 : 0);
@@ -260,16 +273,37 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   for (int r = 0; r < rows; ++r) any_scored |= !s_forced[r];
 
   if (any_scored) {
-    // Scores of the whole group, one k_hat chunk at a time.
-    const float* kg = khat + g * nkb * (int64_t)d;
+    // Scores of the whole group, one k_hat chunk at a time: the next chunk's
+    // float4 loads are in flight while the current chunk is multiplied.
+    const float4* kg4 = reinterpret_cast<const float4*>(khat + g * nkb * (int64_t)d);
+    const int nf4 = d / 4;
     const int r = threadIdx.x / kChunk, j = threadIdx.x % kChunk;
+    constexpr int kPer = kChunk * 256 / 4 / kRowThreads;   // float4 per thread (d <= 256)
+    float4 buf[kPer];
+    auto load_chunk = [&](int64_t c0) {
+      const int total = (int)min64(kChunk, nkb - c0) * nf4;
+#pragma unroll
+      for (int q = 0; q < kPer; ++q) {
+        const int i = threadIdx.x + q * kRowThreads;
+        buf[q] = i < total ? __ldg(kg4 + c0 * nf4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    load_chunk(0);
     for (int64_t c0 = 0; c0 < nkb; c0 += kChunk) {
       const int cn = (int)min64(kChunk, nkb - c0);
-      for (int i = threadIdx.x; i < cn * d; i += blockDim.x) {
-        const int jj = i / d, e = i % d;
-        ks[jj * (d + 1) + e] = kg[(c0 + jj) * d + e];
+#pragma unroll
+      for (int q = 0; q < kPer; ++q) {
+        const int i = threadIdx.x + q * kRowThreads;
+        if (i < cn * nf4) {
+          float* dst = ks + (i / nf4) * (d + 1) + (i % nf4) * 4;
+          dst[0] = buf[q].x;
+          dst[1] = buf[q].y;
+          dst[2] = buf[q].z;
+          dst[3] = buf[q].w;
+        }
       }
       __syncthreads();
+      if (c0 + kChunk < nkb) load_chunk(c0 + kChunk);
       const int64_t kb = c0 + j;
       if (r < rows && j < cn) {
         float s = -INFINITY;
@@ -291,79 +325,91 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
     }
   }
 
-  for (int r = 0; r < rows; ++r) {
-    const int64_t qb = qb0 + r;
-    const int64_t u = bh * nqb + qb;
-    const bool row_forced = s_forced[r] != 0;
-    for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) flags[kb] = 0;
-    if (!row_forced) {
-      const float* srow = sc + r * nkb;
-      float mx = -INFINITY;
-      for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) mx = fmaxf(mx, srow[kb]);
-      mx = block_reduce_max(mx, shf);
-      if (mx > -INFINITY) {
-        for (int64_t kb = threadIdx.x; kb < P2; kb += blockDim.x) {
-          uint64_t key = 0ull;
-          if (kb < nkb) {
-            const float s = srow[kb];
-            const float p = (s == -INFINITY) ? 0.f : expf(s - mx);
-            // key = p bits (p >= 0: integer order = float order) | ~kb
-            key = ((uint64_t)__float_as_uint(p) << 32) | (uint32_t)(~(uint32_t)kb);
-          }
-          keys[kb] = key;
+  if (warp >= rows) return;
+  // ---- warp `warp` finishes row r = warp ----
+  const int r = warp;
+  const int64_t qb = qb0 + r;
+  const int64_t u = bh * nqb + qb;
+  const bool row_forced = s_forced[r] != 0;
+  uint64_t* kw = keys + (size_t)r * P2;
+  uint8_t* fl = flags + (size_t)r * nkb16;
+  for (int64_t kb = lane; kb < nkb; kb += 32) fl[kb] = 0;
+  if (!row_forced) {
+    const float* srow = sc + r * nkb;
+    float mx = -INFINITY;
+    for (int64_t kb = lane; kb < nkb; kb += 32) mx = fmaxf(mx, srow[kb]);
+    mx = warp_max(mx);
+    if (mx > -INFINITY) {
+      for (int kb = lane; kb < P2; kb += 32) {
+        uint64_t key = 0ull;
+        if (kb < nkb) {
+          const float sv = srow[kb];
+          const float p = (sv == -INFINITY) ? 0.f : expf(sv - mx);
+          // key = p bits (p >= 0: integer order = float order) | ~kb
+          key = ((uint64_t)__float_as_uint(p) << 32) | (uint32_t)(~(uint32_t)kb);
         }
-        __syncthreads();
-        // Bitonic sort, descending.
-        for (int k = 2; k <= P2; k <<= 1) {
-          for (int jj = k >> 1; jj > 0; jj >>= 1) {
-            for (int i = threadIdx.x; i < P2; i += blockDim.x) {
-              const int ixj = i ^ jj;
-              if (ixj > i) {
-                const uint64_t a = keys[i], c = keys[ixj];
-                const bool desc = (i & k) == 0;
-                if (desc ? (a < c) : (a > c)) {
-                  keys[i] = c;
-                  keys[ixj] = a;
-                }
+        kw[kb] = key;
+      }
+      __syncwarp();
+      // Bitonic sort, descending.
+      for (int k = 2; k <= P2; k <<= 1) {
+        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+          for (int i = lane; i < P2; i += 32) {
+            const int ixj = i ^ jj;
+            if (ixj > i) {
+              const uint64_t x = kw[i], y = kw[ixj];
+              const bool desc = (i & k) == 0;
+              if (desc ? (x < y) : (x > y)) {
+                kw[i] = y;
+                kw[ixj] = x;
               }
             }
-            __syncthreads();
           }
-        }
-        // Inclusive scan of the sorted probabilities: each thread a contiguous
-        // run, then a block scan of the run totals.
-        const int per = P2 / (int)blockDim.x > 0 ? P2 / (int)blockDim.x : 1;
-        const int beg = threadIdx.x * per;
-        float run = 0.f;
-        for (int i = beg; i < beg + per && i < P2; ++i) run += __uint_as_float((uint32_t)(keys[i] >> 32));
-        scan_part[threadIdx.x] = run;
-        __syncthreads();
-        for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-          const float v = threadIdx.x >= (unsigned)off ? scan_part[threadIdx.x - off] : 0.f;
-          __syncthreads();
-          scan_part[threadIdx.x] += v;
-          __syncthreads();
-        }
-        const float total = scan_part[blockDim.x - 1];
-        const float limit = tau * total;
-        float excl = scan_part[threadIdx.x] - run;
-        for (int i = beg; i < beg + per && i < P2; ++i) {
-          const float p = __uint_as_float((uint32_t)(keys[i] >> 32));
-          const uint32_t kb = ~(uint32_t)keys[i];
-          if (p > 0.f && excl < limit) flags[kb] = 1;
-          excl += p;
+          __syncwarp();
         }
       }
+      // Inclusive scan of the sorted probabilities: lane `lane` owns a
+      // contiguous run, then a warp scan of the run totals.
+      const int per = P2 >= 32 ? P2 / 32 : 1;
+      const int beg = lane * per;
+      float run = 0.f;
+      for (int i = beg; i < beg + per && i < P2; ++i) run += __uint_as_float((uint32_t)(kw[i] >> 32));
+      float incl = run;
+      for (int off = 1; off < 32; off <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      const float total = __shfl_sync(0xffffffffu, incl, 31);
+      const float limit = tau * total;
+      float excl = incl - run;
+      for (int i = beg; i < beg + per && i < P2; ++i) {
+        const float p = __uint_as_float((uint32_t)(kw[i] >> 32));
+        const uint32_t kb = ~(uint32_t)kw[i];
+        if (p > 0.f && excl < limit) fl[kb] = 1;
+        excl += p;
+      }
     }
-    __syncthreads();
-    for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) {
-      const bool col = rules.struct_col(kb) || (guard && sk[g * nkb + kb] < theta);
-      const bool keep = rules.valid(qb, kb) && (row_forced || flags[kb] || col || rules.in_window(qb, kb));
-      flags[kb] = keep ? 1 : 0;
+  }
+  __syncwarp();
+  int cnt = 0, first = 0x7fffffff;
+  uint8_t* mrow = mask + u * nkb;
+  for (int64_t kb = lane; kb < nkb; kb += 32) {
+    const bool col = rules.struct_col(kb) || (guard && sk[g * nkb + kb] < theta);
+    const bool keep = rules.valid(qb, kb) && (row_forced || fl[kb] || col || rules.in_window(qb, kb));
+    mrow[kb] = keep ? 1 : 0;
+    if (keep) {
+      ++cnt;
+      first = min(first, (int)kb);
     }
-    __syncthreads();
-    finish_row(flags, u, qb, nkb, rules, mask + u * nkb, counts, status, shi);
-    __syncthreads();
+  }
+  for (int off = 16; off > 0; off >>= 1) {
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    first = min(first, __shfl_xor_sync(0xffffffffu, first, off));
+  }
+  if (lane == 0) {
+    counts[u] = cnt;
+    const bool empty = rules.causal ? (cnt == 0 || (int64_t)first * rules.bk > qb * rules.bq) : cnt == 0;
+    if (empty) raise_status(status, SA_ERR_EMPTY_ROW);
   }
 }
 
@@ -581,15 +627,16 @@ sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
   }
   int P2 = 1;
   while (P2 < nkb) P2 <<= 1;
-  const size_t smem = score_smem_bytes((int)s.d, nkb, P2) + 16;
+  const int G = score_rows_per_cta(P2);
+  const size_t smem = score_smem_bytes((int)s.d, nkb, P2, G);
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(score_topcdf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(score_topcdf_kernel) failed");
   }
-  dim3 grid((unsigned)ceil_div(nqb, kRowsPerCta), (unsigned)(s.B * s.Hq));
+  dim3 grid((unsigned)ceil_div(nqb, G), (unsigned)(s.B * s.Hq));
   score_topcdf_kernel<<<grid, kRowThreads, smem, st>>>(
-      w.qhat, w.khat, w.sq, w.sk, s.Hq, s.Hkv, nqb, nkb, (int)s.d, P2, p.tau, p.theta,
+      w.qhat, w.khat, w.sq, w.sk, s.Hq, s.Hkv, nqb, nkb, (int)s.d, P2, G, p.tau, p.theta,
       make_rules(s, p), out.block_mask, w.counts, out.status);
   if ((e = check_launch("score_topcdf_kernel"))) return e;
   return launch_lists(s, p.bq, p.bk, w.counts, w.tmp, out, st);

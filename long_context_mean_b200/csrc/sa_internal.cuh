@@ -99,6 +99,7 @@ struct AttnArgs {
   const void* v;
   void* out;
   float* lse;
+  const int32_t* out_perm;  // nullptr = rows stored in place
   uint8_t* skip_log;
   const int32_t* row_ptr;   // nullptr = dense (every causally valid block)
   const int32_t* col_idx;

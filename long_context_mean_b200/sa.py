@@ -102,7 +102,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                       ctypes.POINTER(Mask), P]),
         "sa_attn_workspace": (SZ, []),
         "sa_block_sparse_attn": (I32, [P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F, F,
-                                       P, P, P, P, SZ, I32, P]),
+                                       P, P, P, P, P, SZ, I32, P]),
         "sa_dense_attn": (I32, [P, P, P, ctypes.POINTER(Shape), I32, F, P, P, P, P, SZ, I32, P]),
         "sa_read_status": (I32, [P, P]),
     }
@@ -233,10 +233,11 @@ def _default_attn_ws(device):
 
 
 def block_sparse_attn(q, k, v, shape: Shape, mask: Mask, lam, scale, out, lse=None, skip_log=None,
-                      flags=0, stream=None, ws=None):
+                      flags=0, stream=None, ws=None, out_perm=None):
     ws = ws if ws is not None else _default_attn_ws(q.device)
     _check(load().sa_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), ctypes.byref(mask),
-                                       float(lam), float(scale), _ptr(out), _ptr(lse), _ptr(skip_log),
+                                       float(lam), float(scale), _ptr(out), _ptr(lse), _ptr(out_perm),
+                                       _ptr(skip_log),
                                        _ptr(ws), ws.numel() * ws.element_size(), int(flags),
                                        _stream(stream)))
 
@@ -316,8 +317,6 @@ class Pipeline:
             self.qr = torch.empty(B, Hq, N, d, dtype=tdt, device=device)
             self.kr = torch.empty(B, Hkv, N, d, dtype=tdt, device=device)
             self.vr = torch.empty(B, Hkv, N, dv, dtype=tdt, device=device)
-            self.out_r = torch.empty(B, Hq, N, dv, dtype=tdt, device=device)
-            self.lse_r = torch.empty(B, Hq, N, 1, dtype=torch.float32, device=device)
         self.out = torch.empty(B, Hq, N, dv, dtype=tdt, device=device)
         self.lse = torch.empty(B, Hq, N, 1, dtype=torch.float32, device=device)
         self.ws = workspace(predict_mask_workspace(self.shape, params), device)
@@ -328,19 +327,19 @@ class Pipeline:
 
     def run(self, q, k, v, stream=None):
         if self.identity:
-            qr, kr, vr, out_r, lse_r = q, k, v, self.out, self.lse
+            qr, kr, vr = q, k, v
         else:
             layout_build(self.layout, self.perm, self.inv, self.layout_ws, stream)
             reorder(self.perm, q, self.qr, stream)
             reorder(self.perm, k, self.kr, stream)
             reorder(self.perm, v, self.vr, stream)
-            qr, kr, vr, out_r, lse_r = self.qr, self.kr, self.vr, self.out_r, self.lse_r
+            qr, kr, vr = self.qr, self.kr, self.vr
         predict_mask(qr, kr, self.shape, self.params, self.ws, self.mask.struct, stream)
-        block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, out_r, lse_r,
-                          self.skip_log, self.flags, stream, ws=self.attn_ws)
-        if not self.identity:
-            unreorder(self.perm, out_r, self.out, stream)
-            unreorder(self.perm, lse_r, self.lse, stream)
+        # The inverse reorder of O and LSE is fused into the attention store
+        # (out_perm); sa_unreorder stays available for standalone use.
+        block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, self.out, self.lse,
+                          self.skip_log, self.flags, stream, ws=self.attn_ws,
+                          out_perm=None if self.identity else self.perm)
         return self.out, self.lse
 
     def status(self, stream=None) -> int:

@@ -97,12 +97,12 @@ def test_host_validation_codes(lib):
     m2.bq, m2.bk, m2.nqb, m2.nkb = 128, 64, 3, 5
     WS = ctypes.c_void_p(1 << 20)
     assert lib.sa_block_sparse_attn(FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m2), ctypes.c_float(0.5),
-                                    ctypes.c_float(0), FAKE, null, null, WS, 256, 0, null) == sa.SA_ERR_INVALID_ARG
+                                    ctypes.c_float(0), FAKE, null, null, null, WS, 256, 0, null) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_block_sparse_attn(FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m2), ctypes.c_float(-1),
-                                    ctypes.c_float(0), FAKE, null, null, null, 0, 0, null) == sa.SA_ERR_WORKSPACE
+                                    ctypes.c_float(0), FAKE, null, null, null, null, 0, 0, null) == sa.SA_ERR_WORKSPACE
     m2.nqb = 4   # wrong for N=300, bq=128
     assert lib.sa_block_sparse_attn(FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m2), ctypes.c_float(-1),
-                                    ctypes.c_float(0), FAKE, null, null, WS, 256, 0, null) == sa.SA_ERR_INVALID_ARG
+                                    ctypes.c_float(0), FAKE, null, null, null, WS, 256, 0, null) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_dense_attn(FAKE, FAKE, FAKE, ctypes.byref(s), 2, ctypes.c_float(0), FAKE, null, null, WS, 256,
                              0, null) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_read_status(null, null) == sa.SA_ERR_INVALID_ARG
