@@ -510,6 +510,41 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
           if (key >= p.N || (p.causal && key > row_g)) s[jj] = -INFINITY;
         }
       }
+      // P = exp2(s * scale_log2 - ref), packed to bf16 pairs, and its row sum.
+      uint32_t pk[BK / 2];
+      float row_sum = 0.f;
+      auto compute_p = [&](float ref) {
+        // Pairs of columns on the packed fp32x2 pipe: x = s * scale - ref.
+        const uint64_t sc2 = pack2(sc, sc), neg2 = pack2(-ref, -ref);
+        uint64_t acc[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) acc[jj] = pack2(0.f, 0.f);
+#pragma unroll
+        for (int jj = 0; jj < BK; jj += 2) {
+          const uint64_t x = ffma2(pack2(s[jj], s[jj + 1]), sc2, neg2);
+          float p0, p1;
+          if (((jj >> 1) & 7) < kEmuPairs && !need_mask) {
+            exp2_fma_pair(x, p0, p1);          // FMA pipe, relieves the MUFU
+          } else {
+            float x0, x1;
+            unpack2(x, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          acc[(jj >> 1) & 3] = fadd2(acc[(jj >> 1) & 3], pack2(p0, p1));
+          pk[jj >> 1] = pack_bf16(p0, p1);
+        }
+        const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+        float lo, hi;
+        unpack2(a2, lo, hi);
+        row_sum = lo + hi;
+      };
+      // Speculate with the current reference maximum: P needs the tile's
+      // maximum only when that maximum exceeds the reference by more than
+      // the threshold (then P is recomputed below), so the exponentials and
+      // the max tree are independent work.
+      const bool spec = m_ref > -INFINITY;
+      if (spec) compute_p(m_ref);
       // Row max as a tree of 3-input maxima (independent chains), raw units.
       float mx[BK / 4];
 #pragma unroll
@@ -535,38 +570,11 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
         corr = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
         m_ref = m_new;
         resc = (t > 0);
-      }
-      // P = exp2(s * scale_log2 - m_ref), packed to bf16 pairs; row sum.
-      uint32_t pk[BK / 2];
-      float row_sum = 0.f;
-      if (m_ref > -INFINITY) {
-        // Pairs of columns on the packed fp32x2 pipe: x = s * scale - m_ref.
-        const uint64_t sc2 = pack2(sc, sc), neg2 = pack2(-m_ref, -m_ref);
-        uint64_t acc[4];
+        compute_p(m_ref);                       // the speculation missed
+      } else if (!spec) {
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) acc[jj] = pack2(0.f, 0.f);
-#pragma unroll
-        for (int jj = 0; jj < BK; jj += 2) {
-          const uint64_t x = ffma2(pack2(s[jj], s[jj + 1]), sc2, neg2);
-          float p0, p1;
-          if (((jj >> 1) & 7) < kEmuPairs && !need_mask) {
-            exp2_fma_pair(x, p0, p1);          // FMA pipe, relieves the MUFU
-          } else {
-            float x0, x1;
-            unpack2(x, x0, x1);
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
-          acc[(jj >> 1) & 3] = fadd2(acc[(jj >> 1) & 3], pack2(p0, p1));
-          pk[jj >> 1] = pack_bf16(p0, p1);
-        }
-        const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-        float lo, hi;
-        unpack2(a2, lo, hi);
-        row_sum = lo + hi;
-      } else {
-#pragma unroll
-        for (int jj = 0; jj < BK / 2; ++jj) pk[jj] = 0u;
+        for (int jj = 0; jj < BK / 2; ++jj) pk[jj] = 0u;   // every score so far masked
+        row_sum = 0.f;
       }
       l = l * corr + row_sum;
       // tcgen05.ld/st are warp-collective: a warp rescales when any of its
