@@ -220,6 +220,8 @@ __device__ void finish_row(const uint8_t* flags, int64_t u, int64_t qb, int64_t 
 // ---------------------------------------------------------------------------
 constexpr int kMaxRowsPerCta = 8;
 constexpr int kChunk = 32;
+constexpr int kFastKeys = 16;     // keys per lane on the fast TopCdf path (nkb <= 512)
+constexpr int kFastPicks = 128;   // picks before the fast path defers to the sort
 
 int score_rows_per_cta(int P2) {
   int g = 65536 / (P2 * 8);
@@ -339,7 +341,56 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
     float mx = -INFINITY;
     for (int64_t kb = lane; kb < nkb; kb += 32) mx = fmaxf(mx, srow[kb]);
     mx = warp_max(mx);
-    if (mx > -INFINITY) {
+    bool done = false;
+    if (mx > -INFINITY && P2 <= 32 * kFastKeys) {
+      // Fast path: repeated warp-wide arg-max over register-resident keys,
+      // accumulating the mass in sorted order; TopCdf usually stops after a
+      // few picks.  Gives up after kFastPicks picks (the sort below then
+      // decides the row from scratch).
+      uint64_t key[kFastKeys];
+      float part = 0.f;
+#pragma unroll
+      for (int q = 0; q < kFastKeys; ++q) {
+        const int kb = lane + 32 * q;
+        key[q] = 0ull;
+        if (kb < nkb) {
+          const float sv = srow[kb];
+          const float pv = (sv == -INFINITY) ? 0.f : expf(sv - mx);
+          key[q] = ((uint64_t)__float_as_uint(pv) << 32) | (uint32_t)(~(uint32_t)kb);
+          part += pv;
+        }
+      }
+      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      const float limit = tau * part;
+      float cum = 0.f;
+      for (int pick = 0; pick < kFastPicks; ++pick) {
+        uint64_t best = 0ull;
+#pragma unroll
+        for (int q = 0; q < kFastKeys; ++q) best = key[q] > best ? key[q] : best;
+        for (int off = 16; off > 0; off >>= 1) {
+          const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
+          best = o > best ? o : best;
+        }
+        const float pv = __uint_as_float((uint32_t)(best >> 32));
+        if (!(pv > 0.f) || !(cum < limit)) {
+          done = true;
+          break;
+        }
+        const uint32_t kb = ~(uint32_t)best;
+        if ((int)(kb & 31) == lane) {
+          fl[kb] = 1;
+#pragma unroll
+          for (int q = 0; q < kFastKeys; ++q)        // static indices keep key[] in registers
+            if (q == (int)(kb >> 5)) key[q] = 0ull;
+        }
+        cum += pv;
+      }
+      if (!done) {
+        for (int64_t kb = lane; kb < nkb; kb += 32) fl[kb] = 0;
+      }
+      __syncwarp();
+    }
+    if (mx > -INFINITY && !done) {
       for (int kb = lane; kb < P2; kb += 32) {
         uint64_t key = 0ull;
         if (kb < nkb) {

@@ -103,3 +103,58 @@ def test_full_size_pipeline_sampled(name):
     for b, h in heads:
         sel[b, h] = rows_orig
     oracle_check(w, g, pipe, out, lse, heads, qblocks)
+
+
+def _sampled_heads_check(w, heads, kv_of, qblocks):
+    """Full-size run of the whole path; the oracle recomputes the mask and the
+    attention for the listed (b, h) heads and q-blocks only."""
+    import torch
+    from long_context_mean_b200 import sa
+    g = I.gen_qkv(w)
+    q, k, v = P.qkv_dev(g, w.dtype)
+    pipe = sa.pipeline_for(w, log_skips=True)
+    out, lse = pipe.run(q, k, v)
+    assert pipe.status() == 0
+    out_h = out.float().cpu().numpy()
+    lse_h = lse.cpu().numpy()[..., 0]
+    perm, _ = Y.build_layout(w.order, w.T, w.H, w.W, w.win, w.sink_frames, w.txt_len)
+    nqb, nkb = pipe.mask.struct.nqb, pipe.mask.struct.nkb
+    gmask = pipe.mask.block_mask.cpu().numpy().reshape(w.B, w.Hq, nqb, nkb).astype(bool)
+    rp = pipe.mask.row_ptr.cpu().numpy()
+    ci = pipe.mask.col_idx.cpu().numpy()
+    skip = pipe.skip_log.cpu().numpy()
+    for b, h in heads:
+        g_h = kv_of(h)
+        qh = Y.reorder(g["q"][b:b + 1, h:h + 1], perm)
+        kh = Y.reorder(g["k"][b:b + 1, g_h:g_h + 1], perm)
+        vh = Y.reorder(g["v"][b:b + 1, g_h:g_h + 1], perm)
+        orc = Pr.predict_mask(qh, kh, w.bq, w.bk, w.tau, w.theta, w.causal, w.sink_tokens, w.txt_len,
+                              w.local_window, w.anchor_tokens)
+        P.compare_masks(gmask[b:b + 1, h:h + 1], orc, w.tau, w.theta, 1)
+        m = gmask[b:b + 1, h:h + 1]
+        ref = A.block_sparse_attention_heads(qh, kh, vh, m, w.bq, w.bk, w.causal, w.lam, qblocks=qblocks)
+        if w.lam > -math.inf:
+            over = {}
+            base = (b * w.Hq + h) * nqb
+            for qb in qblocks:
+                u = base + qb
+                for t in range(rp[u], rp[u + 1]):
+                    over[(0, 0, qb, int(ci[t]))] = bool(skip[t])
+            if P.check_skip_decisions(over, ref["skips"], ref["gaps"], w.lam):
+                ref = A.block_sparse_attention_heads(qh, kh, vh, m, w.bq, w.bk, w.causal, w.lam, qblocks=qblocks,
+                                                     skip_override=over, band=P.LAMBDA_BAND)
+        ref_out = Y.unreorder(ref["out"], perm, axis=2)
+        ref_lse = Y.unreorder(ref["lse"], perm, axis=2)
+        P.attention_check(out_h[b:b + 1, h:h + 1], lse_h[b:b + 1, h:h + 1], {"out": ref_out, "lse": ref_lse})
+
+
+def test_video_large_hilbert_sampled():
+    w = I.WORKLOADS["video_large"]
+    nqb = -(-w.N // w.bq)
+    _sampled_heads_check(w, [(0, 0), (0, 23)], lambda h: h, [0, 300, nqb - 1])
+
+
+def test_lm_causal_gqa_sampled():
+    w = I.WORKLOADS["lm_causal"]
+    nqb = -(-w.N // w.bq)
+    _sampled_heads_check(w, [(0, 0), (0, 29)], lambda h: h // (w.Hq // w.Hkv), [0, 1, 40, 513, nqb - 1])
