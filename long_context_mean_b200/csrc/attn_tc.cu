@@ -15,13 +15,13 @@
 //   * per pipeline, warp p (one lane) is the TMA producer (Q tile once per
 //     unit, K and V tiles of the kept key blocks through a STAGES ring) and
 //     warp 2+p (one lane) issues tcgen05.mma: S = Q K^T into one of two TMEM
-//     S buffers and O += P V into the TMEM O accumulator.
-//       bk = 64:  the softmax releases an S buffer as soon as it has loaded
-//                 it and writes P (bf16) to a shared-memory buffer in the
-//                 128-byte-swizzled K-major layout, so S runs two tiles
-//                 ahead of PV (S(t+2) and PV(t) overlap the softmax of t+1);
-//       bk = 128: P overwrites S in TMEM and PV reads it from there, S runs
-//                 one tile ahead.
+//     S buffers and O += P V into the TMEM O accumulator.  The softmax
+//     writes P (bf16 pairs) over its S buffer in TMEM and the PV product
+//     reads it from there (TS form), so S runs one tile ahead of PV: S(t+1)
+//     overlaps the softmax of t, and PV(t) the softmax of t+1.  A variant
+//     with P in a 128-byte-swizzled shared-memory buffer (SS form, S two
+//     tiles ahead) is kept behind Cfg::P_SMEM; on B200 it measured slower
+//     at both block sizes.
 //   * per pipeline, four softmax warps (one thread per query row = TMEM
 //     lane): S from TMEM, masks, running max, exp2 (scale folded into one
 //     packed fp32x2 FMA), P, O rescale in TMEM when the reference maximum

@@ -9,7 +9,7 @@ position n to the source index it takes (y[n] = x[perm[n]]); ``inv`` is its
 inverse (x[i] = y[inv[i]]), the "inverse reorder" of [P1] section 3.4 and
 [P3] section 2.5.
 
-Readings (the pages are silent on these; each is listed in the design doc):
+Readings (the pages are silent on these):
 * The first ``sink_frames`` frames (the first-frame sink of [P2]) stay at the
   front in raster order and are not reordered; text tokens stay last and are
   not reordered ([P3] section 2.5 permutes visual tokens only; [P1] section 5

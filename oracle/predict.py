@@ -21,7 +21,7 @@ Pipeline ([P3] section 2.2, with [P2] rf_v2 / ada_bsa and [P5] anchors):
   6. CSR lists (column indices ascending) and a work order (rows by
      descending kept count, ties by ascending row index).
 
-Readings where the pages are silent or garbled (all listed in the design doc):
+Readings where the pages are silent or garbled:
   * CosSim: the notes print mean(X X^T / |max(X X^T)|) while naming it a
     cosine similarity; the standard mean pairwise cosine (x_hat = x/|x|,
     zero vectors contribute 0) is used.  ``cossim_literal`` keeps the printed
