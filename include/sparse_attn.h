@@ -187,6 +187,24 @@ sa_status sa_predict_mask(const void* q, const void* k, const sa_shape* shape,
                           const sa_mask_params* params, void* ws, size_t ws_bytes,
                           sa_mask* out, void* stream);
 
+/* sa_predict_mask without a caller workspace.  The pages describe no such
+ * call: it exists for callers that cannot allocate device memory at all (code
+ * running inside another runtime's memory pool without access to it, a
+ * plug-in handed only pre-sized inputs and outputs, a serving process whose
+ * device footprint must not grow).  The scratch comes from a 32 MiB array
+ * that the library itself holds on each device for the life of the process;
+ * the function allocates nothing.  Shapes whose sa_predict_mask_workspace()
+ * exceeds 32 MiB are rejected with SA_ERR_WORKSPACE (the largest shipped
+ * workload needs about 25 MiB).  Arguments and results are those of
+ * sa_predict_mask.  Every call shares the one array; each call writes every
+ * scratch value before reading it, so it needs no clearing, but calls that
+ * overlap on the GPU (other streams, other threads) race on it and must be
+ * serialised by the caller.  The first call on a device (with that device
+ * current) looks up the array's address; make it before any stream capture
+ * begins on that device. */
+sa_status sa_predict_mask_noalloc(const void* q, const void* k, const sa_shape* shape,
+                                  const sa_mask_params* params, sa_mask* out, void* stream);
+
 /* A caller-supplied block mask (uint8 [B*Hq, nqb, nkb], nonzero = kept) is
  * ANDed with causal validity, copied to out->block_mask (may alias), checked
  * for empty rows and compacted into lists exactly as sa_predict_mask does. */

@@ -32,7 +32,8 @@ STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3:
 
 EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_attn_workspace", "sa_layout_workspace",
            "sa_layout_build", "sa_reorder", "sa_unreorder", "sa_predict_mask_workspace",
-           "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_mask_from_blocks_workspace",
+           "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_predict_mask_noalloc",
+           "sa_mask_from_blocks_workspace",
            "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status"]
 
 
@@ -97,6 +98,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                             ctypes.POINTER(SZ * 6)]),
         "sa_predict_mask": (I32, [P, P, ctypes.POINTER(Shape), ctypes.POINTER(MaskParams), P, SZ,
                                   ctypes.POINTER(Mask), P]),
+        "sa_predict_mask_noalloc": (I32, [P, P, ctypes.POINTER(Shape), ctypes.POINTER(MaskParams),
+                                          ctypes.POINTER(Mask), P]),
         "sa_mask_from_blocks_workspace": (SZ, [ctypes.POINTER(Shape), I32, I32]),
         "sa_mask_from_blocks": (I32, [P, ctypes.POINTER(Shape), I32, I32, I32, P, SZ,
                                       ctypes.POINTER(Mask), P]),
@@ -203,6 +206,12 @@ def predict_mask_ws_layout(shape: Shape, params: MaskParams):
 def predict_mask(q, k, shape: Shape, params: MaskParams, ws, mask: Mask, stream=None):
     _check(load().sa_predict_mask(_ptr(q), _ptr(k), ctypes.byref(shape), ctypes.byref(params), _ptr(ws),
                                   ws.numel() * ws.element_size(), ctypes.byref(mask), _stream(stream)))
+
+
+def predict_mask_noalloc(q, k, shape: Shape, params: MaskParams, mask: Mask, stream=None):
+    """sa_predict_mask with the library's own fixed scratch array (no workspace argument)."""
+    _check(load().sa_predict_mask_noalloc(_ptr(q), _ptr(k), ctypes.byref(shape), ctypes.byref(params),
+                                          ctypes.byref(mask), _stream(stream)))
 
 
 def mask_from_blocks_workspace(shape: Shape, bq: int, bk: int) -> int:
