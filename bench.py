@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch of the attention kernel from the ncu capture recorded
 # in profiles/attn_tc_video.md, keyed by the sha1 of the kernel code it was
 # taken on (src_sha1); any other code reports null.
-TRAFFIC = {("049cb25953c5c46ea500db3d5126554696a40c4f", "video"): 1.219e9}
+TRAFFIC = {("b5b6ef460c7c7391887a0a133378e43162267090", "video"): 1.216e9}
 
 
 def peaks():
@@ -228,13 +228,14 @@ def run_ours(args, rank, world, local_rank):
         e[0].record(stream)
         if not pipe.identity:
             sa.layout_build(pipe.layout, pipe.perm, pipe.inv, pipe.layout_ws)
-            sa.reorder(pipe.perm, q, pipe.qr)
-            sa.reorder(pipe.perm, k, pipe.kr)
+            # mask prediction with the reorder of Q and K fused into its pooling pass
+            sa.reorder_predict_mask(pipe.perm, q, k, pipe.qr, pipe.kr, pipe.shape, pipe.params, pipe.ws,
+                                    pipe.mask.struct)
             sa.reorder(pipe.perm, v, pipe.vr)
             qr, kr, vr = pipe.qr, pipe.kr, pipe.vr
         else:
             qr, kr, vr = q, k, v
-        sa.predict_mask(qr, kr, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
+            sa.predict_mask(qr, kr, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
         e[1].record(stream)
         # attention with the inverse reorder of O and LSE fused into its store
         sa.block_sparse_attn(qr, kr, vr, pipe.shape, pipe.mask.struct, pipe.lam, pipe.scale, pipe.out, pipe.lse,
@@ -242,7 +243,8 @@ def run_ours(args, rank, world, local_rank):
         e[2].record(stream)
         return e
 
-    launches_per_step = (0 if pipe.identity else (1 if w.order != "hilbert" else 3) + 3) + 6 + 1
+    # layout (1, Hilbert 3) + reorder V; pool Q, pool K, score, row scan, column fill, order; attention
+    launches_per_step = (0 if pipe.identity else (1 if w.order != "hilbert" else 3) + 1) + 6 + 1
 
     for _ in range(args.warmup):
         l2_flush()

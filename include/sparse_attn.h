@@ -187,6 +187,22 @@ sa_status sa_predict_mask(const void* q, const void* k, const sa_shape* shape,
                           const sa_mask_params* params, void* ws, size_t ws_bytes,
                           sa_mask* out, void* stream);
 
+/* ---- a1 + a2-a4 fused: reorder Q and K while pooling them ([P1] 3.4,
+ * [P3] 2.2) ------------------------------------------------------------------
+ * sa_predict_mask on the permuted sequence, for q and k given in the
+ * original token order: the pooling pass reads token n of the permuted
+ * order from row perm[n] of q and k and also writes it to row n of q_r and
+ * k_r (q_r[o, n, :] = q[o, perm[n], :], as sa_reorder), so Q and K cross HBM
+ * once for both steps.  perm: int32 [N], a permutation of [0, N) (an entry
+ * outside that range raises SA_ERR_INVALID_ARG in the status word and the
+ * token is skipped).  q_r, k_r: device buffers of the shapes of q and k,
+ * 16-byte aligned, overlapping neither q, k nor each other.  Workspace, the
+ * other arguments and the results are those of sa_predict_mask (the mask
+ * describes the permuted sequence). */
+sa_status sa_reorder_predict_mask(const int32_t* perm, const void* q, const void* k, void* q_r, void* k_r,
+                                  const sa_shape* shape, const sa_mask_params* params, void* ws,
+                                  size_t ws_bytes, sa_mask* out, void* stream);
+
 /* sa_predict_mask without a caller workspace.  The pages describe no such
  * call: it exists for callers that cannot allocate device memory at all (code
  * running inside another runtime's memory pool without access to it, a

@@ -167,11 +167,13 @@ sa_status sa_predict_mask_ws_layout(const sa_shape* shape, const sa_mask_params*
   return SA_OK;
 }
 
-sa_status sa_predict_mask(const void* q, const void* k, const sa_shape* shape,
-                          const sa_mask_params* params, void* ws, size_t ws_bytes, sa_mask* out,
-                          void* stream) {
+namespace {
+// Validation shared by the two prediction entry points; fills the mask's
+// geometry and the workspace carve-up.
+sa_status predict_prepare(const char* who, const void* q, const void* k, const sa_shape* shape,
+                          const sa_mask_params* params, void* ws, size_t ws_bytes, sa_mask* out) {
   if (sa_status e = check_shape(shape)) return e;
-  if (!q || !k || !params) return set_error(SA_ERR_INVALID_ARG, "NULL argument to sa_predict_mask");
+  if (!q || !k || !params) return set_error(SA_ERR_INVALID_ARG, "NULL argument to %s", who);
   const sa_mask_params& p = *params;
   if (sa_status e = check_blocks(p.bq, p.bk, shape->N)) return e;
   if (sa_status e = check_predict_dims(shape)) return e;
@@ -185,15 +187,46 @@ sa_status sa_predict_mask(const void* q, const void* k, const sa_shape* shape,
   size_t off[6];
   const size_t need = predict_ws_bytes(*shape, p.bq, p.bk, off);
   if (!ws || ws_bytes < need || (uintptr_t)ws % 256)
-    return set_error(SA_ERR_WORKSPACE, "sa_predict_mask needs %zu bytes of 256-byte aligned workspace", need);
+    return set_error(SA_ERR_WORKSPACE, "%s needs %zu bytes of 256-byte aligned workspace", who, need);
   if (sa_status e = check_device()) return e;
   out->nqb = ceil_div(shape->N, p.bq);
   out->nkb = ceil_div(shape->N, p.bk);
   out->bq = p.bq;
   out->bk = p.bk;
   out->causal = p.causal;
-  return launch_predict(q, k, *shape, p, predict_ws_carve(ws, *shape, p.bq, p.bk), *out,
+  return SA_OK;
+}
+
+bool overlaps(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+  return x < y + bytes && y < x + bytes;
+}
+}  // namespace
+
+sa_status sa_predict_mask(const void* q, const void* k, const sa_shape* shape,
+                          const sa_mask_params* params, void* ws, size_t ws_bytes, sa_mask* out,
+                          void* stream) {
+  if (sa_status e = predict_prepare("sa_predict_mask", q, k, shape, params, ws, ws_bytes, out)) return e;
+  return launch_predict(q, k, *shape, *params, predict_ws_carve(ws, *shape, params->bq, params->bk), *out,
                         static_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_reorder_predict_mask(const int32_t* perm, const void* q, const void* k, void* q_r, void* k_r,
+                                  const sa_shape* shape, const sa_mask_params* params, void* ws,
+                                  size_t ws_bytes, sa_mask* out, void* stream) {
+  if (sa_status e = check_shape(shape)) return e;
+  if (!perm || !q_r || !k_r) return set_error(SA_ERR_INVALID_ARG, "NULL perm, q_r or k_r");
+  if ((uintptr_t)q_r % 16 || (uintptr_t)k_r % 16)
+    return set_error(SA_ERR_INVALID_ARG, "q_r and k_r must be 16-byte aligned");
+  const size_t esz = shape->dtype == SA_BF16 ? 2 : 4;
+  const size_t qbytes = (size_t)(shape->B * shape->Hq * shape->N * shape->d) * esz;
+  const size_t kbytes = (size_t)(shape->B * shape->Hkv * shape->N * shape->d) * esz;
+  if (overlaps(q, q_r, qbytes) || overlaps(k, k_r, kbytes) || overlaps(q_r, k_r, qbytes < kbytes ? qbytes : kbytes) ||
+      overlaps(q, k_r, qbytes < kbytes ? qbytes : kbytes) || overlaps(k, q_r, qbytes < kbytes ? qbytes : kbytes))
+    return set_error(SA_ERR_INVALID_ARG, "q_r and k_r must not overlap q, k or each other");
+  if (sa_status e = predict_prepare("sa_reorder_predict_mask", q, k, shape, params, ws, ws_bytes, out)) return e;
+  return launch_predict(q, k, *shape, *params, predict_ws_carve(ws, *shape, params->bq, params->bk), *out,
+                        static_cast<cudaStream_t>(stream), perm, q_r, k_r);
 }
 
 size_t sa_mask_from_blocks_workspace(const sa_shape* shape, int32_t bq, int32_t bk) {

@@ -27,11 +27,14 @@ constexpr int kPoolWarps = kPoolThreads / 32;
 // a2: one CTA per (head, block): block mean and mean pairwise cosine.  A warp
 // covers 32/chunks tokens per step (chunks = 16-byte pieces of a token),
 // four steps in flight; token norms reduce inside each token's lane group.
+// With perm, token n of the block is read from row perm[n] of x and also
+// written to row n of y (a1 fused with a2: the reordered copy is produced by
+// the same pass that pools it).
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
     const T* __restrict__ x, int64_t N, int d, int b, int nB, float* __restrict__ mean_out,
-    float* __restrict__ s_out) {
+    float* __restrict__ s_out, const int32_t* __restrict__ perm, T* __restrict__ y, int32_t* status) {
   constexpr int EPL = 16 / sizeof(T);
   const int blk = blockIdx.x;
   const int64_t bh = blockIdx.y;
@@ -44,7 +47,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
   float ax[EPL], au[EPL];
 #pragma unroll
   for (int e = 0; e < EPL; ++e) ax[e] = au[e] = 0.f;
-  const uint4* base = reinterpret_cast<const uint4*>(x + (bh * N + t0) * (int64_t)d);
+  const uint4* xbh = reinterpret_cast<const uint4*>(x + bh * N * (int64_t)d);
+  uint4* ybh = y ? reinterpret_cast<uint4*>(y + bh * N * (int64_t)d) : nullptr;
   const int step = kPoolWarps * tpw;
   constexpr int kInFlight = 4;
   for (int tb = warp * tpw; tb < cnt; tb += kInFlight * step) {
@@ -53,8 +57,18 @@ __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
 #pragma unroll
     for (int u = 0; u < kInFlight; ++u) {
       const int tok = tb + u * step + sub;
+      const int64_t n = t0 + tok;
       ok[u] = tok < cnt;
-      raw[u] = ok[u] ? __ldg(base + (int64_t)tok * chunks + c) : make_uint4(0, 0, 0, 0);
+      int64_t src = n;
+      if (perm && ok[u]) {
+        src = __ldg(perm + n);
+        if ((uint64_t)src >= (uint64_t)N) {   // not a permutation of [0, N)
+          raise_status(status, SA_ERR_INVALID_ARG);
+          ok[u] = false;
+        }
+      }
+      raw[u] = ok[u] ? __ldg(xbh + src * chunks + c) : make_uint4(0, 0, 0, 0);
+      if (ybh && ok[u]) __stcs(ybh + n * chunks + c, raw[u]);
     }
 #pragma unroll
     for (int u = 0; u < kInFlight; ++u) {
@@ -230,7 +244,7 @@ int score_rows_per_cta(int P2) {
 
 size_t score_smem_bytes(int d, int64_t nkb, int P2, int G) {
   const size_t nkb16 = (size_t)((nkb + 15) / 16) * 16;
-  return (size_t)kMaxRowsPerCta * d * 4 + (size_t)kChunk * (d + 1) * 4 + (size_t)G * nkb * 4 +
+  return (size_t)kMaxRowsPerCta * d * 4 + (size_t)kChunk * (d + 4) * 4 + (size_t)G * nkb * 4 +
          (size_t)G * P2 * 8 + (size_t)G * nkb16;
 }
 
@@ -248,8 +262,10 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   const int nkb16 = (int)((nkb + 15) / 16) * 16;
   float* qs = reinterpret_cast<float*>(smem);
   float* ks = qs + kMaxRowsPerCta * d;
-  float* sc = ks + kChunk * (d + 1);
-  // 8-byte aligned: the float offset 8d + 32(d+1) + G nkb is even (G even
+  // k_hat rows padded to d + 4 floats: 16-byte aligned for float4 reads,
+  // and the 8 rows a quarter-warp reads land in distinct bank groups.
+  float* sc = ks + kChunk * (d + 4);
+  // 8-byte aligned: the float offset 8d + 32(d+4) + G nkb is even (G even
   // or nkb even; see score_rows_per_cta).
   uint64_t* keys = reinterpret_cast<uint64_t*>(sc + G * nkb);
   uint8_t* flags = reinterpret_cast<uint8_t*>(keys + (size_t)G * P2);
@@ -297,11 +313,7 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
       for (int q = 0; q < kPer; ++q) {
         const int i = threadIdx.x + q * kRowThreads;
         if (i < cn * nf4) {
-          float* dst = ks + (i / nf4) * (d + 1) + (i % nf4) * 4;
-          dst[0] = buf[q].x;
-          dst[1] = buf[q].y;
-          dst[2] = buf[q].z;
-          dst[3] = buf[q].w;
+          *reinterpret_cast<float4*>(ks + (i / nf4) * (d + 4) + (i % nf4) * 4) = buf[q];
         }
       }
       __syncthreads();
@@ -310,14 +322,15 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
       if (r < rows && j < cn) {
         float s = -INFINITY;
         if (!s_forced[r] && rules.valid(qb0 + r, kb) && !(guard && sk[g * nkb + kb] < theta)) {
-          const float* qr = qs + r * d;
-          const float* kr = ks + j * (d + 1);
+          const float4* qr = reinterpret_cast<const float4*>(qs + r * d);
+          const float4* kr = reinterpret_cast<const float4*>(ks + j * (d + 4));
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-          for (int e = 0; e < d; e += 4) {
-            a0 = fmaf(qr[e], kr[e], a0);
-            a1 = fmaf(qr[e + 1], kr[e + 1], a1);
-            a2 = fmaf(qr[e + 2], kr[e + 2], a2);
-            a3 = fmaf(qr[e + 3], kr[e + 3], a3);
+          for (int e = 0; e < d / 4; ++e) {
+            const float4 x = qr[e], y = kr[e];
+            a0 = fmaf(x.x, y.x, a0);
+            a1 = fmaf(x.y, y.y, a1);
+            a2 = fmaf(x.z, y.z, a2);
+            a3 = fmaf(x.w, y.w, a3);
           }
           s = ((a0 + a1) + (a2 + a3)) * scale;
         }
@@ -620,10 +633,10 @@ RowRules make_rules(const sa_shape& s, const sa_mask_params& p) {
 
 template <typename T>
 sa_status launch_pool(const void* x, int64_t BH, int64_t N, int d, int b, int64_t nB, float* mean,
-                      float* sim, cudaStream_t st) {
+                      float* sim, const int32_t* perm, void* y, int32_t* status, cudaStream_t st) {
   dim3 grid((unsigned)nB, (unsigned)BH);
   pool_cossim_kernel<T><<<grid, kPoolThreads, 0, st>>>(static_cast<const T*>(x), N, d, b, (int)nB,
-                                                       mean, sim);
+                                                       mean, sim, perm, static_cast<T*>(y), status);
   return check_launch("pool_cossim_kernel");
 }
 
@@ -664,17 +677,25 @@ size_t lists_ws_bytes(const sa_shape& s, int bq, int) {
 
 sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
                          const sa_mask_params& p, const PredictWs& w, sa_mask& out,
-                         cudaStream_t st) {
+                         cudaStream_t st, const int32_t* perm, void* q_r, void* k_r) {
   const int64_t nqb = out.nqb, nkb = out.nkb;
   if (cudaMemsetAsync(out.status, 0, sizeof(int32_t), st) != cudaSuccess)
     return set_error(SA_ERR_CUDA, "cudaMemsetAsync(status) failed");
   sa_status e;
   if (s.dtype == SA_BF16) {
-    if ((e = launch_pool<uint16_t>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, st))) return e;
-    if ((e = launch_pool<uint16_t>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, w.sk, st))) return e;
+    if ((e = launch_pool<uint16_t>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, perm, q_r,
+                                   out.status, st)))
+      return e;
+    if ((e = launch_pool<uint16_t>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, w.sk, perm, k_r,
+                                   out.status, st)))
+      return e;
   } else {
-    if ((e = launch_pool<float>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, st))) return e;
-    if ((e = launch_pool<float>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, w.sk, st))) return e;
+    if ((e = launch_pool<float>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, perm, q_r,
+                                out.status, st)))
+      return e;
+    if ((e = launch_pool<float>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, w.sk, perm, k_r,
+                                out.status, st)))
+      return e;
   }
   int P2 = 1;
   while (P2 < nkb) P2 <<= 1;

@@ -86,9 +86,12 @@ size_t predict_ws_bytes(const sa_shape& s, int bq, int bk, size_t offsets[6]);
 PredictWs predict_ws_carve(void* ws, const sa_shape& s, int bq, int bk);
 size_t lists_ws_bytes(const sa_shape& s, int bq, int bk);
 
+// With perm (nullable), q and k are in the original token order: the pooling
+// pass reads row perm[n] for token n and writes the reordered copies q_r, k_r.
 sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
                          const sa_mask_params& p, const PredictWs& w, sa_mask& out,
-                         cudaStream_t st);
+                         cudaStream_t st, const int32_t* perm = nullptr, void* q_r = nullptr,
+                         void* k_r = nullptr);
 sa_status launch_mask_from_blocks(const uint8_t* in, const sa_shape& s, int bq, int bk,
                                   int causal, int32_t* counts, int32_t* tmp, sa_mask& out,
                                   cudaStream_t st);

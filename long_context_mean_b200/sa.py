@@ -32,7 +32,7 @@ STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3:
 
 EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_attn_workspace", "sa_layout_workspace",
            "sa_layout_build", "sa_reorder", "sa_unreorder", "sa_predict_mask_workspace",
-           "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_predict_mask_noalloc",
+           "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_reorder_predict_mask", "sa_predict_mask_noalloc",
            "sa_mask_from_blocks_workspace",
            "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status"]
 
@@ -98,6 +98,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                             ctypes.POINTER(SZ * 6)]),
         "sa_predict_mask": (I32, [P, P, ctypes.POINTER(Shape), ctypes.POINTER(MaskParams), P, SZ,
                                   ctypes.POINTER(Mask), P]),
+        "sa_reorder_predict_mask": (I32, [P, P, P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(MaskParams), P,
+                                          SZ, ctypes.POINTER(Mask), P]),
         "sa_predict_mask_noalloc": (I32, [P, P, ctypes.POINTER(Shape), ctypes.POINTER(MaskParams),
                                           ctypes.POINTER(Mask), P]),
         "sa_mask_from_blocks_workspace": (SZ, [ctypes.POINTER(Shape), I32, I32]),
@@ -208,6 +210,14 @@ def predict_mask(q, k, shape: Shape, params: MaskParams, ws, mask: Mask, stream=
                                   ws.numel() * ws.element_size(), ctypes.byref(mask), _stream(stream)))
 
 
+def reorder_predict_mask(perm, q, k, q_r, k_r, shape: Shape, params: MaskParams, ws, mask: Mask, stream=None):
+    """Mask prediction on the permuted sequence with q, k in the original order;
+    writes the reordered copies q_r, k_r in the same pass."""
+    _check(load().sa_reorder_predict_mask(_ptr(perm), _ptr(q), _ptr(k), _ptr(q_r), _ptr(k_r), ctypes.byref(shape),
+                                          ctypes.byref(params), _ptr(ws), ws.numel() * ws.element_size(),
+                                          ctypes.byref(mask), _stream(stream)))
+
+
 def predict_mask_noalloc(q, k, shape: Shape, params: MaskParams, mask: Mask, stream=None):
     """sa_predict_mask with the library's own fixed scratch array (no workspace argument)."""
     _check(load().sa_predict_mask_noalloc(_ptr(q), _ptr(k), ctypes.byref(shape), ctypes.byref(params),
@@ -306,9 +316,10 @@ class Pipeline:
 
     Allocates (through torch) the layout, reordered copies, workspace, mask
     lists and outputs once; ``run(q, k, v)`` then enqueues, on the current
-    stream: layout build, reorder of Q, K, V, mask prediction, block-sparse
-    attention and inverse reorder of O and LSE.  Inputs are BNSD in the
-    original token order; ``out``/``lse`` come back in that order too.
+    stream: layout build, mask prediction fused with the reorder of Q and K,
+    reorder of V, block-sparse attention with the inverse reorder of O and
+    LSE fused into its store.  Inputs are BNSD in the original token order;
+    ``out``/``lse`` come back in that order too.
     """
 
     def __init__(self, B, Hq, Hkv, N, d, dv, dtype, *, layout: LayoutDesc, params: MaskParams,
@@ -337,13 +348,14 @@ class Pipeline:
     def run(self, q, k, v, stream=None):
         if self.identity:
             qr, kr, vr = q, k, v
+            predict_mask(qr, kr, self.shape, self.params, self.ws, self.mask.struct, stream)
         else:
             layout_build(self.layout, self.perm, self.inv, self.layout_ws, stream)
-            reorder(self.perm, q, self.qr, stream)
-            reorder(self.perm, k, self.kr, stream)
+            # Q and K are reordered by the pooling pass of the prediction.
+            reorder_predict_mask(self.perm, q, k, self.qr, self.kr, self.shape, self.params, self.ws,
+                                 self.mask.struct, stream)
             reorder(self.perm, v, self.vr, stream)
             qr, kr, vr = self.qr, self.kr, self.vr
-        predict_mask(qr, kr, self.shape, self.params, self.ws, self.mask.struct, stream)
         # The inverse reorder of O and LSE is fused into the attention store
         # (out_perm); sa_unreorder stays available for standalone use.
         block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, self.out, self.lse,

@@ -92,6 +92,12 @@ def test_host_validation_codes(lib):
     s_g = _shape(Hq=3, Hkv=2)
     assert lib.sa_predict_mask(FAKE, FAKE, ctypes.byref(s_g), ctypes.byref(p), FAKE, 1 << 30,
                                ctypes.byref(m), null) == sa.SA_ERR_INVALID_ARG
+    # fused reorder + predict: perm and the copies must be given and must not overlap the inputs
+    QR, KR = ctypes.c_void_p(1 << 30), ctypes.c_void_p(1 << 31)
+    assert lib.sa_reorder_predict_mask(null, FAKE, FAKE, QR, KR, ctypes.byref(s), ctypes.byref(p), FAKE, 1 << 30,
+                                       ctypes.byref(m), null) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_reorder_predict_mask(FAKE, FAKE, ctypes.c_void_p(1 << 20), FAKE, KR, ctypes.byref(s),
+                                       ctypes.byref(p), FAKE, 1 << 30, ctypes.byref(m), null) == sa.SA_ERR_INVALID_ARG
     # attention
     m2 = _mask()
     m2.bq, m2.bk, m2.nqb, m2.nkb = 128, 64, 3, 5

@@ -189,3 +189,71 @@ def test_mask_from_blocks_lists_and_causal_and():
     assert np.array_equal(mb.row_ptr.cpu().numpy(), c["row_ptr"])
     assert np.array_equal(mb.col_idx.cpu().numpy()[:c["kept_total"]], c["col_idx"])
     assert np.array_equal(mb.order.cpu().numpy(), c["order"])
+
+
+def _fused_vs_separate(w, perm_np, q_bits, k_bits):
+    """sa_reorder_predict_mask on original-order inputs against the oracle's
+    reorder (bit-exact copies) and sa_predict_mask on those copies (same
+    pooled values, mask, lists and order)."""
+    import torch
+    from long_context_mean_b200 import sa
+    q_dev, k_dev = P.bf16_dev(q_bits), P.bf16_dev(k_bits)
+    qr_want, kr_want = Y.reorder(q_bits, perm_np), Y.reorder(k_bits, perm_np)
+    prm = sa.make_params(w.bq, w.bk, w.tau, w.theta, w.sink_tokens, w.txt_len, w.local_window,
+                         w.anchor_tokens, w.causal)
+    shape = sa.Shape(q_dev.shape[0], q_dev.shape[1], k_dev.shape[1], q_dev.shape[2], q_dev.shape[3],
+                     q_dev.shape[3], sa.SA_BF16, 0)
+    perm = torch.from_numpy(perm_np.astype(np.int32)).to("cuda")
+    q_r = torch.full_like(q_dev, float("nan"))
+    k_r = torch.full_like(k_dev, float("nan"))
+    ws = sa.workspace(sa.predict_mask_workspace(shape, prm), "cuda")
+    ws.fill_(0xFF)
+    mb = sa.MaskBuffers.allocate(shape.B, shape.Hq, shape.N, prm.bq, prm.bk, "cuda")
+    sa.reorder_predict_mask(perm, q_dev, k_dev, q_r, k_r, shape, prm, ws, mb.struct)
+    assert sa.read_status(mb.status) == sa.SA_OK
+    assert np.array_equal(q_r.cpu().view(torch.int16).numpy().view(np.uint16), qr_want)
+    assert np.array_equal(k_r.cpu().view(torch.int16).numpy().view(np.uint16), kr_want)
+    ref = run_gpu_predict(P.bf16_dev(qr_want), P.bf16_dev(kr_want), w, prm)
+    off = sa.predict_mask_ws_layout(shape, prm)
+    for i, key in ((0, "qhat"), (1, "khat"), (2, "s_q"), (3, "s_k")):
+        n = ref[key].size
+        got = ws[off[i]:off[i] + n * 4].view(torch.float32).cpu().numpy().reshape(ref[key].shape)
+        assert np.array_equal(got, ref[key]), key
+    assert np.array_equal(mb.block_mask.cpu().numpy().reshape(ref["mask"].shape).astype(bool), ref["mask"])
+    kt = int(mb.kept_total.item())
+    assert kt == ref["kept_total"]
+    assert np.array_equal(mb.row_ptr.cpu().numpy(), ref["row_ptr"])
+    assert np.array_equal(mb.col_idx.cpu().numpy()[:kt], ref["col_idx"][:kt])
+    assert np.array_equal(mb.order.cpu().numpy(), ref["order"])
+
+
+def test_reorder_predict_fused_small_window():
+    w = I.Workload("fused_small", 321, 1, 3, 3, 5, 12, 20, 37, 128, 128, "bf16", "field", order="window",
+                   win=(2, 8, 8), sink_frames=1, bq=128, bk=64, tau=0.5, theta=0.3, sigma=(1.0, 2.0, 2.0))
+    g = I.gen_qkv(w)
+    perm, _ = Y.build_layout(w.order, w.T, w.H, w.W, w.win, w.sink_frames, w.txt_len)
+    _fused_vs_separate(w, np.asarray(perm), g["q_bits"], g["k_bits"])
+
+
+def test_reorder_predict_fused_full_size_video():
+    w = I.WORKLOADS["video"]
+    g = I.gen_qkv(w)
+    perm, _ = Y.build_layout(w.order, w.T, w.H, w.W, w.win, w.sink_frames, w.txt_len)
+    _fused_vs_separate(w, np.asarray(perm), g["q_bits"], g["k_bits"])
+
+
+def test_reorder_predict_rejects_out_of_range_perm():
+    import torch
+    from long_context_mean_b200 import sa
+    N = 300
+    shape = sa.Shape(1, 2, 2, N, 128, 128, sa.SA_BF16, 0)
+    prm = sa.make_params(128, 64, 0.5)
+    q = torch.randn(1, 2, N, 128, device="cuda").to(torch.bfloat16)
+    k = torch.randn(1, 2, N, 128, device="cuda").to(torch.bfloat16)
+    perm = torch.arange(N, dtype=torch.int32, device="cuda")
+    perm[17] = N + 5                     # not a permutation: the kernel skips the token
+    q_r, k_r = torch.empty_like(q), torch.empty_like(k)
+    ws = sa.workspace(sa.predict_mask_workspace(shape, prm), "cuda")
+    mb = sa.MaskBuffers.allocate(1, 2, N, 128, 64, "cuda")
+    sa.reorder_predict_mask(perm, q, k, q_r, k_r, shape, prm, ws, mb.struct)
+    assert sa.read_status(mb.status) == sa.SA_ERR_INVALID_ARG
