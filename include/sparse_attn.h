@@ -4,11 +4,16 @@
  *
  * The path, in call order:
  *   sa_layout_build  -> token permutation (identity, [t,h,w] windows, Hilbert)
- *   sa_reorder       -> Q, K, V gathered into the permuted order
- *   sa_predict_mask  -> block mask M_g + CSR kept lists + work order
- *   sa_block_sparse_attn -> O and per-row LSE over the kept blocks
- *   sa_unreorder     -> O (and LSE) scattered back to the original order
+ *   sa_reorder_predict_mask -> Q, K gathered into the permuted order while
+ *                       their blocks are pooled; block mask M_g + CSR kept
+ *                       lists + work order (sa_reorder + sa_predict_mask
+ *                       do the same in two passes)
+ *   sa_reorder       -> V gathered into the permuted order
+ *   sa_block_sparse_attn -> O and per-row LSE over the kept blocks, stored
+ *                       back in the original order (out_perm; sa_unreorder
+ *                       does that as a separate pass)
  *   sa_dense_attn    -> the same kernel with every block kept (reference)
+ *   sa_l1_error      -> relative L1 error of an output (calibration)
  *
  * Sources of the operations (page title, section):
  *   [P1] "AIGC 基本功｜视频稀疏注意力的误差与布局" (jefxiong.cn)
@@ -30,8 +35,9 @@
  *     log).  Query head h reads kv head h / (Hq / Hkv).
  *   - Every pointer argument to data is a DEVICE pointer unless stated;
  *     struct arguments are HOST pointers.  The caller owns all memory; the
- *     library never allocates device memory and keeps no state between
- *     calls except a thread-local error string.
+ *     library never allocates device memory (sa_predict_mask_noalloc uses a
+ *     fixed array that is part of the loaded library) and keeps no state
+ *     between calls except a thread-local error string.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *     enqueued asynchronously on it.  Argument errors are detected on the
  *     host and returned synchronously before anything is enqueued; errors
@@ -264,6 +270,14 @@ sa_status sa_dense_attn(const void* q, const void* k, const void* v, const sa_sh
 /* Synchronises `stream` and returns the device status word's code (0 =
  * SA_OK).  The word is not cleared. */
 sa_status sa_read_status(const int32_t* status, void* stream);
+
+/* ---- calibration support ([P3] 2.4) ---------------------------------------
+ * The per-layer calibration of the SpargeAttention notes bounds the relative
+ * L1 error sum |O - O'| / sum |O| of the sparse output O' against the dense
+ * output O.  sums (device double[2], overwritten) receives sum |ref - x| and
+ * sum |ref| over n elements of dtype; ref and x are 16-byte aligned device
+ * buffers, n a multiple of 8 (bf16) or 4 (fp32).  Asynchronous on stream. */
+sa_status sa_l1_error(const void* ref, const void* x, int64_t n, int32_t dtype, double* sums, void* stream);
 
 #ifdef __cplusplus
 }

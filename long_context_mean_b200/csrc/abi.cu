@@ -357,4 +357,15 @@ sa_status sa_read_status(const int32_t* status, void* stream) {
   return (sa_status)h;
 }
 
+sa_status sa_l1_error(const void* ref, const void* x, int64_t n, int32_t dtype, double* sums, void* stream) {
+  if (!ref || !x || !sums) return set_error(SA_ERR_INVALID_ARG, "NULL argument to sa_l1_error");
+  if (dtype != SA_BF16 && dtype != SA_FP32) return set_error(SA_ERR_INVALID_ARG, "dtype must be SA_BF16 or SA_FP32");
+  const int64_t per_vec = dtype == SA_BF16 ? 8 : 4;
+  if (n < 0 || n % per_vec) return set_error(SA_ERR_INVALID_ARG, "n must be a non-negative multiple of %lld", (long long)per_vec);
+  if ((uintptr_t)ref % 16 || (uintptr_t)x % 16 || (uintptr_t)sums % 8)
+    return set_error(SA_ERR_INVALID_ARG, "ref and x must be 16-byte aligned, sums 8-byte aligned");
+  if (sa_status e = check_device()) return e;
+  return launch_l1(ref, x, n, dtype, sums, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -117,6 +117,7 @@ struct AttnArgs {
   float lambda;
 };
 sa_status launch_attn_simt(const AttnArgs& a, cudaStream_t st);
+sa_status launch_l1(const void* ref, const void* x, int64_t n, int32_t dtype, double* sums, cudaStream_t st);
 sa_status launch_attn_tc(const AttnArgs& a, cudaStream_t st);
 bool attn_tc_supported(const sa_shape& s, int bq, int bk);
 

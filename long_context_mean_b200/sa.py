@@ -34,7 +34,7 @@ EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_attn_worksp
            "sa_layout_build", "sa_reorder", "sa_unreorder", "sa_predict_mask_workspace",
            "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_reorder_predict_mask", "sa_predict_mask_noalloc",
            "sa_mask_from_blocks_workspace",
-           "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status"]
+           "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status", "sa_l1_error"]
 
 
 class SAError(RuntimeError):
@@ -106,6 +106,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sa_mask_from_blocks": (I32, [P, ctypes.POINTER(Shape), I32, I32, I32, P, SZ,
                                       ctypes.POINTER(Mask), P]),
         "sa_attn_workspace": (SZ, []),
+        "sa_l1_error": (I32, [P, P, I64, I32, P, P]),
         "sa_block_sparse_attn": (I32, [P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F, F,
                                        P, P, P, P, P, SZ, I32, P]),
         "sa_dense_attn": (I32, [P, P, P, ctypes.POINTER(Shape), I32, F, P, P, P, P, SZ, I32, P]),
@@ -269,6 +270,12 @@ def dense_attn(q, k, v, shape: Shape, causal, scale, out, lse=None, status=None,
                                 ws.numel() * ws.element_size(), int(flags), _stream(stream)))
 
 
+def l1_error(ref, x, sums, stream=None):
+    """Enqueue sums[0] = sum |ref - x|, sums[1] = sum |ref| (sums: float64
+    device tensor of 2)."""
+    _check(load().sa_l1_error(_ptr(ref), _ptr(x), ref.numel(), dtype_code(ref), _ptr(sums), _stream(stream)))
+
+
 def read_status(status, stream=None) -> int:
     """Synchronises the stream and returns the device status code (no raise)."""
     return int(load().sa_read_status(_ptr(status), _stream(stream)))
@@ -345,7 +352,12 @@ class Pipeline:
         self.skip_log = (torch.zeros(self.mask.col_idx.numel(), dtype=torch.uint8, device=device)
                          if log_skips else None)
 
-    def run(self, q, k, v, stream=None):
+    def run(self, q, k, v, stream=None, out=None, lse=None):
+        """Enqueue the path on ``stream`` (default: the current stream).
+        ``out``/``lse`` (optional) receive the results instead of the
+        pipeline's own buffers."""
+        out = self.out if out is None else out
+        lse = self.lse if lse is None else lse
         if self.identity:
             qr, kr, vr = q, k, v
             predict_mask(qr, kr, self.shape, self.params, self.ws, self.mask.struct, stream)
@@ -358,13 +370,112 @@ class Pipeline:
             qr, kr, vr = self.qr, self.kr, self.vr
         # The inverse reorder of O and LSE is fused into the attention store
         # (out_perm); sa_unreorder stays available for standalone use.
-        block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, self.out, self.lse,
+        block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, out, lse,
                           self.skip_log, self.flags, stream, ws=self.attn_ws,
                           out_perm=None if self.identity else self.perm)
-        return self.out, self.lse
+        return out, lse
 
     def status(self, stream=None) -> int:
         return read_status(self.mask.status, stream)
+
+
+class HostPipeline:
+    """End-to-end pass from pinned host buffers to pinned host buffers.
+
+    Heads are independent, so the problem is cut into ``chunks`` groups of
+    (batch, head) rows (whole kv groups).  Chunk i's host-to-device copy of
+    Q, K, V runs on a copy stream, its path on the compute stream (one
+    ``Pipeline`` sized for a chunk, reused), and its device-to-host copy of
+    O and LSE on a third stream, so the copies of one chunk overlap the
+    kernels of its neighbours.  ``run`` only enqueues: the caller waits on
+    ``done`` (an event recorded after the last copy back) or synchronises.
+    """
+
+    def __init__(self, B, Hq, Hkv, N, d, dv, dtype, *, layout: LayoutDesc, params: MaskParams,
+                 lam=-math.inf, scale=0.0, flags=0, device="cuda", chunks=4):
+        import torch
+        if (B * Hkv) % chunks:
+            raise ValueError(f"chunks={chunks} must divide the {B * Hkv} kv rows")
+        self.device = torch.device(device)
+        tdt = torch.bfloat16 if dtype in ("bf16", SA_BF16) else torch.float32
+        self.g = Hq // Hkv
+        self.chunks = chunks
+        self.rows_kv = B * Hkv // chunks
+        self.rows_q = self.rows_kv * self.g
+        # Flattened (batch, head) rows: query row r reads kv row r // g.
+        self.sub = Pipeline(1, self.rows_q, self.rows_kv, N, d, dv, dtype, layout=layout, params=params,
+                            lam=lam, scale=scale, flags=flags, device=device)
+        self.q = torch.empty(B * Hq, N, d, dtype=tdt, device=device)
+        self.k = torch.empty(B * Hkv, N, d, dtype=tdt, device=device)
+        self.v = torch.empty(B * Hkv, N, dv, dtype=tdt, device=device)
+        self.out = torch.empty(B * Hq, N, dv, dtype=tdt, device=device)
+        self.lse = torch.empty(B * Hq, N, 1, dtype=torch.float32, device=device)
+        self.s_in = torch.cuda.Stream(device=self.device)
+        self.s_out = torch.cuda.Stream(device=self.device)
+        ev = lambda: torch.cuda.Event()
+        self.e_in = [ev() for _ in range(chunks)]
+        self.e_comp = [ev() for _ in range(chunks)]
+        self.e_out = [ev() for _ in range(chunks)]
+        self.done = ev()
+        self.status_word = torch.zeros(1, dtype=torch.int32, device=device)   # worst status over chunks
+        self._first = True
+
+    def run(self, q_host, k_host, v_host, out_host, lse_host, stream=None):
+        """q_host [B, Hq, N, d], k_host/v_host [B, Hkv, N, d|dv], out_host
+        [B, Hq, N, dv], lse_host [B, Hq, N] or [B, Hq, N, 1]: pinned CPU
+        tensors.  Work is ordered after ``stream`` (default: current)."""
+        import torch
+        comp = stream if stream is not None else torch.cuda.current_stream(self.device)
+        start = torch.cuda.Event()
+        with torch.cuda.stream(comp):
+            self.status_word.zero_()
+        start.record(comp)
+        qh, kh, vh = (x.reshape(-1, *x.shape[-2:]) for x in (q_host, k_host, v_host))
+        oh = out_host.reshape(-1, *out_host.shape[-2:])
+        lh = lse_host.reshape(oh.shape[0], -1)
+        rq, rk = self.rows_q, self.rows_kv
+        for i in range(self.chunks):
+            sq, sk = slice(i * rq, (i + 1) * rq), slice(i * rk, (i + 1) * rk)
+            # host -> device (the previous pass's compute of this chunk has read its inputs)
+            self.s_in.wait_event(start)
+            if not self._first:
+                self.s_in.wait_event(self.e_comp[i])
+            with torch.cuda.stream(self.s_in):
+                self.q[sq].copy_(qh[sq], non_blocking=True)
+                self.k[sk].copy_(kh[sk], non_blocking=True)
+                self.v[sk].copy_(vh[sk], non_blocking=True)
+            self.e_in[i].record(self.s_in)
+            # the path on this chunk (its outputs' previous copy back has finished)
+            comp.wait_event(self.e_in[i])
+            if not self._first:
+                comp.wait_event(self.e_out[i])
+            self.sub.run(self.q[sq].unsqueeze(0), self.k[sk].unsqueeze(0), self.v[sk].unsqueeze(0), comp,
+                         out=self.out[sq].unsqueeze(0), lse=self.lse[sq].unsqueeze(0))
+            with torch.cuda.stream(comp):
+                torch.maximum(self.status_word, self.sub.mask.status, out=self.status_word)
+            self.e_comp[i].record(comp)
+            # device -> host
+            self.s_out.wait_event(self.e_comp[i])
+            with torch.cuda.stream(self.s_out):
+                oh[sq].copy_(self.out[sq], non_blocking=True)
+                lh[sq].copy_(self.lse[sq].reshape(rq, -1), non_blocking=True)
+            self.e_out[i].record(self.s_out)
+        comp.wait_event(self.e_out[self.chunks - 1])
+        self.done.record(comp)
+        self._first = False
+
+    def status(self) -> int:
+        """Synchronises; the largest status code any chunk raised (0 = SA_OK)."""
+        return read_status(self.status_word)
+
+
+def host_pipeline_for(w, device="cuda", chunks=4, **kw) -> HostPipeline:
+    """HostPipeline for a workload description from ``inputs.WORKLOADS``."""
+    lay = make_layout(w.T, w.H, w.W, w.txt_len, w.sink_frames, w.order, w.win)
+    prm = make_params(w.bq, w.bk, w.tau, w.theta, w.sink_tokens, w.txt_len, w.local_window,
+                      w.anchor_tokens, w.causal)
+    return HostPipeline(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, w.dtype, layout=lay, params=prm, lam=w.lam,
+                        device=device, chunks=chunks, **kw)
 
 
 def pipeline_for(w, device="cuda", **kw) -> Pipeline:

@@ -158,3 +158,34 @@ def test_lm_causal_gqa_sampled():
     w = I.WORKLOADS["lm_causal"]
     nqb = -(-w.N // w.bq)
     _sampled_heads_check(w, [(0, 0), (0, 29)], lambda h: h // (w.Hq // w.Hkv), [0, 1, 40, 513, nqb - 1])
+
+
+@pytest.mark.parametrize("name,chunks", [("video", 4), ("lm_small", 2)])
+def test_host_pipeline_matches_device_pipeline(name, chunks):
+    """The chunked host-to-host pass (copies overlapped with the kernels)
+    returns exactly what the device pipeline computes: heads are independent
+    and every chunk runs the same kernels on its rows."""
+    import torch
+    from long_context_mean_b200 import sa
+    if name == "lm_small":
+        w = I.Workload("lm_small", 55, 2, 4, 2, 1, 1, 1500, 0, 128, 128, "bf16", "lowrank", bq=128, bk=64,
+                       tau=0.9, causal=True, local_window=300, anchor_tokens=64, sigma_pos=40.0)
+    else:
+        w = I.WORKLOADS[name]
+    g = I.gen_qkv(w)
+    host = {n: torch.from_numpy(g[n + "_bits"].view(np.int16)).view(torch.bfloat16).pin_memory() for n in "qkv"}
+    q, k, v = (host[n].to("cuda") for n in "qkv")
+    pipe = sa.pipeline_for(w)
+    out_d, lse_d = pipe.run(q, k, v)
+    assert pipe.status() == sa.SA_OK
+    hp = sa.host_pipeline_for(w, chunks=chunks)
+    out_h = torch.empty(out_d.shape, dtype=out_d.dtype).pin_memory()
+    lse_h = torch.empty(lse_d.shape, dtype=lse_d.dtype).pin_memory()
+    for _ in range(2):                  # twice: the second pass reuses every buffer
+        out_h.fill_(0)
+        lse_h.fill_(0)
+        hp.run(host["q"], host["k"], host["v"], out_h, lse_h)
+        hp.done.synchronize()
+        assert hp.status() == sa.SA_OK
+        assert torch.equal(out_h, out_d.cpu())
+        assert torch.equal(lse_h, lse_d.cpu())
