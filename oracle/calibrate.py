@@ -22,7 +22,7 @@ measure for lambda is printed):
 
 Pins (tests/test_oracle_calibrate.py): relative L1 on closed-form arrays; the
 selection rule on hand-made tables; on a small problem the full-mask point
-(tau = 1, theta = 0) has L1 = 0 exactly, and the chosen point is feasible
+(tau = 1, theta = 0) has L1 = 0 up to rounding (< 1e-12), and the chosen point is feasible
 and at least as sparse as every other feasible point found by brute force.
 """
 
@@ -77,7 +77,7 @@ def calibrate(q, k, v, bq, bk, taus, thetas, lams, l1, l2, causal=False, sink_to
     q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
     B, Hq, N, _ = q.shape
     group = Hq // k.shape[1]
-    dense = np.stack([np.stack([A.dense_attention(q[b, h], k[b, h // group], v[b, h // group], causal)
+    dense = np.stack([np.stack([A.dense_attention(q[b, h], k[b, h // group], v[b, h // group], causal)[0]
                                 for h in range(Hq)]) for b in range(B)])
     total_valid = B * Hq * valid_tiles(N, bq, bk, causal)
     step1 = []
