@@ -242,11 +242,30 @@ int score_rows_per_cta(int P2) {
   return g < 1 ? 1 : (g > kMaxRowsPerCta ? kMaxRowsPerCta : g);
 }
 
+constexpr int kStages = 3;   // k_hat chunks in flight (cp.async ring)
+
+// Bytes of the region shared by the k_hat chunk ring (score phase) and the
+// sort keys (TopCdf phase): the two are never live at once.
+__host__ __device__ inline size_t score_union_bytes(int d, int P2, int G) {
+  const size_t ring = (size_t)kStages * kChunk * (d + 4) * 4;
+  const size_t keys = (size_t)G * P2 * 8;
+  return ring > keys ? ring : keys;
+}
+
 size_t score_smem_bytes(int d, int64_t nkb, int P2, int G) {
   const size_t nkb16 = (size_t)((nkb + 15) / 16) * 16;
-  return (size_t)kMaxRowsPerCta * d * 4 + (size_t)kChunk * (d + 4) * 4 + (size_t)G * nkb * 4 +
-         (size_t)G * P2 * 8 + (size_t)G * nkb16;
+  return (size_t)kMaxRowsPerCta * d * 4 + score_union_bytes(d, P2, G) + (size_t)G * nkb * 4 +
+         (size_t)G * nkb16;
 }
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ float warp_max(float v) {
   for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
@@ -261,14 +280,15 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   extern __shared__ __align__(16) unsigned char smem[];
   const int nkb16 = (int)((nkb + 15) / 16) * 16;
   float* qs = reinterpret_cast<float*>(smem);
-  float* ks = qs + kMaxRowsPerCta * d;
-  // k_hat rows padded to d + 4 floats: 16-byte aligned for float4 reads,
-  // and the 8 rows a quarter-warp reads land in distinct bank groups.
-  float* sc = ks + kChunk * (d + 4);
-  // 8-byte aligned: the float offset 8d + 32(d+4) + G nkb is even (G even
-  // or nkb even; see score_rows_per_cta).
-  uint64_t* keys = reinterpret_cast<uint64_t*>(sc + G * nkb);
-  uint8_t* flags = reinterpret_cast<uint8_t*>(keys + (size_t)G * P2);
+  // One region holds the ring of k_hat chunks while scores are computed and
+  // the sort keys afterwards.  k_hat rows are padded to d + 4 floats:
+  // 16-byte aligned for cp.async and float4 reads, and the 8 rows a
+  // quarter-warp reads land in distinct bank groups.
+  unsigned char* uni = smem + (size_t)kMaxRowsPerCta * d * 4;
+  float* ks = reinterpret_cast<float*>(uni);
+  uint64_t* keys = reinterpret_cast<uint64_t*>(uni);
+  float* sc = reinterpret_cast<float*>(uni + score_union_bytes(d, P2, G));
+  uint8_t* flags = reinterpret_cast<uint8_t*>(sc + G * nkb);
   __shared__ int s_forced[kMaxRowsPerCta];
 
   const int64_t bh = blockIdx.y;
@@ -291,39 +311,37 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   for (int r = 0; r < rows; ++r) any_scored |= !s_forced[r];
 
   if (any_scored) {
-    // Scores of the whole group, one k_hat chunk at a time: the next chunk's
-    // float4 loads are in flight while the current chunk is multiplied.
+    // Scores of the whole group, one k_hat chunk at a time, the chunks
+    // streamed into a ring of kStages buffers with cp.async so that the next
+    // chunks' loads are in flight while the current one is multiplied.
     const float4* kg4 = reinterpret_cast<const float4*>(khat + g * nkb * (int64_t)d);
     const int nf4 = d / 4;
     const int r = threadIdx.x / kChunk, j = threadIdx.x % kChunk;
-    constexpr int kPer = kChunk * 256 / 4 / kRowThreads;   // float4 per thread (d <= 256)
-    float4 buf[kPer];
-    auto load_chunk = [&](int64_t c0) {
-      const int total = (int)min64(kChunk, nkb - c0) * nf4;
-#pragma unroll
-      for (int q = 0; q < kPer; ++q) {
-        const int i = threadIdx.x + q * kRowThreads;
-        buf[q] = i < total ? __ldg(kg4 + c0 * nf4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int64_t nchunks = (nkb + kChunk - 1) / kChunk;
+    auto issue_chunk = [&](int64_t c) {
+      if (c < nchunks) {
+        const int64_t c0 = c * kChunk;
+        const int total = (int)min64(kChunk, nkb - c0) * nf4;
+        float* dst = ks + (c % kStages) * kChunk * (d + 4);
+        for (int i = threadIdx.x; i < total; i += kRowThreads)
+          cp_async16(dst + (i / nf4) * (d + 4) + (i % nf4) * 4, kg4 + c0 * nf4 + i);
       }
+      cp_async_commit();   // possibly empty: one group per chunk slot keeps the count uniform
     };
-    load_chunk(0);
-    for (int64_t c0 = 0; c0 < nkb; c0 += kChunk) {
+    for (int c = 0; c < kStages - 1; ++c) issue_chunk(c);
+    for (int64_t c = 0; c < nchunks; ++c) {
+      const int64_t c0 = c * kChunk;
       const int cn = (int)min64(kChunk, nkb - c0);
-#pragma unroll
-      for (int q = 0; q < kPer; ++q) {
-        const int i = threadIdx.x + q * kRowThreads;
-        if (i < cn * nf4) {
-          *reinterpret_cast<float4*>(ks + (i / nf4) * (d + 4) + (i % nf4) * 4) = buf[q];
-        }
-      }
-      __syncthreads();
-      if (c0 + kChunk < nkb) load_chunk(c0 + kChunk);
+      cp_async_wait<kStages - 2>();   // chunk c has landed (this thread's part)
+      __syncthreads();                // ... everyone's; and chunk c-1's buffer is free
+      issue_chunk(c + kStages - 1);
+      const float* kc = ks + (c % kStages) * kChunk * (d + 4);
       const int64_t kb = c0 + j;
       if (r < rows && j < cn) {
         float s = -INFINITY;
         if (!s_forced[r] && rules.valid(qb0 + r, kb) && !(guard && sk[g * nkb + kb] < theta)) {
           const float4* qr = reinterpret_cast<const float4*>(qs + r * d);
-          const float4* kr = reinterpret_cast<const float4*>(ks + j * (d + 4));
+          const float4* kr = reinterpret_cast<const float4*>(kc + j * (d + 4));
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
           for (int e = 0; e < d / 4; ++e) {
             const float4 x = qr[e], y = kr[e];
@@ -336,8 +354,9 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
         }
         sc[r * nkb + kb] = s;
       }
-      __syncthreads();
     }
+    cp_async_wait<0>();
+    __syncthreads();   // the chunk ring becomes the sort keys below
   }
 
   if (warp >= rows) return;
@@ -390,12 +409,11 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
           break;
         }
         const uint32_t kb = ~(uint32_t)best;
-        if ((int)(kb & 31) == lane) {
-          fl[kb] = 1;
+        if ((int)(kb & 31) == lane) fl[kb] = 1;
+        // Keys are unique (the block index is part of the key): clearing by
+        // value needs no computed index, so key[] stays in registers.
 #pragma unroll
-          for (int q = 0; q < kFastKeys; ++q)        // static indices keep key[] in registers
-            if (q == (int)(kb >> 5)) key[q] = 0ull;
-        }
+        for (int q = 0; q < kFastKeys; ++q) key[q] = key[q] == best ? 0ull : key[q];
         cum += pv;
       }
       if (!done) {
