@@ -565,52 +565,88 @@ __global__ void fill_cols_kernel(const uint8_t* __restrict__ mask, int64_t R, in
 
 // Work order: stable LSD radix sort of rows by key = 4095 - count (3 passes
 // of 4 bits), i.e. descending count, ties by ascending row index.  One CTA;
-// each thread owns a contiguous range of the current sequence; the digit
-// histogram is kept per (digit, thread) so the scatter stays stable.
+// each thread owns a contiguous range of the current sequence and keeps its
+// 16 digit counts in a padded row of shared memory (stride 17: no bank
+// conflicts); the scatter offsets come from a scan in (digit, thread) order
+// done with warp shuffles, which keeps the scatter stable.  When the rows
+// fit (R <= kOrderSmemRows) the keys and the intermediate sequences live in
+// shared memory and only the final pass writes `order`.
 constexpr int kOrderThreads = 1024;
+constexpr int kOrderWarps = kOrderThreads / 32;
+constexpr int kOrderSmemRows = 8192;
+constexpr int kHistStride = 17;
+
 __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __restrict__ counts,
                                                               int64_t R, int32_t* __restrict__ tmp,
                                                               int32_t* __restrict__ order) {
-  extern __shared__ uint32_t hist[];  // [16][kOrderThreads]
-  __shared__ uint32_t part[kOrderThreads];
-  const int tid = threadIdx.x;
+  extern __shared__ uint32_t dyn[];
+  uint32_t* hist = dyn;                                   // [kOrderThreads][17]
+  const bool in_smem = R <= kOrderSmemRows;
+  uint16_t* skey = reinterpret_cast<uint16_t*>(dyn + kHistStride * kOrderThreads);   // [R] key of row
+  int32_t* sa = reinterpret_cast<int32_t*>(skey + (in_smem ? kOrderSmemRows : 0));   // [R] sequences
+  int32_t* sb = sa + (in_smem ? kOrderSmemRows : 0);
+  __shared__ uint32_t wtot[kOrderWarps][16];              // per-warp digit totals, then warp offsets
+  __shared__ uint32_t dtot[16];                           // digit totals
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t* my = hist + tid * kHistStride;
   const int64_t per = (R + kOrderThreads - 1) / kOrderThreads;
   const int64_t beg = tid * per, end = min(R, beg + per);
+  if (in_smem) {
+    for (int64_t i = tid; i < R; i += kOrderThreads) skey[i] = (uint16_t)(4095u - (uint32_t)counts[i]);
+    __syncthreads();
+  }
+  auto key_of = [&](int32_t row) -> uint32_t {
+    return in_smem ? (uint32_t)skey[row] : 4095u - (uint32_t)counts[row];
+  };
   for (int pass = 0; pass < 3; ++pass) {
-    const int32_t* src = pass == 0 ? nullptr : (pass == 1 ? order : tmp);
-    int32_t* dst = pass == 1 ? tmp : order;
+    // source and destination of this pass: rows in natural order first, the
+    // final pass writes `order`
+    const int32_t* src = pass == 0 ? nullptr : (in_smem ? (pass == 1 ? sa : sb) : (pass == 1 ? order : tmp));
+    int32_t* dst = pass == 2 ? order : (in_smem ? (pass == 0 ? sa : sb) : (pass == 0 ? order : tmp));
     const int shift = 4 * pass;
-    for (int dgt = 0; dgt < 16; ++dgt) hist[dgt * kOrderThreads + tid] = 0;
+#pragma unroll
+    for (int dgt = 0; dgt < 16; ++dgt) my[dgt] = 0;
+    for (int64_t i = beg; i < end; ++i) {
+      const int32_t row = src ? src[i] : (int32_t)i;
+      my[(key_of(row) >> shift) & 15u] += 1;
+    }
+    // Offsets: entry (digit, thread) starts after every entry of smaller
+    // digits and after the same digit's entries of smaller threads.
+    uint32_t c[16], x[16];
+#pragma unroll
+    for (int dgt = 0; dgt < 16; ++dgt) x[dgt] = c[dgt] = my[dgt];
+#pragma unroll
+    for (int dgt = 0; dgt < 16; ++dgt) {
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, x[dgt], off);
+        if (lane >= off) x[dgt] += o;
+      }
+    }
+    if (lane == 31) {
+#pragma unroll
+      for (int dgt = 0; dgt < 16; ++dgt) wtot[warp][dgt] = x[dgt];
+    }
+    __syncthreads();
+    if (tid < 16) {   // thread `dgt`: exclusive scan of the warp totals of its digit
+      uint32_t run = 0;
+      for (int w = 0; w < kOrderWarps; ++w) {
+        const uint32_t t = wtot[w][tid];
+        wtot[w][tid] = run;
+        run += t;
+      }
+      dtot[tid] = run;
+    }
+    __syncthreads();
+    uint32_t base = 0;
+#pragma unroll
+    for (int dgt = 0; dgt < 16; ++dgt) {
+      my[dgt] = base + wtot[warp][dgt] + x[dgt] - c[dgt];
+      base += dtot[dgt];
+    }
     __syncthreads();
     for (int64_t i = beg; i < end; ++i) {
       const int32_t row = src ? src[i] : (int32_t)i;
-      const uint32_t key = 4095u - (uint32_t)counts[row];
-      hist[((key >> shift) & 15u) * kOrderThreads + tid] += 1;
-    }
-    __syncthreads();
-    // Exclusive scan over the 16*1024 entries in (digit, thread) order:
-    // thread j owns entries [16j, 16j+16).
-    uint32_t s = 0;
-    for (int e = 0; e < 16; ++e) s += hist[tid * 16 + e];
-    part[tid] = s;
-    __syncthreads();
-    for (int off = 1; off < kOrderThreads; off <<= 1) {
-      const uint32_t v = tid >= off ? part[tid - off] : 0;
-      __syncthreads();
-      part[tid] += v;
-      __syncthreads();
-    }
-    uint32_t run = part[tid] - s;
-    for (int e = 0; e < 16; ++e) {
-      const uint32_t c = hist[tid * 16 + e];
-      hist[tid * 16 + e] = run;
-      run += c;
-    }
-    __syncthreads();
-    for (int64_t i = beg; i < end; ++i) {
-      const int32_t row = src ? src[i] : (int32_t)i;
-      const uint32_t key = 4095u - (uint32_t)counts[row];
-      uint32_t& slot = hist[((key >> shift) & 15u) * kOrderThreads + tid];
+      uint32_t& slot = my[(key_of(row) >> shift) & 15u];
       dst[slot] = row;
       slot += 1;
     }
@@ -628,7 +664,8 @@ sa_status launch_lists(const sa_shape& s, int bq, int bk, int32_t* counts, int32
   fill_cols_kernel<<<(unsigned)ceil_div(R, warps_per_block), 32 * warps_per_block, 0, st>>>(
       out.block_mask, R, out.nkb, out.row_ptr, out.col_capacity, out.col_idx);
   if (sa_status e = check_launch("fill_cols_kernel")) return e;
-  const size_t hist_bytes = 16 * kOrderThreads * sizeof(uint32_t);
+  size_t hist_bytes = (size_t)kHistStride * kOrderThreads * sizeof(uint32_t);
+  if (R <= kOrderSmemRows) hist_bytes += (size_t)kOrderSmemRows * (2 + 4 + 4);   // keys + two sequences
   if (cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)hist_bytes) != cudaSuccess)
     return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(order_kernel) failed");
