@@ -225,12 +225,13 @@ __device__ void finish_row(const uint8_t* flags, int64_t u, int64_t qb, int64_t 
 // a3 + a4: one CTA per (head, group of G <= 8 query blocks).  The group's
 // q_hat rows and 32-row chunks of the kv head's k_hat are staged in shared
 // memory (padded rows, conflict-free) so every k_hat element is read once per
-// group.  Then warp r alone finishes row r: softmax, bitonic sort of
-// (p, kb) keys descending (ties: lower kb first), scan, TopCdf, the union with
+// group.  Then warp r alone finishes row r: softmax and TopCdf (an arg-max
+// loop over register-resident keys when the row is short and few blocks are
+// picked, else a bisection for the last kept probability), the union with
 // the forced parts and the causal AND -- with warp-level synchronisation
 // only.
-// Dynamic shared memory: q_hat [8][d] | k_hat chunk [32][d+1] |
-// scores [G][nkb] | keys [G][P2] (u64) | flags [G][nkb rounded to 16] (u8).
+// Dynamic shared memory: q_hat [8][d] | k_hat chunk ring [3][32][d+4], reused
+// as p [G][P2] (fp32) | scores [G][nkb] | flags [G][nkb rounded to 16] (u8).
 // ---------------------------------------------------------------------------
 constexpr int kMaxRowsPerCta = 8;
 constexpr int kChunk = 32;
@@ -238,7 +239,7 @@ constexpr int kFastKeys = 16;     // keys per lane on the fast TopCdf path (nkb 
 constexpr int kFastPicks = 128;   // picks before the fast path defers to the sort
 
 int score_rows_per_cta(int P2) {
-  int g = 65536 / (P2 * 8);
+  int g = 65536 / (P2 * 4);
   return g < 1 ? 1 : (g > kMaxRowsPerCta ? kMaxRowsPerCta : g);
 }
 
@@ -248,7 +249,7 @@ constexpr int kStages = 3;   // k_hat chunks in flight (cp.async ring)
 // sort keys (TopCdf phase): the two are never live at once.
 __host__ __device__ inline size_t score_union_bytes(int d, int P2, int G) {
   const size_t ring = (size_t)kStages * kChunk * (d + 4) * 4;
-  const size_t keys = (size_t)G * P2 * 8;
+  const size_t keys = (size_t)G * P2 * 4;
   return ring > keys ? ring : keys;
 }
 
@@ -286,7 +287,7 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   // quarter-warp reads land in distinct bank groups.
   unsigned char* uni = smem + (size_t)kMaxRowsPerCta * d * 4;
   float* ks = reinterpret_cast<float*>(uni);
-  uint64_t* keys = reinterpret_cast<uint64_t*>(uni);
+  float* keys = reinterpret_cast<float*>(uni);
   float* sc = reinterpret_cast<float*>(uni + score_union_bytes(d, P2, G));
   uint8_t* flags = reinterpret_cast<uint8_t*>(sc + G * nkb);
   __shared__ int s_forced[kMaxRowsPerCta];
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   const int64_t qb = qb0 + r;
   const int64_t u = bh * nqb + qb;
   const bool row_forced = s_forced[r] != 0;
-  uint64_t* kw = keys + (size_t)r * P2;
+  float* pr = keys + (size_t)r * P2;
   uint8_t* fl = flags + (size_t)r * nkb16;
   for (int64_t kb = lane; kb < nkb; kb += 32) fl[kb] = 0;
   if (!row_forced) {
@@ -377,7 +378,7 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
     if (mx > -INFINITY && P2 <= 32 * kFastKeys) {
       // Fast path: repeated warp-wide arg-max over register-resident keys,
       // accumulating the mass in sorted order; TopCdf usually stops after a
-      // few picks.  Gives up after kFastPicks picks (the sort below then
+      // few picks.  Gives up after kFastPicks picks (the bisection below then
       // decides the row from scratch).
       uint64_t key[kFastKeys];
       float part = 0.f;
@@ -422,53 +423,48 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
       __syncwarp();
     }
     if (mx > -INFINITY && !done) {
-      for (int kb = lane; kb < P2; kb += 32) {
-        uint64_t key = 0ull;
-        if (kb < nkb) {
-          const float sv = srow[kb];
-          const float p = (sv == -INFINITY) ? 0.f : expf(sv - mx);
-          // key = p bits (p >= 0: integer order = float order) | ~kb
-          key = ((uint64_t)__float_as_uint(p) << 32) | (uint32_t)(~(uint32_t)kb);
-        }
-        kw[kb] = key;
+      // Threshold search for rows the fast path does not settle.  With p
+      // sorted descending (ties by index), block j is kept iff the mass
+      // sorted before it is < tau * total.  Let f(t) be the mass of the p
+      // whose bit pattern exceeds t (p >= 0: bit order = value order); f
+      // falls as t rises.  The smallest t* with f(t*) < tau * total is the
+      // bit pattern of the last value kept: every p above it is kept, and the
+      // blocks whose p equals it are kept in index order while f(t*) + r p <
+      // tau * total (r = rank among them).  t* is found by bisection over the
+      // bit patterns of (0, 1] (p = exp(s - max) <= 1).
+      for (int kb = lane; kb < nkb; kb += 32) {
+        const float sv = srow[kb];
+        pr[kb] = (sv == -INFINITY) ? 0.f : expf(sv - mx);
       }
       __syncwarp();
-      // Bitonic sort, descending.
-      for (int k = 2; k <= P2; k <<= 1) {
-        for (int jj = k >> 1; jj > 0; jj >>= 1) {
-          for (int i = lane; i < P2; i += 32) {
-            const int ixj = i ^ jj;
-            if (ixj > i) {
-              const uint64_t x = kw[i], y = kw[ixj];
-              const bool desc = (i & k) == 0;
-              if (desc ? (x < y) : (x > y)) {
-                kw[i] = y;
-                kw[ixj] = x;
-              }
-            }
-          }
-          __syncwarp();
+      auto mass_above = [&](uint32_t t) -> float {
+        float m = 0.f;
+        for (int kb = lane; kb < nkb; kb += 32) {
+          const float pv = pr[kb];
+          m += __float_as_uint(pv) > t ? pv : 0.f;
         }
+        for (int off = 16; off > 0; off >>= 1) m += __shfl_xor_sync(0xffffffffu, m, off);
+        return m;
+      };
+      const float limit = tau * mass_above(0u);
+      uint32_t lo = 0u, hi = 0x3F800000u;   // f(lo) >= limit (tau <= 1), f(hi) = 0 < limit
+      while (hi - lo > 1u) {
+        const uint32_t mid = lo + (hi - lo) / 2u;
+        if (mass_above(mid) < limit) hi = mid;
+        else lo = mid;
       }
-      // Inclusive scan of the sorted probabilities: lane `lane` owns a
-      // contiguous run, then a warp scan of the run totals.
-      const int per = P2 >= 32 ? P2 / 32 : 1;
-      const int beg = lane * per;
-      float run = 0.f;
-      for (int i = beg; i < beg + per && i < P2; ++i) run += __uint_as_float((uint32_t)(kw[i] >> 32));
-      float incl = run;
-      for (int off = 1; off < 32; off <<= 1) {
-        const float v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      const float total = __shfl_sync(0xffffffffu, incl, 31);
-      const float limit = tau * total;
-      float excl = incl - run;
-      for (int i = beg; i < beg + per && i < P2; ++i) {
-        const float p = __uint_as_float((uint32_t)(kw[i] >> 32));
-        const uint32_t kb = ~(uint32_t)kw[i];
-        if (p > 0.f && excl < limit) fl[kb] = 1;
-        excl += p;
+      const float above = mass_above(hi);
+      const float vstar = __uint_as_float(hi);
+      uint32_t run = 0;
+      for (int64_t kb0 = 0; kb0 < nkb; kb0 += 32) {
+        const int64_t kb = kb0 + lane;
+        const uint32_t bits = kb < nkb ? __float_as_uint(pr[kb]) : 0u;
+        const bool tie = kb < nkb && bits == hi;
+        const unsigned bal = __ballot_sync(0xffffffffu, tie);
+        bool keep = kb < nkb && bits > hi;
+        if (tie) keep = above + (float)(run + __popc(bal & ((1u << lane) - 1u))) * vstar < limit;
+        if (keep) fl[kb] = 1;
+        run += __popc(bal);
       }
     }
   }
