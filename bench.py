@@ -159,6 +159,15 @@ def kept_flops(w, row_ptr, col_idx, skip, nqb):
 # Our arm
 # ----------------------------------------------------------------------------
 
+def workload_config(w, world):
+    """The bench line's config: the workload with its sizes (both arms)."""
+    return {"workload": f"{w.name}: B={w.B} H={w.Hq} N={w.N} ([{w.T},{w.H},{w.W}]+{w.txt_len} text) "
+                        f"d={w.d} {w.order}{list(w.win) if w.order == 'window' else ''} sink_frames={w.sink_frames} "
+                        f"bq={w.bq} bk={w.bk} tau={w.tau} theta={w.theta} lambda={w.lam}",
+            "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"replicas x{world}",
+            "l2": "flushed between timed steps (256 MB write)"}
+
+
 def max_over_ranks(values, world, device):
     """Element-wise maximum of per-rank timings (ms) over all ranks."""
     import torch
@@ -345,11 +354,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded smooth-field generator, bf16)",
-        "config": {"workload": f"{w.name}: B={w.B} H={w.Hq} N={w.N} ([{w.T},{w.H},{w.W}]+{w.txt_len} text) "
-                               f"d={w.d} {w.order}{list(w.win) if w.order == 'window' else ''} sink_frames={w.sink_frames} "
-                               f"bq={w.bq} bk={w.bk} tau={w.tau} theta={w.theta} lambda={w.lam}",
-                   "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"replicas x{world}",
-                   "l2": "flushed between timed steps (256 MB write)"},
+        "config": workload_config(w, world),
         "stages_ms": {"layout_reorder_predict": round(statistics.mean(pre_ms), 4),
                       "attention_with_fused_unreorder": round(statistics.mean(attn_ms), 4)},
         "attn_ms": round(attn_mean, 4),
@@ -452,7 +457,7 @@ def run_reference(args, rank, world):
     return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "seq_len": w.N, "parallelism": "host cores"},
+            "config": workload_config(w, world),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
                              "sample": sample},
