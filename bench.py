@@ -237,10 +237,15 @@ def run_ours(args, rank, world, local_rank):
         e[0].record(stream)
         if not pipe.identity:
             sa.layout_build(pipe.layout, pipe.perm, pipe.inv, pipe.layout_ws)
+            # the V reorder on the pipeline's side stream, beside the prediction
+            pipe.ev_layout.record(stream)
+            pipe.side.wait_event(pipe.ev_layout)
+            sa.reorder(pipe.perm, v, pipe.vr, pipe.side)
+            pipe.ev_v.record(pipe.side)
             # mask prediction with the reorder of Q and K fused into its pooling pass
             sa.reorder_predict_mask(pipe.perm, q, k, pipe.qr, pipe.kr, pipe.shape, pipe.params, pipe.ws,
                                     pipe.mask.struct)
-            sa.reorder(pipe.perm, v, pipe.vr)
+            stream.wait_event(pipe.ev_v)
             qr, kr, vr = pipe.qr, pipe.kr, pipe.vr
         else:
             qr, kr, vr = q, k, v

@@ -323,9 +323,9 @@ class Pipeline:
 
     Allocates (through torch) the layout, reordered copies, workspace, mask
     lists and outputs once; ``run(q, k, v)`` then enqueues, on the current
-    stream: layout build, mask prediction fused with the reorder of Q and K,
-    reorder of V, block-sparse attention with the inverse reorder of O and
-    LSE fused into its store.  Inputs are BNSD in the original token order;
+    stream: layout build, mask prediction fused with the reorder of Q and K
+    (the reorder of V runs beside it on a side stream), block-sparse
+    attention with the inverse reorder of O and LSE fused into its store.  Inputs are BNSD in the original token order;
     ``out``/``lse`` come back in that order too.
     """
 
@@ -351,6 +351,13 @@ class Pipeline:
         self.mask = MaskBuffers.allocate(B, Hq, N, params.bq, params.bk, device)
         self.skip_log = (torch.zeros(self.mask.col_idx.numel(), dtype=torch.uint8, device=device)
                          if log_skips else None)
+        if not self.identity:
+            # The V reorder runs on a side stream beside the prediction: both
+            # need only the layout, and the prediction's scoring and list
+            # kernels leave HBM bandwidth free.
+            self.side = torch.cuda.Stream(device=torch.device(device))
+            self.ev_layout = torch.cuda.Event()
+            self.ev_v = torch.cuda.Event()
 
     def run(self, q, k, v, stream=None, out=None, lse=None):
         """Enqueue the path on ``stream`` (default: the current stream).
@@ -362,11 +369,21 @@ class Pipeline:
             qr, kr, vr = q, k, v
             predict_mask(qr, kr, self.shape, self.params, self.ws, self.mask.struct, stream)
         else:
-            layout_build(self.layout, self.perm, self.inv, self.layout_ws, stream)
+            import torch
+            st = stream if stream is not None else torch.cuda.current_stream(q.device)
+            layout_build(self.layout, self.perm, self.inv, self.layout_ws, st)
+            # V on the side stream, after the layout (and after everything the
+            # caller enqueued before, including the last pass's attention).
+            self.ev_layout.record(st)
+            self.side.wait_event(self.ev_layout)
+            reorder(self.perm, v, self.vr, self.side)
+            v.record_stream(self.side)   # the caller's v stays allocated until the side stream has read it
+            self.ev_v.record(self.side)
             # Q and K are reordered by the pooling pass of the prediction.
             reorder_predict_mask(self.perm, q, k, self.qr, self.kr, self.shape, self.params, self.ws,
-                                 self.mask.struct, stream)
-            reorder(self.perm, v, self.vr, stream)
+                                 self.mask.struct, st)
+            st.wait_event(self.ev_v)
+            stream = st
             qr, kr, vr = self.qr, self.kr, self.vr
         # The inverse reorder of O and LSE is fused into the attention store
         # (out_perm); sa_unreorder stays available for standalone use.
