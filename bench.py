@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch of the attention kernel from the ncu capture recorded
 # in profiles/attn_tc_video.md, keyed by the sha1 of the kernel code it was
 # taken on (src_sha1); any other code reports null.
-TRAFFIC = {("b5b6ef460c7c7391887a0a133378e43162267090", "video"): 1.216e9}
+TRAFFIC = {("ddf27a4b26825447a86d20e705ba53ea13f6274b", "video"): 1.2216e9}
 
 
 def peaks():
@@ -386,6 +386,144 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
+def run_svg(args, rank, world, local_rank):
+    """--path svg: the per-head spatial / temporal path (long_context_mean_b200.svg)
+    on the workload's video shape.  Heads are biased to a frame (two in three)
+    or to a position (one in three); the profile (dense attention and both
+    candidates, sampled-row MSE, argmin) runs once before timing and is timed
+    on its own; a step is the run: Q, K, V into each head's order and the
+    block-sparse attention with the per-head store back."""
+    import numpy as np
+    import torch
+
+    from long_context_mean_b200 import inputs as I
+    from long_context_mean_b200 import sa, svg
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = I.WORKLOADS[args.workload]
+    if w.B != 1 or w.Hq != w.Hkv or w.causal:
+        raise SystemExit("--path svg needs a video workload with B = 1 and Hq = Hkv")
+    bias = ["position" if h % 3 == 0 else "frame" for h in range(w.Hq)]
+    g = I.biased_video_heads(w.T, w.H, w.W, w.txt_len, bias, d=w.d, dv=w.dv, seed=w.seed)
+    q, k, v = (torch.from_numpy(g[n + "_bits"].view(np.int16)).to(dev).view(torch.bfloat16) for n in "qkv")
+    stream = torch.cuda.current_stream(dev)
+    pipe = svg.svg_pipeline_for(w, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    pipe.profile(q, k, v)                                 # warm-up profile
+    prof = []
+    for _ in range(3):
+        flush.fill_(1.0)
+        a, b = ev(), ev()
+        a.record(stream)
+        choice, _ = pipe.profile(q, k, v)
+        b.record(stream)
+        prof.append((a, b))
+    torch.cuda.synchronize(dev)
+    profile_ms = statistics.median(x[0].elapsed_time(x[1]) for x in prof)
+    rp = pipe.mask.row_ptr.cpu().numpy().astype(np.int64)
+    ci = pipe.mask.col_idx.cpu().numpy()
+    nqb, nkb = pipe.mask.struct.nqb, pipe.mask.struct.nkb
+    qk_flops, pv_flops = kept_flops(w, rp, ci, np.zeros(ci.size, dtype=np.uint8), nqb)
+    flops = qk_flops + pv_flops
+    kept = int(rp[-1])
+    sparsity = 1.0 - kept / (w.Hq * nqb * nkb)
+
+    def step_timed():
+        e = [ev() for _ in range(3)]
+        e[0].record(stream)
+        sa.reorder_heads(pipe.perms, q, pipe.qr)
+        sa.reorder_heads(pipe.perms, k, pipe.kr)
+        sa.reorder_heads(pipe.perms, v, pipe.vr)
+        e[1].record(stream)
+        sa.block_sparse_attn(pipe.qr, pipe.kr, pipe.vr, pipe.shape, pipe.mask.struct, pipe.lam, pipe.scale,
+                             pipe.out, pipe.lse, None, sa.SA_FLAG_OUT_PERM_PER_HEAD, ws=pipe.attn_ws,
+                             out_perm=pipe.perms)
+        e[2].record(stream)
+        return e
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step_timed()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    recs = []
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        recs.append(step_timed())
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    if pipe.status() != sa.SA_OK:
+        raise RuntimeError("device status after the timed steps")
+    step_ms = statistics.mean(r[0].elapsed_time(r[2]) for r in recs)
+    attn_ms = statistics.mean(r[1].elapsed_time(r[2]) for r in recs)
+    reorder_ms = statistics.mean(r[0].elapsed_time(r[1]) for r in recs)
+    # dense kernel at the same shape
+    od = torch.empty_like(pipe.out)
+    dst = torch.zeros(1, dtype=torch.int32, device=dev)
+    dense = []
+    for i in range(args.warmup + 5):
+        flush.fill_(1.0)
+        a, b = ev(), ev()
+        a.record(stream)
+        sa.dense_attn(q, k, v, pipe.shape, False, 0.0, od, None, dst, ws=pipe.attn_ws)
+        b.record(stream)
+        if i >= args.warmup:
+            dense.append((a, b))
+    torch.cuda.synchronize(dev)
+    dense_ms = statistics.median(x[0].elapsed_time(x[1]) for x in dense)
+    step_ms, attn_ms = max_over_ranks([step_ms, attn_ms], world, dev)
+    if rank != 0:
+        return None
+    pk, pk_src = peaks()
+    peak_tf = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    attn_tf = flops / (attn_ms * 1e-3) / 1e12
+    n_temporal = sum(1 for c in choice if c == svg.TEMPORAL)
+    return {
+        "metric": "per-head spatial/temporal sparse attn fwd TFLOP/s (kept blocks), video shape, 1xB200",
+        "path": "svg",
+        "value": round(job_tflops(world, flops, step_ms), 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (heads biased to a frame or a position, bf16)",
+        "config": {"workload": f"{w.name} shape: B=1 H={w.Hq} N={w.N} ([{w.T},{w.H},{w.W}]+{w.txt_len} text) "
+                               f"d={w.d} bq={w.bq} bk={w.bk}, per-head spatial/temporal placement",
+                   "global_batch": world, "seq_len": w.N, "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (256 MB write)"},
+        "stages_ms": {"reorder_heads_qkv": round(reorder_ms, 4), "attention_with_per_head_store": round(attn_ms, 4)},
+        "profile_ms": round(profile_ms, 4),
+        "heads_temporal": n_temporal,
+        "heads_spatial": len(choice) - n_temporal,
+        "dense_ms": round(dense_ms, 4),
+        "speedup_vs_dense_whole_step": round(dense_ms / step_ms, 3),
+        "block_sparsity": round(sparsity, 4),
+        "kept_tiles": kept,
+        "roofline": {"bound": "tensor", "achieved": round(attn_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": round(attn_tf / peak_tf, 4), "traffic": None,
+                     "peak_source": f"{pk_src} bf16 dense (burst)", "kernel": "attn_tc_kernel<64>"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+
+
 # ----------------------------------------------------------------------------
 # The oracle on the host cores (CPU baseline and the reference arm)
 # ----------------------------------------------------------------------------
@@ -476,6 +614,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="video")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="sparge", choices=["sparge", "svg"],
+                    help="sparge: the predicted-mask path (the headline); svg: per-head spatial/temporal masks")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-qblocks", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -499,7 +639,7 @@ def main():
             dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                     device_id=torch.device("cuda", local_rank))
         try:
-            res = run_ours(args, rank, world, local_rank)
+            res = (run_svg if args.path == "svg" else run_ours)(args, rank, world, local_rank)
         finally:
             if world > 1:
                 import torch.distributed as dist

@@ -147,6 +147,8 @@ typedef struct {
 /* Flags for the attention entry points. */
 #define SA_FLAG_FORCE_SIMT 1   /* use the portable CUDA-core kernel even where
                                   the tensor-core kernel applies (testing) */
+#define SA_FLAG_OUT_PERM_PER_HEAD 2   /* out_perm is int32 [B*Hq][N], one
+                                         permutation per query head */
 
 /* Library version string and the calling thread's last error message. */
 const char* sa_version(void);
@@ -270,6 +272,49 @@ sa_status sa_dense_attn(const void* q, const void* k, const void* v, const sa_sh
 /* Synchronises `stream` and returns the device status word's code (0 =
  * SA_OK).  The word is not cleared. */
 sa_status sa_read_status(const int32_t* status, void* stream);
+
+/* ---- per-head spatial / temporal placement ([P1] 3.3, 3.4, 4, 5) ---------
+ * The Sparse VideoGen comparison of [P1] section 5.  On a T x H x W video
+ * (P = H*W, nv = T*P frame-major tokens t*P + p, then txt_len text tokens;
+ * N = nv + txt_len) a spatial head keeps the pairs of one frame and a
+ * temporal head the pairs of one position across frames; text tokens pair
+ * with every token.  A spatial head runs in the frame-major order, a
+ * temporal head in the token-major order (place n < nv holds frame n % T of
+ * position n / T; text stays in place), where its pairs fill whole tiles
+ * (the tile ledger of [P1] section 4).
+ *
+ * sa_head_placement, for kinds (device int32 [heads], SA_HEAD_SPATIAL or
+ * SA_HEAD_TEMPORAL):
+ *   perms (device int32 [heads][N], nullable): perms[h][n] = the original
+ *     token at place n of head h's order;
+ *   block_mask (device uint8 [heads][ceil(N/bq)][ceil(N/bk)], nullable): 1
+ *     where the tile of head h's order holds an allowed pair (the block
+ *     cover of the element mask, [P1] section 4); feed it to
+ *     sa_mask_from_blocks.
+ * Another kind value raises SA_ERR_INVALID_ARG in status (device int32,
+ * nullable) and leaves that head's tiles empty.  The usual run: perms and
+ * block_mask from here, Q, K, V through sa_reorder_heads, then
+ * sa_block_sparse_attn with out_perm = perms and SA_FLAG_OUT_PERM_PER_HEAD,
+ * which stores every head back in the original order. */
+#define SA_HEAD_SPATIAL 0
+#define SA_HEAD_TEMPORAL 1
+sa_status sa_head_placement(int64_t T, int64_t H, int64_t W, int64_t txt_len, const int32_t* kinds,
+                            int64_t heads, int32_t bq, int32_t bk, int32_t* perms, uint8_t* block_mask,
+                            int32_t* status, void* stream);
+
+/* y[o, n, :] = x[o, perms[o*N + n], :]: sa_reorder with one permutation per
+ * outer index (x, y [outer, N, row] of dtype; perms device int32
+ * [outer][N], each entry in [0, N)).  x and y must not overlap. */
+sa_status sa_reorder_heads(const int32_t* perms, const void* x, void* y, int64_t outer, int64_t N, int64_t row,
+                           int32_t dtype, void* stream);
+
+/* Sampled-row error of [P1] section 5: out[h] (device double [BH]) = mean of
+ * (ref - x)^2 over the nrows sampled query rows (rows: device int32, each in
+ * [0, N)) and the dv outputs of head h; ref and x are [BH, N, dv] of dtype.
+ * A row outside [0, N) is skipped and raises SA_ERR_INVALID_ARG in status
+ * (device int32, nullable). */
+sa_status sa_rows_mse(const void* ref, const void* x, const int32_t* rows, int64_t nrows, int64_t BH, int64_t N,
+                      int64_t dv, int32_t dtype, double* out, int32_t* status, void* stream);
 
 /* ---- calibration support ([P3] 2.4) ---------------------------------------
  * The per-layer calibration of the SpargeAttention notes bounds the relative

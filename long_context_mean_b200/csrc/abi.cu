@@ -277,6 +277,9 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
   a.out = out;
   a.lse = lse;
   a.out_perm = out_perm;
+  if ((flags & SA_FLAG_OUT_PERM_PER_HEAD) && !out_perm)
+    return set_error(SA_ERR_INVALID_ARG, "SA_FLAG_OUT_PERM_PER_HEAD needs out_perm");
+  a.perm_stride = (flags & SA_FLAG_OUT_PERM_PER_HEAD) ? shape->N : 0;
   if (out_perm && (out == q || out == k || out == v))
     return set_error(SA_ERR_INVALID_ARG, "out must not alias an input when out_perm is given");
   a.skip_log = skip_log;
@@ -366,6 +369,44 @@ sa_status sa_l1_error(const void* ref, const void* x, int64_t n, int32_t dtype, 
     return set_error(SA_ERR_INVALID_ARG, "ref and x must be 16-byte aligned, sums 8-byte aligned");
   if (sa_status e = check_device()) return e;
   return launch_l1(ref, x, n, dtype, sums, static_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_head_placement(int64_t T, int64_t H, int64_t W, int64_t txt_len, const int32_t* kinds,
+                            int64_t heads, int32_t bq, int32_t bk, int32_t* perms, uint8_t* block_mask,
+                            int32_t* status, void* stream) {
+  if (T < 1 || H < 1 || W < 1 || txt_len < 0 || heads < 0)
+    return set_error(SA_ERR_INVALID_ARG, "sa_head_placement: T, H, W >= 1, txt_len and heads >= 0");
+  if (heads > 0 && !kinds) return set_error(SA_ERR_INVALID_ARG, "kinds is NULL");
+  if (block_mask && (bq < 1 || bk < 1 || bq > 128 || bk > 128))
+    return set_error(SA_ERR_INVALID_ARG, "bq, bk must lie in 1..128");
+  const int64_t n = T * H * W + txt_len;
+  if (n > 2147483647) return set_error(SA_ERR_UNSUPPORTED, "sequence too long for int32 orders");
+  if (sa_status e = check_device()) return e;
+  return launch_head_placement(T, H * W, n, kinds, heads, bq, bk, perms, block_mask, status,
+                               static_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_reorder_heads(const int32_t* perms, const void* x, void* y, int64_t outer, int64_t N, int64_t row,
+                           int32_t dtype, void* stream) {
+  if (!perms || !x || !y) return set_error(SA_ERR_INVALID_ARG, "NULL argument to sa_reorder_heads");
+  if (outer <= 0 || N <= 0 || row <= 0) return set_error(SA_ERR_INVALID_ARG, "sizes must be positive");
+  if (dtype != SA_BF16 && dtype != SA_FP32) return set_error(SA_ERR_INVALID_ARG, "unknown dtype");
+  const int64_t bytes = row * elem_size(dtype);
+  if (overlaps(x, y, (size_t)(outer * N * bytes)))
+    return set_error(SA_ERR_INVALID_ARG, "x and y must not overlap");
+  if ((uintptr_t)x % 2 || (uintptr_t)y % 2) return set_error(SA_ERR_INVALID_ARG, "misaligned tensor");
+  if (sa_status e = check_device()) return e;
+  return launch_reorder(perms, x, y, outer, N, bytes, false, static_cast<cudaStream_t>(stream), N);
+}
+
+sa_status sa_rows_mse(const void* ref, const void* x, const int32_t* rows, int64_t nrows, int64_t BH, int64_t N,
+                      int64_t dv, int32_t dtype, double* out, int32_t* status, void* stream) {
+  if (!ref || !x || !out || (nrows > 0 && !rows)) return set_error(SA_ERR_INVALID_ARG, "NULL argument to sa_rows_mse");
+  if (dtype != SA_BF16 && dtype != SA_FP32) return set_error(SA_ERR_INVALID_ARG, "dtype must be SA_BF16 or SA_FP32");
+  if (nrows < 0 || BH < 0 || N < 1 || dv < 1) return set_error(SA_ERR_INVALID_ARG, "bad sizes for sa_rows_mse");
+  if (BH > 2147483647) return set_error(SA_ERR_UNSUPPORTED, "too many heads");
+  if (sa_status e = check_device()) return e;
+  return launch_rows_mse(ref, x, rows, nrows, BH, N, dv, dtype, out, status, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -121,12 +121,12 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
   for (int idx = threadIdx.x; idx < nr * dv; idx += kThreads) {
     const int r = idx / dv, c = idx % dv;
     const float lr = l[r];
-    const int64_t orow = a.out_perm ? a.out_perm[i0 + r] : i0 + r;
+    const int64_t orow = a.out_perm ? a.out_perm[bh * a.perm_stride + i0 + r] : i0 + r;
     Elem<T>::store(out + orow * dv + c, lr > 0.f ? O[idx] / lr : 0.f);
   }
   for (int r = threadIdx.x; r < nr; r += kThreads) {
     if (!(l[r] > 0.f)) raise_status(a.status, SA_ERR_EMPTY_ROW);
-    const int64_t orow = a.out_perm ? a.out_perm[i0 + r] : i0 + r;
+    const int64_t orow = a.out_perm ? a.out_perm[bh * a.perm_stride + i0 + r] : i0 + r;
     if (a.lse) a.lse[bh * a.N + orow] = m[r] + logf(l[r]);
   }
 }

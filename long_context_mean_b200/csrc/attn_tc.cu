@@ -100,6 +100,7 @@ struct TcParams {
   int32_t* status;
   int32_t* counter;      // work counter, zero at launch
   int64_t N, nqb, nkb;
+  int64_t perm_stride;   // 0: one out_perm for every head; N: one per query head
   int32_t Hq, Hkv;
   int32_t num_units;
   int32_t causal;
@@ -625,7 +626,8 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
     mbar_wait(&c->pv_done[gl & 1], (gl >> 1) & 1, g, p.status);
     tc_fence_after();
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    const int64_t out_row = row_valid ? (p.out_perm ? (int64_t)p.out_perm[row_g] : row_g) : 0;
+    const int64_t out_row =
+        row_valid ? (p.out_perm ? (int64_t)p.out_perm[u.bh * p.perm_stride + row_g] : row_g) : 0;
     uint16_t* orow = p.out + (u.bh * p.N + out_row) * 128;
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
@@ -777,6 +779,7 @@ sa_status launch_bk(const AttnArgs& a, cudaStream_t st) {
   p.out = static_cast<uint16_t*>(a.out);
   p.lse = a.lse;
   p.out_perm = a.out_perm;
+  p.perm_stride = a.perm_stride;
   p.skip_log = a.skip_log;
   p.status = a.status;
   p.counter = a.counter;

@@ -162,7 +162,7 @@ int hilbert_bits_for(const sa_layout_desc& d) {
 // UNROLL independent chunk copies in flight.
 // ---------------------------------------------------------------------------
 template <int UNROLL>
-__global__ void __launch_bounds__(256) reorder_vec_kernel(const int32_t* __restrict__ perm,
+__global__ void __launch_bounds__(256) reorder_vec_kernel(const int32_t* __restrict__ perm, int64_t pstride,
                                                           const uint4* __restrict__ src,
                                                           uint4* __restrict__ dst, int64_t outer,
                                                           int64_t N, int64_t cpr, bool scatter) {
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(256) reorder_vec_kernel(const int32_t* __restr
         const int64_t row = i / cpr;
         const int64_t n = row % N;
         const int64_t o = row / N;
-        const int64_t pn = __ldg(perm + n);
+        const int64_t pn = __ldg(perm + o * pstride + n);
         const int64_t s_row = scatter ? row : o * N + pn;
         const int64_t d_row = scatter ? o * N + pn : row;
         v[u] = __ldg(src + s_row * cpr + c);
@@ -194,7 +194,8 @@ __global__ void __launch_bounds__(256) reorder_vec_kernel(const int32_t* __restr
   }
 }
 
-__global__ void reorder_word_kernel(const int32_t* __restrict__ perm, const uint32_t* __restrict__ src,
+__global__ void reorder_word_kernel(const int32_t* __restrict__ perm, int64_t pstride,
+                                    const uint32_t* __restrict__ src,
                                     uint32_t* __restrict__ dst, int64_t outer, int64_t N,
                                     int64_t wpr, bool scatter) {
   const int64_t total = outer * N * wpr;
@@ -204,14 +205,15 @@ __global__ void reorder_word_kernel(const int32_t* __restrict__ perm, const uint
     const int64_t row = i / wpr;
     const int64_t n = row % N;
     const int64_t o = row / N;
-    const int64_t pn = __ldg(perm + n);
+    const int64_t pn = __ldg(perm + o * pstride + n);
     const int64_t s_row = scatter ? row : o * N + pn;
     const int64_t d_row = scatter ? o * N + pn : row;
     dst[d_row * wpr + c] = __ldg(src + s_row * wpr + c);
   }
 }
 
-__global__ void reorder_half_kernel(const int32_t* __restrict__ perm, const uint16_t* __restrict__ src,
+__global__ void reorder_half_kernel(const int32_t* __restrict__ perm, int64_t pstride,
+                                    const uint16_t* __restrict__ src,
                                     uint16_t* __restrict__ dst, int64_t outer, int64_t N,
                                     int64_t hpr, bool scatter) {
   const int64_t total = outer * N * hpr;
@@ -221,7 +223,7 @@ __global__ void reorder_half_kernel(const int32_t* __restrict__ perm, const uint
     const int64_t row = i / hpr;
     const int64_t n = row % N;
     const int64_t o = row / N;
-    const int64_t pn = __ldg(perm + n);
+    const int64_t pn = __ldg(perm + o * pstride + n);
     const int64_t s_row = scatter ? row : o * N + pn;
     const int64_t d_row = scatter ? o * N + pn : row;
     dst[d_row * hpr + c] = __ldg(src + s_row * hpr + c);
@@ -279,7 +281,7 @@ sa_status launch_layout(const sa_layout_desc& d, int32_t* perm, int32_t* inv, vo
 }
 
 sa_status launch_reorder(const int32_t* perm, const void* src, void* dst, int64_t outer,
-                         int64_t N, int64_t row_bytes, bool scatter, cudaStream_t st) {
+                         int64_t N, int64_t row_bytes, bool scatter, cudaStream_t st, int64_t pstride) {
   const int threads = 256;
   const bool aligned16 = ((uintptr_t)src % 16 == 0) && ((uintptr_t)dst % 16 == 0);
   if (row_bytes % 16 == 0 && aligned16) {
@@ -287,19 +289,19 @@ sa_status launch_reorder(const int32_t* perm, const void* src, void* dst, int64_
     const int64_t total = outer * N * cpr;
     constexpr int U = 4;
     reorder_vec_kernel<U><<<grid_for(ceil_div(total, U), threads), threads, 0, st>>>(
-        perm, static_cast<const uint4*>(src), static_cast<uint4*>(dst), outer, N, cpr, scatter);
+        perm, pstride, static_cast<const uint4*>(src), static_cast<uint4*>(dst), outer, N, cpr, scatter);
     return check_launch("reorder_vec_kernel");
   }
   if (row_bytes % 4 == 0 && (uintptr_t)src % 4 == 0 && (uintptr_t)dst % 4 == 0) {
     const int64_t wpr = row_bytes / 4;
     reorder_word_kernel<<<grid_for(outer * N * wpr, threads), threads, 0, st>>>(
-        perm, static_cast<const uint32_t*>(src), static_cast<uint32_t*>(dst), outer, N, wpr,
+        perm, pstride, static_cast<const uint32_t*>(src), static_cast<uint32_t*>(dst), outer, N, wpr,
         scatter);
     return check_launch("reorder_word_kernel");
   }
   const int64_t hpr = row_bytes / 2;
   reorder_half_kernel<<<grid_for(outer * N * hpr, threads), threads, 0, st>>>(
-      perm, static_cast<const uint16_t*>(src), static_cast<uint16_t*>(dst), outer, N, hpr,
+      perm, pstride, static_cast<const uint16_t*>(src), static_cast<uint16_t*>(dst), outer, N, hpr,
       scatter);
   return check_launch("reorder_half_kernel");
 }

@@ -71,8 +71,9 @@ sa_status launch_layout(const sa_layout_desc& d, int32_t* perm, int32_t* inv, vo
                         cudaStream_t st);
 size_t layout_ws_bytes(const sa_layout_desc& d);
 
+// pstride: 0 = one perm for every outer index; N = perm[o * N + n], one per outer index.
 sa_status launch_reorder(const int32_t* perm, const void* src, void* dst, int64_t outer,
-                         int64_t N, int64_t row_bytes, bool scatter, cudaStream_t st);
+                         int64_t N, int64_t row_bytes, bool scatter, cudaStream_t st, int64_t pstride = 0);
 
 struct PredictWs {
   float* qhat;     // [B*Hq, nqb, d]
@@ -103,6 +104,7 @@ struct AttnArgs {
   void* out;
   float* lse;
   const int32_t* out_perm;  // nullptr = rows stored in place
+  int64_t perm_stride;      // 0: out_perm shared by all heads; N: out_perm[bh * N + n]
   uint8_t* skip_log;
   const int32_t* row_ptr;   // nullptr = dense (every causally valid block)
   const int32_t* col_idx;
@@ -117,6 +119,10 @@ struct AttnArgs {
   float lambda;
 };
 sa_status launch_attn_simt(const AttnArgs& a, cudaStream_t st);
+sa_status launch_head_placement(int64_t T, int64_t P, int64_t n, const int32_t* kinds, int64_t heads, int bq,
+                                int bk, int32_t* perms, uint8_t* mask, int32_t* status, cudaStream_t st);
+sa_status launch_rows_mse(const void* ref, const void* x, const int32_t* rows, int64_t nrows, int64_t BH, int64_t N,
+                          int64_t dv, int32_t dtype, double* out, int32_t* status, cudaStream_t st);
 sa_status launch_l1(const void* ref, const void* x, int64_t n, int32_t dtype, double* sums, cudaStream_t st);
 sa_status launch_attn_tc(const AttnArgs& a, cudaStream_t st);
 bool attn_tc_supported(const sa_shape& s, int bq, int bk);

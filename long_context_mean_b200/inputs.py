@@ -255,6 +255,39 @@ def worked_example_inputs():
     return {"q": q, "k": q.copy(), "v": v, "frame": frame, "pixel": pixel, "T": T, "P": P}
 
 
+def biased_video_heads(T, H, W, txt_len, bias, d=128, dv=128, seed=0, amp=15.0, noise=0.15):
+    """Heads biased to one frame or to one position, the worked example's
+    construction carried to any grid and head width: head h gets
+    q = k = amp * code[g(i)] + N(0, noise^2) on video token i, where g is the
+    frame ("frame" bias) or the position ("position" bias) of the token and
+    the codes are random unit vectors of R^d (one per frame or position);
+    text tokens get noise only; v ~ N(0, 1).  bias: one "frame"/"position"
+    per head.  Returns float32 [1, heads, N, d|dv] arrays, bf16-rounded, and
+    their bit patterns (q_bits, k_bits, v_bits)."""
+    P = H * W
+    nv = T * P
+    n = nv + txt_len
+    frame = np.repeat(np.arange(T), P)
+    pixel = np.tile(np.arange(P), T)
+    q = np.empty((1, len(bias), n, d), dtype=np.float32)
+    v = np.empty((1, len(bias), n, dv), dtype=np.float32)
+    for h, kind in enumerate(bias):
+        rng = np.random.default_rng(np.random.SeedSequence([seed, 7919, h]))
+        groups = T if kind == "frame" else P
+        codes = rng.standard_normal((groups, d))
+        codes /= np.linalg.norm(codes, axis=1, keepdims=True)
+        x = noise * rng.standard_normal((n, d))
+        x[:nv] += amp * codes[frame if kind == "frame" else pixel]
+        q[0, h] = x
+        v[0, h] = rng.standard_normal((n, dv))
+    out = {}
+    for name, arr in (("q", q), ("k", q.copy()), ("v", v)):
+        bits = to_bf16_bits(arr)
+        out[name + "_bits"] = bits
+        out[name] = bf16_bits_to_f32(bits)
+    return out
+
+
 def two_key_inputs():
     """q = [1], keys [ln 99, 0], values [0, 100]: probabilities 0.99 / 0.01."""
     return {"q": np.array([[1.0]]), "k": np.array([[math.log(99.0)], [0.0]]),

@@ -34,7 +34,8 @@ EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_attn_worksp
            "sa_layout_build", "sa_reorder", "sa_unreorder", "sa_predict_mask_workspace",
            "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_reorder_predict_mask", "sa_predict_mask_noalloc",
            "sa_mask_from_blocks_workspace",
-           "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status", "sa_l1_error"]
+           "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status", "sa_l1_error",
+           "sa_head_placement", "sa_reorder_heads", "sa_rows_mse"]
 
 
 class SAError(RuntimeError):
@@ -107,6 +108,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                       ctypes.POINTER(Mask), P]),
         "sa_attn_workspace": (SZ, []),
         "sa_l1_error": (I32, [P, P, I64, I32, P, P]),
+        "sa_head_placement": (I32, [I64, I64, I64, I64, P, I64, I32, I32, P, P, P, P]),
+        "sa_reorder_heads": (I32, [P, P, P, I64, I64, I64, I32, P]),
+        "sa_rows_mse": (I32, [P, P, P, I64, I64, I64, I64, I32, P, P, P]),
         "sa_block_sparse_attn": (I32, [P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F, F,
                                        P, P, P, P, P, SZ, I32, P]),
         "sa_dense_attn": (I32, [P, P, P, ctypes.POINTER(Shape), I32, F, P, P, P, P, SZ, I32, P]),
@@ -274,6 +278,35 @@ def l1_error(ref, x, sums, stream=None):
     """Enqueue sums[0] = sum |ref - x|, sums[1] = sum |ref| (sums: float64
     device tensor of 2)."""
     _check(load().sa_l1_error(_ptr(ref), _ptr(x), ref.numel(), dtype_code(ref), _ptr(sums), _stream(stream)))
+
+
+SA_HEAD_SPATIAL, SA_HEAD_TEMPORAL = 0, 1
+
+
+SA_FLAG_OUT_PERM_PER_HEAD = 2
+
+
+def head_placement(T, H, W, txt_len, kinds, bq, bk, perms=None, block_mask=None, status=None, stream=None):
+    """Per-head orders (perms [heads, N]) and tile covers (block_mask) of the
+    spatial / temporal candidates; kinds: int32 device tensor [heads]."""
+    _check(load().sa_head_placement(T, H, W, txt_len, _ptr(kinds), kinds.numel(), bq, bk, _ptr(perms),
+                                    _ptr(block_mask), _ptr(status), _stream(stream)))
+
+
+def reorder_heads(perms, x, y, stream=None):
+    """y[o, n, :] = x[o, perms[o, n], :] for x of shape [..., N, row]."""
+    N, row = x.shape[-2], x.shape[-1]
+    outer = x.numel() // (N * row)
+    _check(load().sa_reorder_heads(_ptr(perms), _ptr(x), _ptr(y), outer, N, row, dtype_code(x), _stream(stream)))
+
+
+def rows_mse(ref, x, rows, out, status=None, stream=None):
+    """out[h] = mean (ref - x)^2 over the sampled rows of head h; ref/x
+    [..., N, dv] device tensors, rows int32 device tensor, out float64 [BH]."""
+    N, dv = ref.shape[-2], ref.shape[-1]
+    BH = ref.numel() // (N * dv)
+    _check(load().sa_rows_mse(_ptr(ref), _ptr(x), _ptr(rows), rows.numel(), BH, N, dv, dtype_code(ref), _ptr(out),
+                              _ptr(status), _stream(stream)))
 
 
 def read_status(status, stream=None) -> int:

@@ -49,17 +49,22 @@ from . import attention as A
 SPATIAL, TEMPORAL = 0, 1
 
 
-def element_mask(T: int, H: int, W: int, txt_len: int, kind: int) -> np.ndarray:
-    """bool [N, N] over the frame-major order, N = T*H*W + txt_len."""
+def element_mask_rows(T: int, H: int, W: int, txt_len: int, kind: int, rows) -> np.ndarray:
+    """Rows ``rows`` (original token indices) of the element mask: bool
+    [len(rows), N] over the frame-major order, N = T*H*W + txt_len."""
     P = H * W
     nv = T * P
     n = nv + txt_len
-    frame = np.repeat(np.arange(T), P)
-    pixel = np.tile(np.arange(P), T)
-    key = frame if kind == SPATIAL else pixel
-    m = np.ones((n, n), dtype=bool)
-    m[:nv, :nv] = key[:, None] == key[None, :]
-    return m
+    rows = np.asarray(rows, dtype=np.int64)
+    group = np.full(n, -1, dtype=np.int64)           # -1: a text token
+    group[:nv] = np.repeat(np.arange(T), P) if kind == SPATIAL else np.tile(np.arange(P), T)
+    gr = group[rows]
+    return (gr[:, None] == group[None, :]) | (gr[:, None] < 0) | (group[None, :] < 0)
+
+
+def element_mask(T: int, H: int, W: int, txt_len: int, kind: int) -> np.ndarray:
+    """bool [N, N] over the frame-major order, N = T*H*W + txt_len."""
+    return element_mask_rows(T, H, W, txt_len, kind, np.arange(T * H * W + txt_len))
 
 
 def token_major_perm(T: int, H: int, W: int, txt_len: int) -> np.ndarray:

@@ -113,6 +113,19 @@ def test_host_validation_codes(lib):
                              0, null) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_read_status(null, null) == sa.SA_ERR_INVALID_ARG
     assert b"status" in lib.sa_last_error()
+    # per-head placement, per-head reorder, sampled-row error
+    assert lib.sa_head_placement(0, 2, 2, 0, FAKE, 2, 4, 4, FAKE, FAKE, null, null) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_head_placement(2, 2, 2, 0, null, 2, 4, 4, FAKE, FAKE, null, null) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_head_placement(2, 2, 2, 0, FAKE, 2, 0, 4, FAKE, FAKE, null, null) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_reorder_heads(FAKE, FAKE, ctypes.c_void_p(4096 + 64), 2, 10, 8, 0, null) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_reorder_heads(null, FAKE, ctypes.c_void_p(1 << 20), 2, 10, 8, 0, null) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_rows_mse(FAKE, FAKE, FAKE, 4, 2, 10, 8, 7, FAKE, null, null) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_rows_mse(FAKE, FAKE, null, 4, 2, 10, 8, 0, FAKE, null, null) == sa.SA_ERR_INVALID_ARG
+    # a per-head output permutation needs out_perm
+    m2.nqb = 3
+    assert lib.sa_block_sparse_attn(FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m2), ctypes.c_float(-1),
+                                    ctypes.c_float(0), FAKE, null, null, null, WS, 256,
+                                    sa.SA_FLAG_OUT_PERM_PER_HEAD, null) == sa.SA_ERR_INVALID_ARG
 
 
 def test_workspace_queries_are_host_only(lib):
