@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch of the attention kernel from the ncu capture recorded
 # in profiles/attn_tc_video.md, keyed by the sha1 of the kernel code it was
 # taken on (src_sha1); any other code reports null.
-TRAFFIC = {("ddf27a4b26825447a86d20e705ba53ea13f6274b", "video"): 1.2216e9}
+TRAFFIC = {("f0b51a04784cb91ddfcc4d14d72a7a39a094f8c2", "video"): 1.2127e9}
 
 
 def peaks():
@@ -199,7 +199,7 @@ def run_ours(args, rank, world, local_rank):
     host = {n: torch.from_numpy(g[n + "_bits"].view(np.int16)).view(torch.bfloat16).pin_memory() for n in "qkv"}
     q, k, v = (host[n].to(dev) for n in "qkv")
     stream = torch.cuda.current_stream(dev)
-    pipe = sa.pipeline_for(w, device=dev, log_skips=True)
+    pipe = sa.pipeline_for(w, device=dev, log_skips=True, qk8=args.qk8)
 
     # Calibration pass (untimed): mask, skip log, FLOPs, sparsity.
     pipe.run(q, k, v)
@@ -245,20 +245,33 @@ def run_ours(args, rank, world, local_rank):
             # mask prediction with the reorder of Q and K fused into its pooling pass
             sa.reorder_predict_mask(pipe.perm, q, k, pipe.qr, pipe.kr, pipe.shape, pipe.params, pipe.ws,
                                     pipe.mask.struct)
+            if args.qk8:   # per-block INT8 codes of Q and K, beside the V reorder
+                sa.quantize_blocks(pipe.qr, w.bq, pipe.q8, pipe.q_scales)
+                sa.quantize_blocks(pipe.kr, w.bk, pipe.k8, pipe.k_scales)
             stream.wait_event(pipe.ev_v)
             qr, kr, vr = pipe.qr, pipe.kr, pipe.vr
         else:
             qr, kr, vr = q, k, v
             sa.predict_mask(qr, kr, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
+            if args.qk8:
+                sa.quantize_blocks(qr, w.bq, pipe.q8, pipe.q_scales)
+                sa.quantize_blocks(kr, w.bk, pipe.k8, pipe.k_scales)
         e[1].record(stream)
         # attention with the inverse reorder of O and LSE fused into its store
-        sa.block_sparse_attn(qr, kr, vr, pipe.shape, pipe.mask.struct, pipe.lam, pipe.scale, pipe.out, pipe.lse,
-                             ws=pipe.attn_ws, out_perm=None if pipe.identity else pipe.perm)
+        if args.qk8:
+            sa.block_sparse_attn_qk8(pipe.q8, pipe.q_scales, pipe.k8, pipe.k_scales, vr, pipe.shape,
+                                     pipe.mask.struct, pipe.lam, pipe.scale, pipe.out, pipe.attn_ws, pipe.lse,
+                                     out_perm=None if pipe.identity else pipe.perm)
+        else:
+            sa.block_sparse_attn(qr, kr, vr, pipe.shape, pipe.mask.struct, pipe.lam, pipe.scale, pipe.out,
+                                 pipe.lse, ws=pipe.attn_ws, out_perm=None if pipe.identity else pipe.perm)
         e[2].record(stream)
         return e
 
     # layout (1, Hilbert 3) + reorder V; pool Q, pool K, score, row scan, column fill, order; attention
     launches_per_step = (0 if pipe.identity else (1 if w.order != "hilbert" else 3) + 1) + 6 + 1
+    if args.qk8:
+        launches_per_step += 3            # two quantisation passes and the tile-scale kernel
 
     for _ in range(args.warmup):
         l2_flush()
@@ -296,11 +309,12 @@ def run_ours(args, rank, world, local_rank):
     dst = torch.zeros(1, dtype=torch.int32, device=dev)
     qr, kr, vr = (pipe.qr, pipe.kr, pipe.vr) if not pipe.identity else (q, k, v)
     dense = []
+    dense_ws = sa.workspace(sa.attn_workspace(), dev)
     for i in range(args.warmup + max(3, min(args.steps, 10))):
         l2_flush()
         a, b = ev(), ev()
         a.record(stream)
-        sa.dense_attn(qr, kr, vr, pipe.shape, w.causal, 0.0, od, ld, dst, ws=pipe.attn_ws)
+        sa.dense_attn(qr, kr, vr, pipe.shape, w.causal, 0.0, od, ld, dst, ws=dense_ws)
         b.record(stream)
         if i >= args.warmup:
             dense.append((a, b))
@@ -312,26 +326,28 @@ def run_ours(args, rank, world, local_rank):
     # so the copies of one chunk overlap the kernels of the others.
     out_host = torch.empty(pipe.out.shape, dtype=pipe.out.dtype).pin_memory()
     lse_host = torch.empty(pipe.lse.shape, dtype=pipe.lse.dtype).pin_memory()
-    hp = sa.host_pipeline_for(w, device=dev, chunks=args.e2e_chunks)
+    e2e_ms = float("nan")
+    if not args.qk8:   # the host-buffer pass runs the bf16 path
+        hp = sa.host_pipeline_for(w, device=dev, chunks=args.e2e_chunks)
 
-    def e2e_step():
-        hp.run(host["q"], host["k"], host["v"], out_host, lse_host, stream)
+        def e2e_step():
+            hp.run(host["q"], host["k"], host["v"], out_host, lse_host, stream)
 
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    e2e = []
-    for _ in range(args.steps):
-        l2_flush()
-        a, b = ev(), ev()
-        a.record(stream)
-        e2e_step()
-        b.record(stream)
-        e2e.append((a, b))
-    torch.cuda.synchronize(dev)
-    if hp.status() != sa.SA_OK:
-        raise RuntimeError("device status after the end-to-end passes")
-    e2e_ms = sum(x[0].elapsed_time(x[1]) for x in e2e) / len(e2e)
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e2e = []
+        for _ in range(args.steps):
+            l2_flush()
+            a, b = ev(), ev()
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+            e2e.append((a, b))
+        torch.cuda.synchronize(dev)
+        if hp.status() != sa.SA_OK:
+            raise RuntimeError("device status after the end-to-end passes")
+        e2e_ms = sum(x[0].elapsed_time(x[1]) for x in e2e) / len(e2e)
     h2d = sum(host[n].numel() * host[n].element_size() for n in "qkv")
     d2h = out_host.numel() * out_host.element_size() + lse_host.numel() * lse_host.element_size()
 
@@ -343,9 +359,15 @@ def run_ours(args, rank, world, local_rank):
 
     pk, pk_src = peaks()
     peak_tf = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_src = f"{pk_src} bf16 dense (burst)"
+    if args.qk8:
+        # QK at the int8 rate (the nominal int8 / bf16 ratio 2 on the measured
+        # bf16 peak), PV at the bf16 rate: the peak of the mixed contraction.
+        peak_tf = flops / (qk_flops / (2 * peak_tf) + pv_flops / peak_tf)
+        peak_src = f"{pk_src} bf16 (burst) x nominal int8/bf16 ratio 2 on the QK half"
     attn_tf = flops / (attn_mean * 1e-3) / 1e12
     sha = src_sha1("attn_tc.cu")
-    traffic = TRAFFIC.get((sha, args.workload))
+    traffic = None if args.qk8 else TRAFFIC.get((sha, args.workload))
     res = {
         "metric": METRIC,
         "value": round(job_tflops(world, flops, mean_ms), 3),
@@ -357,7 +379,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16, QK int8 per block" if args.qk8 else "bf16",
         "data": "synthetic (seeded smooth-field generator, bf16)",
         "config": workload_config(w, world),
         "stages_ms": {"layout_reorder_predict": round(statistics.mean(pre_ms), 4),
@@ -371,17 +393,21 @@ def run_ours(args, rank, world, local_rank):
         "kept_tiles": kept,
         "pv_skipped_tiles": pv_skipped,
         "flops_per_step": {"qk": qk_flops, "pv": pv_flops},
-        "roofline": {"bound": "tensor", "achieved": round(attn_tf, 2), "peak": peak_tf,
+        "roofline": {"bound": "tensor", "achieved": round(attn_tf, 2), "peak": round(peak_tf, 1),
                      "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4), "traffic": traffic,
-                     "peak_source": f"{pk_src} bf16 dense (burst)", "kernel": "attn_tc_kernel<64>"},
-        "e2e": {"value": round(job_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
-                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "chunks": args.e2e_chunks},
+                     "peak_source": peak_src,
+                     "kernel": "attn_tc_kernel<64, int8 QK>" if args.qk8 else "attn_tc_kernel<64>"},
+        "e2e": None if args.qk8 else {
+            "value": round(job_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
+            "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "chunks": args.e2e_chunks},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "wall_s": round(wall, 3),
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if args.qk8:
+        res["qk"] = "int8, per-block scales (Q per query block, K per key block); P, V bf16"
+    if world == 1 and not args.no_cpu_baseline and not args.qk8:
         res["cpu_baseline"] = cpu_baseline(w, g, seconds=args.cpu_seconds)
     return res
 
@@ -614,6 +640,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="video")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--qk8", action="store_true",
+                    help="the predicted-mask path with INT8 QK (per-block quantised Q and K)")
     ap.add_argument("--path", default="sparge", choices=["sparge", "svg"],
                     help="sparge: the predicted-mask path (the headline); svg: per-head spatial/temporal masks")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

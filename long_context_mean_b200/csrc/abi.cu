@@ -257,16 +257,21 @@ sa_status sa_mask_from_blocks(const uint8_t* block_mask, const sa_shape* shape, 
                                  static_cast<cudaStream_t>(stream));
 }
 
+struct Qk8Args {
+  const float* q_scales;   // [B*Hq][nqb]
+  const float* k_scales;   // [B*Hkv][nkb]
+};
+
 static sa_status attn_common(const void* q, const void* k, const void* v, const sa_shape* shape,
                              const sa_mask* mask, int32_t causal, float lambda, float scale, void* out,
                              float* lse, const int32_t* out_perm, uint8_t* skip_log, int32_t* status,
                              void* ws, size_t ws_bytes,
-                             int32_t flags, void* stream) {
+                             int32_t flags, void* stream, const Qk8Args* qk8 = nullptr) {
   if (sa_status e = check_shape(shape)) return e;
   if (!q || !k || !v || !out) return set_error(SA_ERR_INVALID_ARG, "NULL tensor argument");
-  if (!ws || ws_bytes < sa_attn_workspace() || (uintptr_t)ws % 256)
-    return set_error(SA_ERR_WORKSPACE, "attention needs %zu bytes of 256-byte aligned workspace",
-                     sa_attn_workspace());
+  const size_t ws_need = qk8 ? sa_attn_qk8_workspace(mask) : sa_attn_workspace();
+  if (!ws || ws_bytes < ws_need || (uintptr_t)ws % 256)
+    return set_error(SA_ERR_WORKSPACE, "attention needs %zu bytes of 256-byte aligned workspace", ws_need);
   if (std::isnan(lambda) || lambda > 0.f)
     return set_error(SA_ERR_INVALID_ARG, "lambda must be <= 0 (or -INFINITY to disable the PV skip)");
   if (!(scale >= 0.f) || std::isinf(scale)) return set_error(SA_ERR_INVALID_ARG, "scale must be finite and >= 0");
@@ -310,6 +315,25 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
     a.causal = causal;
   }
   const bool tc_ok = !(flags & SA_FLAG_FORCE_SIMT) && is_sm100();
+  if (qk8) {
+    // INT8 QK runs on the tensor-core kernel only: there is no other path.
+    if (!qk8->q_scales || !qk8->k_scales) return set_error(SA_ERR_INVALID_ARG, "NULL scale array");
+    if (!(shape->dtype == SA_BF16 && shape->d == 128 && shape->dv == 128 && a.bq == 128 &&
+          (a.bk == 64 || a.bk == 128)))
+      return set_error(SA_ERR_UNSUPPORTED, "INT8 QK needs bf16 V, d = dv = 128, bq = 128, bk in {64, 128}");
+    if (flags & SA_FLAG_FORCE_SIMT) return set_error(SA_ERR_UNSUPPORTED, "INT8 QK has no CUDA-core kernel");
+    a.nqb = ceil_div(a.N, a.bq);
+    a.nkb = ceil_div(a.N, a.bk);
+    if (sa_status e = check_device()) return e;
+    if (!tc_ok) return set_error(SA_ERR_UNSUPPORTED, "INT8 QK needs an sm_100 device");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* ts = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
+    if (sa_status e = launch_tile_scales(*mask, a.B, a.Hq, a.Hkv, qk8->q_scales, qk8->k_scales,
+                                         a.scale * 1.4426950408889634f, ts, st))
+      return e;
+    a.tile_scale = ts;
+    return launch_attn_tc(a, st);
+  }
   if (!mask) {
     if (tc_ok && attn_tc_supported(*shape, 128, 64)) {
       a.bq = 128;
@@ -336,6 +360,36 @@ sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v, cons
   if (!mask) return set_error(SA_ERR_INVALID_ARG, "mask is NULL");
   return attn_common(q, k, v, shape, mask, 0, lambda, scale, out, lse, out_perm, pv_skip_log, nullptr, ws,
                      ws_bytes, flags, stream);
+}
+
+size_t sa_attn_qk8_workspace(const sa_mask* mask) {
+  if (!mask || mask->col_capacity < 0) return 0;
+  return 256 + align_up((size_t)mask->col_capacity * sizeof(float), 256);
+}
+
+sa_status sa_quantize_blocks(const void* x, int64_t heads, int64_t N, int64_t d, int32_t rows, int32_t dtype,
+                             int8_t* x8, float* scales, void* stream) {
+  if (!x || !x8 || !scales) return set_error(SA_ERR_INVALID_ARG, "NULL argument to sa_quantize_blocks");
+  if (heads < 0 || N < 1 || d < 1 || rows < 1) return set_error(SA_ERR_INVALID_ARG, "bad sizes for sa_quantize_blocks");
+  if (dtype != SA_BF16) return set_error(SA_ERR_UNSUPPORTED, "sa_quantize_blocks takes bf16 input");
+  if (!quant_blocks_fits(d, rows))
+    return set_error(SA_ERR_UNSUPPORTED, "sa_quantize_blocks needs d a multiple of 8 and rows * d <= 16384");
+  if ((uintptr_t)x % 16 || (uintptr_t)x8 % 8 || (uintptr_t)scales % 4)
+    return set_error(SA_ERR_INVALID_ARG, "misaligned tensor (x 16 bytes, x8 8 bytes)");
+  if (sa_status e = check_device()) return e;
+  return launch_quant_blocks(x, heads, N, d, rows, x8, scales, static_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_block_sparse_attn_qk8(const int8_t* q8, const float* q_scales, const int8_t* k8, const float* k_scales,
+                                   const void* v, const sa_shape* shape, const sa_mask* mask, float lambda,
+                                   float scale, void* out, float* lse, const int32_t* out_perm,
+                                   uint8_t* pv_skip_log, void* ws, size_t ws_bytes, int32_t flags, void* stream) {
+  if (!mask) return set_error(SA_ERR_INVALID_ARG, "mask is NULL");
+  if ((uintptr_t)q8 % 16 || (uintptr_t)k8 % 16 || (uintptr_t)v % 16 || (uintptr_t)out % 16)
+    return set_error(SA_ERR_INVALID_ARG, "INT8 QK needs 16-byte aligned q8, k8, v, out");
+  const Qk8Args qk8{q_scales, k_scales};
+  return attn_common(q8, k8, v, shape, mask, 0, lambda, scale, out, lse, out_perm, pv_skip_log, nullptr, ws,
+                     ws_bytes, flags, stream, &qk8);
 }
 
 sa_status sa_dense_attn(const void* q, const void* k, const void* v, const sa_shape* shape, int32_t causal,

@@ -35,7 +35,8 @@ EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_attn_worksp
            "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_reorder_predict_mask", "sa_predict_mask_noalloc",
            "sa_mask_from_blocks_workspace",
            "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status", "sa_l1_error",
-           "sa_head_placement", "sa_reorder_heads", "sa_rows_mse"]
+           "sa_head_placement", "sa_reorder_heads", "sa_rows_mse",
+           "sa_quantize_blocks", "sa_attn_qk8_workspace", "sa_block_sparse_attn_qk8"]
 
 
 class SAError(RuntimeError):
@@ -110,6 +111,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sa_l1_error": (I32, [P, P, I64, I32, P, P]),
         "sa_head_placement": (I32, [I64, I64, I64, I64, P, I64, I32, I32, P, P, P, P]),
         "sa_reorder_heads": (I32, [P, P, P, I64, I64, I64, I32, P]),
+        "sa_quantize_blocks": (I32, [P, I64, I64, I64, I32, I32, P, P, P]),
+        "sa_attn_qk8_workspace": (SZ, [ctypes.POINTER(Mask)]),
+        "sa_block_sparse_attn_qk8": (I32, [P, P, P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F, F,
+                                           P, P, P, P, P, SZ, I32, P]),
         "sa_rows_mse": (I32, [P, P, P, I64, I64, I64, I64, I32, P, P, P]),
         "sa_block_sparse_attn": (I32, [P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F, F,
                                        P, P, P, P, P, SZ, I32, P]),
@@ -266,6 +271,27 @@ def block_sparse_attn(q, k, v, shape: Shape, mask: Mask, lam, scale, out, lse=No
                                        _stream(stream)))
 
 
+def quantize_blocks(x, rows, x8, scales, stream=None):
+    """Per-block INT8 codes x8 and scales of a bf16 [..., N, d] tensor, one
+    scale per `rows` tokens of each head."""
+    N, d = x.shape[-2], x.shape[-1]
+    heads = x.numel() // (N * d)
+    _check(load().sa_quantize_blocks(_ptr(x), heads, N, d, rows, dtype_code(x), _ptr(x8), _ptr(scales),
+                                     _stream(stream)))
+
+
+def attn_qk8_workspace(mask: Mask) -> int:
+    return int(load().sa_attn_qk8_workspace(ctypes.byref(mask)))
+
+
+def block_sparse_attn_qk8(q8, q_scales, k8, k_scales, v, shape: Shape, mask: Mask, lam, scale, out, ws, lse=None,
+                          skip_log=None, flags=0, stream=None, out_perm=None):
+    _check(load().sa_block_sparse_attn_qk8(_ptr(q8), _ptr(q_scales), _ptr(k8), _ptr(k_scales), _ptr(v),
+                                           ctypes.byref(shape), ctypes.byref(mask), float(lam), float(scale),
+                                           _ptr(out), _ptr(lse), _ptr(out_perm), _ptr(skip_log), _ptr(ws),
+                                           ws.numel() * ws.element_size(), int(flags), _stream(stream)))
+
+
 def dense_attn(q, k, v, shape: Shape, causal, scale, out, lse=None, status=None, flags=0, stream=None,
                ws=None):
     ws = ws if ws is not None else _default_attn_ws(q.device)
@@ -363,7 +389,7 @@ class Pipeline:
     """
 
     def __init__(self, B, Hq, Hkv, N, d, dv, dtype, *, layout: LayoutDesc, params: MaskParams,
-                 lam=-math.inf, scale=0.0, flags=0, device="cuda", log_skips=False):
+                 lam=-math.inf, scale=0.0, flags=0, device="cuda", log_skips=False, qk8=False):
         import torch
         tdt = torch.bfloat16 if dtype in ("bf16", SA_BF16) else torch.float32
         self.shape = Shape(B, Hq, Hkv, N, d, dv, SA_BF16 if tdt == torch.bfloat16 else SA_FP32, 0)
@@ -380,8 +406,19 @@ class Pipeline:
         self.out = torch.empty(B, Hq, N, dv, dtype=tdt, device=device)
         self.lse = torch.empty(B, Hq, N, 1, dtype=torch.float32, device=device)
         self.ws = workspace(predict_mask_workspace(self.shape, params), device)
-        self.attn_ws = workspace(attn_workspace(), device)
         self.mask = MaskBuffers.allocate(B, Hq, N, params.bq, params.bk, device)
+        # INT8 QK ([P3] 2.4): Q and K quantised per query / key block after
+        # the prediction, the attention on the codes.
+        self.qk8 = qk8
+        if qk8:
+            nqb, nkb = self.mask.struct.nqb, self.mask.struct.nkb
+            self.q8 = torch.empty(B, Hq, N, d, dtype=torch.int8, device=device)
+            self.k8 = torch.empty(B, Hkv, N, d, dtype=torch.int8, device=device)
+            self.q_scales = torch.empty(B * Hq * nqb, dtype=torch.float32, device=device)
+            self.k_scales = torch.empty(B * Hkv * nkb, dtype=torch.float32, device=device)
+            self.attn_ws = workspace(attn_qk8_workspace(self.mask.struct), device)
+        else:
+            self.attn_ws = workspace(attn_workspace(), device)
         self.skip_log = (torch.zeros(self.mask.col_idx.numel(), dtype=torch.uint8, device=device)
                          if log_skips else None)
         if not self.identity:
@@ -401,6 +438,8 @@ class Pipeline:
         if self.identity:
             qr, kr, vr = q, k, v
             predict_mask(qr, kr, self.shape, self.params, self.ws, self.mask.struct, stream)
+            if self.qk8:
+                self._quantize(qr, kr, stream)
         else:
             import torch
             st = stream if stream is not None else torch.cuda.current_stream(q.device)
@@ -415,15 +454,26 @@ class Pipeline:
             # Q and K are reordered by the pooling pass of the prediction.
             reorder_predict_mask(self.perm, q, k, self.qr, self.kr, self.shape, self.params, self.ws,
                                  self.mask.struct, st)
+            if self.qk8:   # beside the V reorder, which needs no codes
+                self._quantize(self.qr, self.kr, st)
             st.wait_event(self.ev_v)
             stream = st
             qr, kr, vr = self.qr, self.kr, self.vr
         # The inverse reorder of O and LSE is fused into the attention store
         # (out_perm); sa_unreorder stays available for standalone use.
-        block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, out, lse,
-                          self.skip_log, self.flags, stream, ws=self.attn_ws,
-                          out_perm=None if self.identity else self.perm)
+        out_perm = None if self.identity else self.perm
+        if self.qk8:
+            block_sparse_attn_qk8(self.q8, self.q_scales, self.k8, self.k_scales, vr, self.shape, self.mask.struct,
+                                  self.lam, self.scale, out, self.attn_ws, lse, self.skip_log, self.flags, stream,
+                                  out_perm=out_perm)
+        else:
+            block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, out, lse,
+                              self.skip_log, self.flags, stream, ws=self.attn_ws, out_perm=out_perm)
         return out, lse
+
+    def _quantize(self, qr, kr, stream):
+        quantize_blocks(qr, self.params.bq, self.q8, self.q_scales, stream)
+        quantize_blocks(kr, self.params.bk, self.k8, self.k_scales, stream)
 
     def status(self, stream=None) -> int:
         return read_status(self.mask.status, stream)
