@@ -93,3 +93,73 @@ def test_quantised_attention_is_close_to_exact():
     d = np.abs(r8["out"] - r["out"])
     assert d.max() < 3e-2 and d.mean() < 3e-3
     assert np.max(np.abs(r8["lse"] - r["lse"])) < 3e-2
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3
+# --------------------------------------------------------------------------
+
+def _e4m3_table():
+    """Every positive finite E4M3 value from the format definition."""
+    vals = [m * 2.0 ** -9 for m in range(1, 8)]                       # subnormals
+    for e in range(1, 16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue                                              # the NaN code
+            vals.append((1 + m / 8) * 2.0 ** (e - 7))
+    return np.array(vals)
+
+
+def test_e4m3_table_is_fixed_and_byte_codes_round_trip():
+    t = _e4m3_table()
+    assert t.size == 126 and t.max() == 448.0 and t.min() == 2.0 ** -9
+    assert np.array_equal(Q.round_e4m3(t), t) and np.array_equal(Q.round_e4m3(-t), -t)
+    codes = Q.e4m3_byte(np.concatenate([t, -t, [0.0]]))
+    assert np.array_equal(Q.e4m3_value(codes), np.concatenate([t, -t, [0.0]]))
+    assert len(set(codes.tolist())) == 253
+    # hand-picked codes: 1 = 0 0111 000, 448 = 0 1111 110, 2^-9 = 0 0000 001, -1.75 = 1 0111 110
+    assert Q.e4m3_byte([1.0, 448.0, 2.0 ** -9, -1.75]).tolist() == [0x38, 0x7E, 0x01, 0xBE]
+
+
+def test_e4m3_rounding_midpoints_and_saturation():
+    t = _e4m3_table()
+    mids = (t[:-1] + t[1:]) / 2
+    r = Q.round_e4m3(mids)
+    lo, hi = t[:-1], t[1:]
+    # ties to the neighbour whose code is even
+    even_lo = (Q.e4m3_byte(lo) & 1) == 0
+    assert np.array_equal(r, np.where(even_lo, lo, hi))
+    assert Q.round_e4m3([2.0 ** -10, 2.0 ** -11]).tolist() == [0.0, 0.0]      # half of 2^-9 ties to 0
+    assert Q.round_e4m3([1000.0, 464.0, -1e9]).tolist() == [448.0, 448.0, -448.0]
+    x = np.random.default_rng(0).uniform(-448, 448, 10000)
+    r = Q.round_e4m3(x)
+    # nearest: no table value is closer
+    full = np.concatenate([-t[::-1], [0.0], t])
+    best = full[np.abs(x[:, None] - full[None, :]).argmin(axis=1)]
+    assert np.all(np.abs(x - r) <= np.abs(x - best))
+
+
+def test_e4m3_blocks_scale_and_error():
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((2, 200, 32)) * rng.uniform(0.01, 30, size=(2, 200, 1))).astype(np.float32)
+    codes, scales = Q.quantize_blocks(x, 64, "e4m3")
+    assert codes.dtype == np.uint8
+    deq = Q.dequantize(codes, scales, 64, "e4m3")
+    per_row = np.repeat(scales.astype(np.float64), 64, axis=-1)[..., :200, None]
+    # relative 2^-4 for normals, half the subnormal step below 2^-6 (in code units)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, per_row * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(np.abs(deq - x) <= bound)
+    for b in range(4):   # the block's absmax element maps to 448
+        assert np.all(np.abs(deq[..., b * 64:(b + 1) * 64, :]).max(axis=(-2, -1)) / scales[..., b] ==
+                      pytest.approx(448.0, rel=1e-6))
+
+
+def test_e4m3_attention_is_close_to_exact():
+    rng = np.random.default_rng(2)
+    n = 200
+    q, k, v = (rng.standard_normal((1, 1, n, 128)).astype(np.float32) for _ in range(3))
+    kept = np.ones((1, 1, 2, 4), dtype=bool)
+    r8 = Q.block_sparse_attention_qk8_heads(q, k, v, kept, 128, 64, fmt="e4m3")
+    r = A.block_sparse_attention_heads(q, k, v, kept, 128, 64)
+    d = np.abs(r8["out"] - r["out"])
+    assert d.max() < 5e-2 and d.mean() < 5e-3
