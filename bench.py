@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch of the attention kernel from the ncu capture recorded
 # in profiles/attn_tc_video.md, keyed by the sha1 of the kernel code it was
 # taken on (src_sha1); any other code reports null.
-TRAFFIC = {("f0b51a04784cb91ddfcc4d14d72a7a39a094f8c2", "video"): 1.2127e9}
+TRAFFIC = {("79d19421d0daed5604f044fa9c241e28c613ceb9", "video"): 1.2193e9}
 
 
 def peaks():
@@ -246,22 +246,22 @@ def run_ours(args, rank, world, local_rank):
             sa.reorder_predict_mask(pipe.perm, q, k, pipe.qr, pipe.kr, pipe.shape, pipe.params, pipe.ws,
                                     pipe.mask.struct)
             if args.qk8:   # per-block INT8 codes of Q and K, beside the V reorder
-                sa.quantize_blocks(pipe.qr, w.bq, pipe.q8, pipe.q_scales)
-                sa.quantize_blocks(pipe.kr, w.bk, pipe.k8, pipe.k_scales)
+                sa.quantize_blocks(pipe.qr, w.bq, pipe.q8, pipe.q_scales, args.qk8)
+                sa.quantize_blocks(pipe.kr, w.bk, pipe.k8, pipe.k_scales, args.qk8)
             stream.wait_event(pipe.ev_v)
             qr, kr, vr = pipe.qr, pipe.kr, pipe.vr
         else:
             qr, kr, vr = q, k, v
             sa.predict_mask(qr, kr, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
             if args.qk8:
-                sa.quantize_blocks(qr, w.bq, pipe.q8, pipe.q_scales)
-                sa.quantize_blocks(kr, w.bk, pipe.k8, pipe.k_scales)
+                sa.quantize_blocks(qr, w.bq, pipe.q8, pipe.q_scales, args.qk8)
+                sa.quantize_blocks(kr, w.bk, pipe.k8, pipe.k_scales, args.qk8)
         e[1].record(stream)
         # attention with the inverse reorder of O and LSE fused into its store
         if args.qk8:
             sa.block_sparse_attn_qk8(pipe.q8, pipe.q_scales, pipe.k8, pipe.k_scales, vr, pipe.shape,
                                      pipe.mask.struct, pipe.lam, pipe.scale, pipe.out, pipe.attn_ws, pipe.lse,
-                                     out_perm=None if pipe.identity else pipe.perm)
+                                     out_perm=None if pipe.identity else pipe.perm, fmt=args.qk8)
         else:
             sa.block_sparse_attn(qr, kr, vr, pipe.shape, pipe.mask.struct, pipe.lam, pipe.scale, pipe.out,
                                  pipe.lse, ws=pipe.attn_ws, out_perm=None if pipe.identity else pipe.perm)
@@ -361,10 +361,10 @@ def run_ours(args, rank, world, local_rank):
     peak_tf = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     peak_src = f"{pk_src} bf16 dense (burst)"
     if args.qk8:
-        # QK at the int8 rate (the nominal int8 / bf16 ratio 2 on the measured
-        # bf16 peak), PV at the bf16 rate: the peak of the mixed contraction.
+        # QK at the 8-bit rate (the nominal int8 or fp8 / bf16 ratio 2 on the
+        # measured bf16 peak), PV at the bf16 rate: the peak of the mixed contraction.
         peak_tf = flops / (qk_flops / (2 * peak_tf) + pv_flops / peak_tf)
-        peak_src = f"{pk_src} bf16 (burst) x nominal int8/bf16 ratio 2 on the QK half"
+        peak_src = f"{pk_src} bf16 (burst) x nominal {args.qk8}/bf16 ratio 2 on the QK half"
     attn_tf = flops / (attn_mean * 1e-3) / 1e12
     sha = src_sha1("attn_tc.cu")
     traffic = None if args.qk8 else TRAFFIC.get((sha, args.workload))
@@ -379,7 +379,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16, QK int8 per block" if args.qk8 else "bf16",
+        "dtype": f"bf16, QK {args.qk8} per block" if args.qk8 else "bf16",
         "data": "synthetic (seeded smooth-field generator, bf16)",
         "config": workload_config(w, world),
         "stages_ms": {"layout_reorder_predict": round(statistics.mean(pre_ms), 4),
@@ -396,7 +396,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": round(attn_tf, 2), "peak": round(peak_tf, 1),
                      "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4), "traffic": traffic,
                      "peak_source": peak_src,
-                     "kernel": "attn_tc_kernel<64, int8 QK>" if args.qk8 else "attn_tc_kernel<64>"},
+                     "kernel": f"attn_tc_kernel<64, {args.qk8} QK>" if args.qk8 else "attn_tc_kernel<64>"},
         "e2e": None if args.qk8 else {
             "value": round(job_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
             "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -406,7 +406,7 @@ def run_ours(args, rank, world, local_rank):
         "wall_s": round(wall, 3),
     }
     if args.qk8:
-        res["qk"] = "int8, per-block scales (Q per query block, K per key block); P, V bf16"
+        res["qk"] = f"{args.qk8}, per-block scales (Q per query block, K per key block); P, V bf16"
     if world == 1 and not args.no_cpu_baseline and not args.qk8:
         res["cpu_baseline"] = cpu_baseline(w, g, seconds=args.cpu_seconds)
     return res
@@ -640,8 +640,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="video")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--qk8", action="store_true",
-                    help="the predicted-mask path with INT8 QK (per-block quantised Q and K)")
+    ap.add_argument("--qk8", choices=["int8", "e4m3"], default=None,
+                    help="the predicted-mask path with 8-bit QK (per-block quantised Q and K)")
     ap.add_argument("--path", default="sparge", choices=["sparge", "svg"],
                     help="sparge: the predicted-mask path (the headline); svg: per-head spatial/temporal masks")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

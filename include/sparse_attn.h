@@ -261,34 +261,41 @@ sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v,
                                uint8_t* pv_skip_log, void* ws, size_t ws_bytes, int32_t flags,
                                void* stream);
 
-/* ---- INT8 QK ([P3] 2.4: SageAttention's per-block quantisation) ----------
+/* ---- 8-bit QK ([P3] 2.4: SageAttention's per-block quantisation) ---------
  * The QK product on 8-bit codes with per-block dequantisation scales; P and
- * V stay bf16.
+ * V stay bf16.  Two code formats:
+ *   SA_Q_INT8: int8, scale = absmax / 127, code = rint(x * (127 / absmax))
+ *     in float32, round half to even, in [-127, 127];
+ *   SA_Q_E4M3: FP8 E4M3 bytes, scale = absmax / 448, code = the E4M3 value
+ *     nearest to x * (448 / absmax) (float32 product; ties to even,
+ *     saturated to +-448).
+ * An all-zero block gets scale 0 and codes 0.
  *
- * sa_quantize_blocks: x bf16 [heads][N][d] (16-byte aligned) -> x8 int8
- * [heads][N][d] (8-byte aligned) and scales float [heads][ceil(N/rows)].
- * A block is `rows` consecutive tokens of one head; scale = absmax / 127 and
- * x8 = rint(x * (127 / absmax)) in float32, round half to even, in
- * [-127, 127]; an all-zero block gets scale 0 and codes 0.  Needs d a
- * multiple of 8 and rows * d <= 16384.  Quantise Q with rows = the mask's
- * bq and K with rows = its bk.
+ * sa_quantize_blocks: x bf16 [heads][N][d] (16-byte aligned) -> x8 codes
+ * [heads][N][d] (8-byte aligned) and scales float [heads][ceil(N/rows)]; a
+ * block is `rows` consecutive tokens of one head.  Needs d a multiple of 8
+ * and rows * d <= 16384.  Quantise Q with rows = the mask's bq and K with
+ * rows = its bk.
  *
- * sa_block_sparse_attn_qk8: sa_block_sparse_attn with q8, k8 int8 BNSD
- * codes and their scales (q_scales [B*Hq][ceil(N/bq)], k_scales
+ * sa_block_sparse_attn_qk8: sa_block_sparse_attn with q8, k8 BNSD codes of
+ * `format` and their scales (q_scales [B*Hq][ceil(N/bq)], k_scales
  * [B*Hkv][ceil(N/bk)]): the score of a pair is (q8 . k8) * q_scale *
- * k_scale * scale, the int32 dot product exact on the tensor cores.  Same
+ * k_scale * scale (an exact int32 product for INT8, an fp32-accumulated
+ * one for E4M3, on the tensor cores).  Same
  * mask, lambda, out, lse, out_perm, skip log and flags as
  * sa_block_sparse_attn (SA_FLAG_FORCE_SIMT: SA_ERR_UNSUPPORTED; there is no
  * other kernel).  Needs bf16 V and out, d = dv = 128, bq = 128, bk in
  * {64, 128}, an sm_100 device, 16-byte aligned q8, k8, v, out.  ws:
  * sa_attn_qk8_workspace(mask) bytes, 256-byte aligned (the work counter and
  * one scale per list entry). */
+#define SA_Q_INT8 0
+#define SA_Q_E4M3 1
 sa_status sa_quantize_blocks(const void* x, int64_t heads, int64_t N, int64_t d, int32_t rows, int32_t dtype,
-                             int8_t* x8, float* scales, void* stream);
+                             int32_t format, void* x8, float* scales, void* stream);
 size_t sa_attn_qk8_workspace(const sa_mask* mask);
-sa_status sa_block_sparse_attn_qk8(const int8_t* q8, const float* q_scales, const int8_t* k8, const float* k_scales,
-                                   const void* v, const sa_shape* shape, const sa_mask* mask, float lambda,
-                                   float scale, void* out, float* lse, const int32_t* out_perm,
+sa_status sa_block_sparse_attn_qk8(const void* q8, const float* q_scales, const void* k8, const float* k_scales,
+                                   int32_t format, const void* v, const sa_shape* shape, const sa_mask* mask,
+                                   float lambda, float scale, void* out, float* lse, const int32_t* out_perm,
                                    uint8_t* pv_skip_log, void* ws, size_t ws_bytes, int32_t flags, void* stream);
 
 /* ---- a8: dense reference --------------------------------------------------

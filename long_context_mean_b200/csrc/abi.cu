@@ -260,6 +260,7 @@ sa_status sa_mask_from_blocks(const uint8_t* block_mask, const sa_shape* shape, 
 struct Qk8Args {
   const float* q_scales;   // [B*Hq][nqb]
   const float* k_scales;   // [B*Hkv][nkb]
+  int32_t format;          // SA_Q_INT8 or SA_Q_E4M3
 };
 
 static sa_status attn_common(const void* q, const void* k, const void* v, const sa_shape* shape,
@@ -318,6 +319,8 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
   if (qk8) {
     // INT8 QK runs on the tensor-core kernel only: there is no other path.
     if (!qk8->q_scales || !qk8->k_scales) return set_error(SA_ERR_INVALID_ARG, "NULL scale array");
+    if (qk8->format != SA_Q_INT8 && qk8->format != SA_Q_E4M3)
+      return set_error(SA_ERR_INVALID_ARG, "format must be SA_Q_INT8 or SA_Q_E4M3");
     if (!(shape->dtype == SA_BF16 && shape->d == 128 && shape->dv == 128 && a.bq == 128 &&
           (a.bk == 64 || a.bk == 128)))
       return set_error(SA_ERR_UNSUPPORTED, "INT8 QK needs bf16 V, d = dv = 128, bq = 128, bk in {64, 128}");
@@ -332,6 +335,7 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
                                          a.scale * 1.4426950408889634f, ts, st))
       return e;
     a.tile_scale = ts;
+    a.qfmt = qk8->format;
     return launch_attn_tc(a, st);
   }
   if (!mask) {
@@ -368,26 +372,28 @@ size_t sa_attn_qk8_workspace(const sa_mask* mask) {
 }
 
 sa_status sa_quantize_blocks(const void* x, int64_t heads, int64_t N, int64_t d, int32_t rows, int32_t dtype,
-                             int8_t* x8, float* scales, void* stream) {
+                             int32_t format, void* x8, float* scales, void* stream) {
   if (!x || !x8 || !scales) return set_error(SA_ERR_INVALID_ARG, "NULL argument to sa_quantize_blocks");
   if (heads < 0 || N < 1 || d < 1 || rows < 1) return set_error(SA_ERR_INVALID_ARG, "bad sizes for sa_quantize_blocks");
   if (dtype != SA_BF16) return set_error(SA_ERR_UNSUPPORTED, "sa_quantize_blocks takes bf16 input");
+  if (format != SA_Q_INT8 && format != SA_Q_E4M3)
+    return set_error(SA_ERR_INVALID_ARG, "format must be SA_Q_INT8 or SA_Q_E4M3");
   if (!quant_blocks_fits(d, rows))
     return set_error(SA_ERR_UNSUPPORTED, "sa_quantize_blocks needs d a multiple of 8 and rows * d <= 16384");
   if ((uintptr_t)x % 16 || (uintptr_t)x8 % 8 || (uintptr_t)scales % 4)
     return set_error(SA_ERR_INVALID_ARG, "misaligned tensor (x 16 bytes, x8 8 bytes)");
   if (sa_status e = check_device()) return e;
-  return launch_quant_blocks(x, heads, N, d, rows, x8, scales, static_cast<cudaStream_t>(stream));
+  return launch_quant_blocks(x, heads, N, d, rows, format, x8, scales, static_cast<cudaStream_t>(stream));
 }
 
-sa_status sa_block_sparse_attn_qk8(const int8_t* q8, const float* q_scales, const int8_t* k8, const float* k_scales,
-                                   const void* v, const sa_shape* shape, const sa_mask* mask, float lambda,
-                                   float scale, void* out, float* lse, const int32_t* out_perm,
+sa_status sa_block_sparse_attn_qk8(const void* q8, const float* q_scales, const void* k8, const float* k_scales,
+                                   int32_t format, const void* v, const sa_shape* shape, const sa_mask* mask,
+                                   float lambda, float scale, void* out, float* lse, const int32_t* out_perm,
                                    uint8_t* pv_skip_log, void* ws, size_t ws_bytes, int32_t flags, void* stream) {
   if (!mask) return set_error(SA_ERR_INVALID_ARG, "mask is NULL");
   if ((uintptr_t)q8 % 16 || (uintptr_t)k8 % 16 || (uintptr_t)v % 16 || (uintptr_t)out % 16)
     return set_error(SA_ERR_INVALID_ARG, "INT8 QK needs 16-byte aligned q8, k8, v, out");
-  const Qk8Args qk8{q_scales, k_scales};
+  const Qk8Args qk8{q_scales, k_scales, format};
   return attn_common(q8, k8, v, shape, mask, 0, lambda, scale, out, lse, out_perm, pv_skip_log, nullptr, ws,
                      ws_bytes, flags, stream, &qk8);
 }

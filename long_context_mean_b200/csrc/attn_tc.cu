@@ -48,7 +48,7 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-template <int BK, bool QI8>
+template <int BK, int QM>
 struct Cfg {
   // P in shared memory (SS MMA, S two tiles ahead of PV) or over S in TMEM
   // (TS MMA, S one tile ahead).  Measured on B200 at bk = 64 the TMEM form
@@ -56,11 +56,12 @@ struct Cfg {
   // block sizes use it; the shared-memory form stays for other shapes.
   static constexpr bool P_SMEM = false;
   static constexpr int PIPES = BK == 64 ? 2 : 1;
-  // INT8 Q and K halve their tiles, which leaves room for a third stage.
-  static constexpr int STAGES = (BK == 64 && !QI8) ? 2 : 3;
+  // 8-bit Q and K (QM 1: INT8, 2: FP8 E4M3) halve their tiles, which leaves
+  // room for a third stage.
+  static constexpr int STAGES = (BK == 64 && QM == 0) ? 2 : 3;
   static constexpr int LOOKAHEAD = P_SMEM ? 2 : 1;    // S tiles issued ahead of PV
   static constexpr int THREADS = 128 + 128 * PIPES;
-  static constexpr int QK_ELEM = QI8 ? 1 : 2;          // bytes per Q / K element
+  static constexpr int QK_ELEM = QM ? 1 : 2;           // bytes per Q / K element
   static constexpr int Q_BYTES = 128 * 128 * QK_ELEM;
   static constexpr int K_BYTES = BK * 128 * QK_ELEM;
   static constexpr int V_BYTES = BK * 128 * 2;
@@ -93,8 +94,8 @@ struct Ctl {
   volatile int32_t ring[4];
 };
 static_assert(sizeof(Ctl) <= 512, "control block too large");
-static_assert(Cfg<64, false>::SMEM <= 227 * 1024 && Cfg<128, false>::SMEM <= 227 * 1024 &&
-                  Cfg<64, true>::SMEM <= 227 * 1024 && Cfg<128, true>::SMEM <= 227 * 1024,
+static_assert(Cfg<64, 0>::SMEM <= 227 * 1024 && Cfg<128, 0>::SMEM <= 227 * 1024 &&
+                  Cfg<64, 1>::SMEM <= 227 * 1024 && Cfg<128, 1>::SMEM <= 227 * 1024,
               "shared memory above the 227 KB a CTA may use");
 
 struct TcParams {
@@ -109,7 +110,7 @@ struct TcParams {
   int32_t* counter;      // work counter, zero at launch
   int64_t N, nqb, nkb;
   int64_t perm_stride;   // 0: one out_perm for every head; N: one per query head
-  const float* tile_scale;   // INT8 QK: log2-domain scale of each kept tile, CSR order
+  const float* tile_scale;   // 8-bit QK: log2-domain scale of each kept tile, CSR order
   int32_t Hq, Hkv;
   int32_t num_units;
   int32_t causal;
@@ -202,6 +203,15 @@ __device__ __forceinline__ void umma_ss_i8(uint32_t d_tmem, uint64_t a, uint64_t
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// D (TMEM, f32) = A (SMEM desc, e4m3) x B (SMEM desc, e4m3) [+ D]
+__device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
@@ -321,6 +331,11 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N, int b_mn_major) 
 __host__ __device__ constexpr uint32_t make_idesc_s8(int M, int N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// Instruction descriptor, kind::f8f6f4: e4m3 x e4m3 -> f32 (D format 1, A
+// and B format 0 = E4M3), both operands K-major.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 // An int32 in (-2^22, 2^22) as a float biased by 1.5 * 2^23: the bit pattern
 // of 12582912 + x, exact (used on the raw int32 S tile of the INT8 path).
 constexpr int32_t kBiasBits = 0x4B400000;
@@ -356,10 +371,10 @@ __device__ __forceinline__ int64_t kblock_at(const TcParams& p, const Unit& u, i
 // ---------------------------------------------------------------------------
 // Roles
 // ---------------------------------------------------------------------------
-template <int BK, bool QI8>
+template <int BK, int QM>
 __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                          const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, int pipe) {
-  using C = Cfg<BK, QI8>;
+  using C = Cfg<BK, QM>;
   uint32_t kv_it = 0, nq = 0;
   for (uint32_t j = 0;; ++j) {
     // Take the next unit of the work order and announce it to the pipeline's
@@ -377,7 +392,7 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const C
     ++nq;
     mbar_expect_tx(&c->q_full, C::Q_BYTES);
     tma_load_3d(sb + C::off_q(pipe), tmQ, 0, (int)(u.qb * 128), (int)u.bh, &c->q_full);
-    if constexpr (!QI8)   // bf16 rows are two 128-byte chunks; int8 rows one
+    if constexpr (QM == 0)   // bf16 rows are two 128-byte chunks; 8-bit rows one
       tma_load_3d(sb + C::off_q(pipe) + C::Q_BYTES / 2, tmQ, 64, (int)(u.qb * 128), (int)u.bh, &c->q_full);
     for (int64_t t = 0; t < u.n; ++t, ++kv_it) {
       const int kb = (int)kblock_at(p, u, t);
@@ -388,7 +403,7 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const C
       mbar_wait(&c->k_empty[s], ph ^ 1, g, p.status);
       mbar_expect_tx(&c->k_full[s], C::K_BYTES);
       tma_load_3d(kdst, tmK, 0, kb * BK, (int)u.kvh, &c->k_full[s]);
-      if constexpr (!QI8) tma_load_3d(kdst + C::KV_CHUNK, tmK, 64, kb * BK, (int)u.kvh, &c->k_full[s]);
+      if constexpr (QM == 0) tma_load_3d(kdst + C::KV_CHUNK, tmK, 64, kb * BK, (int)u.kvh, &c->k_full[s]);
       mbar_wait(&c->v_empty[s], ph ^ 1, g, p.status);
       mbar_expect_tx(&c->v_full[s], C::V_BYTES);
       tma_load_3d(vdst, tmV, 0, kb * BK, (int)u.kvh, &c->v_full[s]);
@@ -403,10 +418,11 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const C
   }
 }
 
-template <int BK, bool QI8>
+template <int BK, int QM>
 __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint32_t tm, int pipe) {
-  using C = Cfg<BK, QI8>;
-  constexpr uint32_t idesc_s = QI8 ? make_idesc_s8(128, BK) : make_idesc(128, BK, 0);
+  using C = Cfg<BK, QM>;
+  constexpr uint32_t idesc_s =
+      QM == 1 ? make_idesc_s8(128, BK) : (QM == 2 ? make_idesc_e4m3(128, BK) : make_idesc(128, BK, 0));
   constexpr uint32_t idesc_pv = make_idesc(128, 128, 1);
   uint32_t kv_it = 0, gt0 = 0, unit_it = 0;   // unit_it counts units with work
   for (uint32_t j = 0;; ++j) {
@@ -464,13 +480,16 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
       tc_fence_after();
       const uint32_t kbase = sb + C::off_k(pipe) + s * C::K_BYTES;
       const uint32_t qbase = sb + C::off_q(pipe);
-      if constexpr (QI8) {
-        // d = 128 int8 = one 128-byte swizzle row; K = 32 per instruction.
+      if constexpr (QM != 0) {
+        // d = 128 8-bit codes = one 128-byte swizzle row; K = 32 per instruction.
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t a = desc_sw128(qbase + kk * 32, 16, 1024);
           const uint64_t b = desc_sw128(kbase + kk * 32, 16, 1024);
-          umma_ss_i8(tm + C::S_COL + gb * BK, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          if constexpr (QM == 1)
+            umma_ss_i8(tm + C::S_COL + gb * BK, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          else
+            umma_ss_f8(tm + C::S_COL + gb * BK, a, b, idesc_s, kk > 0 ? 1u : 0u);
         }
       } else {
 #pragma unroll
@@ -500,13 +519,13 @@ __device__ __forceinline__ float warp_fmax(float v) {
   return __int_as_float(m >= 0 ? m : m ^ 0x7FFFFFFF);
 }
 
-template <int BK, bool QI8>
+template <int BK, int QM>
 __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, uint32_t tm, int pipe, int wq,
                              int lane) {
-  using C = Cfg<BK, QI8>;
+  using C = Cfg<BK, QM>;
   const int row = wq * 32 + lane;
   const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-  float sc = p.scale_log2;   // log2-domain score scale; INT8 QK: per tile
+  float sc = p.scale_log2;   // log2-domain score scale; 8-bit QK: per tile
   uint8_t* prow = smem + C::off_p(pipe) + (row >> 3) * 1024 + (row & 7) * 128;
   uint32_t gt0 = 0;
   for (uint32_t j = 0;; ++j) {
@@ -526,13 +545,13 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
     float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
     int64_t kb_cur = kblock_at(p, u, 0);
     float sc_next = 0.f;
-    if constexpr (QI8) sc_next = p.tile_scale[u.lo];
+    if constexpr (QM != 0) sc_next = p.tile_scale[u.lo];
     for (int64_t t = 0; t < u.n; ++t) {
       const uint32_t gt = gt0 + (uint32_t)t;
       const int gb = gt & 1;
       const uint32_t scol = tm + lane_off + C::S_COL + gb * BK;
       const int64_t kb_next = (t + 1 < u.n) ? kblock_at(p, u, t + 1) : 0;   // load ahead
-      if constexpr (QI8) {
+      if constexpr (QM != 0) {
         sc = sc_next;
         if (t + 1 < u.n) sc_next = p.tile_scale[u.lo + t + 1];
       }
@@ -542,7 +561,7 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
 #pragma unroll
       for (int cc = 0; cc < BK / 32; ++cc) tmem_ld32(scol + cc * 32, s + cc * 32);
       tmem_wait_ld();
-      if constexpr (QI8) {
+      if constexpr (QM == 1) {
         // int32 scores -> floats biased by kBias (exact); the bias cancels
         // in the exponent offset and the tile maximum below.
 #pragma unroll
@@ -568,7 +587,7 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
       float row_sum = 0.f;
       auto compute_p = [&](float ref) {
         // Pairs of columns on the packed fp32x2 pipe: x = s * scale - ref.
-        const float off = QI8 ? fmaf(-kBias, sc, -ref) : -ref;
+        const float off = QM == 1 ? fmaf(-kBias, sc, -ref) : -ref;
         const uint64_t sc2 = pack2(sc, sc), neg2 = pack2(off, off);
         uint64_t acc[4];
 #pragma unroll
@@ -613,7 +632,7 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
           mx[jj] = max3(a, b, d);
         }
       }
-      const float mloc = (QI8 ? mx[0] - kBias : mx[0]) * sc;   // scale > 0: max commutes
+      const float mloc = (QM == 1 ? mx[0] - kBias : mx[0]) * sc;   // scale > 0: max commutes
       const float m_new = fmaxf(m_run, mloc);
       const float gap = warp_fmax((row_valid && mloc > -INFINITY) ? mloc - m_new : -INFINITY);
       if (lane == 0) c->gapw[gt & 3][wq] = gap;
@@ -708,11 +727,11 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
   }
 }
 
-template <int BK, bool QI8>
-__global__ void __launch_bounds__(Cfg<BK, QI8>::THREADS, 1)
+template <int BK, int QM>
+__global__ void __launch_bounds__(Cfg<BK, QM>::THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, TcParams p) {
-  using C = Cfg<BK, QI8>;
+  using C = Cfg<BK, QM>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -760,19 +779,19 @@ __global__ void __launch_bounds__(Cfg<BK, QI8>::THREADS, 1)
   if (warp < 2) {
     if (warp < C::PIPES && lane == 0) {
       Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + warp * C::CTL_BYTES);
-      producer<BK, QI8>(&tmQ, &tmK, &tmV, p, c, ctl0, sb, warp);
+      producer<BK, QM>(&tmQ, &tmK, &tmV, p, c, ctl0, sb, warp);
     }
   } else if (warp < 4) {
     const int pipe = warp - 2;
     if (pipe < C::PIPES && lane == 0) {
       Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + pipe * C::CTL_BYTES);
-      mma_issuer<BK, QI8>(p, c, ctl0, sb, tmem + pipe * C::TMEM_PIPE, pipe);
+      mma_issuer<BK, QM>(p, c, ctl0, sb, tmem + pipe * C::TMEM_PIPE, pipe);
     }
     __syncwarp();
   } else {
     const int pipe = (warp - 4) >> 2;
     Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + pipe * C::CTL_BYTES);
-    softmax_rows<BK, QI8>(p, c, ctl0, smem, tmem + pipe * C::TMEM_PIPE, pipe, warp & 3, lane);
+    softmax_rows<BK, QM>(p, c, ctl0, smem, tmem + pipe * C::TMEM_PIPE, pipe, warp & 3, lane);
   }
 
   tc_fence_before();
@@ -803,7 +822,7 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over [heads][N][128] elements of 2 (bf16) or 1 (int8) bytes, box
+// 3-D map over [heads][N][128] elements of 2 (bf16) or 1 (8-bit codes) bytes, box
 // [1][rows][one 128-byte chunk], 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, int64_t heads, int64_t N, int rows, int elem = 2) {
   EncodeTiledFn fn = encode_fn();
@@ -818,9 +837,9 @@ bool make_map(CUtensorMap* m, const void* base, int64_t heads, int64_t N, int ro
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BK, bool QI8>
+template <int BK, int QM>
 sa_status launch_bk(const AttnArgs& a, cudaStream_t st) {
-  using C = Cfg<BK, QI8>;
+  using C = Cfg<BK, QM>;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, a.q, a.B * a.Hq, a.N, 128, C::QK_ELEM) || !make_map(&mk, a.k, a.B * a.Hkv, a.N, BK, C::QK_ELEM) ||
       !make_map(&mv, a.v, a.B * a.Hkv, a.N, BK))
@@ -852,12 +871,12 @@ sa_status launch_bk(const AttnArgs& a, cudaStream_t st) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaFuncSetAttribute(attn_tc_kernel<BK, QI8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+  if (cudaFuncSetAttribute(attn_tc_kernel<BK, QM>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(attn_tc_kernel) failed");
   const int want = (p.num_units + C::PIPES - 1) / C::PIPES;
   const int grid = want < sms ? want : sms;
-  attn_tc_kernel<BK, QI8><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, p);
+  attn_tc_kernel<BK, QM><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, p);
   return check_launch("attn_tc_kernel");
 }
 
@@ -870,8 +889,9 @@ bool attn_tc_supported(const sa_shape& s, int bq, int bk) {
 sa_status launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   if ((uintptr_t)a.q % 16 || (uintptr_t)a.k % 16 || (uintptr_t)a.v % 16 || (uintptr_t)a.out % 16)
     return set_error(SA_ERR_INVALID_ARG, "tensor-core path needs 16-byte aligned q, k, v, out");
-  if (a.tile_scale) return a.bk == 64 ? launch_bk<64, true>(a, st) : launch_bk<128, true>(a, st);
-  return a.bk == 64 ? launch_bk<64, false>(a, st) : launch_bk<128, false>(a, st);
+  if (a.tile_scale && a.qfmt == SA_Q_E4M3) return a.bk == 64 ? launch_bk<64, 2>(a, st) : launch_bk<128, 2>(a, st);
+  if (a.tile_scale) return a.bk == 64 ? launch_bk<64, 1>(a, st) : launch_bk<128, 1>(a, st);
+  return a.bk == 64 ? launch_bk<64, 0>(a, st) : launch_bk<128, 0>(a, st);
 }
 
 }  // namespace sa

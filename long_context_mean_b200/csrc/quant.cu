@@ -1,17 +1,21 @@
-// Per-block INT8 quantisation of Q and K for the quantised QK path of the
+// Per-block 8-bit quantisation of Q and K for the quantised QK path of the
 // SpargeAttention notes ([P3] section 2.4: the QK product runs on
 // SageAttention's per-block quantisation with dequantisation scales).
 //
 // A block is `rows` consecutive tokens of one head over all d channels
-// (the query block for Q, the key block for K).  Its scale is
-// absmax / 127; every value becomes rint(x * (127 / absmax)) computed in
-// float32 (round half to even), in [-127, 127]; an all-zero block has scale
-// 0 and codes 0.  Both divisions are correctly rounded (__fdiv_rn), so the
-// codes do not depend on compiler flags.
+// (the query block for Q, the key block for K).  INT8: scale absmax / 127,
+// every value becomes rint(x * (127 / absmax)) computed in float32 (round
+// half to even), in [-127, 127].  FP8 E4M3: scale absmax / 448, every value
+// becomes the E4M3 value nearest to x * (448 / absmax) (float32 product,
+// hardware conversion: ties to even, saturated to +-448).  An all-zero block
+// has scale 0 and codes 0.  Both divisions are correctly rounded
+// (__fdiv_rn), so the codes do not depend on compiler flags.
 //
 // The attention kernel multiplies the exact int32 tile of q8 . k8 by one
 // float per kept tile: scale * log2(e) * scale_q(query block) *
 // scale_k(key block), written in CSR order by tile_scales_kernel.
+#include <cuda_fp8.h>
+
 #include "sa_internal.cuh"
 
 namespace sa {
@@ -31,15 +35,26 @@ __device__ __forceinline__ uint32_t bf16_abs_max4(uint4 v) {
   return m;
 }
 
-__device__ __forceinline__ int8_t quant1(uint32_t bits16, float inv) {
+__device__ __forceinline__ uint32_t quant1(uint32_t bits16, float inv) {
   const float f = __uint_as_float(bits16 << 16);
   int q = __float2int_rn(f * inv);
   q = max(-127, min(127, q));
-  return (int8_t)q;
+  return (uint32_t)(uint8_t)(int8_t)q;
+}
+// Two bf16 values (low, high half of w) to two 8-bit codes (low byte first).
+template <int FMT>
+__device__ __forceinline__ uint32_t quant2(uint32_t w, float inv) {
+  if constexpr (FMT == SA_Q_E4M3) {
+    const float2 f = make_float2(__uint_as_float(w << 16) * inv, __uint_as_float(w & 0xFFFF0000u) * inv);
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+  } else {
+    return quant1(w & 0xFFFFu, inv) | (quant1(w >> 16, inv) << 8);
+  }
 }
 
-// One CTA per (head, block).  x: bf16 [heads][N][d]; x8: int8 [heads][N][d];
-// scales: float [heads][nblk].
+// One CTA per (head, block).  x: bf16 [heads][N][d]; x8: 8-bit codes
+// [heads][N][d]; scales: float [heads][nblk].
+template <int FMT>
 __global__ void __launch_bounds__(kQuantThreads) quant_blocks_kernel(const uint4* __restrict__ x, int64_t N, int d,
                                                                      int rows, int64_t nblk, uint2* __restrict__ x8,
                                                                      float* __restrict__ scales) {
@@ -68,21 +83,15 @@ __global__ void __launch_bounds__(kQuantThreads) quant_blocks_kernel(const uint4
 #pragma unroll
   for (int w = 0; w < kQuantThreads / 32; ++w) m = max(m, wmax[w]);
   const float amax = __uint_as_float(m << 16);
-  const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
-  if (threadIdx.x == 0) scales[blockIdx.x] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
+  const float qmax = FMT == SA_Q_E4M3 ? 448.0f : 127.0f;
+  const float inv = amax > 0.f ? __fdiv_rn(qmax, amax) : 0.f;
+  if (threadIdx.x == 0) scales[blockIdx.x] = amax > 0.f ? __fdiv_rn(amax, qmax) : 0.f;
 #pragma unroll
   for (int i = 0; i < kQuantMaxVec; ++i) {
     const int64_t e = threadIdx.x + (int64_t)i * kQuantThreads;
     if (e < total) {
-      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        lo |= (uint32_t)(uint8_t)quant1(w[j] & 0xFFFFu, inv) << (16 * j);
-        lo |= (uint32_t)(uint8_t)quant1(w[j] >> 16, inv) << (16 * j + 8);
-        hi |= (uint32_t)(uint8_t)quant1(w[j + 2] & 0xFFFFu, inv) << (16 * j);
-        hi |= (uint32_t)(uint8_t)quant1(w[j + 2] >> 16, inv) << (16 * j + 8);
-      }
+      const uint32_t lo = quant2<FMT>(v[i].x, inv) | (quant2<FMT>(v[i].y, inv) << 16);
+      const uint32_t hi = quant2<FMT>(v[i].z, inv) | (quant2<FMT>(v[i].w, inv) << 16);
       x8[base + e] = make_uint2(lo, hi);
     }
   }
@@ -108,14 +117,18 @@ __global__ void __launch_bounds__(256) tile_scales_kernel(const int32_t* __restr
 
 }  // namespace
 
-sa_status launch_quant_blocks(const void* x, int64_t heads, int64_t N, int64_t d, int rows, int8_t* x8,
+sa_status launch_quant_blocks(const void* x, int64_t heads, int64_t N, int64_t d, int rows, int32_t fmt, void* x8,
                               float* scales, cudaStream_t st) {
   const int64_t nblk = ceil_div(N, rows);
   const int64_t ctas = heads * nblk;
   if (ctas == 0) return SA_OK;
   if (ctas > 2147483647) return set_error(SA_ERR_UNSUPPORTED, "too many blocks");
-  quant_blocks_kernel<<<(unsigned)ctas, kQuantThreads, 0, st>>>(static_cast<const uint4*>(x), N, (int)d, rows, nblk,
-                                                                reinterpret_cast<uint2*>(x8), scales);
+  if (fmt == SA_Q_E4M3)
+    quant_blocks_kernel<SA_Q_E4M3><<<(unsigned)ctas, kQuantThreads, 0, st>>>(
+        static_cast<const uint4*>(x), N, (int)d, rows, nblk, static_cast<uint2*>(x8), scales);
+  else
+    quant_blocks_kernel<SA_Q_INT8><<<(unsigned)ctas, kQuantThreads, 0, st>>>(
+        static_cast<const uint4*>(x), N, (int)d, rows, nblk, static_cast<uint2*>(x8), scales);
   return check_launch("quant_blocks_kernel");
 }
 

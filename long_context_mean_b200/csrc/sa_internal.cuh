@@ -105,8 +105,9 @@ struct AttnArgs {
   float* lse;
   const int32_t* out_perm;  // nullptr = rows stored in place
   int64_t perm_stride;      // 0: out_perm shared by all heads; N: out_perm[bh * N + n]
-  const float* tile_scale;  // non-null: q, k are int8 codes and this holds each kept tile's
+  const float* tile_scale;  // non-null: q, k are 8-bit codes and this holds each kept tile's
                             // log2-domain score scale in CSR order (tensor-core kernel only)
+  int32_t qfmt;             // the codes' format: SA_Q_INT8 or SA_Q_E4M3
   uint8_t* skip_log;
   const int32_t* row_ptr;   // nullptr = dense (every causally valid block)
   const int32_t* col_idx;
@@ -125,7 +126,7 @@ sa_status launch_head_placement(int64_t T, int64_t P, int64_t n, const int32_t* 
                                 int bk, int32_t* perms, uint8_t* mask, int32_t* status, cudaStream_t st);
 sa_status launch_rows_mse(const void* ref, const void* x, const int32_t* rows, int64_t nrows, int64_t BH, int64_t N,
                           int64_t dv, int32_t dtype, double* out, int32_t* status, cudaStream_t st);
-sa_status launch_quant_blocks(const void* x, int64_t heads, int64_t N, int64_t d, int rows, int8_t* x8,
+sa_status launch_quant_blocks(const void* x, int64_t heads, int64_t N, int64_t d, int rows, int32_t fmt, void* x8,
                               float* scales, cudaStream_t st);
 bool quant_blocks_fits(int64_t d, int rows);
 sa_status launch_tile_scales(const sa_mask& m, int64_t B, int64_t Hq, int64_t Hkv, const float* qs, const float* ks,

@@ -111,10 +111,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sa_l1_error": (I32, [P, P, I64, I32, P, P]),
         "sa_head_placement": (I32, [I64, I64, I64, I64, P, I64, I32, I32, P, P, P, P]),
         "sa_reorder_heads": (I32, [P, P, P, I64, I64, I64, I32, P]),
-        "sa_quantize_blocks": (I32, [P, I64, I64, I64, I32, I32, P, P, P]),
+        "sa_quantize_blocks": (I32, [P, I64, I64, I64, I32, I32, I32, P, P, P]),
         "sa_attn_qk8_workspace": (SZ, [ctypes.POINTER(Mask)]),
-        "sa_block_sparse_attn_qk8": (I32, [P, P, P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F, F,
-                                           P, P, P, P, P, SZ, I32, P]),
+        "sa_block_sparse_attn_qk8": (I32, [P, P, P, P, I32, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F,
+                                           F, P, P, P, P, P, SZ, I32, P]),
         "sa_rows_mse": (I32, [P, P, P, I64, I64, I64, I64, I32, P, P, P]),
         "sa_block_sparse_attn": (I32, [P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F, F,
                                        P, P, P, P, P, SZ, I32, P]),
@@ -271,13 +271,17 @@ def block_sparse_attn(q, k, v, shape: Shape, mask: Mask, lam, scale, out, lse=No
                                        _stream(stream)))
 
 
-def quantize_blocks(x, rows, x8, scales, stream=None):
-    """Per-block INT8 codes x8 and scales of a bf16 [..., N, d] tensor, one
-    scale per `rows` tokens of each head."""
+SA_Q_INT8, SA_Q_E4M3 = 0, 1
+Q_FORMATS = {"int8": SA_Q_INT8, "e4m3": SA_Q_E4M3}
+
+
+def quantize_blocks(x, rows, x8, scales, fmt="int8", stream=None):
+    """Per-block 8-bit codes x8 ("int8" or "e4m3") and scales of a bf16
+    [..., N, d] tensor, one scale per `rows` tokens of each head."""
     N, d = x.shape[-2], x.shape[-1]
     heads = x.numel() // (N * d)
-    _check(load().sa_quantize_blocks(_ptr(x), heads, N, d, rows, dtype_code(x), _ptr(x8), _ptr(scales),
-                                     _stream(stream)))
+    _check(load().sa_quantize_blocks(_ptr(x), heads, N, d, rows, dtype_code(x), Q_FORMATS[fmt], _ptr(x8),
+                                     _ptr(scales), _stream(stream)))
 
 
 def attn_qk8_workspace(mask: Mask) -> int:
@@ -285,8 +289,9 @@ def attn_qk8_workspace(mask: Mask) -> int:
 
 
 def block_sparse_attn_qk8(q8, q_scales, k8, k_scales, v, shape: Shape, mask: Mask, lam, scale, out, ws, lse=None,
-                          skip_log=None, flags=0, stream=None, out_perm=None):
-    _check(load().sa_block_sparse_attn_qk8(_ptr(q8), _ptr(q_scales), _ptr(k8), _ptr(k_scales), _ptr(v),
+                          skip_log=None, flags=0, stream=None, out_perm=None, fmt="int8"):
+    _check(load().sa_block_sparse_attn_qk8(_ptr(q8), _ptr(q_scales), _ptr(k8), _ptr(k_scales), Q_FORMATS[fmt],
+                                           _ptr(v),
                                            ctypes.byref(shape), ctypes.byref(mask), float(lam), float(scale),
                                            _ptr(out), _ptr(lse), _ptr(out_perm), _ptr(skip_log), _ptr(ws),
                                            ws.numel() * ws.element_size(), int(flags), _stream(stream)))
@@ -409,11 +414,13 @@ class Pipeline:
         self.mask = MaskBuffers.allocate(B, Hq, N, params.bq, params.bk, device)
         # INT8 QK ([P3] 2.4): Q and K quantised per query / key block after
         # the prediction, the attention on the codes.
-        self.qk8 = qk8
-        if qk8:
+        self.qk8 = {True: "int8", False: None}.get(qk8, qk8)    # None, "int8" or "e4m3"
+        if self.qk8:
+            if self.qk8 not in Q_FORMATS:
+                raise ValueError(f"qk8 must be one of {sorted(Q_FORMATS)}")
             nqb, nkb = self.mask.struct.nqb, self.mask.struct.nkb
-            self.q8 = torch.empty(B, Hq, N, d, dtype=torch.int8, device=device)
-            self.k8 = torch.empty(B, Hkv, N, d, dtype=torch.int8, device=device)
+            self.q8 = torch.empty(B, Hq, N, d, dtype=torch.uint8, device=device)
+            self.k8 = torch.empty(B, Hkv, N, d, dtype=torch.uint8, device=device)
             self.q_scales = torch.empty(B * Hq * nqb, dtype=torch.float32, device=device)
             self.k_scales = torch.empty(B * Hkv * nkb, dtype=torch.float32, device=device)
             self.attn_ws = workspace(attn_qk8_workspace(self.mask.struct), device)
@@ -465,15 +472,15 @@ class Pipeline:
         if self.qk8:
             block_sparse_attn_qk8(self.q8, self.q_scales, self.k8, self.k_scales, vr, self.shape, self.mask.struct,
                                   self.lam, self.scale, out, self.attn_ws, lse, self.skip_log, self.flags, stream,
-                                  out_perm=out_perm)
+                                  out_perm=out_perm, fmt=self.qk8)
         else:
             block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, out, lse,
                               self.skip_log, self.flags, stream, ws=self.attn_ws, out_perm=out_perm)
         return out, lse
 
     def _quantize(self, qr, kr, stream):
-        quantize_blocks(qr, self.params.bq, self.q8, self.q_scales, stream)
-        quantize_blocks(kr, self.params.bk, self.k8, self.k_scales, stream)
+        quantize_blocks(qr, self.params.bq, self.q8, self.q_scales, self.qk8, stream)
+        quantize_blocks(kr, self.params.bk, self.k8, self.k_scales, self.qk8, stream)
 
     def status(self, stream=None) -> int:
         return read_status(self.mask.status, stream)

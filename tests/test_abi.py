@@ -122,26 +122,30 @@ def test_host_validation_codes(lib):
     assert lib.sa_rows_mse(FAKE, FAKE, FAKE, 4, 2, 10, 8, 7, FAKE, null, null) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_rows_mse(FAKE, FAKE, null, 4, 2, 10, 8, 0, FAKE, null, null) == sa.SA_ERR_INVALID_ARG
     # INT8 QK
-    assert lib.sa_quantize_blocks(null, 2, 10, 128, 64, 0, FAKE, FAKE, null) == sa.SA_ERR_INVALID_ARG
-    assert lib.sa_quantize_blocks(FAKE, 2, 10, 128, 64, 1, FAKE, FAKE, null) == sa.SA_ERR_UNSUPPORTED
-    assert lib.sa_quantize_blocks(FAKE, 2, 10, 128, 256, 0, FAKE, FAKE, null) == sa.SA_ERR_UNSUPPORTED
+    assert lib.sa_quantize_blocks(null, 2, 10, 128, 64, 0, 0, FAKE, FAKE, null) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_quantize_blocks(FAKE, 2, 10, 128, 64, 1, 0, FAKE, FAKE, null) == sa.SA_ERR_UNSUPPORTED
+    assert lib.sa_quantize_blocks(FAKE, 2, 10, 128, 256, 0, 0, FAKE, FAKE, null) == sa.SA_ERR_UNSUPPORTED
+    assert lib.sa_quantize_blocks(FAKE, 2, 10, 128, 64, 0, 5, FAKE, FAKE, null) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_attn_qk8_workspace(None) == 0
     m3 = _mask()
     m3.bq, m3.bk, m3.nqb, m3.nkb, m3.col_capacity = 128, 64, 3, 5, 15
     assert lib.sa_attn_qk8_workspace(ctypes.byref(m3)) == 256 + 256
     WS8 = ctypes.c_void_p(1 << 21)
-    assert lib.sa_block_sparse_attn_qk8(FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(s), None, ctypes.c_float(-1),
+    assert lib.sa_block_sparse_attn_qk8(FAKE, FAKE, FAKE, FAKE, 0, FAKE, ctypes.byref(s), None, ctypes.c_float(-1),
                                         ctypes.c_float(0), FAKE, null, null, null, WS8, 512, 0,
                                         null) == sa.SA_ERR_INVALID_ARG
-    assert lib.sa_block_sparse_attn_qk8(FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m3),
+    assert lib.sa_block_sparse_attn_qk8(FAKE, FAKE, FAKE, FAKE, 0, FAKE, ctypes.byref(s), ctypes.byref(m3),
                                         ctypes.c_float(-1), ctypes.c_float(0), FAKE, null, null, null, WS8, 256, 0,
                                         null) == sa.SA_ERR_WORKSPACE
-    assert lib.sa_block_sparse_attn_qk8(FAKE, null, FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m3),
+    assert lib.sa_block_sparse_attn_qk8(FAKE, null, FAKE, FAKE, 0, FAKE, ctypes.byref(s), ctypes.byref(m3),
                                         ctypes.c_float(-1), ctypes.c_float(0), FAKE, null, null, null, WS8, 512, 0,
                                         null) == sa.SA_ERR_INVALID_ARG
-    assert lib.sa_block_sparse_attn_qk8(FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m3),
+    assert lib.sa_block_sparse_attn_qk8(FAKE, FAKE, FAKE, FAKE, 0, FAKE, ctypes.byref(s), ctypes.byref(m3),
                                         ctypes.c_float(-1), ctypes.c_float(0), FAKE, null, null, null, WS8, 512,
                                         sa.SA_FLAG_FORCE_SIMT, null) == sa.SA_ERR_UNSUPPORTED
+    assert lib.sa_block_sparse_attn_qk8(FAKE, FAKE, FAKE, FAKE, 9, FAKE, ctypes.byref(s), ctypes.byref(m3),
+                                        ctypes.c_float(-1), ctypes.c_float(0), FAKE, null, null, null, WS8, 512, 0,
+                                        null) == sa.SA_ERR_INVALID_ARG
     # a per-head output permutation needs out_perm
     m2.nqb = 3
     assert lib.sa_block_sparse_attn(FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m2), ctypes.c_float(-1),
