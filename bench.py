@@ -242,20 +242,23 @@ def run_ours(args, rank, world, local_rank):
             pipe.side.wait_event(pipe.ev_layout)
             sa.reorder(pipe.perm, v, pipe.vr, pipe.side)
             pipe.ev_v.record(pipe.side)
-            # mask prediction with the reorder of Q and K fused into its pooling pass
-            sa.reorder_predict_mask(pipe.perm, q, k, pipe.qr, pipe.kr, pipe.shape, pipe.params, pipe.ws,
-                                    pipe.mask.struct)
-            if args.qk8:   # per-block INT8 codes of Q and K, beside the V reorder
-                sa.quantize_blocks(pipe.qr, w.bq, pipe.q8, pipe.q_scales, args.qk8)
-                sa.quantize_blocks(pipe.kr, w.bk, pipe.k8, pipe.k_scales, args.qk8)
+            # mask prediction with the reorder of Q and K fused into its pooling
+            # pass (the 8-bit path: reorder and quantisation)
+            if args.qk8:
+                sa.reorder_predict_mask_q8(pipe.perm, q, k, args.qk8, pipe.q8, pipe.q_scales, pipe.k8,
+                                           pipe.k_scales, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
+            else:
+                sa.reorder_predict_mask(pipe.perm, q, k, pipe.qr, pipe.kr, pipe.shape, pipe.params, pipe.ws,
+                                        pipe.mask.struct)
             stream.wait_event(pipe.ev_v)
-            qr, kr, vr = pipe.qr, pipe.kr, pipe.vr
+            qr, kr, vr = (q, k, pipe.vr) if args.qk8 else (pipe.qr, pipe.kr, pipe.vr)
         else:
             qr, kr, vr = q, k, v
-            sa.predict_mask(qr, kr, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
             if args.qk8:
-                sa.quantize_blocks(qr, w.bq, pipe.q8, pipe.q_scales, args.qk8)
-                sa.quantize_blocks(kr, w.bk, pipe.k8, pipe.k_scales, args.qk8)
+                sa.reorder_predict_mask_q8(None, q, k, args.qk8, pipe.q8, pipe.q_scales, pipe.k8, pipe.k_scales,
+                                           pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
+            else:
+                sa.predict_mask(qr, kr, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
         e[1].record(stream)
         # attention with the inverse reorder of O and LSE fused into its store
         if args.qk8:
@@ -271,7 +274,7 @@ def run_ours(args, rank, world, local_rank):
     # layout (1, Hilbert 3) + reorder V; pool Q, pool K, score, row scan, column fill, order; attention
     launches_per_step = (0 if pipe.identity else (1 if w.order != "hilbert" else 3) + 1) + 6 + 1
     if args.qk8:
-        launches_per_step += 3            # two quantisation passes and the tile-scale kernel
+        launches_per_step += 1            # the tile-scale kernel (codes come from the pooling pass)
 
     for _ in range(args.warmup):
         l2_flush()
@@ -307,7 +310,7 @@ def run_ours(args, rank, world, local_rank):
     od = torch.empty_like(pipe.out)
     ld = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=dev)
     dst = torch.zeros(1, dtype=torch.int32, device=dev)
-    qr, kr, vr = (pipe.qr, pipe.kr, pipe.vr) if not pipe.identity else (q, k, v)
+    qr, kr, vr = (pipe.qr, pipe.kr, pipe.vr) if not (pipe.identity or args.qk8) else (q, k, v)
     dense = []
     dense_ws = sa.workspace(sa.attn_workspace(), dev)
     for i in range(args.warmup + max(3, min(args.steps, 10))):

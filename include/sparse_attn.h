@@ -293,6 +293,16 @@ sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v,
 sa_status sa_quantize_blocks(const void* x, int64_t heads, int64_t N, int64_t d, int32_t rows, int32_t dtype,
                              int32_t format, void* x8, float* scales, void* stream);
 size_t sa_attn_qk8_workspace(const sa_mask* mask);
+/* sa_reorder_predict_mask with the quantisation fused into its pooling
+ * pass: instead of reordered bf16 copies it writes the reordered 8-bit
+ * codes q8 [B*Hq][N][d], k8 [B*Hkv][N][d] (16-byte aligned) and the block
+ * scales q_scales [B*Hq][ceil(N/bq)], k_scales [B*Hkv][ceil(N/bk)], equal
+ * to sa_quantize_blocks of the reordered tensors (query blocks for Q, key
+ * blocks for K).  perm may be NULL (the original order).  bf16 q, k only. */
+sa_status sa_reorder_predict_mask_q8(const int32_t* perm, const void* q, const void* k, int32_t format, void* q8,
+                                     float* q_scales, void* k8, float* k_scales, const sa_shape* shape,
+                                     const sa_mask_params* params, void* ws, size_t ws_bytes, sa_mask* out,
+                                     void* stream);
 sa_status sa_block_sparse_attn_qk8(const void* q8, const float* q_scales, const void* k8, const float* k_scales,
                                    int32_t format, const void* v, const sa_shape* shape, const sa_mask* mask,
                                    float lambda, float scale, void* out, float* lse, const int32_t* out_perm,
@@ -344,6 +354,23 @@ sa_status sa_head_placement(int64_t T, int64_t H, int64_t W, int64_t txt_len, co
  * [outer][N], each entry in [0, N)).  x and y must not overlap. */
 sa_status sa_reorder_heads(const int32_t* perms, const void* x, void* y, int64_t outer, int64_t N, int64_t row,
                            int32_t dtype, void* stream);
+
+/* Attention of a few query rows, the online profile of [P1] section 5 (only
+ * the sampled rows are computed).  For each query head bh = b*Hq + h and
+ * sampled row r, the query token rows[r] (device int32, in [0, N)) attends
+ * to: every key (block_mask NULL), or the keys of the kept tiles of its
+ * query block in head bh's order (block_mask uint8 [B*Hq][ceil(N/bq)]
+ * [ceil(N/bk)], e.g. from sa_head_placement; perms int32 [B*Hq][N], the
+ * token at each place of that order, NULL = the original order).  q, k, v
+ * BNSD (bf16 or fp32, 16-byte aligned, d = dv in {64, 128},
+ * N / bk <= 4096); scale
+ * 0 means 1/sqrt(d).  out: float [B*Hq][nrows][dv], lse (nullable): float
+ * [B*Hq][nrows], natural log.  A row outside [0, N) or missing from its
+ * head's order raises SA_ERR_INVALID_ARG in status (device int32,
+ * nullable) and is not written; a row with no key raises SA_ERR_EMPTY_ROW. */
+sa_status sa_rows_attn(const void* q, const void* k, const void* v, const sa_shape* shape, const int32_t* rows,
+                       int64_t nrows, const int32_t* perms, const uint8_t* block_mask, int32_t bq, int32_t bk,
+                       float scale, float* out, float* lse, int32_t* status, void* stream);
 
 /* Sampled-row error of [P1] section 5: out[h] (device double [BH]) = mean of
  * (ref - x)^2 over the nrows sampled query rows (rows: device int32, each in

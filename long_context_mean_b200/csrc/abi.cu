@@ -201,6 +201,11 @@ bool overlaps(const void* a, const void* b, size_t bytes) {
   const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
   return x < y + bytes && y < x + bytes;
 }
+// [a, a + na) and [b, b + nb) share a byte.
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+  return x < y + nb && y < x + na;
+}
 }  // namespace
 
 sa_status sa_predict_mask(const void* q, const void* k, const sa_shape* shape,
@@ -221,12 +226,36 @@ sa_status sa_reorder_predict_mask(const int32_t* perm, const void* q, const void
   const size_t esz = shape->dtype == SA_BF16 ? 2 : 4;
   const size_t qbytes = (size_t)(shape->B * shape->Hq * shape->N * shape->d) * esz;
   const size_t kbytes = (size_t)(shape->B * shape->Hkv * shape->N * shape->d) * esz;
-  if (overlaps(q, q_r, qbytes) || overlaps(k, k_r, kbytes) || overlaps(q_r, k_r, qbytes < kbytes ? qbytes : kbytes) ||
-      overlaps(q, k_r, qbytes < kbytes ? qbytes : kbytes) || overlaps(k, q_r, qbytes < kbytes ? qbytes : kbytes))
+  if (ranges_overlap(q, qbytes, q_r, qbytes) || ranges_overlap(k, kbytes, k_r, kbytes) ||
+      ranges_overlap(q_r, qbytes, k_r, kbytes) || ranges_overlap(q, qbytes, k_r, kbytes) ||
+      ranges_overlap(k, kbytes, q_r, qbytes))
     return set_error(SA_ERR_INVALID_ARG, "q_r and k_r must not overlap q, k or each other");
   if (sa_status e = predict_prepare("sa_reorder_predict_mask", q, k, shape, params, ws, ws_bytes, out)) return e;
   return launch_predict(q, k, *shape, *params, predict_ws_carve(ws, *shape, params->bq, params->bk), *out,
                         static_cast<cudaStream_t>(stream), perm, q_r, k_r);
+}
+
+sa_status sa_reorder_predict_mask_q8(const int32_t* perm, const void* q, const void* k, int32_t format, void* q8,
+                                     float* q_scales, void* k8, float* k_scales, const sa_shape* shape,
+                                     const sa_mask_params* params, void* ws, size_t ws_bytes, sa_mask* out,
+                                     void* stream) {
+  if (sa_status e = check_shape(shape)) return e;
+  if (!q8 || !k8 || !q_scales || !k_scales) return set_error(SA_ERR_INVALID_ARG, "NULL code or scale array");
+  if (format != SA_Q_INT8 && format != SA_Q_E4M3)
+    return set_error(SA_ERR_INVALID_ARG, "format must be SA_Q_INT8 or SA_Q_E4M3");
+  if (shape->dtype != SA_BF16) return set_error(SA_ERR_UNSUPPORTED, "8-bit codes are written from bf16 input");
+  if ((uintptr_t)q8 % 16 || (uintptr_t)k8 % 16 || (uintptr_t)q_scales % 4 || (uintptr_t)k_scales % 4)
+    return set_error(SA_ERR_INVALID_ARG, "q8 and k8 must be 16-byte aligned");
+  const size_t qbytes = (size_t)(shape->B * shape->Hq * shape->N * shape->d);
+  const size_t kbytes = (size_t)(shape->B * shape->Hkv * shape->N * shape->d);
+  if (ranges_overlap(q, 2 * qbytes, q8, qbytes) || ranges_overlap(k, 2 * kbytes, k8, kbytes) ||
+      ranges_overlap(q8, qbytes, k8, kbytes) || ranges_overlap(q, 2 * qbytes, k8, kbytes) ||
+      ranges_overlap(k, 2 * kbytes, q8, qbytes))
+    return set_error(SA_ERR_INVALID_ARG, "q8 and k8 must not overlap q, k or each other");
+  if (sa_status e = predict_prepare("sa_reorder_predict_mask_q8", q, k, shape, params, ws, ws_bytes, out)) return e;
+  const PoolCodes codes{format, q8, q_scales, k8, k_scales};
+  return launch_predict(q, k, *shape, *params, predict_ws_carve(ws, *shape, params->bq, params->bk), *out,
+                        static_cast<cudaStream_t>(stream), perm, nullptr, nullptr, &codes);
 }
 
 size_t sa_mask_from_blocks_workspace(const sa_shape* shape, int32_t bq, int32_t bk) {
@@ -457,6 +486,24 @@ sa_status sa_reorder_heads(const int32_t* perms, const void* x, void* y, int64_t
   if ((uintptr_t)x % 2 || (uintptr_t)y % 2) return set_error(SA_ERR_INVALID_ARG, "misaligned tensor");
   if (sa_status e = check_device()) return e;
   return launch_reorder(perms, x, y, outer, N, bytes, false, static_cast<cudaStream_t>(stream), N);
+}
+
+sa_status sa_rows_attn(const void* q, const void* k, const void* v, const sa_shape* shape, const int32_t* rows,
+                       int64_t nrows, const int32_t* perms, const uint8_t* block_mask, int32_t bq, int32_t bk,
+                       float scale, float* out, float* lse, int32_t* status, void* stream) {
+  if (sa_status e = check_shape(shape)) return e;
+  if (!q || !k || !v || !out || (nrows > 0 && !rows)) return set_error(SA_ERR_INVALID_ARG, "NULL argument to sa_rows_attn");
+  if (nrows < 0) return set_error(SA_ERR_INVALID_ARG, "nrows must be >= 0");
+  if (bq < 1 || bk < 1) return set_error(SA_ERR_INVALID_ARG, "bq, bk must be positive");
+  if (!(scale >= 0.f) || std::isinf(scale)) return set_error(SA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (!rows_attn_supported(shape->d, shape->dv, shape->N, bk))
+    return set_error(SA_ERR_UNSUPPORTED, "sa_rows_attn needs d = dv in {64, 128} and N / bk <= 4096");
+  if ((uintptr_t)q % 16 || (uintptr_t)k % 16 || (uintptr_t)v % 16)
+    return set_error(SA_ERR_INVALID_ARG, "q, k, v must be 16-byte aligned");
+  if (sa_status e = check_device()) return e;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)shape->d);
+  return launch_rows_attn(q, k, v, *shape, rows, nrows, perms, block_mask, bq, bk, sc, out, lse, status,
+                          static_cast<cudaStream_t>(stream));
 }
 
 sa_status sa_rows_mse(const void* ref, const void* x, const int32_t* rows, int64_t nrows, int64_t BH, int64_t N,

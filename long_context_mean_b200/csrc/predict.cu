@@ -29,12 +29,16 @@ constexpr int kPoolWarps = kPoolThreads / 32;
 // four steps in flight; token norms reduce inside each token's lane group.
 // With perm, token n of the block is read from row perm[n] of x and also
 // written to row n of y (a1 fused with a2: the reordered copy is produced by
-// the same pass that pools it).
+// the same pass that pools it).  QF = 1 + SA_Q_INT8 or 1 + SA_Q_E4M3 (bf16
+// input): instead of the copy, the pass writes the block's 8-bit codes to
+// row n of y8 and its scale (absmax / 127 or / 448) to qscale, reading the
+// block a second time (from L2) once its absmax is known.
 // ---------------------------------------------------------------------------
-template <typename T>
+template <typename T, int QF = 0>
 __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
     const T* __restrict__ x, int64_t N, int d, int b, int nB, float* __restrict__ mean_out,
-    float* __restrict__ s_out, const int32_t* __restrict__ perm, T* __restrict__ y, int32_t* status) {
+    float* __restrict__ s_out, const int32_t* __restrict__ perm, T* __restrict__ y, int32_t* status,
+    uint2* __restrict__ y8 = nullptr, float* __restrict__ qscale = nullptr) {
   constexpr int EPL = 16 / sizeof(T);
   const int blk = blockIdx.x;
   const int64_t bh = blockIdx.y;
@@ -47,6 +51,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
   float ax[EPL], au[EPL];
 #pragma unroll
   for (int e = 0; e < EPL; ++e) ax[e] = au[e] = 0.f;
+  float amax = 0.f;                        // QF: block absmax
   const uint4* xbh = reinterpret_cast<const uint4*>(x + bh * N * (int64_t)d);
   uint4* ybh = y ? reinterpret_cast<uint4*>(y + bh * N * (int64_t)d) : nullptr;
   const int step = kPoolWarps * tpw;
@@ -83,6 +88,10 @@ __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
       for (int e = 0; e < EPL; ++e) {
         ax[e] += v[e];
         au[e] = fmaf(v[e], inv, au[e]);
+      }
+      if constexpr (QF != 0) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) amax = fmaxf(amax, fabsf(v[e]));
       }
     }
   }
@@ -122,6 +131,29 @@ __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
     float tot = 0.f;
     for (int w = 0; w < kPoolWarps; ++w) tot += red[w];
     s_out[bh * nB + blk] = tot / ((float)cnt * (float)cnt);
+  }
+  if constexpr (QF != 0) {
+    static_assert(sizeof(T) == 2, "8-bit codes are written from bf16 input");
+    constexpr int FMT = QF - 1;
+    __shared__ float wmax[kPoolWarps];
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) wmax[warp] = amax;
+    __syncthreads();
+    float A = 0.f;
+#pragma unroll
+    for (int w = 0; w < kPoolWarps; ++w) A = fmaxf(A, wmax[w]);
+    const float qmax = FMT == SA_Q_E4M3 ? 448.0f : 127.0f;
+    const float qinv = A > 0.f ? __fdiv_rn(qmax, A) : 0.f;
+    if (threadIdx.x == 0) qscale[bh * nB + blk] = A > 0.f ? __fdiv_rn(A, qmax) : 0.f;
+    uint2* y8bh = y8 + bh * N * (int64_t)chunks;
+    for (int tb = warp * tpw; tb < cnt; tb += step) {
+      const int tok = tb + sub;
+      if (tok >= cnt) continue;
+      const int64_t n = t0 + tok;
+      const int64_t src = perm ? (int64_t)__ldg(perm + n) : n;
+      if ((uint64_t)src >= (uint64_t)N) continue;          // raised in the first pass
+      y8bh[n * chunks + c] = quant8<FMT>(__ldg(xbh + src * chunks + c), qinv);
+    }
   }
 }
 
@@ -691,6 +723,22 @@ sa_status launch_pool(const void* x, int64_t BH, int64_t N, int d, int b, int64_
   return check_launch("pool_cossim_kernel");
 }
 
+// Pooling with 8-bit codes and block scales instead of the reordered copy.
+sa_status launch_pool_codes(const void* x, int64_t BH, int64_t N, int d, int b, int64_t nB, float* mean,
+                            float* sim, const int32_t* perm, int32_t fmt, void* y8, float* qscale, int32_t* status,
+                            cudaStream_t st) {
+  dim3 grid((unsigned)nB, (unsigned)BH);
+  if (fmt == SA_Q_E4M3)
+    pool_cossim_kernel<uint16_t, 1 + SA_Q_E4M3><<<grid, kPoolThreads, 0, st>>>(
+        static_cast<const uint16_t*>(x), N, d, b, (int)nB, mean, sim, perm, nullptr, status,
+        static_cast<uint2*>(y8), qscale);
+  else
+    pool_cossim_kernel<uint16_t, 1 + SA_Q_INT8><<<grid, kPoolThreads, 0, st>>>(
+        static_cast<const uint16_t*>(x), N, d, b, (int)nB, mean, sim, perm, nullptr, status,
+        static_cast<uint2*>(y8), qscale);
+  return check_launch("pool_cossim_kernel");
+}
+
 }  // namespace
 
 size_t predict_ws_bytes(const sa_shape& s, int bq, int bk, size_t off[6]) {
@@ -728,12 +776,19 @@ size_t lists_ws_bytes(const sa_shape& s, int bq, int) {
 
 sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
                          const sa_mask_params& p, const PredictWs& w, sa_mask& out,
-                         cudaStream_t st, const int32_t* perm, void* q_r, void* k_r) {
+                         cudaStream_t st, const int32_t* perm, void* q_r, void* k_r, const PoolCodes* codes) {
   const int64_t nqb = out.nqb, nkb = out.nkb;
   if (cudaMemsetAsync(out.status, 0, sizeof(int32_t), st) != cudaSuccess)
     return set_error(SA_ERR_CUDA, "cudaMemsetAsync(status) failed");
   sa_status e;
-  if (s.dtype == SA_BF16) {
+  if (codes) {   // bf16 input: codes and scales instead of reordered copies
+    if ((e = launch_pool_codes(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, perm, codes->format,
+                               codes->q8, codes->q_scales, out.status, st)))
+      return e;
+    if ((e = launch_pool_codes(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, w.sk, perm, codes->format,
+                               codes->k8, codes->k_scales, out.status, st)))
+      return e;
+  } else if (s.dtype == SA_BF16) {
     if ((e = launch_pool<uint16_t>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, perm, q_r,
                                    out.status, st)))
       return e;

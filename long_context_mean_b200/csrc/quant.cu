@@ -14,8 +14,6 @@
 // The attention kernel multiplies the exact int32 tile of q8 . k8 by one
 // float per kept tile: scale * log2(e) * scale_q(query block) *
 // scale_k(key block), written in CSR order by tile_scales_kernel.
-#include <cuda_fp8.h>
-
 #include "sa_internal.cuh"
 
 namespace sa {
@@ -33,23 +31,6 @@ __device__ __forceinline__ uint32_t bf16_abs_max4(uint4 v) {
     m = max(m, (w[i] >> 16) & 0x7FFFu);
   }
   return m;
-}
-
-__device__ __forceinline__ uint32_t quant1(uint32_t bits16, float inv) {
-  const float f = __uint_as_float(bits16 << 16);
-  int q = __float2int_rn(f * inv);
-  q = max(-127, min(127, q));
-  return (uint32_t)(uint8_t)(int8_t)q;
-}
-// Two bf16 values (low, high half of w) to two 8-bit codes (low byte first).
-template <int FMT>
-__device__ __forceinline__ uint32_t quant2(uint32_t w, float inv) {
-  if constexpr (FMT == SA_Q_E4M3) {
-    const float2 f = make_float2(__uint_as_float(w << 16) * inv, __uint_as_float(w & 0xFFFF0000u) * inv);
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
-  } else {
-    return quant1(w & 0xFFFFu, inv) | (quant1(w >> 16, inv) << 8);
-  }
 }
 
 // One CTA per (head, block).  x: bf16 [heads][N][d]; x8: 8-bit codes
@@ -90,9 +71,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_blocks_kernel(const uint4
   for (int i = 0; i < kQuantMaxVec; ++i) {
     const int64_t e = threadIdx.x + (int64_t)i * kQuantThreads;
     if (e < total) {
-      const uint32_t lo = quant2<FMT>(v[i].x, inv) | (quant2<FMT>(v[i].y, inv) << 16);
-      const uint32_t hi = quant2<FMT>(v[i].z, inv) | (quant2<FMT>(v[i].w, inv) << 16);
-      x8[base + e] = make_uint2(lo, hi);
+      x8[base + e] = quant8<FMT>(v[i], inv);
     }
   }
 }

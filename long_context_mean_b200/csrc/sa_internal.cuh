@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include "sparse_attn.h"
@@ -30,6 +31,32 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
 __device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
   __nv_bfloat16 h = __float2bfloat16_rn(f);
   return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// 8-bit codes of two bf16 values (low, high half of w), low byte first:
+// INT8 rint(x * inv) clamped to [-127, 127]; E4M3 by the saturating
+// hardware conversion of x * inv (ties to even).  Used by the standalone
+// quantisation kernel and by the pooling pass that writes codes directly.
+__device__ __forceinline__ uint32_t quant_int8(uint32_t bits16, float inv) {
+  const float f = __uint_as_float(bits16 << 16);
+  int q = __float2int_rn(f * inv);
+  q = max(-127, min(127, q));
+  return (uint32_t)(uint8_t)(int8_t)q;
+}
+template <int FMT>
+__device__ __forceinline__ uint32_t quant2(uint32_t w, float inv) {
+  if constexpr (FMT == SA_Q_E4M3) {
+    const float2 f = make_float2(__uint_as_float(w << 16) * inv, __uint_as_float(w & 0xFFFF0000u) * inv);
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+  } else {
+    return quant_int8(w & 0xFFFFu, inv) | (quant_int8(w >> 16, inv) << 8);
+  }
+}
+// Eight bf16 values (one 16-byte vector) to eight codes.
+template <int FMT>
+__device__ __forceinline__ uint2 quant8(const uint4& v, float inv) {
+  return make_uint2(quant2<FMT>(v.x, inv) | (quant2<FMT>(v.y, inv) << 16),
+                    quant2<FMT>(v.z, inv) | (quant2<FMT>(v.w, inv) << 16));
 }
 
 template <typename T> struct Elem;
@@ -89,10 +116,20 @@ size_t lists_ws_bytes(const sa_shape& s, int bq, int bk);
 
 // With perm (nullable), q and k are in the original token order: the pooling
 // pass reads row perm[n] for token n and writes the reordered copies q_r, k_r.
+// Optional 8-bit outputs of the pooling pass (instead of reordered bf16
+// copies): the codes and block scales of Q (per query block) and K (per key
+// block) in `format`.
+struct PoolCodes {
+  int32_t format;
+  void* q8;
+  float* q_scales;
+  void* k8;
+  float* k_scales;
+};
 sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
                          const sa_mask_params& p, const PredictWs& w, sa_mask& out,
                          cudaStream_t st, const int32_t* perm = nullptr, void* q_r = nullptr,
-                         void* k_r = nullptr);
+                         void* k_r = nullptr, const PoolCodes* codes = nullptr);
 sa_status launch_mask_from_blocks(const uint8_t* in, const sa_shape& s, int bq, int bk,
                                   int causal, int32_t* counts, int32_t* tmp, sa_mask& out,
                                   cudaStream_t st);
@@ -124,6 +161,10 @@ struct AttnArgs {
 sa_status launch_attn_simt(const AttnArgs& a, cudaStream_t st);
 sa_status launch_head_placement(int64_t T, int64_t P, int64_t n, const int32_t* kinds, int64_t heads, int bq,
                                 int bk, int32_t* perms, uint8_t* mask, int32_t* status, cudaStream_t st);
+bool rows_attn_supported(int64_t d, int64_t dv, int64_t N, int bk);
+sa_status launch_rows_attn(const void* q, const void* k, const void* v, const sa_shape& s, const int32_t* rows,
+                           int64_t nrows, const int32_t* perms, const uint8_t* block_mask, int bq, int bk,
+                           float scale, float* out, float* lse, int32_t* status, cudaStream_t st);
 sa_status launch_rows_mse(const void* ref, const void* x, const int32_t* rows, int64_t nrows, int64_t BH, int64_t N,
                           int64_t dv, int32_t dtype, double* out, int32_t* status, cudaStream_t st);
 sa_status launch_quant_blocks(const void* x, int64_t heads, int64_t N, int64_t d, int rows, int32_t fmt, void* x8,

@@ -35,8 +35,9 @@ EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_attn_worksp
            "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_reorder_predict_mask", "sa_predict_mask_noalloc",
            "sa_mask_from_blocks_workspace",
            "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status", "sa_l1_error",
-           "sa_head_placement", "sa_reorder_heads", "sa_rows_mse",
-           "sa_quantize_blocks", "sa_attn_qk8_workspace", "sa_block_sparse_attn_qk8"]
+           "sa_head_placement", "sa_reorder_heads", "sa_rows_attn", "sa_rows_mse",
+           "sa_quantize_blocks", "sa_attn_qk8_workspace", "sa_block_sparse_attn_qk8",
+           "sa_reorder_predict_mask_q8"]
 
 
 class SAError(RuntimeError):
@@ -113,9 +114,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sa_reorder_heads": (I32, [P, P, P, I64, I64, I64, I32, P]),
         "sa_quantize_blocks": (I32, [P, I64, I64, I64, I32, I32, I32, P, P, P]),
         "sa_attn_qk8_workspace": (SZ, [ctypes.POINTER(Mask)]),
+        "sa_reorder_predict_mask_q8": (I32, [P, P, P, I32, P, P, P, P, ctypes.POINTER(Shape),
+                                             ctypes.POINTER(MaskParams), P, SZ, ctypes.POINTER(Mask), P]),
         "sa_block_sparse_attn_qk8": (I32, [P, P, P, P, I32, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F,
                                            F, P, P, P, P, P, SZ, I32, P]),
         "sa_rows_mse": (I32, [P, P, P, I64, I64, I64, I64, I32, P, P, P]),
+        "sa_rows_attn": (I32, [P, P, P, ctypes.POINTER(Shape), P, I64, P, P, I32, I32, F, P, P, P, P]),
         "sa_block_sparse_attn": (I32, [P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(Mask), F, F,
                                        P, P, P, P, P, SZ, I32, P]),
         "sa_dense_attn": (I32, [P, P, P, ctypes.POINTER(Shape), I32, F, P, P, P, P, SZ, I32, P]),
@@ -284,6 +288,16 @@ def quantize_blocks(x, rows, x8, scales, fmt="int8", stream=None):
                                      _ptr(scales), _stream(stream)))
 
 
+def reorder_predict_mask_q8(perm, q, k, fmt, q8, q_scales, k8, k_scales, shape: Shape, params: MaskParams, ws,
+                            mask: Mask, stream=None):
+    """Mask prediction whose pooling pass writes the reordered 8-bit codes
+    and block scales of Q and K (perm None: the original order)."""
+    _check(load().sa_reorder_predict_mask_q8(_ptr(perm), _ptr(q), _ptr(k), Q_FORMATS[fmt], _ptr(q8), _ptr(q_scales),
+                                             _ptr(k8), _ptr(k_scales), ctypes.byref(shape), ctypes.byref(params),
+                                             _ptr(ws), ws.numel() * ws.element_size(), ctypes.byref(mask),
+                                             _stream(stream)))
+
+
 def attn_qk8_workspace(mask: Mask) -> int:
     return int(load().sa_attn_qk8_workspace(ctypes.byref(mask)))
 
@@ -329,6 +343,16 @@ def reorder_heads(perms, x, y, stream=None):
     N, row = x.shape[-2], x.shape[-1]
     outer = x.numel() // (N * row)
     _check(load().sa_reorder_heads(_ptr(perms), _ptr(x), _ptr(y), outer, N, row, dtype_code(x), _stream(stream)))
+
+
+def rows_attn(q, k, v, shape: Shape, rows, out, lse=None, perms=None, block_mask=None, bq=128, bk=64, scale=0.0,
+              status=None, stream=None):
+    """Attention of the sampled query rows only: out [B*Hq, nrows, dv] and
+    lse [B*Hq, nrows] (float32), over every key or over a candidate's kept
+    tiles in each head's order (perms, block_mask from head_placement)."""
+    _check(load().sa_rows_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), _ptr(rows), rows.numel(), _ptr(perms),
+                               _ptr(block_mask), bq, bk, float(scale), _ptr(out), _ptr(lse), _ptr(status),
+                               _stream(stream)))
 
 
 def rows_mse(ref, x, rows, out, status=None, stream=None):
@@ -405,8 +429,9 @@ class Pipeline:
         self.inv = torch.empty(N, dtype=torch.int32, device=device)
         self.layout_ws = workspace(layout_workspace(layout), device)
         if not self.identity:
-            self.qr = torch.empty(B, Hq, N, d, dtype=tdt, device=device)
-            self.kr = torch.empty(B, Hkv, N, d, dtype=tdt, device=device)
+            if not qk8:   # the 8-bit path gets codes from the pooling pass instead
+                self.qr = torch.empty(B, Hq, N, d, dtype=tdt, device=device)
+                self.kr = torch.empty(B, Hkv, N, d, dtype=tdt, device=device)
             self.vr = torch.empty(B, Hkv, N, dv, dtype=tdt, device=device)
         self.out = torch.empty(B, Hq, N, dv, dtype=tdt, device=device)
         self.lse = torch.empty(B, Hq, N, 1, dtype=torch.float32, device=device)
@@ -444,9 +469,10 @@ class Pipeline:
         lse = self.lse if lse is None else lse
         if self.identity:
             qr, kr, vr = q, k, v
-            predict_mask(qr, kr, self.shape, self.params, self.ws, self.mask.struct, stream)
             if self.qk8:
-                self._quantize(qr, kr, stream)
+                self._predict_codes(None, q, k, stream)
+            else:
+                predict_mask(qr, kr, self.shape, self.params, self.ws, self.mask.struct, stream)
         else:
             import torch
             st = stream if stream is not None else torch.cuda.current_stream(q.device)
@@ -458,14 +484,16 @@ class Pipeline:
             reorder(self.perm, v, self.vr, self.side)
             v.record_stream(self.side)   # the caller's v stays allocated until the side stream has read it
             self.ev_v.record(self.side)
-            # Q and K are reordered by the pooling pass of the prediction.
-            reorder_predict_mask(self.perm, q, k, self.qr, self.kr, self.shape, self.params, self.ws,
-                                 self.mask.struct, st)
-            if self.qk8:   # beside the V reorder, which needs no codes
-                self._quantize(self.qr, self.kr, st)
+            # Q and K are reordered (or reordered and quantised) by the
+            # pooling pass of the prediction.
+            if self.qk8:
+                self._predict_codes(self.perm, q, k, st)
+            else:
+                reorder_predict_mask(self.perm, q, k, self.qr, self.kr, self.shape, self.params, self.ws,
+                                     self.mask.struct, st)
             st.wait_event(self.ev_v)
             stream = st
-            qr, kr, vr = self.qr, self.kr, self.vr
+            qr, kr, vr = (None, None, self.vr) if self.qk8 else (self.qr, self.kr, self.vr)
         # The inverse reorder of O and LSE is fused into the attention store
         # (out_perm); sa_unreorder stays available for standalone use.
         out_perm = None if self.identity else self.perm
@@ -478,9 +506,9 @@ class Pipeline:
                               self.skip_log, self.flags, stream, ws=self.attn_ws, out_perm=out_perm)
         return out, lse
 
-    def _quantize(self, qr, kr, stream):
-        quantize_blocks(qr, self.params.bq, self.q8, self.q_scales, self.qk8, stream)
-        quantize_blocks(kr, self.params.bk, self.k8, self.k_scales, self.qk8, stream)
+    def _predict_codes(self, perm, q, k, stream):
+        reorder_predict_mask_q8(perm, q, k, self.qk8, self.q8, self.q_scales, self.k8, self.k_scales, self.shape,
+                                self.params, self.ws, self.mask.struct, stream)
 
     def status(self, stream=None) -> int:
         return read_status(self.mask.status, stream)

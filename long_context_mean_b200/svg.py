@@ -6,7 +6,9 @@ Each head runs one of two fixed candidates: spatial (the pairs of one frame,
 frame-major order) or temporal (the pairs of one position across frames,
 token-major order); text tokens pair with every token.  ``profile`` draws a
 few query rows, computes dense attention and both candidates, and picks per
-head the candidate with the smaller mean squared output error on those rows.
+head the candidate with the smaller mean squared output error on those rows;
+only the sampled rows are computed (``sa_rows_attn``), densely and under
+each candidate.
 ``run`` then enqueues, on one stream: Q, K, V into every head's own order
 (one ``sa_reorder_heads`` pass each), block-sparse attention over the tile
 covers, and the store back into the original order fused into the
@@ -85,23 +87,29 @@ class SvgPipeline:
         return out, lse
 
     def profile(self, q, k, v, stream=None):
-        """Online profiling: dense attention and both candidates on every
-        head, the sampled-row MSE of each against dense, argmin per head
-        (ties to spatial).  Places the choice and returns (choice list,
-        mse [2, heads] on the host)."""
+        """Online profiling on the sampled rows: their dense attention and
+        their attention under each candidate (every head on that candidate),
+        the MSE of each against dense, argmin per head (ties to spatial).
+        Places the choice and returns (choice list, mse [2, heads] on the
+        host)."""
         import torch
         BH = self.kinds.numel()
-        dense = torch.empty_like(self.out)
-        cand = torch.empty_like(self.out)
+        nr = self.rows.numel()
+        dv = self.shape.dv
+        dense = torch.empty(BH, nr, dv, dtype=torch.float32, device=self.device)
+        cand = torch.empty_like(dense)
+        every = torch.arange(nr, dtype=torch.int32, device=self.device)
         st = torch.zeros(1, dtype=torch.int32, device=self.device)
-        sa.dense_attn(q, k, v, self.shape, False, self.scale, dense, None, st, self.flags, stream,
-                      ws=self.attn_ws)
+        sa.rows_attn(q, k, v, self.shape, self.rows, dense, None, bq=self.bq, bk=self.bk, scale=self.scale,
+                     status=st, stream=stream)
         for c in (SPATIAL, TEMPORAL):
-            self.place([c] * BH, stream)
-            self.run(q, k, v, stream, out=cand, lse=self.lse)
-            sa.rows_mse(dense, cand, self.rows, self.mse[c], st, stream)
             with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream(self.device)):
-                torch.maximum(st, self.mask.status, out=st)   # keep this candidate's status
+                self.kinds.fill_(c)
+            sa.head_placement(self.T, self.Hg, self.Wg, self.txt_len, self.kinds, self.bq, self.bk, self.perms,
+                              self.mask.block_mask, st, stream)
+            sa.rows_attn(q, k, v, self.shape, self.rows, cand, None, self.perms, self.mask.block_mask, self.bq,
+                         self.bk, self.scale, st, stream)
+            sa.rows_mse(dense, cand, every, self.mse[c], st, stream)
         if sa.read_status(st, stream) != sa.SA_OK:
             raise RuntimeError("device status raised during profiling")
         mse = self.mse.cpu()

@@ -146,3 +146,46 @@ def test_pipeline_qk8_video_sampled(fmt):
         ref_out = Y.unreorder(ref["out"], perm, axis=2)
         ref_lse = Y.unreorder(ref["lse"], perm, axis=2)
         P.attention_check(out[:, h:h + 1], lse[:, h:h + 1], {"out": ref_out, "lse": ref_lse})
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("reordered", [True, False])
+def test_fused_codes_match_quantised_reordered_inputs(fmt, reordered):
+    """sa_reorder_predict_mask_q8 on the video workload: the codes and scales
+    its pooling pass writes equal the oracle's quantisation of the reordered
+    (or original) Q and K, and the mask equals the bf16 prediction's."""
+    import torch
+    from long_context_mean_b200 import sa
+    w = I.WORKLOADS["video"]
+    g = I.gen_qkv(w)
+    q, k, v = P.qkv_dev(g, w.dtype)
+    pipe = sa.pipeline_for(w)
+    shape = pipe.shape
+    if reordered:
+        sa.layout_build(pipe.layout, pipe.perm, pipe.inv, pipe.layout_ws)
+        perm, _ = Y.build_layout(w.order, w.T, w.H, w.W, w.win, w.sink_frames, w.txt_len)
+        assert np.array_equal(pipe.perm.cpu().numpy(), perm)
+        perm_dev = pipe.perm
+    else:
+        perm_dev, perm = None, np.arange(w.N)
+    nqb, nkb = pipe.mask.struct.nqb, pipe.mask.struct.nkb
+    q8 = torch.empty(q.shape, dtype=torch.uint8, device="cuda")
+    k8 = torch.empty(k.shape, dtype=torch.uint8, device="cuda")
+    qs = torch.empty(w.B * w.Hq * nqb, dtype=torch.float32, device="cuda")
+    ks = torch.empty(w.B * w.Hkv * nkb, dtype=torch.float32, device="cuda")
+    m8 = sa.MaskBuffers.allocate(w.B, w.Hq, w.N, w.bq, w.bk, "cuda")
+    sa.reorder_predict_mask_q8(perm_dev, q, k, fmt, q8, qs, k8, ks, shape, pipe.params, pipe.ws, m8.struct)
+    assert sa.read_status(m8.status) == 0
+    qr = torch.empty_like(q)
+    kr = torch.empty_like(k)
+    mb = sa.MaskBuffers.allocate(w.B, w.Hq, w.N, w.bq, w.bk, "cuda")
+    if reordered:
+        sa.reorder_predict_mask(pipe.perm, q, k, qr, kr, shape, pipe.params, pipe.ws, mb.struct)
+    else:
+        sa.predict_mask(q, k, shape, pipe.params, pipe.ws, mb.struct)
+    assert sa.read_status(mb.status) == 0
+    assert torch.equal(m8.block_mask, mb.block_mask)
+    for x8, sc, name, rows in ((q8, qs, "q", w.bq), (k8, ks, "k", w.bk)):
+        ref8, refs = Q.quantize_blocks(Y.reorder(g[name], perm), rows, fmt)
+        assert np.array_equal(x8.cpu().numpy().view(ref8.dtype), ref8)
+        assert np.array_equal(sc.cpu().numpy().reshape(refs.shape).view(np.uint32), refs.view(np.uint32))

@@ -86,6 +86,62 @@ def test_rows_mse_is_the_oracle():
     assert sa.read_status(st) == sa.SA_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("dt,d,Hq,Hkv", [("bf16", 128, 4, 2), ("fp32", 64, 2, 2)])
+def test_rows_attn_dense_vs_oracle(dt, d, Hq, Hkv):
+    """Sampled rows (with a repeat and both ends) against the dense softmax."""
+    import torch
+    from long_context_mean_b200 import sa
+    N = 421
+    w = I.Workload("rows", 77, 1, Hq, Hkv, 1, 1, N, 0, d, d, dt, "iid")
+    g = I.gen_qkv(w)
+    q, k, v = P.qkv_dev(g, dt)
+    rows = np.array([0, N - 1, 200, 200, 17, 399], dtype=np.int32)
+    out = torch.empty(Hq, rows.size, d, dtype=torch.float32, device="cuda")
+    lse = torch.empty(Hq, rows.size, dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.rows_attn(q, k, v, sa.make_shape(q, k, v), torch.from_numpy(rows).cuda(), out, lse, status=st)
+    assert sa.read_status(st) == 0
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for h in range(Hq):
+        y, _, l = A.masked_attention(g["q"][0, h][rows], g["k"][0, h // (Hq // Hkv)], g["v"][0, h // (Hq // Hkv)],
+                                     np.ones((rows.size, N), bool))
+        assert np.abs(out[h] - y).max() < 1e-4
+        assert np.abs(lse[h] - l).max() < 1e-4
+
+
+def test_rows_attn_candidates_vs_oracle():
+    """Sampled rows under each head's candidate (placement from the GPU)
+    against the oracle's candidate attention at those rows."""
+    import torch
+    from long_context_mean_b200 import sa
+    T, Hg, Wg, txt = SMALL["T"], SMALL["Hg"], SMALL["Wg"], SMALL["txt"]
+    bias = ["frame", "position", "position", "frame"]
+    kinds = [S.SPATIAL, S.TEMPORAL, S.SPATIAL, S.TEMPORAL]
+    g = I.biased_video_heads(T, Hg, Wg, txt, bias, seed=5)
+    q, k, v = (P.bf16_dev(g[n + "_bits"]) for n in "qkv")
+    n = T * Hg * Wg + txt
+    perms = torch.empty(4, n, dtype=torch.int32, device="cuda")
+    bm = torch.empty(4, -(-n // 128), -(-n // 64), dtype=torch.uint8, device="cuda")
+    kd = torch.tensor(kinds, dtype=torch.int32, device="cuda")
+    sa.head_placement(T, Hg, Wg, txt, kd, 128, 64, perms, bm)
+    rows = np.array([0, 5, 130, 383, 384, 420, 250], dtype=np.int32)
+    out = torch.empty(4, rows.size, 128, dtype=torch.float32, device="cuda")
+    lse = torch.empty(4, rows.size, dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.rows_attn(q, k, v, sa.make_shape(q, k, v), torch.from_numpy(rows).cuda(), out, lse, perms, bm, 128, 64,
+                 status=st)
+    assert sa.read_status(st) == 0
+    out_h, lse_h = out.cpu().numpy(), lse.cpu().numpy()
+    for h, c in enumerate(kinds):
+        y, l = S.candidate_attention(g["q"][0, h], g["k"][0, h], g["v"][0, h], T, Hg, Wg, txt, c, 128, 64)
+        assert np.abs(out_h[h] - y[rows]).max() < 1e-4
+        assert np.abs(lse_h[h] - l[rows]).max() < 1e-4
+    bad = torch.tensor([0, n], dtype=torch.int32, device="cuda")
+    out2 = torch.empty(4, 2, 128, dtype=torch.float32, device="cuda")
+    sa.rows_attn(q, k, v, sa.make_shape(q, k, v), bad, out2, None, perms, bm, 128, 64, status=st)
+    assert sa.read_status(st) == sa.SA_ERR_INVALID_ARG
+
+
 def _small_pipe(bias, flags=0, **kw):
     from long_context_mean_b200 import svg
     g = I.biased_video_heads(SMALL["T"], SMALL["Hg"], SMALL["Wg"], SMALL["txt"], bias, seed=11)
