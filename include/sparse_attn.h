@@ -171,7 +171,9 @@ sa_status sa_layout_build(const sa_layout_desc* desc, int32_t* perm, int32_t* in
  * x, y are [outer, N, row] arrays of `row` elements of `dtype` per token
  * (outer = B*H).  sa_reorder: y[o, n, :] = x[o, perm[n], :].
  * sa_unreorder: x[o, perm[n], :] = y[o, n, :] (pass the same perm).
- * x and y must not overlap.  row = 1 with SA_FP32 reorders LSE. */
+ * perm must be a permutation of [0, N) (device int32; not checked here:
+ * sa_layout_build produces one).  x and y must not overlap.  row = 1 with
+ * SA_FP32 reorders LSE. */
 sa_status sa_reorder(const int32_t* perm, const void* x, void* y, int64_t outer,
                      int64_t N, int64_t row, int32_t dtype, void* stream);
 sa_status sa_unreorder(const int32_t* perm, const void* y, void* x, int64_t outer,
