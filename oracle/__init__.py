@@ -26,8 +26,16 @@ The pages are cited by title and section:
 * [P5] "78. Attention Access Pattern Benchmark" (datawhale llm-algo-leetcode),
   Steps 2 and 4 (selective sparse = window + anchors, coverage ledger).
 
+Modules: ``attention`` (restricted softmax, tile recurrence, PV skip),
+``layout`` (identity, window and Hilbert orders), ``predict`` (pooling,
+CosSim, TopCdf, forced blocks), ``ledger`` (pair and tile ledgers),
+``calibrate`` ((tau, theta) then lambda under L1 bounds, [P3] 2.4), ``quant``
+(per-block INT8 / FP8 E4M3 QK, [P3] 2.4), ``svg`` (per-head spatial /
+temporal candidates and their sampled-row choice, [P1] 3.3-5),
+``tune_tau`` (the script that froze the workloads' tau).
+
 Parity status per function is stated in each module header; the one part the
 pages leave unpinned is the exact Hilbert curve (see ``oracle.layout``).
 """
 
-from . import attention, layout, predict, ledger  # noqa: F401
+from . import attention, layout, predict, ledger, calibrate, quant, svg  # noqa: F401
