@@ -171,3 +171,41 @@ def test_kernel_path_selection(lib):
     s32 = _shape(dtype=sa.SA_FP32, d=16, dv=16)
     assert sa.attn_kernel_path(s32, 16, 16) == 0
     assert sa.attn_kernel_path(s, 129, 64) == -1
+
+
+def _declarations():
+    """name -> list of parameter type strings, from the header's prototypes."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(?:sa_status|size_t|int32_t|const char\*)\s+(sa_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        # drop the parameter name; an array parameter (size_t offsets[6]) is a pointer
+        out[m.group(1)] = [p.rsplit(None, 1)[0] + ("*" if "[" in p else "") for p in params]
+    return out
+
+
+def _category(ctype_param):
+    """Compare a header parameter type with a ctypes argtype by kind and width."""
+    if "*" in ctype_param:
+        return "pointer"
+    base = ctype_param.replace("const", "").strip()
+    return {"int32_t": "i32", "int64_t": "i64", "size_t": "size", "float": "f32"}[base]
+
+
+def _ctypes_category(t):
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "pointer"
+    return {ctypes.c_int32: "i32", ctypes.c_int64: "i64", ctypes.c_size_t: "size", ctypes.c_float: "f32"}[t]
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every ctypes argtype list has the header's parameter count and kinds
+    (pointer, int32, int64, size_t, float), so a changed prototype cannot
+    silently shift the arguments of a call."""
+    decls = _declarations()
+    assert set(decls) == set(sa.EXPORTS)
+    for name, params in decls.items():
+        argtypes = getattr(lib, name).argtypes or []
+        assert len(argtypes) == len(params), (name, params, argtypes)
+        for p, t in zip(params, argtypes):
+            assert _category(p) == _ctypes_category(t), (name, p, t)
