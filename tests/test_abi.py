@@ -209,3 +209,28 @@ def test_binding_signatures_match_the_header(lib):
         assert len(argtypes) == len(params), (name, params, argtypes)
         for p, t in zip(params, argtypes):
             assert _category(p) == _ctypes_category(t), (name, p, t)
+
+
+def test_header_is_plain_c(tmp_path):
+    """The boundary is a C ABI: the header compiles as strict C99 and as C++."""
+    import shutil
+    import subprocess
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "sparse_attn.h"\nint main(void) { return (int)sizeof(sa_shape) == 0; }\n')
+    inc = os.path.dirname(HEADER)
+    for comp, flags in (("gcc", ["-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror"]),
+                        ("g++", ["-std=c++17", "-Wall", "-Werror", "-x", "c++"])):
+        if shutil.which(comp) is None:
+            pytest.skip(f"{comp} not installed")
+        r = subprocess.run([comp, *flags, "-fsyntax-only", "-I", inc, str(src)], capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+
+
+def test_binding_return_types_match_the_header(lib):
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    kinds = {"sa_status": ctypes.c_int32, "size_t": ctypes.c_size_t, "int32_t": ctypes.c_int32,
+             "const char*": ctypes.c_char_p}
+    found = re.findall(r"\b(sa_status|size_t|int32_t|const char\*)\s+(sa_[a-z0-9_]+)\s*\(", text)
+    assert {n for _, n in found} == set(sa.EXPORTS)
+    for ret, name in found:
+        assert getattr(lib, name).restype is kinds[ret], (name, ret)
