@@ -234,3 +234,47 @@ def test_binding_return_types_match_the_header(lib):
     assert {n for _, n in found} == set(sa.EXPORTS)
     for ret, name in found:
         assert getattr(lib, name).restype is kinds[ret], (name, ret)
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "sparse_attn.h"
+
+int main(void) {
+  sa_shape s = {1, 2, 2, 300, 128, 128, SA_BF16, 0};
+  sa_mask_params p;
+  memset(&p, 0, sizeof p);
+  p.bq = 128; p.bk = 64; p.tau = 0.5f; p.theta = 0.0f;
+  if (strstr(sa_version(), "sm_100a") == NULL) return 10;
+  if (sa_attn_workspace() == 0) return 11;
+  if (sa_predict_mask_workspace(&s, &p) == 0) return 12;
+  /* argument errors are reported before anything touches a device */
+  if (sa_reorder(NULL, (void*)4096, (void*)8192, 1, 10, 128, SA_BF16, NULL) != SA_ERR_INVALID_ARG) return 13;
+  if (sa_read_status(NULL, NULL) != SA_ERR_INVALID_ARG) return 14;
+  if (sa_last_error()[0] == '\0') return 15;
+  printf("c client ok\n");
+  return 0;
+}
+"""
+
+
+def test_plain_c_client_links_and_calls(tmp_path):
+    """A C program (no Python, no torch) includes the header, links the
+    shared library and gets its host-side answers."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not installed")
+    if not os.path.exists(sa.LIB_PATH):
+        from long_context_mean_b200 import build
+        build.build()
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(sa.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                        "-L", libdir, "-l:libsparseattn.so", f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0 and "c client ok" in run.stdout, (run.returncode, run.stdout, run.stderr)
