@@ -11,9 +11,10 @@
 // has scale 0 and codes 0.  Both divisions are correctly rounded
 // (__fdiv_rn), so the codes do not depend on compiler flags.
 //
-// The attention kernel multiplies the exact int32 tile of q8 . k8 by one
-// float per kept tile: scale * log2(e) * scale_q(query block) *
-// scale_k(key block), written in CSR order by tile_scales_kernel.
+// The attention kernel multiplies the tile of q8 . k8 (exact int32 for
+// INT8, fp32-accumulated for E4M3) by one float per kept tile:
+// scale * log2(e) * scale_q(query block) * scale_k(key block), written in
+// CSR order by tile_scales_kernel.
 #include "sa_internal.cuh"
 
 namespace sa {
