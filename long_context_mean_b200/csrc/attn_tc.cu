@@ -33,6 +33,11 @@
 //   maximum that only moves when the running max exceeds it by more than
 //   2^8 (O / l is the same quotient).  A row whose maximum moves has a gap of
 //   0, so a tile that needs a rescale is never skipped.
+// 8-bit QK ([P3] 2.4, QM = 1: INT8, 2: FP8 E4M3): Q and K tiles hold one
+// code per element (one 128-byte swizzle row per token), S is four
+// kind::i8 / kind::f8f6f4 steps, and the softmax multiplies each tile by its
+// own scale (the two block scales of the quantisation); INT8 scores are
+// int32 and reach the float path through an exact biased-float add.
 // Every mbarrier wait is bounded (2 s); on expiry the kernel raises
 // SA_ERR_TIMEOUT, every later wait returns at once, the producers drain
 // their own loads (bounded) and the TMEM allocation is released.
