@@ -34,8 +34,10 @@ CosSim, TopCdf, forced blocks), ``ledger`` (pair and tile ledgers),
 temporal candidates and their sampled-row choice, [P1] 3.3-5),
 ``tune_tau`` (the script that froze the workloads' tau).
 
-Parity status per function is stated in each module header; the one part the
-pages leave unpinned is the exact Hilbert curve (see ``oracle.layout``).
+Parity status per function is stated in each module header.  The pages name
+no Hilbert variant; ``oracle.layout`` pins Skilling's curve against an
+independent two-dimensional construction and the three-dimensional defining
+properties of a Hilbert curve.
 """
 
 from . import attention, layout, predict, ledger, calibrate, quant, svg  # noqa: F401

@@ -27,10 +27,17 @@ Readings (the pages are silent on these):
 Parity: window and identity are pinned by closed forms ([P1] section 4:
 window [T,1,1] equals the stable argsort by pixel; a window covering the
 whole grid is the identity; the 4x4 temporal ledger goes from 64 to 16
-tiles).  The Hilbert curve is pinned by properties only -- bijection, unit
-steps between consecutive points on a full cube, index 0 at the origin --
-the pages do not fix which Hilbert curve: **parity unpinned** beyond those
-properties (the GPU must still match this oracle bit for bit).
+tiles).  The Hilbert index is pinned, in two dimensions, to an independent
+construction: the classic rotate-and-reflect Hilbert curve, equal index for
+index on every grid up to 64 x 64 (Skilling's algorithm is generic in the
+number of axes, so the same inversion, exchange, Gray-encode and interleave
+steps serve both).  In three dimensions it is pinned by the defining
+properties of a Hilbert curve: bijection and unit steps on full cubes, start
+at the origin and end at (2^b - 1, 0, 0), octants in binary-reflected Gray
+order with t most significant, and exact self-similarity (every order is
+eight isometric copies of the order below, by the same eight isometries).
+The pages name no Hilbert variant; among the three-axis variants this one is
+Skilling's by the algorithm the two-dimensional pin checks.
 """
 
 from __future__ import annotations

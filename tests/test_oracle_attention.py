@@ -38,11 +38,18 @@ def test_worked_example_reproduces_printed_values():
         y_full, _, _ = A.masked_attention(q[head], k[head], v, m["full"])
         y_u, _, _ = A.masked_attention(q[head], k[head], v, m["union"])
         mses.append(float(np.mean((y_u - y_full) ** 2)))
-    assert mses == pytest.approx(g["union_mse"], rel=1e-6)
+    # The page prints the two MSEs to 11 significant digits (5.5294485880e-08,
+    # 5.0711107889e-06): the oracle's values, rounded to those digits, are
+    # the printed ones (agreement within half a unit of the last digit,
+    # about 1e-11 relative).
+    for got, printed in zip(mses, g["union_mse"]):
+        assert float(f"{got:.10e}") == printed
+        assert abs(got - printed) <= 0.5e-10 * 10.0 ** math.floor(math.log10(printed))
     dec = A.error_decomposition(q[0], k[0], v, m["spatial"])
     err = np.linalg.norm(dec["y_tilde"] - dec["y"], axis=-1)
-    assert err.max() == pytest.approx(g["spatial_head_spatial_mask_max_row_error"], abs=1e-10)
-    assert dec["bound"].max() == pytest.approx(g["spatial_head_spatial_mask_max_bound"], abs=1e-10)
+    # printed to 10 decimals (0.0008639397, 0.0117092274)
+    assert round(float(err.max()), 10) == g["spatial_head_spatial_mask_max_row_error"]
+    assert round(float(dec["bound"].max()), 10) == g["spatial_head_spatial_mask_max_bound"]
     assert np.all(err <= dec["bound"] + 1e-12)
 
 

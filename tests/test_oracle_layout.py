@@ -98,3 +98,91 @@ def test_reorder_unreorder_round_trip():
     y = Y.reorder(x, perm)
     assert np.array_equal(Y.unreorder(y, perm), x)
     assert np.array_equal(np.take(y, inv, axis=-2), x)
+
+
+def _classic_hilbert_d(n, x, y):
+    """Distance along the classic two-dimensional Hilbert curve on an n x n
+    grid (n a power of two): at each scale s the quadrant (rx, ry) gives
+    s*s*((3*rx) ^ ry), then the point is reflected and its axes swapped
+    into the quadrant's frame.  Written independently of Skilling's
+    transpose algorithm; the two must agree in two dimensions, where the
+    Hilbert curve from (0, 0) to (n-1, 0) is unique."""
+    d = 0
+    s = n // 2
+    while s > 0:
+        rx = 1 if x & s else 0
+        ry = 1 if y & s else 0
+        d += s * s * ((3 * rx) ^ ry)
+        if ry == 0:
+            if rx == 1:
+                x, y = n - 1 - x, n - 1 - y
+            x, y = y, x
+        s //= 2
+    return d
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6])
+def test_hilbert_2d_equals_the_classic_construction(bits):
+    """Skilling's algorithm is generic in the number of axes: in two
+    dimensions it must give exactly the classic Hilbert curve (the same
+    loops -- the inversion/exchange pass, the Gray encoding, the bit
+    interleave -- that serve the three-axis layout)."""
+    n = 1 << bits
+    x, y = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+    pts = np.stack([x.ravel(), y.ravel()], axis=1)
+    idx = Y.hilbert_index(pts, bits)
+    ref = np.array([_classic_hilbert_d(n, int(a), int(b)) for a, b in pts])
+    assert np.array_equal(idx, ref)
+
+
+def _curve3(bits):
+    n = 1 << bits
+    t, h, w = np.meshgrid(np.arange(n), np.arange(n), np.arange(n), indexing="ij")
+    pts = np.stack([t.ravel(), h.ravel(), w.ravel()], axis=1)
+    return pts[np.argsort(Y.hilbert_index(pts, bits))]
+
+
+def _octant_isometries(bits):
+    """For each of the 8 octants of the order-`bits` curve (in curve order):
+    the cube isometry (axis permutation, reflections) that maps the
+    order-(bits-1) curve onto the octant's piece of the curve."""
+    import itertools
+    big, small = _curve3(bits), _curve3(bits - 1)
+    m = (1 << (bits - 1)) - 1
+    L = len(small)
+    found = []
+    for c in range(8):
+        piece = big[c * L:(c + 1) * L]
+        rel = piece - (piece[0] // (m + 1)) * (m + 1)
+        match = []
+        for perm in itertools.permutations(range(3)):
+            for flips in itertools.product([0, 1], repeat=3):
+                q = small[:, list(perm)].copy()
+                for a in range(3):
+                    if flips[a]:
+                        q[:, a] = m - q[:, a]
+                if np.array_equal(q, rel):
+                    match.append((perm, flips))
+        assert len(match) == 1            # each piece is one isometric copy
+        found.append(match[0])
+    return found
+
+
+def test_hilbert_3d_gray_order_end_corner_and_self_similarity():
+    """Three axes: at every order the curve runs from the origin to
+    (2^b - 1, 0, 0), visits the octants in binary-reflected Gray-code order
+    of their (t, h, w) bits with t most significant, and each octant holds an
+    isometric copy of the curve one order down, by the same eight isometries
+    at every order (one generator, as a Hilbert curve is defined)."""
+    gray = [(g >> 2 & 1, g >> 1 & 1, g & 1) for g in (i ^ (i >> 1) for i in range(8))]
+    gen = None
+    for bits in range(1, 6):
+        path = _curve3(bits)
+        n = 1 << bits
+        assert tuple(path[0]) == (0, 0, 0) and tuple(path[-1]) == (n - 1, 0, 0)
+        octs = [tuple(int(v) for v in p) for p in path[::len(path) // 8] // max(1, n // 2)]
+        assert octs == gray
+        if bits >= 2:
+            iso = _octant_isometries(bits)
+            gen = iso if gen is None else gen
+            assert iso == gen
