@@ -227,7 +227,8 @@ sa_status sa_reorder_predict_mask(const int32_t* perm, const void* q, const void
  * overlap on the GPU (other streams, other threads) race on it and must be
  * serialised by the caller.  The first call on a device (with that device
  * current) looks up the array's address; make it before any stream capture
- * begins on that device. */
+ * begins on that device.  The address is kept for the life of the process,
+ * so do not use this entry point across a cudaDeviceReset of the device. */
 sa_status sa_predict_mask_noalloc(const void* q, const void* k, const sa_shape* shape,
                                   const sa_mask_params* params, sa_mask* out, void* stream);
 
@@ -255,8 +256,13 @@ size_t sa_attn_workspace(void);
  * inverse reorder into the store: row n of the problem is written to row
  * out_perm[n] of out and lse (pass the layout's perm to get the original
  * token order back; out must not alias q).  pv_skip_log (nullable) gets one
- * byte per kept tile in CSR order, 1 = PV skipped.  The mask's status word
- * also receives kernel errors. */
+ * byte per kept tile in CSR order, 1 = PV skipped; size it like col_idx
+ * (mask->col_capacity bytes).  The mask's status word also receives kernel
+ * errors.  A row whose list reaches past mask->col_capacity (the mask's
+ * builder raised SA_ERR_CAPACITY) is not computed: its O and LSE rows are
+ * left as they were, and nothing past col_capacity is read or written, so
+ * the call may be enqueued right after the builder, before the status is
+ * read. */
 sa_status sa_block_sparse_attn(const void* q, const void* k, const void* v,
                                const sa_shape* shape, const sa_mask* mask, float lambda,
                                float scale, void* out, float* lse, const int32_t* out_perm,

@@ -244,14 +244,31 @@ sa_status sa_reorder_predict_mask_q8(const int32_t* perm, const void* q, const v
   if (format != SA_Q_INT8 && format != SA_Q_E4M3)
     return set_error(SA_ERR_INVALID_ARG, "format must be SA_Q_INT8 or SA_Q_E4M3");
   if (shape->dtype != SA_BF16) return set_error(SA_ERR_UNSUPPORTED, "8-bit codes are written from bf16 input");
-  if ((uintptr_t)q8 % 16 || (uintptr_t)k8 % 16 || (uintptr_t)q_scales % 4 || (uintptr_t)k_scales % 4)
+  if ((uintptr_t)q8 % 16 || (uintptr_t)k8 % 16)
     return set_error(SA_ERR_INVALID_ARG, "q8 and k8 must be 16-byte aligned");
+  if ((uintptr_t)q_scales % 4 || (uintptr_t)k_scales % 4)
+    return set_error(SA_ERR_INVALID_ARG, "q_scales and k_scales must be 4-byte aligned");
   const size_t qbytes = (size_t)(shape->B * shape->Hq * shape->N * shape->d);
   const size_t kbytes = (size_t)(shape->B * shape->Hkv * shape->N * shape->d);
   if (ranges_overlap(q, 2 * qbytes, q8, qbytes) || ranges_overlap(k, 2 * kbytes, k8, kbytes) ||
       ranges_overlap(q8, qbytes, k8, kbytes) || ranges_overlap(q, 2 * qbytes, k8, kbytes) ||
       ranges_overlap(k, 2 * kbytes, q8, qbytes))
     return set_error(SA_ERR_INVALID_ARG, "q8 and k8 must not overlap q, k or each other");
+  if (params && params->bq >= 1 && params->bk >= 1) {
+    // The scale arrays: one float per query block (Q) and per key block (K).
+    const size_t qsb = (size_t)(shape->B * shape->Hq * ceil_div(shape->N, params->bq)) * sizeof(float);
+    const size_t ksb = (size_t)(shape->B * shape->Hkv * ceil_div(shape->N, params->bk)) * sizeof(float);
+    const void* spans[4] = {q, k, q8, k8};
+    const size_t lens[4] = {2 * qbytes, 2 * kbytes, qbytes, kbytes};
+    bool bad = ranges_overlap(q_scales, qsb, k_scales, ksb) ||
+               (ws && ws_bytes && (ranges_overlap(q_scales, qsb, ws, ws_bytes) ||
+                                   ranges_overlap(k_scales, ksb, ws, ws_bytes)));
+    for (int i = 0; i < 4; ++i)
+      bad = bad || ranges_overlap(q_scales, qsb, spans[i], lens[i]) || ranges_overlap(k_scales, ksb, spans[i], lens[i]);
+    if (bad)
+      return set_error(SA_ERR_INVALID_ARG,
+                       "q_scales and k_scales must overlap neither each other, q, k, q8, k8 nor the workspace");
+  }
   if (sa_status e = predict_prepare("sa_reorder_predict_mask_q8", q, k, shape, params, ws, ws_bytes, out)) return e;
   const PoolCodes codes{format, q8, q_scales, k8, k_scales};
   return launch_predict(q, k, *shape, *params, predict_ws_carve(ws, *shape, params->bq, params->bk), *out,
@@ -335,6 +352,7 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
       return set_error(SA_ERR_INVALID_ARG, "mask does not match the shape (was it built for this shape?)");
     a.row_ptr = mask->row_ptr;
     a.col_idx = mask->col_idx;
+    a.col_capacity = mask->col_capacity;
     a.order = mask->order;
     a.status = mask->status;
     a.bq = mask->bq;
@@ -346,18 +364,18 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
   }
   const bool tc_ok = !(flags & SA_FLAG_FORCE_SIMT) && is_sm100();
   if (qk8) {
-    // INT8 QK runs on the tensor-core kernel only: there is no other path.
+    // 8-bit QK runs on the tensor-core kernel only: there is no other path.
     if (!qk8->q_scales || !qk8->k_scales) return set_error(SA_ERR_INVALID_ARG, "NULL scale array");
     if (qk8->format != SA_Q_INT8 && qk8->format != SA_Q_E4M3)
       return set_error(SA_ERR_INVALID_ARG, "format must be SA_Q_INT8 or SA_Q_E4M3");
     if (!(shape->dtype == SA_BF16 && shape->d == 128 && shape->dv == 128 && a.bq == 128 &&
           (a.bk == 64 || a.bk == 128)))
-      return set_error(SA_ERR_UNSUPPORTED, "INT8 QK needs bf16 V, d = dv = 128, bq = 128, bk in {64, 128}");
-    if (flags & SA_FLAG_FORCE_SIMT) return set_error(SA_ERR_UNSUPPORTED, "INT8 QK has no CUDA-core kernel");
+      return set_error(SA_ERR_UNSUPPORTED, "8-bit QK needs bf16 V, d = dv = 128, bq = 128, bk in {64, 128}");
+    if (flags & SA_FLAG_FORCE_SIMT) return set_error(SA_ERR_UNSUPPORTED, "8-bit QK has no CUDA-core kernel");
     a.nqb = ceil_div(a.N, a.bq);
     a.nkb = ceil_div(a.N, a.bk);
     if (sa_status e = check_device()) return e;
-    if (!tc_ok) return set_error(SA_ERR_UNSUPPORTED, "INT8 QK needs an sm_100 device");
+    if (!tc_ok) return set_error(SA_ERR_UNSUPPORTED, "8-bit QK needs an sm_100 device");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* ts = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
     if (sa_status e = launch_tile_scales(*mask, a.B, a.Hq, a.Hkv, qk8->q_scales, qk8->k_scales,
@@ -421,7 +439,7 @@ sa_status sa_block_sparse_attn_qk8(const void* q8, const float* q_scales, const 
                                    uint8_t* pv_skip_log, void* ws, size_t ws_bytes, int32_t flags, void* stream) {
   if (!mask) return set_error(SA_ERR_INVALID_ARG, "mask is NULL");
   if ((uintptr_t)q8 % 16 || (uintptr_t)k8 % 16 || (uintptr_t)v % 16 || (uintptr_t)out % 16)
-    return set_error(SA_ERR_INVALID_ARG, "INT8 QK needs 16-byte aligned q8, k8, v, out");
+    return set_error(SA_ERR_INVALID_ARG, "8-bit QK needs 16-byte aligned q8, k8, v, out");
   const Qk8Args qk8{q_scales, k_scales, format};
   return attn_common(q8, k8, v, shape, mask, 0, lambda, scale, out, lse, out_perm, pv_skip_log, nullptr, ws,
                      ws_bytes, flags, stream, &qk8);

@@ -49,6 +49,12 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
   if (a.row_ptr) {
     lo = a.row_ptr[u];
     hi = a.row_ptr[u + 1];
+    if (hi > a.col_capacity || lo > hi) {
+      // The list reaches past col_idx: the builder raised SA_ERR_CAPACITY;
+      // the row is not computed.
+      if (threadIdx.x == 0) raise_status(a.status, SA_ERR_CAPACITY);
+      return;
+    }
   } else {
     const int64_t last_row = i0 + nr - 1;
     hi = a.causal ? (last_row / bk + 1) : a.nkb;
@@ -57,6 +63,10 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
 
   for (int64_t t = lo; t < hi; ++t) {
     const int64_t kb = a.row_ptr ? a.col_idx[t] : t;
+    if (kb < 0 || kb >= a.nkb) {   // not a list a mask builder wrote
+      if (threadIdx.x == 0) raise_status(a.status, SA_ERR_INVALID_ARG);
+      continue;
+    }
     const int64_t j0 = kb * bk;
     const int nc = (int)min64(bk, a.N - j0);
     // Scores.

@@ -106,6 +106,7 @@ static_assert(Cfg<64, 0>::SMEM <= 227 * 1024 && Cfg<128, 0>::SMEM <= 227 * 1024 
 struct TcParams {
   const int32_t* row_ptr;
   const int32_t* col_idx;
+  int64_t col_capacity;
   const int32_t* order;
   uint16_t* out;
   float* lse;
@@ -360,7 +361,10 @@ __device__ __forceinline__ Unit unit_at(const TcParams& p, int i, int BK) {
   u.kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
   if (p.row_ptr) {
     u.lo = p.row_ptr[id];
-    u.n = p.row_ptr[id + 1] - u.lo;
+    const int64_t hi = p.row_ptr[id + 1];
+    // A list that reaches past col_idx (the builder raised SA_ERR_CAPACITY)
+    // is not computed: n = -1 tells every role to pass the unit by.
+    u.n = (hi > p.col_capacity || u.lo > hi) ? -1 : hi - u.lo;
   } else {
     u.lo = 0;
     const int64_t last_row = min64(p.N, (u.qb + 1) * 128) - 1;
@@ -544,7 +548,7 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
     const int64_t row_g = u.qb * 128 + row;
     const bool row_valid = row_g < p.N;
     if (u.n <= 0) {
-      if (row_valid) raise_status(p.status, SA_ERR_EMPTY_ROW);
+      if (row_valid) raise_status(p.status, u.n < 0 ? SA_ERR_CAPACITY : SA_ERR_EMPTY_ROW);
       continue;
     }
     float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
@@ -852,6 +856,7 @@ sa_status launch_bk(const AttnArgs& a, cudaStream_t st) {
   TcParams p;
   p.row_ptr = a.row_ptr;
   p.col_idx = a.col_idx;
+  p.col_capacity = a.col_capacity;
   p.order = a.order;
   p.out = static_cast<uint16_t*>(a.out);
   p.lse = a.lse;

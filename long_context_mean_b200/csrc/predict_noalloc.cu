@@ -21,7 +21,10 @@
 //
 // The device address of the array is looked up with cudaGetSymbolAddress the
 // first time the entry point runs on a device (with that device current);
-// make that first call before any stream capture begins on the device.
+// make that first call before any stream capture begins on the device.  The
+// address is kept for the life of the process: after cudaDeviceReset (or any
+// other teardown of the device's primary context) the library would hold a
+// stale address, so the entry point must not be used across a device reset.
 #include <mutex>
 
 #include "sa_internal.cuh"

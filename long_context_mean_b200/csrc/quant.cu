@@ -78,10 +78,13 @@ __global__ void __launch_bounds__(kQuantThreads) quant_blocks_kernel(const uint4
 }
 
 // ts[e] = scale_log2 * q_scales[row] * k_scales[kv head][col_idx[e]] for
-// every list entry e of row (bh, qb); one warp per row.
+// every list entry e of row (bh, qb); one warp per row.  A row whose list
+// reaches past the capacity of col_idx (and of ts) is left out: the mask's
+// builder has raised SA_ERR_CAPACITY for it.
 __global__ void __launch_bounds__(256) tile_scales_kernel(const int32_t* __restrict__ row_ptr,
                                                           const int32_t* __restrict__ col_idx, int64_t R,
-                                                          int64_t nqb, int64_t nkb, int64_t Hq, int64_t Hkv,
+                                                          int64_t capacity, int64_t nqb, int64_t nkb,
+                                                          int64_t Hq, int64_t Hkv,
                                                           const float* __restrict__ qs, const float* __restrict__ ks,
                                                           float scale_log2, float* __restrict__ ts) {
   const int64_t r = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -92,7 +95,11 @@ __global__ void __launch_bounds__(256) tile_scales_kernel(const int32_t* __restr
   const float a = scale_log2 * __ldg(qs + r);
   const float* kr = ks + kvh * nkb;
   const int32_t e1 = __ldg(row_ptr + r + 1);
-  for (int32_t e = __ldg(row_ptr + r) + lane; e < e1; e += 32) ts[e] = a * __ldg(kr + __ldg(col_idx + e));
+  if (e1 > capacity) return;
+  for (int32_t e = __ldg(row_ptr + r) + lane; e < e1; e += 32) {
+    const int32_t kb = __ldg(col_idx + e);
+    ts[e] = (kb >= 0 && kb < nkb) ? a * __ldg(kr + kb) : 0.f;
+  }
 }
 
 }  // namespace
@@ -118,8 +125,8 @@ sa_status launch_tile_scales(const sa_mask& m, int64_t B, int64_t Hq, int64_t Hk
                              float scale_log2, float* ts, cudaStream_t st) {
   const int64_t R = B * Hq * m.nqb;
   if (R == 0) return SA_OK;
-  tile_scales_kernel<<<(unsigned)ceil_div(R, 8), 256, 0, st>>>(m.row_ptr, m.col_idx, R, m.nqb, m.nkb, Hq, Hkv, qs, ks,
-                                                               scale_log2, ts);
+  tile_scales_kernel<<<(unsigned)ceil_div(R, 8), 256, 0, st>>>(m.row_ptr, m.col_idx, R, m.col_capacity, m.nqb,
+                                                               m.nkb, Hq, Hkv, qs, ks, scale_log2, ts);
   return check_launch("tile_scales_kernel");
 }
 

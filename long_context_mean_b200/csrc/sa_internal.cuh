@@ -148,6 +148,8 @@ struct AttnArgs {
   uint8_t* skip_log;
   const int32_t* row_ptr;   // nullptr = dense (every causally valid block)
   const int32_t* col_idx;
+  int64_t col_capacity;     // entries col_idx holds: a row whose list reaches past it is not
+                            // computed (the mask's builder raised SA_ERR_CAPACITY)
   const int32_t* order;     // nullptr = natural row order
   int32_t* status;
   int32_t* counter;         // attention workspace: the work counter

@@ -174,8 +174,13 @@ __global__ void __launch_bounds__(32 * kRowsWarps) rows_attn_kernel(
     const int64_t j0 = (int64_t)s_tiles[t] * bk, j1 = min64(N, j0 + bk);
     for (int64_t jj = j0; jj < j1; jj += kRowsGroups) {    // uniform over the warp
       const int64_t j = jj + grp;
-      const bool valid = j < j1;
-      const int64_t key = valid ? (perm ? (int64_t)__ldg(perm + j) : j) : j0;
+      int64_t key = j < j1 ? (perm ? (int64_t)__ldg(perm + j) : j) : j0;
+      // An entry of perms outside [0, N) (not a permutation) is reported and
+      // left out, as the pooling pass does.
+      const bool in_range = (uint64_t)key < (uint64_t)N;
+      if (j < j1 && !in_range) raise_status(status, SA_ERR_INVALID_ARG);
+      const bool valid = j < j1 && in_range;
+      if (!in_range) key = j0;
       const uint4* kp = reinterpret_cast<const uint4*>(kh + key * D);
       const uint4* vp = reinterpret_cast<const uint4*>(vh + key * D);
       float kf[DL], vf[DL];

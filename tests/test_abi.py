@@ -121,7 +121,7 @@ def test_host_validation_codes(lib):
     assert lib.sa_reorder_heads(null, FAKE, ctypes.c_void_p(1 << 20), 2, 10, 8, 0, null) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_rows_mse(FAKE, FAKE, FAKE, 4, 2, 10, 8, 7, FAKE, null, null) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_rows_mse(FAKE, FAKE, null, 4, 2, 10, 8, 0, FAKE, null, null) == sa.SA_ERR_INVALID_ARG
-    # INT8 QK
+    # 8-bit QK
     assert lib.sa_quantize_blocks(null, 2, 10, 128, 64, 0, 0, FAKE, FAKE, null) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_quantize_blocks(FAKE, 2, 10, 128, 64, 1, 0, FAKE, FAKE, null) == sa.SA_ERR_UNSUPPORTED
     assert lib.sa_quantize_blocks(FAKE, 2, 10, 128, 256, 0, 0, FAKE, FAKE, null) == sa.SA_ERR_UNSUPPORTED
@@ -151,6 +151,30 @@ def test_host_validation_codes(lib):
     assert lib.sa_block_sparse_attn(FAKE, FAKE, FAKE, ctypes.byref(s), ctypes.byref(m2), ctypes.c_float(-1),
                                     ctypes.c_float(0), FAKE, null, null, null, WS, 256,
                                     sa.SA_FLAG_OUT_PERM_PER_HEAD, null) == sa.SA_ERR_INVALID_ARG
+
+
+def test_q8_scale_arrays_are_checked(lib):
+    """sa_reorder_predict_mask_q8 rejects misaligned or overlapping scale
+    arrays on the host with their own message."""
+    null = ctypes.c_void_p(None)
+    s = sa.Shape(1, 2, 1, 1024, 128, 128, sa.SA_BF16, 0)
+    pr = sa.make_params(128, 64, 0.5)
+    m = _mask()
+    q, k = ctypes.c_void_p(1 << 24), ctypes.c_void_p(1 << 25)
+    q8, k8 = ctypes.c_void_p(1 << 26), ctypes.c_void_p(1 << 27)
+    qs, ks = ctypes.c_void_p(1 << 28), ctypes.c_void_p((1 << 28) + 4096)
+    ws = ctypes.c_void_p(1 << 29)
+    call = lambda qs_, ks_: lib.sa_reorder_predict_mask_q8(null, q, k, 0, q8, qs_, k8, ks_, ctypes.byref(s),
+                                                          ctypes.byref(pr), ws, 1 << 20, ctypes.byref(m), null)
+    assert call(ctypes.c_void_p((1 << 28) + 2), ks) == sa.SA_ERR_INVALID_ARG
+    assert b"q_scales and k_scales must be 4-byte aligned" in lib.sa_last_error()
+    # q_scales (2 heads x 8 blocks = 64 bytes) inside q
+    assert call(ctypes.c_void_p((1 << 24) + 64), ks) == sa.SA_ERR_INVALID_ARG
+    assert b"q_scales and k_scales" in lib.sa_last_error()
+    # k_scales overlapping q_scales, and inside the workspace
+    assert call(qs, ctypes.c_void_p((1 << 28) + 32)) == sa.SA_ERR_INVALID_ARG
+    assert call(qs, ctypes.c_void_p((1 << 29) + 256)) == sa.SA_ERR_INVALID_ARG
+    assert b"workspace" in lib.sa_last_error()
 
 
 def test_workspace_queries_are_host_only(lib):

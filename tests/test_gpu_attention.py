@@ -159,3 +159,54 @@ def test_pv_skip_exercised(flags, causal):
     n_skip = sum(ref["skips"].values())
     assert n_skip >= 10, n_skip
     P.attention_check(r["out"], r["lse"], ref)
+
+
+@pytest.mark.parametrize("path", ["tc", "simt", "int8", "e4m3"])
+def test_undersized_mask_attention_stays_in_bounds(path):
+    """A mask whose lists overflow col_capacity (the builder raises
+    SA_ERR_CAPACITY), handed to attention on the same stream before the
+    status is read: the attention kernels must not read or write past the
+    capacity.  Canary bytes after the skip log's and the 8-bit path's
+    tile-scale entries stay untouched, and the status word keeps
+    SA_ERR_CAPACITY."""
+    import torch
+    from long_context_mean_b200 import sa
+    N, bq, bk, cap = 512, 128, 64, 31          # 4 x 8 = 32 kept tiles, one over
+    rng = np.random.default_rng(11)
+    q, k, v = (P.bf16_dev(I.to_bf16_bits(rng.standard_normal((1, 1, N, 128)).astype(np.float32)))
+               for _ in range(3))
+    shape = sa.make_shape(q, k, v)
+    mb = sa.MaskBuffers.allocate(1, 1, N, bq, bk, "cuda", capacity=cap)
+    ws = sa.workspace(sa.mask_from_blocks_workspace(shape, bq, bk), "cuda")
+    sa.mask_from_blocks(torch.ones(4 * 8, dtype=torch.uint8, device="cuda"), shape, bq, bk, False, ws, mb.struct)
+    canary = 0xA5
+    skip = torch.full((cap + 64,), canary, dtype=torch.uint8, device="cuda")
+    out = torch.zeros((1, 1, N, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((1, 1, N), dtype=torch.float32, device="cuda")
+    if path in ("tc", "simt"):
+        flags = sa.SA_FLAG_FORCE_SIMT if path == "simt" else 0
+        sa.block_sparse_attn(q, k, v, shape, mb.struct, -1.0, 0.0, out, lse, skip, flags)
+        aws = None
+    else:
+        q8 = torch.empty((1, 1, N, 128), dtype=torch.uint8, device="cuda")
+        k8 = torch.empty_like(q8)
+        qs = torch.empty(N // bq, dtype=torch.float32, device="cuda")
+        ks = torch.empty(N // bk, dtype=torch.float32, device="cuda")
+        sa.quantize_blocks(q, bq, q8, qs, path)
+        sa.quantize_blocks(k, bk, k8, ks, path)
+        need = sa.attn_qk8_workspace(mb.struct)
+        aws = torch.full((need + 256,), canary, dtype=torch.uint8, device="cuda")
+        sa.block_sparse_attn_qk8(q8, qs, k8, ks, v, shape, mb.struct, -1.0, 0.0, out, aws, lse, skip, fmt=path)
+    assert sa.read_status(mb.status) == sa.SA_ERR_CAPACITY
+    sk = skip.cpu().numpy()
+    assert (sk[cap:] == canary).all(), "skip log written past col_capacity"
+    rp = mb.row_ptr.cpu().numpy()
+    assert rp[-1] == 32 and rp[3] == 24
+    assert set(sk[:24].tolist()) <= {0, 1}, "rows inside the capacity must still be computed"
+    if aws is not None:
+        a = aws.cpu().numpy()
+        assert (a[256 + 4 * cap:] == canary).all(), "tile scales written past col_capacity"
+    # rows of query blocks 0-2 were computed; block 3 (list past capacity) was left alone
+    o = out.float().cpu().numpy()[0, 0]
+    assert np.isfinite(o[:3 * bq]).all() and (np.abs(o[:3 * bq]).sum(axis=1) > 0).all()
+    assert (o[3 * bq:] == 0).all()
