@@ -324,6 +324,35 @@ sa_status sa_dense_attn(const void* q, const void* k, const void* v, const sa_sh
                         int32_t causal, float scale, void* out, float* lse, int32_t* status,
                         void* ws, size_t ws_bytes, int32_t flags, void* stream);
 
+/* ---- a0-a7 end to end from host buffers ([P1] 6: the permutation and the
+ * data movement count in end-to-end time) -----------------------------------
+ * The whole path for host buffers (pinned, so that the copies are
+ * asynchronous): q_host [B*Hq][N][d], k_host and v_host [B*Hkv][N][d | dv],
+ * out_host [B*Hq][N][dv] in the input dtype and lse_host float [B*Hq][N], all
+ * in the original token order.  The problem is cut into `chunks` groups of
+ * (batch, head) rows (chunks divides B*Hkv, at most 16; query row r reads kv
+ * row r / (Hq/Hkv)).  Chunk i's copies in run on streams[1], its path on
+ * streams[0] (sa_layout_build once; sa_reorder_predict_mask and sa_reorder of
+ * V, or sa_predict_mask for the identity layout; sa_block_sparse_attn with
+ * out_perm = the layout's perm) and its copies out on streams[2], so the
+ * copies of one chunk overlap the kernels of its neighbours.  The work is
+ * ordered after what the caller enqueued on streams[0] before the call, and
+ * is complete on streams[0] once the last copy out is; the three streams may
+ * be one stream (no overlap).  shape->N must equal the layout's token count.
+ * ws: sa_forward_host_workspace() bytes, 256-byte aligned, owned by the
+ * caller (device copies of the inputs and outputs, one chunk's reordered
+ * copies, mask and scratch); calls sharing it must not overlap.  status
+ * (device int32 [1]) is cleared and then receives the largest status code of
+ * any chunk.  The host buffers must stay valid until the work completes.
+ * Argument and CUDA errors return synchronously; work already enqueued stays
+ * enqueued. */
+size_t sa_forward_host_workspace(const sa_shape* shape, const sa_layout_desc* layout,
+                                 const sa_mask_params* params, int32_t chunks);
+sa_status sa_forward_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                          float* lse_host, const sa_shape* shape, const sa_layout_desc* layout,
+                          const sa_mask_params* params, float lambda, float scale, int32_t chunks,
+                          void* ws, size_t ws_bytes, int32_t* status, void* const streams[3]);
+
 /* Synchronises `stream` and returns the device status word's code (0 =
  * SA_OK).  The word is not cleared. */
 sa_status sa_read_status(const int32_t* status, void* stream);

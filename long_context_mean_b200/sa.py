@@ -37,7 +37,7 @@ EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_attn_worksp
            "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status", "sa_l1_error",
            "sa_head_placement", "sa_reorder_heads", "sa_rows_attn", "sa_rows_mse",
            "sa_quantize_blocks", "sa_attn_qk8_workspace", "sa_block_sparse_attn_qk8",
-           "sa_reorder_predict_mask_q8"]
+           "sa_reorder_predict_mask_q8", "sa_forward_host_workspace", "sa_forward_host"]
 
 
 class SAError(RuntimeError):
@@ -124,6 +124,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                        P, P, P, P, P, SZ, I32, P]),
         "sa_dense_attn": (I32, [P, P, P, ctypes.POINTER(Shape), I32, F, P, P, P, P, SZ, I32, P]),
         "sa_read_status": (I32, [P, P]),
+        "sa_forward_host_workspace": (SZ, [ctypes.POINTER(Shape), ctypes.POINTER(LayoutDesc),
+                                           ctypes.POINTER(MaskParams), I32]),
+        "sa_forward_host": (I32, [P, P, P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(LayoutDesc),
+                                  ctypes.POINTER(MaskParams), F, F, I32, P, SZ, P, ctypes.POINTER(P * 3)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -515,15 +519,17 @@ class Pipeline:
 
 
 class HostPipeline:
-    """End-to-end pass from pinned host buffers to pinned host buffers.
+    """End-to-end pass from pinned host buffers to pinned host buffers: the
+    library's ``sa_forward_host`` (one C call per pass).
 
-    Heads are independent, so the problem is cut into ``chunks`` groups of
-    (batch, head) rows (whole kv groups).  Chunk i's host-to-device copy of
-    Q, K, V runs on a copy stream, its path on the compute stream (one
-    ``Pipeline`` sized for a chunk, reused), and its device-to-host copy of
-    O and LSE on a third stream, so the copies of one chunk overlap the
-    kernels of its neighbours.  ``run`` only enqueues: the caller waits on
-    ``done`` (an event recorded after the last copy back) or synchronises.
+    Heads are independent, so the library cuts the problem into ``chunks``
+    groups of (batch, head) rows; chunk i's host-to-device copy runs on a
+    copy stream, its path on the compute stream and its copy back on a third
+    stream, so the copies of one chunk overlap the kernels of its
+    neighbours.  The workspace and the two copy streams are allocated here
+    once (through torch).  ``run`` only enqueues: the caller waits on
+    ``done`` (an event recorded on the compute stream after the call) or
+    synchronises.
     """
 
     def __init__(self, B, Hq, Hkv, N, d, dv, dtype, *, layout: LayoutDesc, params: MaskParams,
@@ -533,27 +539,18 @@ class HostPipeline:
             raise ValueError(f"chunks={chunks} must divide the {B * Hkv} kv rows")
         self.device = torch.device(device)
         tdt = torch.bfloat16 if dtype in ("bf16", SA_BF16) else torch.float32
-        self.g = Hq // Hkv
-        self.chunks = chunks
-        self.rows_kv = B * Hkv // chunks
-        self.rows_q = self.rows_kv * self.g
-        # Flattened (batch, head) rows: query row r reads kv row r // g.
-        self.sub = Pipeline(1, self.rows_q, self.rows_kv, N, d, dv, dtype, layout=layout, params=params,
-                            lam=lam, scale=scale, flags=flags, device=device)
-        self.q = torch.empty(B * Hq, N, d, dtype=tdt, device=device)
-        self.k = torch.empty(B * Hkv, N, d, dtype=tdt, device=device)
-        self.v = torch.empty(B * Hkv, N, dv, dtype=tdt, device=device)
-        self.out = torch.empty(B * Hq, N, dv, dtype=tdt, device=device)
-        self.lse = torch.empty(B * Hq, N, 1, dtype=torch.float32, device=device)
+        self.shape = Shape(B, Hq, Hkv, N, d, dv, SA_BF16 if tdt == torch.bfloat16 else SA_FP32, 0)
+        self.layout, self.params = layout, params
+        self.lam, self.scale, self.chunks = lam, scale, chunks
+        nbytes = load().sa_forward_host_workspace(ctypes.byref(self.shape), ctypes.byref(layout),
+                                                  ctypes.byref(params), int(chunks))
+        if nbytes == 0:
+            raise SAError(SA_ERR_INVALID_ARG, load().sa_last_error().decode(errors="replace"))
+        self.ws = workspace(nbytes, device)
         self.s_in = torch.cuda.Stream(device=self.device)
         self.s_out = torch.cuda.Stream(device=self.device)
-        ev = lambda: torch.cuda.Event()
-        self.e_in = [ev() for _ in range(chunks)]
-        self.e_comp = [ev() for _ in range(chunks)]
-        self.e_out = [ev() for _ in range(chunks)]
-        self.done = ev()
+        self.done = torch.cuda.Event()
         self.status_word = torch.zeros(1, dtype=torch.int32, device=device)   # worst status over chunks
-        self._first = True
 
     def run(self, q_host, k_host, v_host, out_host, lse_host, stream=None):
         """q_host [B, Hq, N, d], k_host/v_host [B, Hkv, N, d|dv], out_host
@@ -561,43 +558,13 @@ class HostPipeline:
         tensors.  Work is ordered after ``stream`` (default: current)."""
         import torch
         comp = stream if stream is not None else torch.cuda.current_stream(self.device)
-        start = torch.cuda.Event()
-        with torch.cuda.stream(comp):
-            self.status_word.zero_()
-        start.record(comp)
-        qh, kh, vh = (x.reshape(-1, *x.shape[-2:]) for x in (q_host, k_host, v_host))
-        oh = out_host.reshape(-1, *out_host.shape[-2:])
-        lh = lse_host.reshape(oh.shape[0], -1)
-        rq, rk = self.rows_q, self.rows_kv
-        for i in range(self.chunks):
-            sq, sk = slice(i * rq, (i + 1) * rq), slice(i * rk, (i + 1) * rk)
-            # host -> device (the previous pass's compute of this chunk has read its inputs)
-            self.s_in.wait_event(start)
-            if not self._first:
-                self.s_in.wait_event(self.e_comp[i])
-            with torch.cuda.stream(self.s_in):
-                self.q[sq].copy_(qh[sq], non_blocking=True)
-                self.k[sk].copy_(kh[sk], non_blocking=True)
-                self.v[sk].copy_(vh[sk], non_blocking=True)
-            self.e_in[i].record(self.s_in)
-            # the path on this chunk (its outputs' previous copy back has finished)
-            comp.wait_event(self.e_in[i])
-            if not self._first:
-                comp.wait_event(self.e_out[i])
-            self.sub.run(self.q[sq].unsqueeze(0), self.k[sk].unsqueeze(0), self.v[sk].unsqueeze(0), comp,
-                         out=self.out[sq].unsqueeze(0), lse=self.lse[sq].unsqueeze(0))
-            with torch.cuda.stream(comp):
-                torch.maximum(self.status_word, self.sub.mask.status, out=self.status_word)
-            self.e_comp[i].record(comp)
-            # device -> host
-            self.s_out.wait_event(self.e_comp[i])
-            with torch.cuda.stream(self.s_out):
-                oh[sq].copy_(self.out[sq], non_blocking=True)
-                lh[sq].copy_(self.lse[sq].reshape(rq, -1), non_blocking=True)
-            self.e_out[i].record(self.s_out)
-        comp.wait_event(self.e_out[self.chunks - 1])
+        streams = (ctypes.c_void_p * 3)(comp.cuda_stream, self.s_in.cuda_stream, self.s_out.cuda_stream)
+        _check(load().sa_forward_host(_ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(out_host), _ptr(lse_host),
+                                      ctypes.byref(self.shape), ctypes.byref(self.layout), ctypes.byref(self.params),
+                                      float(self.lam), float(self.scale), int(self.chunks), _ptr(self.ws),
+                                      self.ws.numel() * self.ws.element_size(), _ptr(self.status_word),
+                                      ctypes.byref(streams)))
         self.done.record(comp)
-        self._first = False
 
     def status(self) -> int:
         """Synchronises; the largest status code any chunk raised (0 = SA_OK)."""

@@ -177,6 +177,34 @@ def test_q8_scale_arrays_are_checked(lib):
     assert b"workspace" in lib.sa_last_error()
 
 
+def test_forward_host_validation(lib):
+    """sa_forward_host checks its arguments on the host before enqueueing:
+    NULL buffers, a chunk count that does not divide B*Hkv, a shape whose N
+    differs from the layout's tokens, an undersized workspace."""
+    null = ctypes.c_void_p(None)
+    s = sa.Shape(1, 4, 2, 64, 128, 128, sa.SA_BF16, 0)
+    lay = sa.make_layout(4, 4, 4, 0, 0, "window", (2, 2, 2))
+    pr = sa.make_params(16, 16, 0.5)
+    assert lib.sa_forward_host_workspace(ctypes.byref(s), ctypes.byref(lay), ctypes.byref(pr), 3) == 0
+    need = lib.sa_forward_host_workspace(ctypes.byref(s), ctypes.byref(lay), ctypes.byref(pr), 2)
+    assert need > 0 and need % 256 == 0
+    # one chunk holds the whole problem: at least the device copies of q, k, v, out (4 x 16 KB x heads)
+    one = lib.sa_forward_host_workspace(ctypes.byref(s), ctypes.byref(lay), ctypes.byref(pr), 1)
+    assert one >= (4 + 2 + 2 + 4) * 64 * 128 * 2
+    st = (ctypes.c_void_p * 3)(None, None, None)
+    H = ctypes.c_void_p(1 << 30)
+    WS = ctypes.c_void_p(1 << 31)
+    call = lambda q, shape, lay_, chunks, ws_bytes: lib.sa_forward_host(
+        q, H, H, H, H, ctypes.byref(shape), ctypes.byref(lay_), ctypes.byref(pr), ctypes.c_float(-1.0),
+        ctypes.c_float(0.0), chunks, WS, ws_bytes, FAKE, ctypes.byref(st))
+    assert call(null, s, lay, 2, need) == sa.SA_ERR_INVALID_ARG
+    assert call(H, s, lay, 3, need) == sa.SA_ERR_INVALID_ARG
+    assert b"chunks" in lib.sa_last_error()
+    s_bad = sa.Shape(1, 4, 2, 65, 128, 128, sa.SA_BF16, 0)
+    assert call(H, s_bad, lay, 2, need) == sa.SA_ERR_INVALID_ARG
+    assert call(H, s, lay, 2, need - 256) == sa.SA_ERR_WORKSPACE
+
+
 def test_workspace_queries_are_host_only(lib):
     s = _shape(N=20506, Hq=24, Hkv=24)
     p = sa.make_params(128, 64, 0.5)
