@@ -185,28 +185,6 @@ struct RowRules {
 
 constexpr int kRowThreads = 256;
 
-__device__ __forceinline__ float block_reduce_max(float v, float* sh) {
-  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0) sh[warp] = v;
-  __syncthreads();
-  float r = -INFINITY;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, sh[w]);
-  return r;
-}
-
-__device__ __forceinline__ float block_reduce_sum(float v, float* sh) {
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0) sh[warp] = v;
-  __syncthreads();
-  float r = 0.f;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += sh[w];
-  return r;
-}
-
 __device__ __forceinline__ int block_reduce_sum_int(int v, int* sh) {
   for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -254,19 +232,21 @@ __device__ void finish_row(const uint8_t* flags, int64_t u, int64_t qb, int64_t 
 }
 
 // ---------------------------------------------------------------------------
-// a3 + a4: one CTA per (head, group of G <= 8 query blocks).  The group's
-// q_hat rows and 32-row chunks of the kv head's k_hat are staged in shared
-// memory (padded rows, conflict-free) so every k_hat element is read once per
-// group.  Then warp r alone finishes row r: softmax and TopCdf (an arg-max
-// loop over register-resident keys when the row is short and few blocks are
-// picked, else a bisection for the last kept probability), the union with
-// the forced parts and the causal AND -- with warp-level synchronisation
-// only.
-// Dynamic shared memory: q_hat [8][d] | k_hat chunk ring [3][32][d+4], reused
-// as p [G][P2] (fp32) | scores [G][nkb] | flags [G][nkb rounded to 16] (u8).
+// a3 + a4: one CTA per (head, group of G <= 8 query blocks).  Scores: thread
+// i takes the key blocks kb = i, i + 256, ... and computes q_hat[r] . k_hat[kb]
+// for every row r of the group, reading its k_hat row from global memory
+// (L2-resident, each element read once per group) and the q_hat rows from
+// shared memory (the same address in every lane: broadcast), so the loop is
+// bound by the FMA pipe.  Then warp r alone finishes row r: softmax and
+// TopCdf (an arg-max loop over register-resident keys when the row is short
+// and few blocks are picked, else a bisection for the last kept
+// probability), the union with the forced parts and the causal AND -- with
+// warp-level synchronisation only.
+// Dynamic shared memory: q_hat [8][d] | scores [G][nkb rounded to 4] (fp32;
+// the bisection turns a row's scores into its probabilities in place, the
+// padding holding zeros) | flags [G][nkb rounded to 16] (u8).
 // ---------------------------------------------------------------------------
 constexpr int kMaxRowsPerCta = 8;
-constexpr int kChunk = 32;
 constexpr int kFastKeys = 16;     // keys per lane on the fast TopCdf path (nkb <= 512)
 constexpr int kFastPicks = 128;   // picks before the fast path defers to the sort
 
@@ -275,30 +255,12 @@ int score_rows_per_cta(int P2) {
   return g < 1 ? 1 : (g > kMaxRowsPerCta ? kMaxRowsPerCta : g);
 }
 
-constexpr int kStages = 3;   // k_hat chunks in flight (cp.async ring)
-
-// Bytes of the region shared by the k_hat chunk ring (score phase) and the
-// sort keys (TopCdf phase): the two are never live at once.
-__host__ __device__ inline size_t score_union_bytes(int d, int P2, int G) {
-  const size_t ring = (size_t)kStages * kChunk * (d + 4) * 4;
-  const size_t keys = (size_t)G * P2 * 4;
-  return ring > keys ? ring : keys;
-}
-
 size_t score_smem_bytes(int d, int64_t nkb, int P2, int G) {
+  (void)P2;
   const size_t nkb16 = (size_t)((nkb + 15) / 16) * 16;
-  return (size_t)kMaxRowsPerCta * d * 4 + score_union_bytes(d, P2, G) + (size_t)G * nkb * 4 +
-         (size_t)G * nkb16;
+  const size_t nkb4 = (size_t)((nkb + 3) / 4) * 4;
+  return (size_t)kMaxRowsPerCta * d * 4 + (size_t)G * nkb4 * 4 + (size_t)G * nkb16;
 }
-
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
-               "l"(gsrc)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ float warp_max(float v) {
   for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
@@ -312,16 +274,10 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
     int32_t* __restrict__ counts, int32_t* status) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int nkb16 = (int)((nkb + 15) / 16) * 16;
+  const int nkb4 = (int)((nkb + 3) / 4) * 4;   // score row stride: float4-aligned rows
   float* qs = reinterpret_cast<float*>(smem);
-  // One region holds the ring of k_hat chunks while scores are computed and
-  // the sort keys afterwards.  k_hat rows are padded to d + 4 floats:
-  // 16-byte aligned for cp.async and float4 reads, and the 8 rows a
-  // quarter-warp reads land in distinct bank groups.
-  unsigned char* uni = smem + (size_t)kMaxRowsPerCta * d * 4;
-  float* ks = reinterpret_cast<float*>(uni);
-  float* keys = reinterpret_cast<float*>(uni);
-  float* sc = reinterpret_cast<float*>(uni + score_union_bytes(d, P2, G));
-  uint8_t* flags = reinterpret_cast<uint8_t*>(sc + G * nkb);
+  float* sc = reinterpret_cast<float*>(smem + (size_t)kMaxRowsPerCta * d * 4);
+  uint8_t* flags = reinterpret_cast<uint8_t*>(sc + G * nkb4);
   __shared__ int s_forced[kMaxRowsPerCta];
 
   const int64_t bh = blockIdx.y;
@@ -344,52 +300,40 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   for (int r = 0; r < rows; ++r) any_scored |= !s_forced[r];
 
   if (any_scored) {
-    // Scores of the whole group, one k_hat chunk at a time, the chunks
-    // streamed into a ring of kStages buffers with cp.async so that the next
-    // chunks' loads are in flight while the current one is multiplied.
     const float4* kg4 = reinterpret_cast<const float4*>(khat + g * nkb * (int64_t)d);
+    const float4* qs4 = reinterpret_cast<const float4*>(qs);
     const int nf4 = d / 4;
-    const int r = threadIdx.x / kChunk, j = threadIdx.x % kChunk;
-    const int64_t nchunks = (nkb + kChunk - 1) / kChunk;
-    auto issue_chunk = [&](int64_t c) {
-      if (c < nchunks) {
-        const int64_t c0 = c * kChunk;
-        const int total = (int)min64(kChunk, nkb - c0) * nf4;
-        float* dst = ks + (c % kStages) * kChunk * (d + 4);
-        for (int i = threadIdx.x; i < total; i += kRowThreads)
-          cp_async16(dst + (i / nf4) * (d + 4) + (i % nf4) * 4, kg4 + c0 * nf4 + i);
-      }
-      cp_async_commit();   // possibly empty: one group per chunk slot keeps the count uniform
-    };
-    for (int c = 0; c < kStages - 1; ++c) issue_chunk(c);
-    for (int64_t c = 0; c < nchunks; ++c) {
-      const int64_t c0 = c * kChunk;
-      const int cn = (int)min64(kChunk, nkb - c0);
-      cp_async_wait<kStages - 2>();   // chunk c has landed (this thread's part)
-      __syncthreads();                // ... everyone's; and chunk c-1's buffer is free
-      issue_chunk(c + kStages - 1);
-      const float* kc = ks + (c % kStages) * kChunk * (d + 4);
-      const int64_t kb = c0 + j;
-      if (r < rows && j < cn) {
-        float s = -INFINITY;
-        if (!s_forced[r] && rules.valid(qb0 + r, kb) && !(guard && sk[g * nkb + kb] < theta)) {
-          const float4* qr = reinterpret_cast<const float4*>(qs + r * d);
-          const float4* kr = reinterpret_cast<const float4*>(kc + j * (d + 4));
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-          for (int e = 0; e < d / 4; ++e) {
-            const float4 x = qr[e], y = kr[e];
-            a0 = fmaf(x.x, y.x, a0);
-            a1 = fmaf(x.y, y.y, a1);
-            a2 = fmaf(x.z, y.z, a2);
-            a3 = fmaf(x.w, y.w, a3);
+    for (int64_t kb = threadIdx.x; kb < nkb; kb += kRowThreads) {
+      uint32_t need = 0;   // rows of the group that score this key block
+      const bool col_ok = !(guard && sk[g * nkb + kb] < theta);
+#pragma unroll
+      for (int r = 0; r < kMaxRowsPerCta; ++r)
+        if (r < rows && col_ok && !s_forced[r] && rules.valid(qb0 + r, kb)) need |= 1u << r;
+      float a[kMaxRowsPerCta][4];
+#pragma unroll
+      for (int r = 0; r < kMaxRowsPerCta; ++r) a[r][0] = a[r][1] = a[r][2] = a[r][3] = 0.f;
+      if (need) {
+        const float4* kr = kg4 + kb * nf4;
+        for (int e = 0; e < nf4; ++e) {
+          const float4 y = __ldg(kr + e);
+#pragma unroll
+          for (int r = 0; r < kMaxRowsPerCta; ++r) {
+            if (r < rows) {
+              const float4 x = qs4[r * nf4 + e];
+              a[r][0] = fmaf(x.x, y.x, a[r][0]);
+              a[r][1] = fmaf(x.y, y.y, a[r][1]);
+              a[r][2] = fmaf(x.z, y.z, a[r][2]);
+              a[r][3] = fmaf(x.w, y.w, a[r][3]);
+            }
           }
-          s = ((a0 + a1) + (a2 + a3)) * scale;
         }
-        sc[r * nkb + kb] = s;
       }
+#pragma unroll
+      for (int r = 0; r < kMaxRowsPerCta; ++r)
+        if (r < rows) sc[r * nkb4 + kb] = ((need >> r) & 1u) ? ((a[r][0] + a[r][1]) + (a[r][2] + a[r][3])) * scale
+                                                              : -INFINITY;
     }
-    cp_async_wait<0>();
-    __syncthreads();   // the chunk ring becomes the sort keys below
+    __syncthreads();
   }
 
   if (warp >= rows) return;
@@ -398,11 +342,11 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   const int64_t qb = qb0 + r;
   const int64_t u = bh * nqb + qb;
   const bool row_forced = s_forced[r] != 0;
-  float* pr = keys + (size_t)r * P2;
+  float* pr = sc + (size_t)r * nkb4;   // probabilities replace the scores (bisection)
   uint8_t* fl = flags + (size_t)r * nkb16;
   for (int64_t kb = lane; kb < nkb; kb += 32) fl[kb] = 0;
   if (!row_forced) {
-    const float* srow = sc + r * nkb;
+    const float* srow = sc + r * nkb4;
     float mx = -INFINITY;
     for (int64_t kb = lane; kb < nkb; kb += 32) mx = fmaxf(mx, srow[kb]);
     mx = warp_max(mx);
@@ -464,17 +408,20 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
       // blocks whose p equals it are kept in index order while f(t*) + r p <
       // tau * total (r = rank among them).  t* is found by bisection over the
       // bit patterns of (0, 1] (p = exp(s - max) <= 1).
-      for (int kb = lane; kb < nkb; kb += 32) {
-        const float sv = srow[kb];
+      for (int kb = lane; kb < nkb4; kb += 32) {
+        const float sv = kb < nkb ? srow[kb] : -INFINITY;
         pr[kb] = (sv == -INFINITY) ? 0.f : expf(sv - mx);
       }
       __syncwarp();
+      const float4* pr4 = reinterpret_cast<const float4*>(pr);
       auto mass_above = [&](uint32_t t) -> float {
-        float m = 0.f;
-        for (int kb = lane; kb < nkb; kb += 32) {
-          const float pv = pr[kb];
-          m += __float_as_uint(pv) > t ? pv : 0.f;
+        float m0 = 0.f, m1 = 0.f;
+        for (int q = lane; q < nkb4 / 4; q += 32) {
+          const float4 v = pr4[q];
+          m0 += (__float_as_uint(v.x) > t ? v.x : 0.f) + (__float_as_uint(v.y) > t ? v.y : 0.f);
+          m1 += (__float_as_uint(v.z) > t ? v.z : 0.f) + (__float_as_uint(v.w) > t ? v.w : 0.f);
         }
+        float m = m0 + m1;
         for (int off = 16; off > 0; off >>= 1) m += __shfl_xor_sync(0xffffffffu, m, off);
         return m;
       };
