@@ -12,16 +12,17 @@
 //     mask's work order (descending kept count), from a global counter by
 //     each pipeline's producer and announced to its MMA and softmax warps
 //     through a 4-slot ring.
-//   * per pipeline, warp p (one lane) is the TMA producer (Q tile once per
-//     unit, K and V tiles of the kept key blocks through a STAGES ring) and
-//     warp 2+p (one lane) issues tcgen05.mma: S = Q K^T into one of two TMEM
-//     S buffers and O += P V into the TMEM O accumulator.  The softmax
-//     writes P (bf16 pairs) over its S buffer in TMEM and the PV product
-//     reads it from there (TS form), so S runs one tile ahead of PV: S(t+1)
-//     overlaps the softmax of t, and PV(t) the softmax of t+1.  A variant
-//     with P in a 128-byte-swizzled shared-memory buffer (SS form, S two
-//     tiles ahead) is kept behind Cfg::P_SMEM; on B200 it measured slower
-//     at both block sizes.
+//   * per pipeline, warp p is the TMA producer: lane 0 loads the Q tile once
+//     per unit and the K tiles of the kept key blocks through a 3-stage ring,
+//     lane 1 the V tiles through their own ring (a K load never waits behind
+//     a V stage that the previous P V still holds).  Warp 2+p (one lane)
+//     issues tcgen05.mma: S = Q K^T into one of two TMEM S buffers and
+//     O += P V into the TMEM O accumulator.  The softmax writes P (bf16
+//     pairs) over its S buffer in TMEM and the P V product reads it from
+//     there (TS form), so S runs one tile ahead of P V: S(t+1) overlaps the
+//     softmax of t, and P V(t) the softmax of t+1.  (Q copied into TMEM with
+//     a TS-form S and one S buffer per pipeline measured 40% slower on B200:
+//     each pipeline's chain softmax -> P V -> S becomes serial.)
 //   * per pipeline, four softmax warps (one thread per query row = TMEM
 //     lane): S from TMEM, masks, running max, exp2 (scale folded into one
 //     packed fp32x2 FMA), P, O rescale in TMEM when the reference maximum
@@ -55,53 +56,69 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 template <int BK, int QM>
 struct Cfg {
-  // P in shared memory (SS MMA, S two tiles ahead of PV) or over S in TMEM
-  // (TS MMA, S one tile ahead).  Measured on B200 at bk = 64 the TMEM form
-  // is faster (the SS form adds 16 KB of operand reads per tile), so both
-  // block sizes use it; the shared-memory form stays for other shapes.
-  static constexpr bool P_SMEM = false;
   static constexpr int PIPES = BK == 64 ? 2 : 1;
-  // 8-bit Q and K (QM 1: INT8, 2: FP8 E4M3) halve their tiles, which leaves
-  // room for a third stage.
-  static constexpr int STAGES = (BK == 64 && QM == 0) ? 2 : 3;
-  static constexpr int LOOKAHEAD = P_SMEM ? 2 : 1;    // S tiles issued ahead of PV
-  static constexpr int THREADS = 128 + 128 * PIPES;
+  static constexpr int S_BUFS = 2;                    // TMEM S buffers per pipeline
+  static constexpr int LOOKAHEAD = 1;                 // S tiles issued ahead of P V
+  // K and V rings.  K is needed one softmax ahead of V, so it gets the deeper
+  // ring: three stages everywhere (the TMA latency, about 1 us, is longer
+  // than a tile); V two stages for bf16 at bk = 64 (shared memory: 2 x 112 KB)
+  // and three where the tiles are smaller (8-bit Q and K) or one pipeline.
+  static constexpr int K_STAGES = 3;
+  static constexpr int V_STAGES = (BK == 64 && QM == 0) ? 2 : 3;
+  // Softmax warps per TMEM lane quarter.  Two (16 rows each, half of a
+  // row's columns per thread, 640 threads) measured 6% slower than one at
+  // bk = 64 on B200, so one warp owns each quarter.
+  static constexpr int SPLIT = 1;
+  static constexpr int SM_WARPS = 4 * SPLIT;          // softmax warps per pipeline
+  static constexpr int THREADS = 128 + 32 * SM_WARPS * PIPES;
   static constexpr int QK_ELEM = QM ? 1 : 2;           // bytes per Q / K element
   static constexpr int Q_BYTES = 128 * 128 * QK_ELEM;
   static constexpr int K_BYTES = BK * 128 * QK_ELEM;
   static constexpr int V_BYTES = BK * 128 * 2;
   static constexpr int KV_CHUNK = BK * 128;          // one 128-byte-wide chunk: BK rows x 128 B
-  static constexpr int P_BYTES = P_SMEM ? 128 * BK * 2 : 0;
-  static constexpr int PIPE_BYTES = Q_BYTES + STAGES * (K_BYTES + V_BYTES) + P_BYTES;
+  static constexpr int PIPE_BYTES = Q_BYTES + K_STAGES * K_BYTES + V_STAGES * V_BYTES;
   static constexpr int OFF_CTL = PIPES * PIPE_BYTES;
   static constexpr int CTL_BYTES = 512;
   static constexpr int SMEM = OFF_CTL + PIPES * CTL_BYTES + 1024;   // + alignment slack
-  static constexpr int TMEM_PIPE = (128 + 2 * BK) <= 256 ? 256 : 512;
+  // TMEM columns of a pipeline: O [0, 128), then the S buffers (BK fp32
+  // columns each).
+  static constexpr int S_COL = 128;
+  static constexpr int TMEM_PIPE = (S_COL + S_BUFS * BK) <= 256 ? 256 : 512;
   static constexpr int TMEM_COLS = PIPES * TMEM_PIPE;
-  static constexpr int S_COL = 128;                  // O occupies columns 0..127 of a pipe
+  // buffer and phase of tile gt in the S / P / PV-done rings
+  static __host__ __device__ constexpr int sbuf(uint32_t gt) { return (int)(gt & 1); }
+  static __host__ __device__ constexpr uint32_t sphase(uint32_t gt) { return (gt >> 1) & 1; }
   static __host__ __device__ constexpr int off_q(int p) { return p * PIPE_BYTES; }
   static __host__ __device__ constexpr int off_k(int p) { return p * PIPE_BYTES + Q_BYTES; }
-  static __host__ __device__ constexpr int off_v(int p) { return p * PIPE_BYTES + Q_BYTES + STAGES * K_BYTES; }
-  static __host__ __device__ constexpr int off_p(int p) {
-    return p * PIPE_BYTES + Q_BYTES + STAGES * (K_BYTES + V_BYTES);
-  }
+  static __host__ __device__ constexpr int off_v(int p) { return p * PIPE_BYTES + Q_BYTES + K_STAGES * K_BYTES; }
 };
 
 // Per-pipeline control block (8-byte mbarriers first).
 struct Ctl {
   uint64_t q_full, q_empty, o_free;
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
-  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
+  uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t u_full[4], u_empty[4];          // unit announcement ring
   uint32_t tmem_base;
   volatile uint32_t abort;
-  float gapw[4][4];                        // [tile & 3][softmax warp]
-  volatile int32_t ring[4];
+  float gapw[4][8];                        // [tile & 3][softmax warp]
+  // Unit announcements: the producer resolves each unit once (work-order
+  // entry, list offsets) and the other roles read it from here.  i < 0 ends
+  // the work.
+  struct Slot {
+    int32_t i, n, lo, bh, qb, kvh;
+  };
+  volatile Slot ring[4];
 };
 static_assert(sizeof(Ctl) <= 512, "control block too large");
 static_assert(Cfg<64, 0>::SMEM <= 227 * 1024 && Cfg<128, 0>::SMEM <= 227 * 1024 &&
-                  Cfg<64, 1>::SMEM <= 227 * 1024 && Cfg<128, 1>::SMEM <= 227 * 1024,
+                  Cfg<64, 1>::SMEM <= 227 * 1024 && Cfg<128, 1>::SMEM <= 227 * 1024 &&
+                  Cfg<64, 2>::SMEM <= 227 * 1024 && Cfg<128, 2>::SMEM <= 227 * 1024,
               "shared memory above the 227 KB a CTA may use");
+static_assert(Cfg<64, 0>::K_STAGES <= 3 && Cfg<64, 0>::V_STAGES <= 3 && Cfg<128, 1>::V_STAGES <= 3,
+              "the control block holds three stages per ring");
+static_assert(Cfg<64, 0>::TMEM_COLS <= 512 && Cfg<128, 0>::TMEM_COLS <= 512 && Cfg<64, 1>::TMEM_COLS <= 512,
+              "TMEM holds 512 columns");
 
 struct TcParams {
   const int32_t* row_ptr;
@@ -192,8 +209,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-// Generic-proxy shared-memory writes become visible to the tensor core.
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // D (TMEM) = A (SMEM desc) x B (SMEM desc) [+ D]
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -259,6 +274,53 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+// 16x32bx2 shapes: 16 TMEM lanes from the lane in taddr; thread t < 16 gets
+// lane t at columns [c, c + n), thread t + 16 lane t at [c + IMM, c + IMM + n).
+template <int IMM>
+__device__ __forceinline__ void tmem_ld_16x32bx2_x32(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr), "n"(IMM));
+}
+template <int IMM>
+__device__ __forceinline__ void tmem_st_16x32bx2_x32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, "
+      "{%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};" ::"r"(taddr), "n"(IMM),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+template <int IMM>
+__device__ __forceinline__ void tmem_ld_16x32bx2_x16(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr), "n"(IMM));
+}
+template <int IMM>
+__device__ __forceinline__ void tmem_st_16x32bx2_x16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, "
+      "{%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17};" ::"r"(taddr), "n"(IMM),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ float ex2(float x) {
@@ -289,33 +351,6 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
-}
-// 2^x for a pair of arguments on the FMA pipe.  Cody-Waite range reduction
-// (n = round(x) by the 1.5 * 2^23 addition, f = x - n in [-1/2, 1/2]), a cubic
-// for 2^f fitted for minimax relative error by csrc/fit_exp2.py (max relative
-// error 1.5e-4 in float32, below the bf16 rounding of P), and n added to the
-// exponent field.  x is clamped at -125 so the result stays a normal number;
-// the caller never passes masked (-inf) scores.
-constexpr float kExpC0 = 9.999280572e-01f, kExpC1 = 6.932609677e-01f;
-constexpr float kExpC2 = 2.426109314e-01f, kExpC3 = 5.517149344e-02f;
-constexpr int kEmuPairs = 0;   // of every 8 column pairs, this many use the FMA pipe
-                               // (0: measured slower on B200 at bk = 64 -- the
-                               // softmax is latency-bound, not MUFU-bound)
-__device__ __forceinline__ void exp2_fma_pair(uint64_t x2, float& r0, float& r1) {
-  float x0, x1;
-  unpack2(x2, x0, x1);
-  x2 = pack2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t magic = pack2(12582912.f, 12582912.f);
-  const uint64_t t = fadd2(x2, magic);
-  const uint64_t f = ffma2(fadd2(t, pack2(-12582912.f, -12582912.f)), pack2(-1.f, -1.f), x2);
-  uint64_t q = ffma2(pack2(kExpC3, kExpC3), f, pack2(kExpC2, kExpC2));
-  q = ffma2(q, f, pack2(kExpC1, kExpC1));
-  q = ffma2(q, f, pack2(kExpC0, kExpC0));
-  float q0, q1, t0, t1;
-  unpack2(q, q0, q1);
-  unpack2(t, t0, t1);
-  r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -377,25 +412,48 @@ __device__ __forceinline__ int64_t kblock_at(const TcParams& p, const Unit& u, i
   return p.row_ptr ? p.col_idx[u.lo + t] : t;
 }
 
+// Publish unit i (or the end of the work, i < 0) in a ring slot; read it back.
+__device__ __forceinline__ void post_unit(Ctl* c, int slot, int i, const Unit& u) {
+  volatile Ctl::Slot& s = c->ring[slot];
+  s.i = i;
+  s.n = (int32_t)u.n;
+  s.lo = (int32_t)u.lo;
+  s.bh = (int32_t)u.bh;
+  s.qb = (int32_t)u.qb;
+  s.kvh = (int32_t)u.kvh;
+}
+__device__ __forceinline__ int read_unit(Ctl* c, int slot, Unit& u) {
+  const volatile Ctl::Slot& s = c->ring[slot];
+  u.n = s.n;
+  u.lo = s.lo;
+  u.bh = s.bh;
+  u.qb = s.qb;
+  u.kvh = s.kvh;
+  return s.i;
+}
+
 // ---------------------------------------------------------------------------
 // Roles
 // ---------------------------------------------------------------------------
 template <int BK, int QM>
 __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                          const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, int pipe) {
+  // Lane 0 claims the units and loads Q and the K tiles; it announces each
+  // unit through the ring.
   using C = Cfg<BK, QM>;
-  uint32_t kv_it = 0, nq = 0;
+  uint32_t k_it = 0, nq = 0;
   for (uint32_t j = 0;; ++j) {
     // Take the next unit of the work order and announce it to the pipeline's
-    // MMA and softmax warps through a 4-slot ring.
+    // V loader, MMA and softmax warps through a 4-slot ring.
     const int slot = j & 3;
     mbar_wait(&c->u_empty[slot], ((j >> 2) & 1) ^ 1, g, p.status);
     int i = atomicAdd(p.counter, 1);
     if (i >= p.num_units) i = -1;
-    c->ring[slot] = i;
+    Unit u{};
+    if (i >= 0) u = unit_at(p, i, BK);
+    post_unit(c, slot, i, u);
     mbar_arrive(&c->u_full[slot]);
     if (i < 0) break;
-    const Unit u = unit_at(p, i, BK);
     if (u.n <= 0) continue;
     mbar_wait(&c->q_empty, (nq & 1) ^ 1, g, p.status);
     ++nq;
@@ -403,28 +461,49 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const C
     tma_load_3d(sb + C::off_q(pipe), tmQ, 0, (int)(u.qb * 128), (int)u.bh, &c->q_full);
     if constexpr (QM == 0)   // bf16 rows are two 128-byte chunks; 8-bit rows one
       tma_load_3d(sb + C::off_q(pipe) + C::Q_BYTES / 2, tmQ, 64, (int)(u.qb * 128), (int)u.bh, &c->q_full);
-    for (int64_t t = 0; t < u.n; ++t, ++kv_it) {
+    for (int64_t t = 0; t < u.n; ++t, ++k_it) {
       const int kb = (int)kblock_at(p, u, t);
-      const int s = kv_it % C::STAGES;
-      const uint32_t ph = (kv_it / C::STAGES) & 1;
+      const int s = k_it % C::K_STAGES;
+      const uint32_t ph = (k_it / C::K_STAGES) & 1;
       const uint32_t kdst = sb + C::off_k(pipe) + s * C::K_BYTES;
-      const uint32_t vdst = sb + C::off_v(pipe) + s * C::V_BYTES;
       mbar_wait(&c->k_empty[s], ph ^ 1, g, p.status);
       mbar_expect_tx(&c->k_full[s], C::K_BYTES);
       tma_load_3d(kdst, tmK, 0, kb * BK, (int)u.kvh, &c->k_full[s]);
       if constexpr (QM == 0) tma_load_3d(kdst + C::KV_CHUNK, tmK, 64, kb * BK, (int)u.kvh, &c->k_full[s]);
+    }
+  }
+  // Drain: the last loads of every stage (and the last Q) have landed.
+  if (nq > 0) mbar_drain(&c->q_full, (nq - 1) & 1);
+  for (uint32_t j = k_it > (uint32_t)C::K_STAGES ? k_it - C::K_STAGES : 0; j < k_it; ++j)
+    mbar_drain(&c->k_full[j % C::K_STAGES], (j / C::K_STAGES) & 1);
+}
+
+// Lane 1 of the producer warp loads the V tiles on their own ring, so a K
+// load never waits behind a V stage that the previous P V still holds.
+template <int BK, int QM>
+__device__ void v_loader(const CUtensorMap* tmV, const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, int pipe) {
+  using C = Cfg<BK, QM>;
+  uint32_t v_it = 0;
+  for (uint32_t j = 0;; ++j) {
+    const int slot = j & 3;
+    mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status);
+    Unit u;
+    const int i = read_unit(c, slot, u);
+    mbar_arrive(&c->u_empty[slot]);
+    if (i < 0) break;
+    for (int64_t t = 0; t < u.n; ++t, ++v_it) {
+      const int kb = (int)kblock_at(p, u, t);
+      const int s = v_it % C::V_STAGES;
+      const uint32_t ph = (v_it / C::V_STAGES) & 1;
+      const uint32_t vdst = sb + C::off_v(pipe) + s * C::V_BYTES;
       mbar_wait(&c->v_empty[s], ph ^ 1, g, p.status);
       mbar_expect_tx(&c->v_full[s], C::V_BYTES);
       tma_load_3d(vdst, tmV, 0, kb * BK, (int)u.kvh, &c->v_full[s]);
       tma_load_3d(vdst + C::KV_CHUNK, tmV, 64, kb * BK, (int)u.kvh, &c->v_full[s]);
     }
   }
-  // Drain: the last loads of every stage (and the last Q) have landed.
-  if (nq > 0) mbar_drain(&c->q_full, (nq - 1) & 1);
-  for (uint32_t j = kv_it > (uint32_t)C::STAGES ? kv_it - C::STAGES : 0; j < kv_it; ++j) {
-    mbar_drain(&c->k_full[j % C::STAGES], (j / C::STAGES) & 1);
-    mbar_drain(&c->v_full[j % C::STAGES], (j / C::STAGES) & 1);
-  }
+  for (uint32_t j = v_it > (uint32_t)C::V_STAGES ? v_it - C::V_STAGES : 0; j < v_it; ++j)
+    mbar_drain(&c->v_full[j % C::V_STAGES], (j / C::V_STAGES) & 1);
 }
 
 template <int BK, int QM>
@@ -437,23 +516,27 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
   for (uint32_t j = 0;; ++j) {
     const int slot = j & 3;
     mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status);
-    const int i = c->ring[slot];
+    Unit u;
+    const int i = read_unit(c, slot, u);
     mbar_arrive(&c->u_empty[slot]);
     if (i < 0) break;
-    const Unit u = unit_at(p, i, BK);
     if (u.n <= 0) continue;
     mbar_wait(&c->q_full, unit_it & 1, g, p.status);
     tc_fence_after();
+    const uint32_t qbase = sb + C::off_q(pipe);
     bool first_pv = true;
     auto do_pv = [&](int64_t tt) {
       const uint32_t it = kv_it + (uint32_t)tt, gt = gt0 + (uint32_t)tt;
-      const int s = it % C::STAGES;
-      const uint32_t ph = (it / C::STAGES) & 1;
-      const int gb = gt & 1;
-      mbar_wait(&c->p_full[gb], (gt >> 1) & 1, g, p.status);
+      const int s = it % C::V_STAGES;
+      const uint32_t ph = (it / C::V_STAGES) & 1;
+      const int gb = C::sbuf(gt);
+      mbar_wait(&c->p_full[gb], C::sphase(gt), g, p.status);
       tc_fence_after();
       const float* gw = c->gapw[gt & 3];
-      const bool skip = fmaxf(fmaxf(gw[0], gw[1]), fmaxf(gw[2], gw[3])) < p.lam_log2;
+      float gmax = gw[0];
+#pragma unroll
+      for (int w = 1; w < C::SM_WARPS; ++w) gmax = fmaxf(gmax, gw[w]);
+      const bool skip = gmax < p.lam_log2;
       if (p.skip_log && p.row_ptr) p.skip_log[u.lo + tt] = skip ? 1 : 0;
       if (tt == 0) {
         mbar_wait(&c->o_free, (unit_it & 1) ^ 1, g, p.status);
@@ -467,12 +550,7 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t b = desc_sw128(vbase + kk * 2048, C::KV_CHUNK, 1024);
           const uint32_t acc = (first_pv && kk == 0) ? 0u : 1u;
-          if constexpr (C::P_SMEM) {
-            const uint64_t a = desc_sw128(sb + C::off_p(pipe) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            umma_ss(tm, a, b, idesc_pv, acc);
-          } else {
-            umma_ts(tm, tm + C::S_COL + gb * BK + kk * 8, b, idesc_pv, acc);   // P over the S buffer
-          }
+          umma_ts(tm, tm + C::S_COL + gb * BK + kk * 8, b, idesc_pv, acc);   // P over the S buffer
         }
         first_pv = false;
       }
@@ -481,14 +559,12 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
     };
     for (int64_t t = 0; t < u.n; ++t) {
       const uint32_t it = kv_it + (uint32_t)t, gt = gt0 + (uint32_t)t;
-      const int s = it % C::STAGES;
-      const uint32_t ph = (it / C::STAGES) & 1;
-      const int gb = gt & 1;
+      const int s = it % C::K_STAGES;
+      const uint32_t ph = (it / C::K_STAGES) & 1;
+      const uint32_t scol = tm + C::S_COL + C::sbuf(gt) * BK;
       mbar_wait(&c->k_full[s], ph, g, p.status);
-      if constexpr (C::P_SMEM) mbar_wait(&c->s_empty[gb], ((gt >> 1) & 1) ^ 1, g, p.status);
       tc_fence_after();
       const uint32_t kbase = sb + C::off_k(pipe) + s * C::K_BYTES;
-      const uint32_t qbase = sb + C::off_q(pipe);
       if constexpr (QM != 0) {
         // d = 128 8-bit codes = one 128-byte swizzle row; K = 32 per instruction.
 #pragma unroll
@@ -496,19 +572,19 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
           const uint64_t a = desc_sw128(qbase + kk * 32, 16, 1024);
           const uint64_t b = desc_sw128(kbase + kk * 32, 16, 1024);
           if constexpr (QM == 1)
-            umma_ss_i8(tm + C::S_COL + gb * BK, a, b, idesc_s, kk > 0 ? 1u : 0u);
+            umma_ss_i8(scol, a, b, idesc_s, kk > 0 ? 1u : 0u);
           else
-            umma_ss_f8(tm + C::S_COL + gb * BK, a, b, idesc_s, kk > 0 ? 1u : 0u);
+            umma_ss_f8(scol, a, b, idesc_s, kk > 0 ? 1u : 0u);
         }
       } else {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t a = desc_sw128(qbase + (kk >> 2) * (C::Q_BYTES / 2) + (kk & 3) * 32, 16, 1024);
           const uint64_t b = desc_sw128(kbase + (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32, 16, 1024);
-          umma_ss(tm + C::S_COL + gb * BK, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          umma_ss(scol, a, b, idesc_s, kk > 0 ? 1u : 0u);
         }
       }
-      umma_commit(&c->s_full[gb]);
+      umma_commit(&c->s_full[C::sbuf(gt)]);
       umma_commit(&c->k_empty[s]);
       if (t == u.n - 1) umma_commit(&c->q_empty);
       if (t >= C::LOOKAHEAD) do_pv(t - C::LOOKAHEAD);
@@ -528,71 +604,87 @@ __device__ __forceinline__ float warp_fmax(float v) {
   return __int_as_float(m >= 0 ? m : m ^ 0x7FFFFFFF);
 }
 
+// One softmax thread holds NC = BK / SPLIT score columns of one query row.
+// SPLIT = 1: a warp owns the 32 rows (TMEM lanes) of its quarter, one row a
+// thread (32x32b shapes).  SPLIT = 2: two warps share a quarter, 16 rows
+// each; threads t and t + 16 hold columns [0, NC) and [NC, 2 NC) of the same
+// row (16x32bx2 shapes), so the row's maximum and sum take one shuffle.
 template <int BK, int QM>
-__device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, uint32_t tm, int pipe, int wq,
-                             int lane) {
+__device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int wq, int half, int lane) {
   using C = Cfg<BK, QM>;
-  const int row = wq * 32 + lane;
-  const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+  constexpr int SPLIT = C::SPLIT;
+  constexpr int NC = BK / SPLIT;                                  // score columns per thread
+  const int rlane = SPLIT == 2 ? half * 16 + (lane & 15) : lane;  // TMEM lane within the quarter
+  const int row = wq * 32 + rlane;
+  const int cpart = SPLIT == 2 ? (lane >> 4) : 0;                 // which column part of the row
+  const uint32_t lane_off = (uint32_t)(wq * 32 + (SPLIT == 2 ? half * 16 : 0)) << 16;
+  const int widx = wq * SPLIT + half;                              // this warp among the pipeline's
+  const bool row_owner = SPLIT == 1 || lane < 16;                  // one thread per row stores LSE
   float sc = p.scale_log2;   // log2-domain score scale; 8-bit QK: per tile
-  uint8_t* prow = smem + C::off_p(pipe) + (row >> 3) * 1024 + (row & 7) * 128;
   uint32_t gt0 = 0;
   for (uint32_t j = 0;; ++j) {
     const int slot = j & 3;
     mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status);
-    const int i = c->ring[slot];
+    Unit u;
+    const int i = read_unit(c, slot, u);
     __syncwarp();
     if (lane == 0) mbar_arrive(&c->u_empty[slot]);
     if (i < 0) break;
-    const Unit u = unit_at(p, i, BK);
     const int64_t row_g = u.qb * 128 + row;
     const bool row_valid = row_g < p.N;
+    // The row's destination (the inverse reorder), fetched now so that the
+    // load is long done when the epilogue stores through it.
+    const int64_t out_row =
+        row_valid ? (p.out_perm ? (int64_t)p.out_perm[u.bh * p.perm_stride + row_g] : row_g) : 0;
     if (u.n <= 0) {
-      if (row_valid) raise_status(p.status, u.n < 0 ? SA_ERR_CAPACITY : SA_ERR_EMPTY_ROW);
+      if (row_valid && row_owner) raise_status(p.status, u.n < 0 ? SA_ERR_CAPACITY : SA_ERR_EMPTY_ROW);
       continue;
     }
+    // m_run, m_ref are the row's (equal in both threads of a row); l is this
+    // thread's part of the row sum.
     float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
     int64_t kb_cur = kblock_at(p, u, 0);
     float sc_next = 0.f;
     if constexpr (QM != 0) sc_next = p.tile_scale[u.lo];
     for (int64_t t = 0; t < u.n; ++t) {
       const uint32_t gt = gt0 + (uint32_t)t;
-      const int gb = gt & 1;
+      const int gb = C::sbuf(gt);
       const uint32_t scol = tm + lane_off + C::S_COL + gb * BK;
       const int64_t kb_next = (t + 1 < u.n) ? kblock_at(p, u, t + 1) : 0;   // load ahead
       if constexpr (QM != 0) {
         sc = sc_next;
         if (t + 1 < u.n) sc_next = p.tile_scale[u.lo + t + 1];
       }
-      mbar_wait(&c->s_full[gb], (gt >> 1) & 1, g, p.status);
+      mbar_wait(&c->s_full[gb], C::sphase(gt), g, p.status);
       tc_fence_after();
-      float s[BK];
+      float s[NC];
+      if constexpr (SPLIT == 2) {
+        tmem_ld_16x32bx2_x32<NC>(scol, s);
+      } else {
 #pragma unroll
-      for (int cc = 0; cc < BK / 32; ++cc) tmem_ld32(scol + cc * 32, s + cc * 32);
+        for (int cc = 0; cc < NC / 32; ++cc) tmem_ld32(scol + cc * 32, s + cc * 32);
+      }
       tmem_wait_ld();
       if constexpr (QM == 1) {
         // int32 scores -> floats biased by kBias (exact); the bias cancels
         // in the exponent offset and the tile maximum below.
 #pragma unroll
-        for (int jj = 0; jj < BK; ++jj) s[jj] = __int_as_float(__float_as_int(s[jj]) + kBiasBits);
-      }
-      if constexpr (C::P_SMEM) {
-        tc_fence_before();
-        mbar_arrive(&c->s_empty[gb]);          // S buffer free for S(t+2)
+        for (int jj = 0; jj < NC; ++jj) s[jj] = __int_as_float(__float_as_int(s[jj]) + kBiasBits);
       }
 
-      const int64_t k0 = kb_cur * BK;
+      const int64_t kt0 = kb_cur * BK;            // first key of the tile
       kb_cur = kb_next;
-      const bool need_mask = (k0 + BK > p.N) || (p.causal && k0 + BK - 1 > u.qb * 128);
+      const int64_t k0 = kt0 + cpart * NC;        // key of this thread's first column
+      const bool need_mask = (kt0 + BK > p.N) || (p.causal && kt0 + BK - 1 > u.qb * 128);
       if (need_mask) {
 #pragma unroll
-        for (int jj = 0; jj < BK; ++jj) {
+        for (int jj = 0; jj < NC; ++jj) {
           const int64_t key = k0 + jj;
           if (key >= p.N || (p.causal && key > row_g)) s[jj] = -INFINITY;
         }
       }
-      // P = exp2(s * scale_log2 - ref), packed to bf16 pairs, and its row sum.
-      uint32_t pk[BK / 2];
+      // P = exp2(s * scale_log2 - ref), packed to bf16 pairs, and its sum.
+      uint32_t pk[NC / 2];
       float row_sum = 0.f;
       auto compute_p = [&](float ref) {
         // Pairs of columns on the packed fp32x2 pipe: x = s * scale - ref.
@@ -602,17 +694,11 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) acc[jj] = pack2(0.f, 0.f);
 #pragma unroll
-        for (int jj = 0; jj < BK; jj += 2) {
+        for (int jj = 0; jj < NC; jj += 2) {
           const uint64_t x = ffma2(pack2(s[jj], s[jj + 1]), sc2, neg2);
-          float p0, p1;
-          if (((jj >> 1) & 7) < kEmuPairs && !need_mask) {
-            exp2_fma_pair(x, p0, p1);          // FMA pipe, relieves the MUFU
-          } else {
-            float x0, x1;
-            unpack2(x, x0, x1);
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
+          float x0, x1;
+          unpack2(x, x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
           acc[(jj >> 1) & 3] = fadd2(acc[(jj >> 1) & 3], pack2(p0, p1));
           pk[jj >> 1] = pack_bf16(p0, p1);
         }
@@ -628,11 +714,11 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
       const bool spec = m_ref > -INFINITY;
       if (spec) compute_p(m_ref);
       // Row max as a tree of 3-input maxima (independent chains), raw units.
-      float mx[BK / 4];
+      float mx[NC / 4];
 #pragma unroll
-      for (int jj = 0; jj < BK / 4; ++jj) mx[jj] = max3(fmaxf(s[4 * jj], s[4 * jj + 1]), s[4 * jj + 2], s[4 * jj + 3]);
+      for (int jj = 0; jj < NC / 4; ++jj) mx[jj] = max3(fmaxf(s[4 * jj], s[4 * jj + 1]), s[4 * jj + 2], s[4 * jj + 3]);
 #pragma unroll
-      for (int w = BK / 4; w > 1; w = (w + 2) / 3) {
+      for (int w = NC / 4; w > 1; w = (w + 2) / 3) {
 #pragma unroll
         for (int jj = 0; jj < (w + 2) / 3; ++jj) {
           const float a = mx[3 * jj];
@@ -641,10 +727,12 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
           mx[jj] = max3(a, b, d);
         }
       }
-      const float mloc = (QM == 1 ? mx[0] - kBias : mx[0]) * sc;   // scale > 0: max commutes
+      float mraw = mx[0];
+      if constexpr (SPLIT == 2) mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 16));
+      const float mloc = (QM == 1 ? mraw - kBias : mraw) * sc;   // scale > 0: max commutes
       const float m_new = fmaxf(m_run, mloc);
       const float gap = warp_fmax((row_valid && mloc > -INFINITY) ? mloc - m_new : -INFINITY);
-      if (lane == 0) c->gapw[gt & 3][wq] = gap;
+      if (lane == 0) c->gapw[gt & 3][widx] = gap;
       m_run = m_new;
       float corr = 1.f;
       bool resc = false;
@@ -655,68 +743,73 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
         compute_p(m_ref);                       // the speculation missed
       } else if (!spec) {
 #pragma unroll
-        for (int jj = 0; jj < BK / 2; ++jj) pk[jj] = 0u;   // every score so far masked
+        for (int jj = 0; jj < NC / 2; ++jj) pk[jj] = 0u;   // every score so far masked
         row_sum = 0.f;
       }
       l = l * corr + row_sum;
       // tcgen05.ld/st are warp-collective: a warp rescales when any of its
       // rows needs it (corr is 1 for the others).  A rescale implies the
       // tile is not skipped, so PV(t-1) is the last product to wait for.
-      bool pv_prev_done = false;
       if (__any_sync(0xffffffffu, resc)) {
         const uint32_t gp = gt - 1;
-        mbar_wait(&c->pv_done[gp & 1], (gp >> 1) & 1, g, p.status);
-        pv_prev_done = true;
+        mbar_wait(&c->pv_done[C::sbuf(gp)], C::sphase(gp), g, p.status);
         tc_fence_after();
         const float f = resc ? corr : 1.f;
+        if constexpr (SPLIT == 2) {
+          // this thread's 64 columns of the row, 16 at a time
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            float o[16];
+            tmem_ld_16x32bx2_x16<64>(tm + lane_off + cc * 16, o);
+            tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float o[32];
-          tmem_ld32(tm + lane_off + cc * 32, o);
-          tmem_wait_ld();
+            for (int jj = 0; jj < 16; ++jj) o[jj] *= f;
+            tmem_st_16x32bx2_x16<64>(tm + lane_off + cc * 16, reinterpret_cast<const uint32_t*>(o));
+          }
+        } else {
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) o[jj] *= f;
-          tmem_st32(tm + lane_off + cc * 32, reinterpret_cast<const uint32_t*>(o));
+          for (int cc = 0; cc < 4; ++cc) {
+            float o[32];
+            tmem_ld32(tm + lane_off + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) o[jj] *= f;
+            tmem_st32(tm + lane_off + cc * 32, reinterpret_cast<const uint32_t*>(o));
+          }
         }
         tmem_wait_st();
       }
-      if constexpr (C::P_SMEM) {
-        // The single P buffer is free once PV of the previous tile is done.
-        if (gt >= 1 && !pv_prev_done) {
-          const uint32_t gp = gt - 1;
-          mbar_wait(&c->pv_done[gp & 1], (gp >> 1) & 1, g, p.status);
-        }
-#pragma unroll
-        for (int cc = 0; cc < BK / 8; ++cc) {
-          const uint4 v4 = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-          *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) = v4;
-        }
-        fence_async_smem();
+      if constexpr (SPLIT == 2) {
+        tmem_st_16x32bx2_x16<NC / 2>(scol, pk);   // P over the first BK / 2 columns of S
       } else {
 #pragma unroll
         for (int cc = 0; cc < BK / 64; ++cc) tmem_st32(scol + cc * 32, pk + cc * 32);
-        tmem_wait_st();
       }
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&c->p_full[gb]);
     }
     // Epilogue: O / l from TMEM once the unit's last PV has landed.
     const uint32_t gl = gt0 + (uint32_t)u.n - 1;
-    mbar_wait(&c->pv_done[gl & 1], (gl >> 1) & 1, g, p.status);
+    mbar_wait(&c->pv_done[C::sbuf(gl)], C::sphase(gl), g, p.status);
     tc_fence_after();
+    if constexpr (SPLIT == 2) l += __shfl_xor_sync(0xffffffffu, l, 16);   // the row's two parts
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    const int64_t out_row =
-        row_valid ? (p.out_perm ? (int64_t)p.out_perm[u.bh * p.perm_stride + row_g] : row_g) : 0;
-    uint16_t* orow = p.out + (u.bh * p.N + out_row) * 128;
+    // SPLIT = 2: this thread stores the row's output columns [64 cpart, 64 cpart + 64).
+    uint16_t* orow = p.out + (u.bh * p.N + out_row) * 128 + cpart * 64;
+    constexpr int OCH = SPLIT == 2 ? 16 : 32;   // output columns per TMEM load
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      float o[32];
-      tmem_ld32(tm + lane_off + cc * 32, o);
+    for (int cc = 0; cc < 128 / SPLIT / OCH; ++cc) {
+      float o[OCH];
+      if constexpr (SPLIT == 2)
+        tmem_ld_16x32bx2_x16<64>(tm + lane_off + cc * OCH, o);
+      else
+        tmem_ld32(tm + lane_off + cc * OCH, o);
       tmem_wait_ld();
       if (row_valid) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+        uint4* dst = reinterpret_cast<uint4*>(orow + cc * OCH);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int q4 = 0; q4 < OCH / 8; ++q4) {
           uint4 v;
           v.x = pack_bf16(o[8 * q4 + 0] * inv_l, o[8 * q4 + 1] * inv_l);
           v.y = pack_bf16(o[8 * q4 + 2] * inv_l, o[8 * q4 + 3] * inv_l);
@@ -728,7 +821,7 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint8_t* smem, u
     }
     tc_fence_before();
     mbar_arrive(&c->o_free);
-    if (row_valid) {
+    if (row_valid && row_owner) {
       if (!(l > 0.f)) raise_status(p.status, SA_ERR_EMPTY_ROW);
       if (p.lse) p.lse[u.bh * p.N + out_row] = (m_ref + __log2f(l)) * kLn2;
     }
@@ -752,22 +845,23 @@ __global__ void __launch_bounds__(Cfg<BK, QM>::THREADS, 1)
       Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + q * C::CTL_BYTES);
       mbar_init(&c->q_full, 1);
       mbar_init(&c->q_empty, 1);
-      mbar_init(&c->o_free, 128);
-      for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&c->o_free, 32 * C::SM_WARPS);
+      for (int s = 0; s < C::K_STAGES; ++s) {
         mbar_init(&c->k_full[s], 1);
         mbar_init(&c->k_empty[s], 1);
+      }
+      for (int s = 0; s < C::V_STAGES; ++s) {
         mbar_init(&c->v_full[s], 1);
         mbar_init(&c->v_empty[s], 1);
       }
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < C::S_BUFS; ++b) {
         mbar_init(&c->s_full[b], 1);
-        mbar_init(&c->s_empty[b], 128);
-        mbar_init(&c->p_full[b], 128);
+        mbar_init(&c->p_full[b], 32 * C::SM_WARPS);
         mbar_init(&c->pv_done[b], 1);
       }
       for (int r = 0; r < 4; ++r) {
         mbar_init(&c->u_full[r], 1);
-        mbar_init(&c->u_empty[r], 1 + 4);   // the MMA lane + one lane per softmax warp
+        mbar_init(&c->u_empty[r], 2 + C::SM_WARPS);   // the V lane, the MMA lane, one lane per softmax warp
       }
       c->abort = 0;
     }
@@ -786,9 +880,12 @@ __global__ void __launch_bounds__(Cfg<BK, QM>::THREADS, 1)
   const uint32_t tmem = ctl0->tmem_base;
 
   if (warp < 2) {
-    if (warp < C::PIPES && lane == 0) {
+    if (warp < C::PIPES && lane < 2) {
       Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + warp * C::CTL_BYTES);
-      producer<BK, QM>(&tmQ, &tmK, &tmV, p, c, ctl0, sb, warp);
+      if (lane == 0)
+        producer<BK, QM>(&tmQ, &tmK, &tmV, p, c, ctl0, sb, warp);
+      else
+        v_loader<BK, QM>(&tmV, p, c, ctl0, sb, warp);
     }
   } else if (warp < 4) {
     const int pipe = warp - 2;
@@ -798,9 +895,13 @@ __global__ void __launch_bounds__(Cfg<BK, QM>::THREADS, 1)
     }
     __syncwarp();
   } else {
-    const int pipe = (warp - 4) >> 2;
+    // Softmax warp 4 + 4 (SPLIT pipe + half) + quarter: the quarter is warp % 4,
+    // the TMEM lanes a warp may access.
+    const int sw = warp - 4;
+    const int pipe = sw / C::SM_WARPS;
+    const int half = (sw >> 2) % C::SPLIT;
     Ctl* c = reinterpret_cast<Ctl*>(smem + C::OFF_CTL + pipe * C::CTL_BYTES);
-    softmax_rows<BK, QM>(p, c, ctl0, smem, tmem + pipe * C::TMEM_PIPE, pipe, warp & 3, lane);
+    softmax_rows<BK, QM>(p, c, ctl0, tmem + pipe * C::TMEM_PIPE, warp & 3, half, lane);
   }
 
   tc_fence_before();
