@@ -44,9 +44,9 @@ if ROOT not in sys.path:
 METRIC = "sparse attn fwd ms & TFLOP/s (kept blocks) vs dense, N=20.5K video, 1×B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes per launch of the attention kernel from the ncu capture recorded
-# in profiles/attn_tc_video.md, keyed by the sha1 of the kernel code it was
-# taken on (src_sha1); any other code reports null.
+# DRAM bytes per launch of the attention kernel from the recorded ncu
+# capture, keyed by the sha1 of the kernel code it was taken on (src_sha1);
+# any other code reports null.
 TRAFFIC = {("79d19421d0daed5604f044fa9c241e28c613ceb9", "video"): 1.2193e9}
 
 
@@ -155,6 +155,35 @@ def kept_flops(w, row_ptr, col_idx, skip, nqb):
     return qk, pv
 
 
+def dense_flops(w):
+    """Dense-equivalent op count of the attention: 2*(d + dv) per visible
+    query-key pair over every head ([P3] 3.2: the "Speed" of a sparse kernel
+    is this count divided by its latency, prediction included)."""
+    pairs = w.N * (w.N + 1) / 2 if w.causal else float(w.N) * w.N
+    return w.B * w.Hq * 2.0 * (w.d + w.dv) * pairs
+
+
+def combined_sparsity(valid_tiles, kept, pv_skipped):
+    """SpargeAttn's sparsity over both products ([P3] Table 6): skipped
+    QK^T tiles plus skipped PV tiles over twice the valid tiles."""
+    return (2.0 * (valid_tiles - kept) + pv_skipped) / (2.0 * valid_tiles)
+
+
+def valid_tile_count(w, nqb, nkb):
+    """Causally valid (query block, key block) tiles over batch and heads."""
+    if w.causal:
+        return w.B * w.Hq * sum(min(nkb, (min(w.N, (qb + 1) * w.bq) - 1) // w.bk + 1) for qb in range(nqb))
+    return w.B * w.Hq * nqb * nkb
+
+
+def spread(xs):
+    """Median, p10 and p90 of a list of times (ms)."""
+    import numpy as np
+    a = np.asarray(xs, dtype=np.float64)
+    return {"median": round(float(np.median(a)), 4), "p10": round(float(np.percentile(a, 10)), 4),
+            "p90": round(float(np.percentile(a, 90)), 4), "mean": round(float(a.mean()), 4), "n": int(a.size)}
+
+
 # ----------------------------------------------------------------------------
 # Our arm
 # ----------------------------------------------------------------------------
@@ -213,11 +242,7 @@ def run_ours(args, rank, world, local_rank):
     qk_flops, pv_flops = kept_flops(w, rp, ci, skip, nqb)
     flops = qk_flops + pv_flops
     kept = int(rp[-1])
-    R = w.B * w.Hq * nqb
-    if w.causal:
-        valid_tiles = w.B * w.Hq * sum(min(nkb, (min(w.N, (qb + 1) * w.bq) - 1) // w.bk + 1) for qb in range(nqb))
-    else:
-        valid_tiles = R * nkb
+    valid_tiles = valid_tile_count(w, nqb, nkb)
     sparsity = 1.0 - kept / valid_tiles
     pv_skipped = int(skip[:kept].sum())
     pipe.skip_log = None                      # timed steps run without the log
@@ -323,10 +348,23 @@ def run_ours(args, rank, world, local_rank):
             dense.append((a, b))
     torch.cuda.synchronize(dev)
     dense_ms = statistics.median(x[0].elapsed_time(x[1]) for x in dense)
+    # Per-row dropped mass alpha = 1 - exp(LSE_sparse - LSE_dense) ([P1] 3.2),
+    # every row; the dense LSE comes back to the original token order when the
+    # dense kernel ran on the reordered tensors.
+    ld_h = ld.cpu().numpy().astype(np.float64)
+    if qr is not q:
+        perm_h = pipe.perm.cpu().numpy()
+        back = np.empty_like(ld_h)
+        back[..., perm_h] = ld_h
+        ld_h = back
+    alpha = 1.0 - np.exp(pipe.lse.cpu().numpy()[..., 0].astype(np.float64) - ld_h)
+    worst = [int(x) for x in np.unravel_index(int(np.argmax(alpha)), alpha.shape)]
+    alpha_rep = {"mean": float(alpha.mean()), "max": float(alpha.max()), "min": float(alpha.min()),
+                 "worst_b_h_row": worst, "rows": int(alpha.size)}
 
-    # End to end through the public API with host buffers (sa.HostPipeline):
-    # pinned H2D of Q, K, V, the step, D2H of O and LSE, cut into head chunks
-    # so the copies of one chunk overlap the kernels of the others.
+    # End to end through the C ABI with host buffers (sa_forward_host, one call
+    # per pass): pinned H2D of Q, K, V, the whole path, D2H of O and LSE, cut
+    # into head chunks so the copies of one chunk overlap the kernels of the others.
     out_host = torch.empty(pipe.out.shape, dtype=pipe.out.dtype).pin_memory()
     lse_host = torch.empty(pipe.lse.shape, dtype=pipe.lse.dtype).pin_memory()
     e2e_ms = float("nan")
@@ -387,13 +425,19 @@ def run_ours(args, rank, world, local_rank):
         "config": workload_config(w, world),
         "stages_ms": {"layout_reorder_predict": round(statistics.mean(pre_ms), 4),
                       "attention_with_fused_unreorder": round(statistics.mean(attn_ms), 4)},
+        "timing_ms": {"step": spread(step_ms), "attention": spread(attn_ms), "prediction": spread(pre_ms)},
         "attn_ms": round(attn_mean, 4),
         "attn_tflops": round(attn_tf, 2),
         "dense_ms": round(dense_ms, 4),
         "speedup_vs_dense": round(dense_ms / attn_mean, 3),
         "speedup_vs_dense_whole_step": round(dense_ms / mean_ms, 3),
         "block_sparsity": round(sparsity, 4),
+        "combined_qk_pv_sparsity": round(combined_sparsity(valid_tiles, kept, pv_skipped), 4),
+        "dropped_mass_alpha": alpha_rep,
+        "speed_dense_equiv_tops": round(dense_flops(w) / (mean_ms * 1e-3) / 1e12, 2),
+        "speed_note": "dense op count / step time incl. prediction ([P3] 3.2 Speed)",
         "kept_tiles": kept,
+        "valid_tiles": valid_tiles,
         "pv_skipped_tiles": pv_skipped,
         "flops_per_step": {"qk": qk_flops, "pv": pv_flops},
         "roofline": {"bound": "tensor", "achieved": round(attn_tf, 2), "peak": round(peak_tf, 1),
@@ -403,7 +447,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": None if args.qk8 else {
             "value": round(job_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
             "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "chunks": args.e2e_chunks},
+            "chunks": args.e2e_chunks, "entry_point": "sa_forward_host"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "wall_s": round(wall, 3),
@@ -553,6 +597,123 @@ def run_svg(args, rank, world, local_rank):
     }
 
 
+SWEEP_TARGETS = (0.5, 0.6, 0.7, 0.8, 0.9, 0.95)
+SWEEP_WORKLOADS = ("image", "video", "video_large")
+
+
+def run_sweep(args, rank, world, local_rank):
+    """--sweep: attention throughput against block sparsity ([P3] Fig. 10
+    and Table 11: kernel speed as sparsity rises).  For each workload shape
+    the similarity guard is off (theta = 0; the smooth-field generator's
+    blocks sit below theta = 0.6, which would force every block) and tau is
+    bisected on the library's own mask prediction until the kept-tile count
+    reaches each target block sparsity; targets below the forced blocks'
+    floor (sink and text rows and columns) report the floor.  One JSON line
+    per point: tau, theta, the achieved sparsity, attention time (median of
+    L2-flushed launches), kept-tile TFLOP/s, roofline fraction, dense time and
+    speedup beside the ideal 1 / (1 - s)."""
+    import numpy as np
+    import torch
+
+    from long_context_mean_b200 import inputs as I
+    from long_context_mean_b200 import sa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    pk, pk_src = peaks()
+    peak_tf = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    names = args.sweep.split(",") if args.sweep != "all" else list(SWEEP_WORKLOADS)
+    lines = []
+    for name in names:
+        w = I.WORKLOADS[name].with_(theta=0.0)
+        g = I.gen_qkv(w)
+        q, k, v = (torch.from_numpy(g[n + "_bits"].view(np.int16)).to(dev).view(torch.bfloat16) for n in "qkv")
+        del g
+        pipe = sa.pipeline_for(w, device=dev, log_skips=True)
+        pipe.run(q, k, v)
+        if pipe.status() != sa.SA_OK:
+            raise RuntimeError(f"{name}: device status {pipe.status()}")
+        qr, kr, vr = (q, k, v) if pipe.identity else (pipe.qr, pipe.kr, pipe.vr)
+        nqb, nkb = pipe.mask.struct.nqb, pipe.mask.struct.nkb
+        valid = valid_tile_count(w, nqb, nkb)
+
+        def timed(fn, n):
+            ts = []
+            for i in range(args.warmup + n):
+                flush.fill_(1.0)
+                a, b = ev(), ev()
+                a.record(stream)
+                fn()
+                b.record(stream)
+                if i >= args.warmup:
+                    ts.append((a, b))
+            torch.cuda.synchronize(dev)
+            return [x[0].elapsed_time(x[1]) for x in ts]
+
+        od = torch.empty_like(pipe.out)
+        dst = torch.zeros(1, dtype=torch.int32, device=dev)
+        dense_ms = statistics.median(timed(lambda: sa.dense_attn(qr, kr, vr, pipe.shape, w.causal, 0.0, od, None,
+                                                                 dst, ws=pipe.attn_ws), 5))
+
+        def predict(tau):
+            pipe.params.tau = float(tau)
+            if pipe.identity:
+                sa.predict_mask(q, k, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
+            else:
+                sa.reorder_predict_mask(pipe.perm, q, k, pipe.qr, pipe.kr, pipe.shape, pipe.params, pipe.ws,
+                                        pipe.mask.struct)
+            if pipe.status() != sa.SA_OK:
+                raise RuntimeError(f"{name}: device status {pipe.status()} at tau {tau}")
+            return 1.0 - int(pipe.mask.kept_total.item()) / valid
+
+        floor = predict(1e-9)              # tau -> 0: one TopCdf block per row plus the forced ones
+        for target in SWEEP_TARGETS:
+            lo, hi, tau = 0.0, 1.0, 0.5
+            s = predict(tau)
+            for _ in range(30):             # sparsity falls as tau grows
+                if abs(s - target) <= 0.002:
+                    break
+                lo, hi = (tau, hi) if s > target else (lo, tau)
+                tau = 0.5 * (lo + hi)
+                s = predict(tau)
+            if target > floor:
+                tau, s = 1e-9, predict(1e-9)
+            skip = torch.zeros(pipe.mask.col_idx.numel(), dtype=torch.uint8, device=dev)
+            sa.block_sparse_attn(qr, kr, vr, pipe.shape, pipe.mask.struct, w.lam, 0.0, pipe.out, pipe.lse, skip,
+                                 ws=pipe.attn_ws, out_perm=None if pipe.identity else pipe.perm)
+            rp = pipe.mask.row_ptr.cpu().numpy().astype(np.int64)
+            ci = pipe.mask.col_idx.cpu().numpy()
+            sk = skip.cpu().numpy()
+            qk, pv = kept_flops(w, rp, ci, sk, nqb)
+            kept = int(rp[-1])
+            ms = timed(lambda: sa.block_sparse_attn(qr, kr, vr, pipe.shape, pipe.mask.struct, w.lam, 0.0, pipe.out,
+                                                    pipe.lse, ws=pipe.attn_ws,
+                                                    out_perm=None if pipe.identity else pipe.perm), 10)
+            if pipe.status() != sa.SA_OK:
+                raise RuntimeError(f"{name}: device status after the sweep point")
+            att = statistics.median(ms)
+            tf = (qk + pv) / (att * 1e-3) / 1e12
+            line = {"sweep": name, "target_sparsity": target, "tau": round(tau, 6), "theta": 0.0, "lambda": w.lam,
+                    "block_sparsity": round(s, 4), "forced_floor_sparsity": round(floor, 4),
+                    "reached": abs(s - target) <= 0.005,
+                    "combined_qk_pv_sparsity": round(combined_sparsity(valid, kept, int(sk[:kept].sum())), 4),
+                    "kept_tiles": kept, "pv_skipped_tiles": int(sk[:kept].sum()),
+                    "attn_ms": spread(ms), "attn_tflops": round(tf, 2),
+                    "roofline_frac": round(tf / peak_tf, 4), "peak": peak_tf, "peak_source": f"{pk_src} bf16 (burst)",
+                    "dense_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / att, 3),
+                    "ideal_speedup": round(1.0 / max(1e-9, 1.0 - s), 3),
+                    "speed_dense_equiv_tops": round(dense_flops(w) / (att * 1e-3) / 1e12, 2)}
+            lines.append(line)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+        del pipe, q, k, v, qr, kr, vr
+        torch.cuda.empty_cache()
+    return None
+
+
 # ----------------------------------------------------------------------------
 # The oracle on the host cores (CPU baseline and the reference arm)
 # ----------------------------------------------------------------------------
@@ -650,6 +811,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-qblocks", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", default=None,
+                    help="attention throughput against block sparsity: 'all' or a comma list of workloads "
+                         "(one JSON line per point instead of the headline line)")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="head chunks of the end-to-end pass (copies overlap the kernels)")
     args = ap.parse_args()
@@ -670,7 +834,10 @@ def main():
             dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                     device_id=torch.device("cuda", local_rank))
         try:
-            res = (run_svg if args.path == "svg" else run_ours)(args, rank, world, local_rank)
+            if args.sweep:
+                res = run_sweep(args, rank, world, local_rank)
+            else:
+                res = (run_svg if args.path == "svg" else run_ours)(args, rank, world, local_rank)
         finally:
             if world > 1:
                 import torch.distributed as dist

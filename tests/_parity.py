@@ -83,8 +83,22 @@ def compare_masks(gpu_mask, orc, tau, theta, group):
     return int(diff.sum())
 
 
-def attention_check(out_gpu, lse_gpu, ref, rows=None):
-    """Element-wise comparison on the rows the oracle computed."""
+def report(label, **fields):
+    """Record one parity figure: printed, and appended as a JSON line to the
+    file named by SA_PARITY_REPORT when that is set."""
+    import json
+    import os
+    rec = {"case": label, **fields}
+    print("parity", json.dumps(rec))
+    path = os.environ.get("SA_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
+def attention_check(out_gpu, lse_gpu, ref, rows=None, label=None):
+    """Element-wise comparison on the rows the oracle computed.  The plain
+    max-abs is reported beside the held figure (relative above |O| = 1)."""
     o = np.asarray(out_gpu, dtype=np.float64)
     r = ref["out"]
     sel = ~np.isnan(r[..., 0])
@@ -92,12 +106,34 @@ def attention_check(out_gpu, lse_gpu, ref, rows=None):
         sel &= rows
     d = np.abs(o[sel] - r[sel])
     scaled = d / np.maximum(1.0, np.abs(r[sel]))
-    assert scaled.max() <= OUT_MAX_ABS, f"max abs (relative above 1) {scaled.max()} (plain max abs {d.max()})"
-    assert d.mean() <= OUT_MEAN_ABS, f"mean abs {d.mean()}"
+    dl = None
     if lse_gpu is not None:
         dl = np.abs(np.asarray(lse_gpu, dtype=np.float64)[sel] - ref["lse"][sel])
+    if label is not None:
+        report(label, rows=int(sel.sum()), out_max_abs=float(d.max()), out_max_rel_above_1=float(scaled.max()),
+               out_mean_abs=float(d.mean()), lse_max_abs=None if dl is None else float(dl.max()))
+    assert scaled.max() <= OUT_MAX_ABS, f"max abs (relative above 1) {scaled.max()} (plain max abs {d.max()})"
+    assert d.mean() <= OUT_MEAN_ABS, f"mean abs {d.mean()}"
+    if dl is not None:
         assert dl.max() <= LSE_ABS, f"lse max abs {dl.max()}"
     return float(d.max()), float(d.mean())
+
+
+def alpha_report(label, lse_sparse, lse_dense, sel=None):
+    """Per-row dropped probability mass alpha = 1 - exp(LSE_sparse -
+    LSE_dense) ([P1] 3.2: z = exp(LSE_kept - LSE_full) is the kept mass),
+    computed by the oracle; reports mean, max and the worst (b, h, row).
+    A restricted softmax keeps at most the full mass, so alpha >= 0 up to the
+    two LSEs' tolerance."""
+    a = A.dropped_mass_from_lse(lse_sparse, lse_dense)
+    if sel is None:
+        sel = np.isfinite(a)
+    vals = a[sel]
+    worst = np.unravel_index(int(np.argmax(np.where(sel, a, -np.inf))), a.shape)
+    report(label, alpha_rows=int(sel.sum()), alpha_mean=float(vals.mean()), alpha_max=float(vals.max()),
+           alpha_min=float(vals.min()), alpha_worst=[int(x) for x in worst])
+    assert vals.min() >= -2 * LSE_ABS, f"alpha {vals.min()} below 0 beyond the LSE tolerance"
+    return a
 
 
 def skip_override_from_gpu(skip_log, row_ptr, col_idx, nqb, B, Hq):

@@ -48,7 +48,23 @@ def oracle_check(w, g, pipe, out, lse, heads, qblocks):
     # back to the original token order
     ref_out = Y.unreorder(ref["out"], perm, axis=2)
     ref_lse = Y.unreorder(ref["lse"], perm, axis=2)
-    return P.attention_check(out, lse, {"out": ref_out, "lse": ref_lse})
+    return P.attention_check(out, lse, {"out": ref_out, "lse": ref_lse}, label=f"{w.name} pipeline")
+
+
+def dense_lse_gpu(w, g):
+    """LSE of dense attention (sa_dense_attn) on the original-order inputs:
+    dense attention is permutation-equivariant, so its rows line up with the
+    pipeline's original-order LSE."""
+    import torch
+    from long_context_mean_b200 import sa
+    q, k, v = P.qkv_dev(g, w.dtype)
+    shape = sa.make_shape(q, k, v)
+    out = torch.empty((w.B, w.Hq, w.N, w.dv), dtype=q.dtype, device="cuda")
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.dense_attn(q, k, v, shape, w.causal, 0.0, out, lse, st)
+    assert sa.read_status(st) == sa.SA_OK
+    return lse.cpu().numpy()
 
 
 @pytest.mark.parametrize("flags", [0, 1])
@@ -58,6 +74,10 @@ def test_toy_pipeline(flags):
     pipe, out, lse, st = run_pipeline(w, g, flags)
     assert st == 0
     oracle_check(w, g, pipe, out, lse, None, None)
+    # dropped mass of every row against the oracle's dense attention
+    dense = np.stack([[A.dense_attention(g["q"][b, h], g["k"][b, h], g["v"][b, h], w.causal)[1]
+                       for h in range(w.Hq)] for b in range(w.B)])
+    P.alpha_report(f"toy pipeline flags={flags}", lse, dense)
 
 
 def test_toy_full_and_same_frame_masks():
@@ -84,12 +104,67 @@ def test_toy_full_and_same_frame_masks():
         assert np.abs(lse.cpu().numpy()[0, 0] - l).max() < 1e-5
 
 
-@pytest.mark.parametrize("name", ["video", "image"])
+def gpu_block_sparsity(w, pipe):
+    """1 - kept / causally valid tiles of the GPU's mask, over batch and heads."""
+    nqb, nkb = pipe.mask.struct.nqb, pipe.mask.struct.nkb
+    kept = int(pipe.mask.row_ptr.cpu().numpy()[-1])
+    if w.causal:
+        valid = w.B * w.Hq * sum(min(nkb, (min(w.N, (qb + 1) * w.bq) - 1) // w.bk + 1) for qb in range(nqb))
+    else:
+        valid = w.B * w.Hq * nqb * nkb
+    return 1.0 - kept / valid
+
+
+def test_toy_same_position_mask_through_the_window_reorder():
+    """The toy grid's third fixed mask ([P1] 3.3: each token with the same
+    pixel in every frame, 256 pairs): the [T,1,1] window layout puts a pixel's
+    frames next to each other ([P1] 3.4, token-major order), where the mask is
+    block-diagonal with 4-token blocks (bq = bk = 4, 16 of 256 tiles).  Layout,
+    reorder, attention and inverse reorder run on the GPU; the oracle applies
+    the element mask in the original order."""
+    import torch
+    from long_context_mean_b200 import sa
+    from oracle import ledger as L
+    w = I.WORKLOADS["toy"]
+    g = I.gen_qkv(w)
+    q, k, v = P.qkv_dev(g, "fp32")
+    lay = sa.make_layout(4, 4, 4, 0, 0, "window", (4, 1, 1))
+    perm = torch.empty(64, dtype=torch.int32, device="cuda")
+    inv = torch.empty_like(perm)
+    sa.layout_build(lay, perm, inv)
+    ref_perm, _ = Y.build_layout("window", 4, 4, 4, (4, 1, 1), 0, 0)
+    assert np.array_equal(perm.cpu().numpy(), ref_perm)
+    qr, kr, vr = (torch.empty_like(x) for x in (q, k, v))
+    for x, y in ((q, qr), (k, kr), (v, vr)):
+        sa.reorder(perm, x, y)
+    shape = sa.make_shape(q, k, v)
+    blocks = np.eye(16, dtype=bool)
+    mb = sa.MaskBuffers.allocate(1, 1, 64, 4, 4, "cuda")
+    ws = sa.workspace(sa.mask_from_blocks_workspace(shape, 4, 4), "cuda")
+    sa.mask_from_blocks(torch.from_numpy(blocks.astype(np.uint8).ravel()).cuda(), shape, 4, 4, False, ws,
+                        mb.struct)
+    out = torch.empty_like(q)
+    lse = torch.empty(1, 1, 64, 1, dtype=torch.float32, device="cuda")
+    sa.block_sparse_attn(qr, kr, vr, shape, mb.struct, -math.inf, 0.0, out, lse, out_perm=perm)
+    assert sa.read_status(mb.status) == 0
+    assert int(mb.kept_total.item()) == 16
+    tok = L.video_masks(4, 4, 4)["temporal"]
+    assert int(tok.sum()) == 256
+    y, _, l = A.masked_attention(g["q"][0, 0], g["k"][0, 0], g["v"][0, 0], tok)
+    assert np.abs(out.cpu().numpy()[0, 0] - y).max() < 1e-5
+    assert np.abs(lse.cpu().numpy()[0, 0, :, 0] - l).max() < 1e-5
+
+
+@pytest.mark.parametrize("name", ["video", "image", "image_s60"])
 def test_full_size_pipeline_sampled(name):
     w = I.WORKLOADS[name]
     g = I.gen_qkv(w)
     pipe, out, lse, st = run_pipeline(w, g)
     assert st == 0
+    if w.theta <= 0 and w.target_sparsity > 0:
+        s = gpu_block_sparsity(w, pipe)
+        P.report(f"{name} block sparsity", sparsity=s, target=w.target_sparsity)
+        assert abs(s - w.target_sparsity) <= 0.01
     nqb = pipe.mask.struct.nqb
     heads = [(0, 0), (0, w.Hq - 1)] + ([(1, 5)] if w.B > 1 else [(0, 7)])
     qblocks = sorted({0, 1, nqb // 2, nqb - 2, nqb - 1})
@@ -103,6 +178,7 @@ def test_full_size_pipeline_sampled(name):
     for b, h in heads:
         sel[b, h] = rows_orig
     oracle_check(w, g, pipe, out, lse, heads, qblocks)
+    P.alpha_report(f"{name} pipeline, every row", lse, dense_lse_gpu(w, g))
 
 
 def _sampled_heads_check(w, heads, kv_of, qblocks):
@@ -145,13 +221,27 @@ def _sampled_heads_check(w, heads, kv_of, qblocks):
                                                      skip_override=over, band=P.LAMBDA_BAND)
         ref_out = Y.unreorder(ref["out"], perm, axis=2)
         ref_lse = Y.unreorder(ref["lse"], perm, axis=2)
-        P.attention_check(out_h[b:b + 1, h:h + 1], lse_h[b:b + 1, h:h + 1], {"out": ref_out, "lse": ref_lse})
+        P.attention_check(out_h[b:b + 1, h:h + 1], lse_h[b:b + 1, h:h + 1], {"out": ref_out, "lse": ref_lse},
+                          label=f"{w.name} sampled head ({b},{h})")
+    P.alpha_report(f"{w.name} pipeline, every row", lse_h, dense_lse_gpu(w, g))
+    return pipe
 
 
 def test_video_large_hilbert_sampled():
     w = I.WORKLOADS["video_large"]
     nqb = -(-w.N // w.bq)
     _sampled_heads_check(w, [(0, 0), (0, 23)], lambda h: h, [0, 300, nqb - 1])
+
+
+def test_video_large_hilbert_at_sparsity_085_sampled():
+    """The large Hilbert video at its stated block sparsity (guard off):
+    TopCdf, the ragged lists and the scheduler do real work at this size."""
+    w = I.WORKLOADS["video_large_s85"]
+    nqb = -(-w.N // w.bq)
+    pipe = _sampled_heads_check(w, [(0, 0), (0, 11), (0, 23)], lambda h: h, [0, 29, 300, 411, nqb - 1])
+    s = gpu_block_sparsity(w, pipe)
+    P.report("video_large_s85 block sparsity", sparsity=s, target=w.target_sparsity)
+    assert abs(s - w.target_sparsity) <= 0.01
 
 
 def test_lm_causal_gqa_sampled():
