@@ -149,6 +149,13 @@ typedef struct {
                                   the tensor-core kernel applies (testing) */
 #define SA_FLAG_OUT_PERM_PER_HEAD 2   /* out_perm is int32 [B*Hq][N], one
                                          permutation per query head */
+#define SA_FLAG_TEST_STALL 4          /* testing the timeout path: on the
+                                         tensor-core kernel, the first CTA loads
+                                         no K tile, so its bounded waits (10 ms
+                                         under this flag instead of 2 s) run out
+                                         and the status word gets
+                                         SA_ERR_TIMEOUT; that CTA's query rows are
+                                         not computed.  Never set in normal use. */
 
 /* Library version string and the calling thread's last error message. */
 const char* sa_version(void);

@@ -332,6 +332,7 @@ static sa_status attn_common(const void* q, const void* k, const void* v, const 
   if ((flags & SA_FLAG_OUT_PERM_PER_HEAD) && !out_perm)
     return set_error(SA_ERR_INVALID_ARG, "SA_FLAG_OUT_PERM_PER_HEAD needs out_perm");
   a.perm_stride = (flags & SA_FLAG_OUT_PERM_PER_HEAD) ? shape->N : 0;
+  a.flags = flags;
   if (out_perm && (out == q || out == k || out == v))
     return set_error(SA_ERR_INVALID_ARG, "out must not alias an input when out_perm is given");
   a.skip_log = skip_log;

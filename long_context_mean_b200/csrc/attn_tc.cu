@@ -39,9 +39,12 @@
 // kind::i8 / kind::f8f6f4 steps, and the softmax multiplies each tile by its
 // own scale (the two block scales of the quantisation); INT8 scores are
 // int32 and reach the float path through an exact biased-float add.
-// Every mbarrier wait is bounded (2 s); on expiry the kernel raises
-// SA_ERR_TIMEOUT, every later wait returns at once, the producers drain
-// their own loads (bounded) and the TMEM allocation is released.
+// Every mbarrier wait is bounded (2 s; 10 ms under SA_FLAG_TEST_STALL); on
+// expiry the kernel raises SA_ERR_TIMEOUT and sets the CTA's abort flag, after
+// which every wait returns at once and every role stops issuing: the loaders
+// drain the copies they issued, the MMA warp waits (bounded) for the tensor
+// operations it issued, the softmax warps leave together, and the TMEM
+// allocation is released.
 #include <cuda.h>
 
 #include "sa_internal.cuh"
@@ -49,7 +52,8 @@
 namespace sa {
 namespace {
 
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;       // 2 s
+constexpr unsigned long long kTestWaitLimitNs = 10000000ull;     // 10 ms (SA_FLAG_TEST_STALL)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -99,6 +103,8 @@ struct Ctl {
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t u_full[4], u_empty[4];          // unit announcement ring
+  uint64_t mma_done;                       // the MMA warp's last tensor operations have completed
+  unsigned long long wait_ns;              // limit of every wait
   uint32_t tmem_base;
   volatile uint32_t abort;
   float gapw[4][8];                        // [tile & 3][softmax warp]
@@ -139,6 +145,8 @@ struct TcParams {
   int32_t causal;
   float scale_log2;
   float lam_log2;
+  unsigned long long wait_ns;   // limit of every mbarrier wait
+  int32_t stall;                // test hook: CTA 0 issues no K loads (its waits run out)
 };
 
 // ---------------------------------------------------------------------------
@@ -185,7 +193,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl* g
   for (;;) {
     if (mbar_try(bar, parity)) return true;
     if (g->abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > g->wait_ns) {
       g->abort = 1;
       raise_status(status, SA_ERR_TIMEOUT);
       return false;
@@ -193,10 +201,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl* g
   }
 }
 // Bounded wait that ignores the abort flag (draining in-flight copies).
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, unsigned long long limit) {
   const unsigned long long t0 = globaltimer();
   while (!mbar_try(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) return;
+    if (globaltimer() - t0 > limit) return;
   }
 }
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
@@ -446,7 +454,7 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const C
     // Take the next unit of the work order and announce it to the pipeline's
     // V loader, MMA and softmax warps through a 4-slot ring.
     const int slot = j & 3;
-    mbar_wait(&c->u_empty[slot], ((j >> 2) & 1) ^ 1, g, p.status);
+    if (!mbar_wait(&c->u_empty[slot], ((j >> 2) & 1) ^ 1, g, p.status)) break;
     int i = atomicAdd(p.counter, 1);
     if (i >= p.num_units) i = -1;
     Unit u{};
@@ -455,27 +463,33 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const C
     mbar_arrive(&c->u_full[slot]);
     if (i < 0) break;
     if (u.n <= 0) continue;
-    mbar_wait(&c->q_empty, (nq & 1) ^ 1, g, p.status);
+    if (!mbar_wait(&c->q_empty, (nq & 1) ^ 1, g, p.status)) break;
     ++nq;
     mbar_expect_tx(&c->q_full, C::Q_BYTES);
     tma_load_3d(sb + C::off_q(pipe), tmQ, 0, (int)(u.qb * 128), (int)u.bh, &c->q_full);
     if constexpr (QM == 0)   // bf16 rows are two 128-byte chunks; 8-bit rows one
       tma_load_3d(sb + C::off_q(pipe) + C::Q_BYTES / 2, tmQ, 64, (int)(u.qb * 128), (int)u.bh, &c->q_full);
-    for (int64_t t = 0; t < u.n; ++t, ++k_it) {
+    if (p.stall && blockIdx.x == 0) continue;   // test hook: no K tile arrives here
+    bool ok = true;
+    for (int64_t t = 0; t < u.n && ok; ++t) {
       const int kb = (int)kblock_at(p, u, t);
       const int s = k_it % C::K_STAGES;
       const uint32_t ph = (k_it / C::K_STAGES) & 1;
       const uint32_t kdst = sb + C::off_k(pipe) + s * C::K_BYTES;
-      mbar_wait(&c->k_empty[s], ph ^ 1, g, p.status);
+      ok = mbar_wait(&c->k_empty[s], ph ^ 1, g, p.status);
+      if (!ok) break;
       mbar_expect_tx(&c->k_full[s], C::K_BYTES);
       tma_load_3d(kdst, tmK, 0, kb * BK, (int)u.kvh, &c->k_full[s]);
       if constexpr (QM == 0) tma_load_3d(kdst + C::KV_CHUNK, tmK, 64, kb * BK, (int)u.kvh, &c->k_full[s]);
+      ++k_it;
     }
+    if (!ok) break;
   }
-  // Drain: the last loads of every stage (and the last Q) have landed.
-  if (nq > 0) mbar_drain(&c->q_full, (nq - 1) & 1);
+  // Drain: the last copies issued into every stage (and the last Q) have
+  // landed before the CTA may exit.
+  if (nq > 0) mbar_drain(&c->q_full, (nq - 1) & 1, g->wait_ns);
   for (uint32_t j = k_it > (uint32_t)C::K_STAGES ? k_it - C::K_STAGES : 0; j < k_it; ++j)
-    mbar_drain(&c->k_full[j % C::K_STAGES], (j / C::K_STAGES) & 1);
+    mbar_drain(&c->k_full[j % C::K_STAGES], (j / C::K_STAGES) & 1, g->wait_ns);
 }
 
 // Lane 1 of the producer warp loads the V tiles on their own ring, so a K
@@ -486,24 +500,28 @@ __device__ void v_loader(const CUtensorMap* tmV, const TcParams& p, Ctl* c, Ctl*
   uint32_t v_it = 0;
   for (uint32_t j = 0;; ++j) {
     const int slot = j & 3;
-    mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status);
+    if (!mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status)) break;
     Unit u;
     const int i = read_unit(c, slot, u);
     mbar_arrive(&c->u_empty[slot]);
     if (i < 0) break;
-    for (int64_t t = 0; t < u.n; ++t, ++v_it) {
+    bool ok = true;
+    for (int64_t t = 0; t < u.n; ++t) {
       const int kb = (int)kblock_at(p, u, t);
       const int s = v_it % C::V_STAGES;
       const uint32_t ph = (v_it / C::V_STAGES) & 1;
       const uint32_t vdst = sb + C::off_v(pipe) + s * C::V_BYTES;
-      mbar_wait(&c->v_empty[s], ph ^ 1, g, p.status);
+      ok = mbar_wait(&c->v_empty[s], ph ^ 1, g, p.status);
+      if (!ok) break;
       mbar_expect_tx(&c->v_full[s], C::V_BYTES);
       tma_load_3d(vdst, tmV, 0, kb * BK, (int)u.kvh, &c->v_full[s]);
       tma_load_3d(vdst + C::KV_CHUNK, tmV, 64, kb * BK, (int)u.kvh, &c->v_full[s]);
+      ++v_it;
     }
+    if (!ok) break;
   }
   for (uint32_t j = v_it > (uint32_t)C::V_STAGES ? v_it - C::V_STAGES : 0; j < v_it; ++j)
-    mbar_drain(&c->v_full[j % C::V_STAGES], (j / C::V_STAGES) & 1);
+    mbar_drain(&c->v_full[j % C::V_STAGES], (j / C::V_STAGES) & 1, g->wait_ns);
 }
 
 template <int BK, int QM>
@@ -513,24 +531,26 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
       QM == 1 ? make_idesc_s8(128, BK) : (QM == 2 ? make_idesc_e4m3(128, BK) : make_idesc(128, BK, 0));
   constexpr uint32_t idesc_pv = make_idesc(128, 128, 1);
   uint32_t kv_it = 0, gt0 = 0, unit_it = 0;   // unit_it counts units with work
-  for (uint32_t j = 0;; ++j) {
+  bool ok = true;                             // false once a wait gave up: issue nothing more
+  for (uint32_t j = 0; ok; ++j) {
     const int slot = j & 3;
-    mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status);
+    if (!(ok = mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status))) break;
     Unit u;
     const int i = read_unit(c, slot, u);
     mbar_arrive(&c->u_empty[slot]);
     if (i < 0) break;
     if (u.n <= 0) continue;
-    mbar_wait(&c->q_full, unit_it & 1, g, p.status);
+    if (!(ok = mbar_wait(&c->q_full, unit_it & 1, g, p.status))) break;
     tc_fence_after();
     const uint32_t qbase = sb + C::off_q(pipe);
     bool first_pv = true;
     auto do_pv = [&](int64_t tt) {
+      if (!ok) return;
       const uint32_t it = kv_it + (uint32_t)tt, gt = gt0 + (uint32_t)tt;
       const int s = it % C::V_STAGES;
       const uint32_t ph = (it / C::V_STAGES) & 1;
       const int gb = C::sbuf(gt);
-      mbar_wait(&c->p_full[gb], C::sphase(gt), g, p.status);
+      if (!(ok = mbar_wait(&c->p_full[gb], C::sphase(gt), g, p.status))) return;
       tc_fence_after();
       const float* gw = c->gapw[gt & 3];
       float gmax = gw[0];
@@ -539,10 +559,10 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
       const bool skip = gmax < p.lam_log2;
       if (p.skip_log && p.row_ptr) p.skip_log[u.lo + tt] = skip ? 1 : 0;
       if (tt == 0) {
-        mbar_wait(&c->o_free, (unit_it & 1) ^ 1, g, p.status);
+        if (!(ok = mbar_wait(&c->o_free, (unit_it & 1) ^ 1, g, p.status))) return;
         tc_fence_after();
       }
-      mbar_wait(&c->v_full[s], ph, g, p.status);
+      if (!(ok = mbar_wait(&c->v_full[s], ph, g, p.status))) return;
       tc_fence_after();
       if (!skip) {
         const uint32_t vbase = sb + C::off_v(pipe) + s * C::V_BYTES;
@@ -557,12 +577,12 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
       umma_commit(&c->v_empty[s]);
       umma_commit(&c->pv_done[gb]);
     };
-    for (int64_t t = 0; t < u.n; ++t) {
+    for (int64_t t = 0; t < u.n && ok; ++t) {
       const uint32_t it = kv_it + (uint32_t)t, gt = gt0 + (uint32_t)t;
       const int s = it % C::K_STAGES;
       const uint32_t ph = (it / C::K_STAGES) & 1;
       const uint32_t scol = tm + C::S_COL + C::sbuf(gt) * BK;
-      mbar_wait(&c->k_full[s], ph, g, p.status);
+      if (!(ok = mbar_wait(&c->k_full[s], ph, g, p.status))) break;
       tc_fence_after();
       const uint32_t kbase = sb + C::off_k(pipe) + s * C::K_BYTES;
       if constexpr (QM != 0) {
@@ -594,6 +614,10 @@ __device__ void mma_issuer(const TcParams& p, Ctl* c, Ctl* g, uint32_t sb, uint3
     gt0 += (uint32_t)u.n;
     ++unit_it;
   }
+  // Every tensor operation this thread issued has completed before the TMEM
+  // allocation can be released (on the normal path they already have).
+  umma_commit(&c->mma_done);
+  mbar_drain(&c->mma_done, 0, g->wait_ns);
 }
 
 // Largest value of a float over the warp (order-preserving int key).
@@ -624,7 +648,9 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
   uint32_t gt0 = 0;
   for (uint32_t j = 0;; ++j) {
     const int slot = j & 3;
-    mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status);
+    // A wait that gives up (the CTA is aborting) ends the warp's work; the
+    // decision is warp-uniform, as tcgen05.ld/st are warp-collective.
+    if (!__all_sync(0xffffffffu, mbar_wait(&c->u_full[slot], (j >> 2) & 1, g, p.status))) return;
     Unit u;
     const int i = read_unit(c, slot, u);
     __syncwarp();
@@ -655,7 +681,7 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
         sc = sc_next;
         if (t + 1 < u.n) sc_next = p.tile_scale[u.lo + t + 1];
       }
-      mbar_wait(&c->s_full[gb], C::sphase(gt), g, p.status);
+      if (!__all_sync(0xffffffffu, mbar_wait(&c->s_full[gb], C::sphase(gt), g, p.status))) return;
       tc_fence_after();
       float s[NC];
       if constexpr (SPLIT == 2) {
@@ -752,7 +778,7 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
       // tile is not skipped, so PV(t-1) is the last product to wait for.
       if (__any_sync(0xffffffffu, resc)) {
         const uint32_t gp = gt - 1;
-        mbar_wait(&c->pv_done[C::sbuf(gp)], C::sphase(gp), g, p.status);
+        if (!__all_sync(0xffffffffu, mbar_wait(&c->pv_done[C::sbuf(gp)], C::sphase(gp), g, p.status))) return;
         tc_fence_after();
         const float f = resc ? corr : 1.f;
         if constexpr (SPLIT == 2) {
@@ -791,7 +817,7 @@ __device__ void softmax_rows(const TcParams& p, Ctl* c, Ctl* g, uint32_t tm, int
     }
     // Epilogue: O / l from TMEM once the unit's last PV has landed.
     const uint32_t gl = gt0 + (uint32_t)u.n - 1;
-    mbar_wait(&c->pv_done[C::sbuf(gl)], C::sphase(gl), g, p.status);
+    if (!__all_sync(0xffffffffu, mbar_wait(&c->pv_done[C::sbuf(gl)], C::sphase(gl), g, p.status))) return;
     tc_fence_after();
     if constexpr (SPLIT == 2) l += __shfl_xor_sync(0xffffffffu, l, 16);   // the row's two parts
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -863,6 +889,8 @@ __global__ void __launch_bounds__(Cfg<BK, QM>::THREADS, 1)
         mbar_init(&c->u_full[r], 1);
         mbar_init(&c->u_empty[r], 2 + C::SM_WARPS);   // the V lane, the MMA lane, one lane per softmax warp
       }
+      mbar_init(&c->mma_done, 1);
+      c->wait_ns = p.wait_ns;
       c->abort = 0;
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -976,6 +1004,8 @@ sa_status launch_bk(const AttnArgs& a, cudaStream_t st) {
   p.causal = a.causal;
   p.scale_log2 = a.scale * kLog2e;
   p.lam_log2 = a.lambda * kLog2e;
+  p.stall = (a.flags & SA_FLAG_TEST_STALL) ? 1 : 0;
+  p.wait_ns = p.stall ? kTestWaitLimitNs : kWaitLimitNs;
   if (p.num_units == 0) return SA_OK;
   if (cudaMemsetAsync(p.counter, 0, sizeof(int32_t), st) != cudaSuccess)
     return set_error(SA_ERR_CUDA, "cudaMemsetAsync(work counter) failed");

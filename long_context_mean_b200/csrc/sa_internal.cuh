@@ -159,6 +159,7 @@ struct AttnArgs {
   int64_t nqb, nkb;
   float scale;
   float lambda;
+  int32_t flags;            // SA_FLAG_* of the call
 };
 sa_status launch_attn_simt(const AttnArgs& a, cudaStream_t st);
 sa_status launch_head_placement(int64_t T, int64_t P, int64_t n, const int32_t* kinds, int64_t heads, int bq,

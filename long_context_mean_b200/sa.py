@@ -333,6 +333,7 @@ SA_HEAD_SPATIAL, SA_HEAD_TEMPORAL = 0, 1
 
 
 SA_FLAG_OUT_PERM_PER_HEAD = 2
+SA_FLAG_TEST_STALL = 4   # testing the timeout path only (see the header)
 
 
 def head_placement(T, H, W, txt_len, kinds, bq, bk, perms=None, block_mask=None, status=None, stream=None):

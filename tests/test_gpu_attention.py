@@ -210,3 +210,29 @@ def test_undersized_mask_attention_stays_in_bounds(path):
     o = out.float().cpu().numpy()[0, 0]
     assert np.isfinite(o[:3 * bq]).all() and (np.abs(o[:3 * bq]).sum(axis=1) > 0).all()
     assert (o[3 * bq:] == 0).all()
+
+
+@pytest.mark.parametrize("bk", [64, 128])
+def test_timeout_path_reports_and_recovers(bk):
+    """The bounded waits' error path in the form this pool allows (no GPU
+    fault, no endless wait): SA_FLAG_TEST_STALL makes the first CTA of the
+    tensor-core kernel load no K tile, so its waits run out after 10 ms.  The
+    call must report SA_ERR_TIMEOUT, every role must stop issuing and drain,
+    the CTA must release its TMEM, and later calls on the same context must
+    run normally and match the oracle (twice, so a leak of TMEM or of a
+    barrier phase would show)."""
+    from long_context_mean_b200 import sa
+    N, bq = 2048, 128
+    w = I.Workload("stall", 4321, 1, 4, 4, 1, 1, N, 0, 128, 128, "bf16", "field", sigma=(0.0, 0.0, 8.0), noise=0.5)
+    g = I.gen_qkv(w)
+    q, k, v = P.qkv_dev(g, "bf16")
+    rng = np.random.default_rng(bk)
+    m = random_mask(rng, 1, 4, N, bq, bk, False, 0.5)
+    assert sa.attn_kernel_path(sa.make_shape(q, k, v), bq, bk) == 1
+    for _ in range(2):
+        r = run_sparse(q, k, v, m, bq, bk, False, -math.inf, sa.SA_FLAG_TEST_STALL, log=False)
+        assert r["status"] == sa.SA_ERR_TIMEOUT
+        r = run_sparse(q, k, v, m, bq, bk, False, -math.inf, 0, log=False)
+        assert r["status"] == sa.SA_OK
+        ref = A.block_sparse_attention_heads(g["q"], g["k"], g["v"], m, bq, bk, False)
+        P.attention_check(r["out"], r["lse"], ref)
