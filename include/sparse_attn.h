@@ -110,13 +110,22 @@ typedef struct {
  *   local_window  w > 0 keeps every block pair holding some (i, j) with
  *                 0 <= i - j < w ([P4], block level); 0 = off.
  *   anchor_tokens tokens at the front whose key blocks get full columns.
- *   causal        1 = key j visible to query i only if j <= i. */
+ *   causal        1 = key j visible to query i only if j <= i.
+ *   order_group   the work order of the mask's rows (sa_mask.order).  0:
+ *                 every row by descending kept count, ties by ascending row
+ *                 index.  g > 0: rows in groups of g consecutive (batch,
+ *                 query head) pairs, the groups in order, and the rows of a
+ *                 group by descending count, ties by ascending row index, so
+ *                 that the rows running at the same time share their heads'
+ *                 K and V in L2.  sa_order_group_hint() gives the library's
+ *                 choice for a shape.  Must be >= 0, and order_group * nqb
+ *                 <= 32768. */
 typedef struct {
   int32_t bq, bk;
   float tau, theta;
   int64_t sink_tokens, txt_len, local_window, anchor_tokens;
   int32_t causal;
-  int32_t reserved;
+  int32_t order_group;
 } sa_mask_params;
 
 /* A block mask and its compacted lists.  All pointers are device buffers
@@ -194,10 +203,20 @@ sa_status sa_unreorder(const int32_t* perm, const void* y, void* x, int64_t oute
  * anchors and local window, ANDs causal validity, checks that every query
  * row keeps a key, and builds the CSR lists and work order into *out.
  * Needs d a power of two with d*elem_size a multiple of 16 and d <= 256,
- * N/bk <= 4095.  ws: sa_predict_mask_workspace() bytes, 256-byte aligned;
- * its layout (pooled means and similarities, fp32) is reported by
- * sa_predict_mask_ws_layout() for inspection. */
+ * N/bk <= 4095.  ws: sa_predict_mask_workspace() bytes, 256-byte aligned.
+ * sa_predict_mask_ws_layout() reports the byte offsets of its regions, for
+ * inspection: [0] q_hat fp32 [B*Hq, nqb, d]; [1] k_hat fp32 [B*Hkv, d, nkb4]
+ * (feature-major, nkb4 = nkb rounded up to a multiple of 4, columns >= nkb
+ * unused); [2] query-block similarity fp32 [B*Hq, nqb]; [3] key-block
+ * similarity fp32 [B*Hkv, nkb]; [4] row counts int32 [B*Hq*nqb]; [5] sort
+ * scratch. */
 size_t sa_predict_mask_workspace(const sa_shape* shape, const sa_mask_params* params);
+/* order_group for a shape: 0 (one global order) when the K and V of one KV
+ * head take less than 32 MiB (several heads' K/V stay in L2 anyway);
+ * otherwise the largest power of two g <= B*Hq whose g consecutive query
+ * heads touch at most 96 MiB of K and V (at least 1).  -1 for an invalid
+ * shape. */
+int32_t sa_order_group_hint(const sa_shape* shape);
 sa_status sa_predict_mask_ws_layout(const sa_shape* shape, const sa_mask_params* params,
                                     size_t offsets[6]);
 sa_status sa_predict_mask(const void* q, const void* k, const sa_shape* shape,

@@ -160,6 +160,18 @@ size_t sa_predict_mask_workspace(const sa_shape* shape, const sa_mask_params* p)
   return predict_ws_bytes(*shape, p->bq, p->bk, off);
 }
 
+int32_t sa_order_group_hint(const sa_shape* shape) {
+  if (check_shape(shape) != SA_OK) return -1;
+  const double kv_head = (double)shape->N * (double)(shape->d + shape->dv) * elem_size(shape->dtype);
+  const double lo = 32.0 * 1024 * 1024, hi = 96.0 * 1024 * 1024;
+  if (kv_head < lo) return 0;
+  const int64_t rep = shape->Hq / shape->Hkv;   // query heads per KV head
+  const int64_t heads = shape->B * shape->Hq;
+  int64_t g = 1;
+  while (2 * g <= heads && (double)ceil_div(2 * g, rep) * kv_head <= hi) g *= 2;
+  return (int32_t)g;
+}
+
 sa_status sa_predict_mask_ws_layout(const sa_shape* shape, const sa_mask_params* p, size_t offsets[6]) {
   if (sa_status e = check_shape(shape)) return e;
   if (!p || !offsets || p->bq < 1 || p->bk < 1) return set_error(SA_ERR_INVALID_ARG, "bad arguments");
@@ -182,6 +194,9 @@ sa_status predict_prepare(const char* who, const void* q, const void* k, const s
   if (p.sink_tokens < 0 || p.txt_len < 0 || p.local_window < 0 || p.anchor_tokens < 0)
     return set_error(SA_ERR_INVALID_ARG, "token counts must be non-negative");
   if (p.causal != 0 && p.causal != 1) return set_error(SA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (p.order_group < 0) return set_error(SA_ERR_INVALID_ARG, "order_group must be >= 0");
+  if (p.order_group > 0 && (int64_t)p.order_group * ceil_div(shape->N, p.bq) > 32768)
+    return set_error(SA_ERR_UNSUPPORTED, "order_group * nqb must be <= 32768");
   if (sa_status e = check_mask_out(out)) return e;
   if ((uintptr_t)q % 16 || (uintptr_t)k % 16) return set_error(SA_ERR_INVALID_ARG, "q and k must be 16-byte aligned");
   size_t off[6];

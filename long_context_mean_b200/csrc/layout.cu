@@ -194,6 +194,42 @@ __global__ void __launch_bounds__(256) reorder_vec_kernel(const int32_t* __restr
   }
 }
 
+// Rows of 16 * 2^cpr_shift bytes: one CTA moves STEPS * (256 >> cpr_shift)
+// consecutive rows n of one outer index o (blockIdx.y), chunk c of row rr of
+// a step in thread rr * cpr + c, so a warp copies whole 128-byte lines and no
+// index needs a division.  All STEPS loads of a thread are issued before
+// its first store.
+template <int STEPS>
+__global__ void __launch_bounds__(256) reorder_rows_kernel(const int32_t* __restrict__ perm, int64_t pstride,
+                                                           const uint4* __restrict__ src,
+                                                           uint4* __restrict__ dst, int64_t N, int cpr_shift,
+                                                           bool scatter) {
+  const int64_t o = blockIdx.y;
+  const int rows_per_step = 256 >> cpr_shift;
+  const int64_t n0 = (int64_t)blockIdx.x * rows_per_step * STEPS;
+  const int64_t cpr = (int64_t)1 << cpr_shift;
+  const int c = threadIdx.x & ((1 << cpr_shift) - 1);
+  const int rr = threadIdx.x >> cpr_shift;
+  const int32_t* po = perm + o * pstride;
+  int64_t soff[STEPS], doff[STEPS];
+#pragma unroll
+  for (int u = 0; u < STEPS; ++u) {
+    const int64_t n = n0 + u * rows_per_step + rr;
+    soff[u] = doff[u] = -1;
+    if (n < N) {
+      const int64_t pn = __ldg(po + n);
+      soff[u] = (o * N + (scatter ? n : pn)) * cpr + c;
+      doff[u] = (o * N + (scatter ? pn : n)) * cpr + c;
+    }
+  }
+  uint4 v[STEPS];
+#pragma unroll
+  for (int u = 0; u < STEPS; ++u) v[u] = soff[u] >= 0 ? __ldg(src + soff[u]) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int u = 0; u < STEPS; ++u)
+    if (doff[u] >= 0) __stcs(dst + doff[u], v[u]);
+}
+
 __global__ void reorder_word_kernel(const int32_t* __restrict__ perm, int64_t pstride,
                                     const uint32_t* __restrict__ src,
                                     uint32_t* __restrict__ dst, int64_t outer, int64_t N,
@@ -286,6 +322,16 @@ sa_status launch_reorder(const int32_t* perm, const void* src, void* dst, int64_
   const bool aligned16 = ((uintptr_t)src % 16 == 0) && ((uintptr_t)dst % 16 == 0);
   if (row_bytes % 16 == 0 && aligned16) {
     const int64_t cpr = row_bytes / 16;
+    int shift = 0;
+    while (((int64_t)1 << shift) < cpr) ++shift;
+    if (((int64_t)1 << shift) == cpr && cpr <= 256 && outer <= 65535) {
+      constexpr int STEPS = 4;
+      const int64_t rows_per_cta = (256 >> shift) * STEPS;
+      dim3 grid((unsigned)ceil_div(N, rows_per_cta), (unsigned)outer);
+      reorder_rows_kernel<STEPS><<<grid, threads, 0, st>>>(perm, pstride, static_cast<const uint4*>(src),
+                                                            static_cast<uint4*>(dst), N, shift, scatter);
+      return check_launch("reorder_rows_kernel");
+    }
     const int64_t total = outer * N * cpr;
     constexpr int U = 4;
     reorder_vec_kernel<U><<<grid_for(ceil_div(total, U), threads), threads, 0, st>>>(

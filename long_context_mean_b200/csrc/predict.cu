@@ -20,141 +20,260 @@
 namespace sa {
 namespace {
 
-constexpr int kPoolThreads = 128;
+constexpr int kPoolThreads = 256;
 constexpr int kPoolWarps = kPoolThreads / 32;
+constexpr int kPoolStages = 3;   // blocks a CTA holds in shared memory: one in use, two arriving
+
+__device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_stages() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPoolStages - 1) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Two fp32 values in one 64-bit register for the packed fp32x2 pipe.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// A 16-byte vector of elements as fp32 pairs (8 bf16 -> 4 pairs, 4 fp32 -> 2).
+__device__ __forceinline__ void pairs16(const uint4& u, uint16_t, uint64_t* p) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+__device__ __forceinline__ void pairs16(const uint4& u, float, uint64_t* p) {
+  p[0] = f2(__uint_as_float(u.x), __uint_as_float(u.y));
+  p[1] = f2(__uint_as_float(u.z), __uint_as_float(u.w));
+}
 
 // ---------------------------------------------------------------------------
-// a2: one CTA per (head, block): block mean and mean pairwise cosine.  A warp
-// covers 32/chunks tokens per step (chunks = 16-byte pieces of a token),
-// four steps in flight; token norms reduce inside each token's lane group.
-// With perm, token n of the block is read from row perm[n] of x and also
-// written to row n of y (a1 fused with a2: the reordered copy is produced by
-// the same pass that pools it).  QF = 1 + SA_Q_INT8 or 1 + SA_Q_E4M3 (bf16
-// input): instead of the copy, the pass writes the block's 8-bit codes to
-// row n of y8 and its scale (absmax / 127 or / 448) to qscale, reading the
-// block a second time (from L2) once its absmax is known.
+// a2: block mean and mean pairwise cosine of every (head, block) unit.  A
+// persistent CTA takes units blockIdx.x, + gridDim.x, ... and streams their
+// tokens through a ring of kPoolStages blocks in shared memory with
+// cp.async, so two blocks are arriving while a third is reduced.  Thread i
+// owns chunk c = i % CH (CH = 16-byte pieces of a token) of tokens i / CH,
+// + 256 / CH, ...: it copies exactly the chunks it later reads, so the ring
+// needs no barrier of its own.  The arithmetic runs on fp32 pairs (packed
+// FMA/ADD), the token norm reduces inside the token's lane group and its
+// inverse is the hardware reciprocal square root; the block sums reduce
+// across lanes and warps.  With perm, token n of the block is read from row
+// perm[n] of x (an entry outside [0, N) raises SA_ERR_INVALID_ARG and the
+// token reads as zeros and is not written) and also written to row n of y
+// (a1 fused with a2: the reordered copy is produced by the same pass that
+// pools it).  The block mean goes to mean_out[(bh * nB + blk) * d + i], or
+// with mean_tstride > 0 to mean_out[(bh * d + i) * mean_tstride + blk]
+// (transposed: one row per feature, blocks contiguous).  QF = 1 + SA_Q_INT8
+// or 1 + SA_Q_E4M3 (bf16 input): instead of the copy, the pass writes the
+// block's 8-bit codes to row n of y8 and its scale (absmax / 127 or / 448)
+// to qscale, quantising from shared memory once the block's absmax is known.
+// Dynamic shared memory: ring [kPoolStages][b * CH] 16-byte chunks | block
+// sums [2][kPoolWarps][d] fp32 | token flags [kPoolStages][128].
 // ---------------------------------------------------------------------------
-template <typename T, int QF = 0>
+size_t pool_smem_bytes(int d, int b, int elem) {
+  return (size_t)kPoolStages * b * d * elem + (size_t)2 * kPoolWarps * d * 4 + (size_t)kPoolStages * 128;
+}
+
+template <typename T, int CH, int QF = 0>
 __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
-    const T* __restrict__ x, int64_t N, int d, int b, int nB, float* __restrict__ mean_out,
-    float* __restrict__ s_out, const int32_t* __restrict__ perm, T* __restrict__ y, int32_t* status,
-    uint2* __restrict__ y8 = nullptr, float* __restrict__ qscale = nullptr) {
-  constexpr int EPL = 16 / sizeof(T);
-  const int blk = blockIdx.x;
-  const int64_t bh = blockIdx.y;
-  const int64_t t0 = (int64_t)blk * b;
-  const int cnt = (int)min64(b, N - t0);
-  const int chunks = d / EPL;
-  const int tpw = 32 / chunks;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = lane / chunks, c = lane % chunks;
-  float ax[EPL], au[EPL];
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) ax[e] = au[e] = 0.f;
-  float amax = 0.f;                        // QF: block absmax
-  const uint4* xbh = reinterpret_cast<const uint4*>(x + bh * N * (int64_t)d);
-  uint4* ybh = y ? reinterpret_cast<uint4*>(y + bh * N * (int64_t)d) : nullptr;
-  const int step = kPoolWarps * tpw;
-  constexpr int kInFlight = 4;
-  for (int tb = warp * tpw; tb < cnt; tb += kInFlight * step) {
-    uint4 raw[kInFlight];
-    bool ok[kInFlight];
-#pragma unroll
-    for (int u = 0; u < kInFlight; ++u) {
-      const int tok = tb + u * step + sub;
-      const int64_t n = t0 + tok;
-      ok[u] = tok < cnt;
-      int64_t src = n;
-      if (perm && ok[u]) {
-        src = __ldg(perm + n);
-        if ((uint64_t)src >= (uint64_t)N) {   // not a permutation of [0, N)
-          raise_status(status, SA_ERR_INVALID_ARG);
-          ok[u] = false;
+    const T* __restrict__ x, int64_t BH, int64_t N, int b, int nB, float* __restrict__ mean_out,
+    int64_t mean_tstride, float* __restrict__ s_out, const int32_t* __restrict__ perm, T* __restrict__ y,
+    int32_t* status, uint2* __restrict__ y8 = nullptr, float* __restrict__ qscale = nullptr) {
+  constexpr int EPL = 16 / sizeof(T);   // elements per chunk
+  constexpr int NP = EPL / 2;           // fp32 pairs per chunk
+  constexpr int d = CH * EPL;
+  constexpr int TPP = kPoolThreads / CH;   // tokens per pass of the CTA
+  static_assert(CH >= 1 && CH <= 32 && (CH & (CH - 1)) == 0, "chunks per token: a power of two <= 32");
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint4* ring = reinterpret_cast<uint4*>(smem);
+  const int stage_chunks = b * CH;
+  float* sx = reinterpret_cast<float*>(ring + kPoolStages * stage_chunks);   // [kPoolWarps][d]
+  float* su = sx + kPoolWarps * d;
+  uint8_t* tok_ok = reinterpret_cast<uint8_t*>(su + kPoolWarps * d);        // [kPoolStages][128]
+  __shared__ float red[kPoolWarps];
+  __shared__ float wmax[kPoolWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int sub = tid / CH, c = tid % CH;
+  const int64_t units = BH * nB;
+
+  // Copies of this thread's chunks of unit `unit` into stage `st` (one
+  // commit group per call, empty past the last unit).
+  auto issue = [&](int64_t unit, int st) {
+    if (unit < units) {
+      const int64_t bh = unit / nB;
+      const int blk = (int)(unit - bh * nB);
+      const int64_t t0 = (int64_t)blk * b;
+      const int cnt = (int)min64(b, N - t0);
+      const uint4* xbh = reinterpret_cast<const uint4*>(x + bh * N * (int64_t)d) + c;
+      uint4* dst = ring + st * stage_chunks + c;
+      for (int tok = sub; tok < cnt; tok += TPP) {
+        const int64_t n = t0 + tok;
+        const int64_t src = perm ? (int64_t)__ldg(perm + n) : n;
+        const bool ok = (uint64_t)src < (uint64_t)N;
+        if (!ok) {   // not a permutation of [0, N)
+          if (c == 0) raise_status(status, SA_ERR_INVALID_ARG);
+          dst[tok * CH] = make_uint4(0, 0, 0, 0);
+        } else {
+          cp_async16((uint32_t)__cvta_generic_to_shared(dst + tok * CH), xbh + src * CH);
         }
+        if (c == 0) tok_ok[st * 128 + tok] = ok ? 1 : 0;
       }
-      raw[u] = ok[u] ? __ldg(xbh + src * chunks + c) : make_uint4(0, 0, 0, 0);
-      if (ybh && ok[u]) __stcs(ybh + n * chunks + c, raw[u]);
+    }
+    cp_async_commit();
+  };
+
+  int64_t unit = blockIdx.x;
+#pragma unroll 1
+  for (int j = 0; j < kPoolStages - 1; ++j) issue(unit + (int64_t)j * gridDim.x, j);
+#pragma unroll 1
+  for (int it = 0; unit < units; ++it, unit += gridDim.x) {
+    const int st = it % kPoolStages;
+    issue(unit + (int64_t)(kPoolStages - 1) * gridDim.x, (it + kPoolStages - 1) % kPoolStages);
+    cp_async_wait_stages();   // this thread's copies of `unit` have landed
+    __syncthreads();          // token flags of `unit` written by other threads
+    const int64_t bh = unit / nB;
+    const int blk = (int)(unit - bh * nB);
+    const int64_t t0 = (int64_t)blk * b;
+    const int cnt = (int)min64(b, N - t0);
+    const uint4* ring_st = ring + st * stage_chunks + c;
+    const uint8_t* ok_st = tok_ok + st * 128;
+    uint4* ybh = y ? reinterpret_cast<uint4*>(y + bh * N * (int64_t)d) + t0 * CH + c : nullptr;
+    // Every token of this thread at once: the smem reads, then the norms
+    // (independent shuffle chains), then the sums.  The token loops have a
+    // uniform trip count: the shuffles need every lane.
+    constexpr int MAXP = (128 + TPP - 1) / TPP;
+    uint4 raw[MAXP];
+#pragma unroll
+    for (int ip = 0; ip < MAXP; ++ip) {
+      const int tok = ip * TPP + sub;
+      raw[ip] = tok < cnt ? ring_st[tok * CH] : make_uint4(0, 0, 0, 0);
+    }
+    if (ybh) {
+#pragma unroll
+      for (int ip = 0; ip < MAXP; ++ip) {
+        const int tok = ip * TPP + sub;
+        if (tok < cnt && ok_st[tok]) __stcs(ybh + tok * CH, raw[ip]);
+      }
+    }
+    float ssum[MAXP];
+#pragma unroll
+    for (int ip = 0; ip < MAXP; ++ip) {
+      uint64_t v[NP];
+      pairs16(raw[ip], T(), v);
+      uint64_t s2 = f2(0.f, 0.f);
+#pragma unroll
+      for (int e = 0; e < NP; ++e) s2 = f2_fma(v[e], v[e], s2);
+      float s0, s1;
+      f2_split(s2, s0, s1);
+      ssum[ip] = s0 + s1;
     }
 #pragma unroll
-    for (int u = 0; u < kInFlight; ++u) {
-      float v[EPL];
-      unpack16(raw[u], T(), v);
-      float ss = 0.f;
+    for (int off = CH >> 1; off > 0; off >>= 1) {
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) ss = fmaf(v[e], v[e], ss);
-      for (int off = chunks >> 1; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-      const float inv = (ok[u] && ss > 0.f) ? 1.0f / sqrtf(ss) : 0.f;
+      for (int ip = 0; ip < MAXP; ++ip) ssum[ip] += __shfl_xor_sync(0xffffffffu, ssum[ip], off);
+    }
+    uint64_t ax[NP], au[NP];
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        ax[e] += v[e];
-        au[e] = fmaf(v[e], inv, au[e]);
+    for (int e = 0; e < NP; ++e) ax[e] = au[e] = f2(0.f, 0.f);
+    float amax = 0.f;
+#pragma unroll
+    for (int ip = 0; ip < MAXP; ++ip) {
+      uint64_t v[NP];
+      pairs16(raw[ip], T(), v);
+      const float inv = ssum[ip] > 0.f ? rsqrtf(ssum[ip]) : 0.f;
+      const uint64_t inv2 = f2(inv, inv);
+#pragma unroll
+      for (int e = 0; e < NP; ++e) {
+        ax[e] = f2_add(ax[e], v[e]);
+        au[e] = f2_fma(v[e], inv2, au[e]);
       }
       if constexpr (QF != 0) {
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) amax = fmaxf(amax, fabsf(v[e]));
+        for (int e = 0; e < NP; ++e) {
+          float lo, hi;
+          f2_split(v[e], lo, hi);
+          amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+        }
       }
     }
-  }
-  for (int off = chunks; off < 32; off <<= 1) {
+    float axs[EPL], aus[EPL];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      ax[e] += __shfl_xor_sync(0xffffffffu, ax[e], off);
-      au[e] += __shfl_xor_sync(0xffffffffu, au[e], off);
+    for (int e = 0; e < NP; ++e) {
+      f2_split(ax[e], axs[2 * e], axs[2 * e + 1]);
+      f2_split(au[e], aus[2 * e], aus[2 * e + 1]);
     }
-  }
-  __shared__ float sx[kPoolWarps][256];
-  __shared__ float su[kPoolWarps][256];
-  __shared__ float red[kPoolWarps];
-  if (lane < chunks) {
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      sx[warp][c * EPL + e] = ax[e];
-      su[warp][c * EPL + e] = au[e];
-    }
-  }
-  __syncthreads();
-  float part = 0.f;
-  for (int i = threadIdx.x; i < d; i += kPoolThreads) {
-    float X = 0.f, U = 0.f;
+    for (int off = CH; off < 32; off <<= 1) {
 #pragma unroll
-    for (int w = 0; w < kPoolWarps; ++w) {
-      X += sx[w][i];
-      U += su[w][i];
+      for (int e = 0; e < EPL; ++e) {
+        axs[e] += __shfl_xor_sync(0xffffffffu, axs[e], off);
+        aus[e] += __shfl_xor_sync(0xffffffffu, aus[e], off);
+      }
     }
-    mean_out[(bh * nB + blk) * (int64_t)d + i] = X / (float)cnt;
-    part = fmaf(U, U, part);
-  }
-  for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-  if (lane == 0) red[warp] = part;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float tot = 0.f;
-    for (int w = 0; w < kPoolWarps; ++w) tot += red[w];
-    s_out[bh * nB + blk] = tot / ((float)cnt * (float)cnt);
-  }
-  if constexpr (QF != 0) {
-    static_assert(sizeof(T) == 2, "8-bit codes are written from bf16 input");
-    constexpr int FMT = QF - 1;
-    __shared__ float wmax[kPoolWarps];
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (lane == 0) wmax[warp] = amax;
+    if (lane < CH) {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        sx[warp * d + c * EPL + e] = axs[e];
+        su[warp * d + c * EPL + e] = aus[e];
+      }
+    }
+    if constexpr (QF != 0) {
+      for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      if (lane == 0) wmax[warp] = amax;
+    }
     __syncthreads();
-    float A = 0.f;
+    float part = 0.f;
+    for (int i = tid; i < d; i += kPoolThreads) {
+      float X = 0.f, U = 0.f;
 #pragma unroll
-    for (int w = 0; w < kPoolWarps; ++w) A = fmaxf(A, wmax[w]);
-    const float qmax = FMT == SA_Q_E4M3 ? 448.0f : 127.0f;
-    const float qinv = A > 0.f ? __fdiv_rn(qmax, A) : 0.f;
-    if (threadIdx.x == 0) qscale[bh * nB + blk] = A > 0.f ? __fdiv_rn(A, qmax) : 0.f;
-    uint2* y8bh = y8 + bh * N * (int64_t)chunks;
-    for (int tb = warp * tpw; tb < cnt; tb += step) {
-      const int tok = tb + sub;
-      if (tok >= cnt) continue;
-      const int64_t n = t0 + tok;
-      const int64_t src = perm ? (int64_t)__ldg(perm + n) : n;
-      if ((uint64_t)src >= (uint64_t)N) continue;          // raised in the first pass
-      y8bh[n * chunks + c] = quant8<FMT>(__ldg(xbh + src * chunks + c), qinv);
+      for (int w = 0; w < kPoolWarps; ++w) {
+        X += sx[w * d + i];
+        U += su[w * d + i];
+      }
+      const float mv = X / (float)cnt;
+      if (mean_tstride > 0) mean_out[(bh * d + i) * mean_tstride + blk] = mv;
+      else mean_out[(bh * nB + blk) * (int64_t)d + i] = mv;
+      part = fmaf(U, U, part);
+    }
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (lane == 0) red[warp] = part;
+    if constexpr (QF != 0) {
+      static_assert(sizeof(T) == 2, "8-bit codes are written from bf16 input");
+      constexpr int FMT = QF - 1;
+      float A = 0.f;
+#pragma unroll
+      for (int w = 0; w < kPoolWarps; ++w) A = fmaxf(A, wmax[w]);
+      const float qmax = FMT == SA_Q_E4M3 ? 448.0f : 127.0f;
+      const float qinv = A > 0.f ? __fdiv_rn(qmax, A) : 0.f;
+      if (tid == 0) qscale[bh * nB + blk] = A > 0.f ? __fdiv_rn(A, qmax) : 0.f;
+      uint2* y8bh = y8 + (bh * N + t0) * (int64_t)CH + c;
+      for (int tok = sub; tok < cnt; tok += TPP)
+        if (ok_st[tok]) y8bh[tok * CH] = quant8<FMT>(ring_st[tok * CH], qinv);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      float tot = 0.f;
+      for (int w = 0; w < kPoolWarps; ++w) tot += red[w];
+      s_out[bh * nB + blk] = tot / ((float)cnt * (float)cnt);
     }
   }
+  cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -234,10 +353,11 @@ __device__ void finish_row(const uint8_t* flags, int64_t u, int64_t qb, int64_t 
 // ---------------------------------------------------------------------------
 // a3 + a4: one CTA per (head, group of G <= 8 query blocks).  Scores: thread
 // i takes the key blocks kb = i, i + 256, ... and computes q_hat[r] . k_hat[kb]
-// for every row r of the group, reading its k_hat row from global memory
-// (L2-resident, each element read once per group) and the q_hat rows from
-// shared memory (the same address in every lane: broadcast), so the loop is
-// bound by the FMA pipe.  Then warp r alone finishes row r: softmax and
+// for every row r of the group, reading k_hat (stored transposed, feature-
+// major, L2-resident, each element read once per group: a warp's load of a
+// feature is one 128-byte line) and the q_hat rows from shared memory (the
+// same address in every lane: broadcast, four features per load), so the
+// loop is bound by the FMA pipe.  Then warp r alone finishes row r: softmax and
 // TopCdf (an arg-max loop over register-resident keys when the row is short
 // and few blocks are picked, else a bisection for the last kept
 // probability), the union with the forced parts and the causal AND -- with
@@ -247,6 +367,7 @@ __device__ void finish_row(const uint8_t* flags, int64_t u, int64_t qb, int64_t 
 // padding holding zeros) | flags [G][nkb rounded to 16] (u8).
 // ---------------------------------------------------------------------------
 constexpr int kMaxRowsPerCta = 8;
+constexpr int kSelectRegs = 4;    // TopCdf: candidates a lane holds once at most 128 remain
 constexpr int kFastKeys = 16;     // keys per lane on the fast TopCdf path (nkb <= 512)
 constexpr int kFastPicks = 128;   // picks before the fast path defers to the sort
 
@@ -259,7 +380,8 @@ size_t score_smem_bytes(int d, int64_t nkb, int P2, int G) {
   (void)P2;
   const size_t nkb16 = (size_t)((nkb + 15) / 16) * 16;
   const size_t nkb4 = (size_t)((nkb + 3) / 4) * 4;
-  return (size_t)kMaxRowsPerCta * d * 4 + (size_t)G * nkb4 * 4 + (size_t)G * nkb16;
+  return (size_t)kMaxRowsPerCta * d * 4 + (size_t)G * nkb4 * 4 + (size_t)G * nkb16 +
+         (size_t)kMaxRowsPerCta * kSelectRegs * 32 * 4;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -278,7 +400,9 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   float* qs = reinterpret_cast<float*>(smem);
   float* sc = reinterpret_cast<float*>(smem + (size_t)kMaxRowsPerCta * d * 4);
   uint8_t* flags = reinterpret_cast<uint8_t*>(sc + G * nkb4);
+  float* cand = reinterpret_cast<float*>(flags + (size_t)G * nkb16);   // [8][kSelectRegs * 32]
   __shared__ int s_forced[kMaxRowsPerCta];
+  __shared__ int s_klim[kMaxRowsPerCta];   // last key block row r scores (-1: none)
 
   const int64_t bh = blockIdx.y;
   const int64_t qb0 = (int64_t)blockIdx.x * G;
@@ -293,6 +417,10 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
     const int r = threadIdx.x;
     const int64_t u = bh * nqb + qb0 + r;
     s_forced[r] = (r >= rows) ? 1 : ((rules.struct_row(qb0 + r) || (guard && sq[u] < theta)) ? 1 : 0);
+    // causal validity of kb for row qb is kb * bk <= last query row of qb
+    s_klim[r] = s_forced[r] ? -1
+                            : (rules.causal ? (int)((min64(rules.N, (qb0 + r + 1) * rules.bq) - 1) / rules.bk)
+                                            : (int)nkb - 1);
   }
   for (int i = threadIdx.x; i < rows * d; i += blockDim.x) qs[i] = qhat[(bh * nqb + qb0) * (int64_t)d + i];
   __syncthreads();
@@ -300,38 +428,46 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   for (int r = 0; r < rows; ++r) any_scored |= !s_forced[r];
 
   if (any_scored) {
-    const float4* kg4 = reinterpret_cast<const float4*>(khat + g * nkb * (int64_t)d);
+    // k_hat is stored transposed, [d][nkb4] per KV head: thread i takes key
+    // blocks kb = i, i + 256, ..., so a warp's loads of one feature are one
+    // 128-byte line.
+    const float* kT = khat + g * (int64_t)d * nkb4;
     const float4* qs4 = reinterpret_cast<const float4*>(qs);
     const int nf4 = d / 4;
-    for (int64_t kb = threadIdx.x; kb < nkb; kb += kRowThreads) {
-      uint32_t need = 0;   // rows of the group that score this key block
-      const bool col_ok = !(guard && sk[g * nkb + kb] < theta);
+    for (int kb = threadIdx.x; kb < nkb; kb += kRowThreads) {
+      uint32_t need = 0;   // bit r: row r of the group scores this key block
+      if (!(guard && sk[g * nkb + kb] < theta)) {
 #pragma unroll
-      for (int r = 0; r < kMaxRowsPerCta; ++r)
-        if (r < rows && col_ok && !s_forced[r] && rules.valid(qb0 + r, kb)) need |= 1u << r;
-      float a[kMaxRowsPerCta][4];
+        for (int r = 0; r < kMaxRowsPerCta; ++r)
+          if (kb <= s_klim[r]) need |= 1u << r;
+      }
+      // Row r's dot product as two packed partial sums: features (4e, 4e+1)
+      // and (4e+2, 4e+3) of each group of four.
+      uint64_t a[kMaxRowsPerCta];
 #pragma unroll
-      for (int r = 0; r < kMaxRowsPerCta; ++r) a[r][0] = a[r][1] = a[r][2] = a[r][3] = 0.f;
+      for (int r = 0; r < kMaxRowsPerCta; ++r) a[r] = f2(0.f, 0.f);
       if (need) {
-        const float4* kr = kg4 + kb * nf4;
-        for (int e = 0; e < nf4; ++e) {
-          const float4 y = __ldg(kr + e);
+        const float* kc = kT + kb;
+#pragma unroll 4
+        for (int e4 = 0; e4 < nf4; ++e4) {
+          const uint64_t k01 = f2(__ldg(kc + (int64_t)(4 * e4) * nkb4), __ldg(kc + (int64_t)(4 * e4 + 1) * nkb4));
+          const uint64_t k23 = f2(__ldg(kc + (int64_t)(4 * e4 + 2) * nkb4), __ldg(kc + (int64_t)(4 * e4 + 3) * nkb4));
 #pragma unroll
           for (int r = 0; r < kMaxRowsPerCta; ++r) {
-            if (r < rows) {
-              const float4 x = qs4[r * nf4 + e];
-              a[r][0] = fmaf(x.x, y.x, a[r][0]);
-              a[r][1] = fmaf(x.y, y.y, a[r][1]);
-              a[r][2] = fmaf(x.z, y.z, a[r][2]);
-              a[r][3] = fmaf(x.w, y.w, a[r][3]);
-            }
+            const float4 x = qs4[r * nf4 + e4];
+            a[r] = f2_fma(f2(x.x, x.y), k01, a[r]);
+            a[r] = f2_fma(f2(x.z, x.w), k23, a[r]);
           }
         }
       }
 #pragma unroll
-      for (int r = 0; r < kMaxRowsPerCta; ++r)
-        if (r < rows) sc[r * nkb4 + kb] = ((need >> r) & 1u) ? ((a[r][0] + a[r][1]) + (a[r][2] + a[r][3])) * scale
-                                                              : -INFINITY;
+      for (int r = 0; r < kMaxRowsPerCta; ++r) {
+        if (r < rows) {
+          float lo, hi;
+          f2_split(a[r], lo, hi);
+          sc[r * nkb4 + kb] = ((need >> r) & 1u) ? (lo + hi) * scale : -INFINITY;
+        }
+      }
     }
     __syncthreads();
   }
@@ -414,25 +550,79 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
       }
       __syncwarp();
       const float4* pr4 = reinterpret_cast<const float4*>(pr);
-      auto mass_above = [&](uint32_t t) -> float {
+      // Float4 groups that can hold a positive p: key blocks past the row's
+      // last valid one (causal) have p = 0.
+      const int nq_row = min(nkb4 / 4, (s_klim[r] + 4) / 4);
+      // f(t) and the number of p whose bits exceed t, over the whole row.
+      auto pass_full = [&](uint32_t t, int& count) -> float {
         float m0 = 0.f, m1 = 0.f;
-        for (int q = lane; q < nkb4 / 4; q += 32) {
+        int c = 0;
+        for (int q = lane; q < nq_row; q += 32) {
           const float4 v = pr4[q];
-          m0 += (__float_as_uint(v.x) > t ? v.x : 0.f) + (__float_as_uint(v.y) > t ? v.y : 0.f);
-          m1 += (__float_as_uint(v.z) > t ? v.z : 0.f) + (__float_as_uint(v.w) > t ? v.w : 0.f);
+          const bool g0 = __float_as_uint(v.x) > t, g1 = __float_as_uint(v.y) > t;
+          const bool g2 = __float_as_uint(v.z) > t, g3 = __float_as_uint(v.w) > t;
+          m0 += (g0 ? v.x : 0.f) + (g1 ? v.y : 0.f);
+          m1 += (g2 ? v.z : 0.f) + (g3 ? v.w : 0.f);
+          c += (int)g0 + (int)g1 + (int)g2 + (int)g3;
         }
         float m = m0 + m1;
         for (int off = 16; off > 0; off >>= 1) m += __shfl_xor_sync(0xffffffffu, m, off);
+        count = __reduce_add_sync(0xffffffffu, c);
         return m;
       };
-      const float limit = tau * mass_above(0u);
+      int c_lo = 0, c_hi = 0, c_mid = 0;   // how many p have bits above lo, hi
+      const float limit = tau * pass_full(0u, c_lo);
       uint32_t lo = 0u, hi = 0x3F800000u;   // f(lo) >= limit (tau <= 1), f(hi) = 0 < limit
-      while (hi - lo > 1u) {
+      float f_hi = 0.f;                     // f(hi)
+      while (hi - lo > 1u && c_lo - c_hi > kSelectRegs * 32) {
         const uint32_t mid = lo + (hi - lo) / 2u;
-        if (mass_above(mid) < limit) hi = mid;
-        else lo = mid;
+        const float m = pass_full(mid, c_mid);
+        if (m < limit) {
+          hi = mid;
+          f_hi = m;
+          c_hi = c_mid;
+        } else {
+          lo = mid;
+          c_lo = c_mid;
+        }
       }
-      const float above = mass_above(hi);
+      if (hi - lo > 1u) {
+        // At most kSelectRegs * 32 p lie in (lo, hi]: gather them (in block
+        // order) into the warp's buffer, then into registers, and finish the
+        // search there: f(t) = f(hi on entry) + the mass of the gathered p
+        // above t.
+        float* cbuf = cand + warp * kSelectRegs * 32;
+        int n = 0;
+        for (int kb0 = 0; kb0 < 4 * nq_row; kb0 += 32) {
+          const int kb = kb0 + lane;
+          const float v = kb < 4 * nq_row ? pr[kb] : 0.f;
+          const uint32_t bits = __float_as_uint(v);
+          const bool in = bits > lo && bits <= hi;
+          const unsigned bal = __ballot_sync(0xffffffffu, in);
+          if (in) cbuf[n + __popc(bal & ((1u << lane) - 1u))] = v;
+          n += __popc(bal);
+        }
+        __syncwarp();
+        float cv[kSelectRegs];
+#pragma unroll
+        for (int j = 0; j < kSelectRegs; ++j) cv[j] = lane + 32 * j < n ? cbuf[lane + 32 * j] : 0.f;
+        const float f_base = f_hi;   // f(hi) on entry: every gathered p is <= hi
+        while (hi - lo > 1u) {
+          const uint32_t mid = lo + (hi - lo) / 2u;
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < kSelectRegs; ++j) s += __float_as_uint(cv[j]) > mid ? cv[j] : 0.f;
+          for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+          const float m = f_base + s;
+          if (m < limit) {
+            hi = mid;
+            f_hi = m;
+          } else {
+            lo = mid;
+          }
+        }
+      }
+      const float above = f_hi;
       const float vstar = __uint_as_float(hi);
       uint32_t run = 0;
       for (int64_t kb0 = 0; kb0 < nkb; kb0 += 32) {
@@ -486,35 +676,58 @@ __global__ void __launch_bounds__(kRowThreads) mask_copy_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// CSR: one CTA scans the row counts into row_ptr and checks capacity.
+// CSR: one CTA scans the row counts into row_ptr and checks capacity.  The
+// counts are read kScanBatch chunks of 1024 at a time (coalesced, all loads
+// of a batch in flight together); each chunk is one block-wide scan (warp
+// shuffles, then one warp over the 32 warp totals) on top of the running
+// total of the chunks before it.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) rows_scan_kernel(const int32_t* __restrict__ counts,
-                                                         int64_t R, int64_t capacity,
-                                                         int32_t* __restrict__ row_ptr,
-                                                         int64_t* kept_total, int32_t* status) {
-  __shared__ int64_t part[1024];
-  const int64_t per = (R + blockDim.x - 1) / blockDim.x;
-  const int64_t beg = threadIdx.x * per, end = min(R, beg + per);
-  int64_t s = 0;
-  for (int64_t i = beg; i < end; ++i) s += counts[i];
-  part[threadIdx.x] = s;
-  __syncthreads();
-  for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-    const int64_t v = threadIdx.x >= (unsigned)off ? part[threadIdx.x - off] : 0;
-    __syncthreads();
-    part[threadIdx.x] += v;
-    __syncthreads();
+constexpr int kScanThreads = 1024;
+constexpr int kScanBatch = 8;
+
+__global__ void __launch_bounds__(kScanThreads) rows_scan_kernel(const int32_t* __restrict__ counts,
+                                                                 int64_t R, int64_t capacity,
+                                                                 int32_t* __restrict__ row_ptr,
+                                                                 int64_t* kept_total, int32_t* status) {
+  __shared__ int32_t wsum[kScanThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int64_t carry = 0;   // kept blocks of all rows before the current chunk
+  for (int64_t base = 0; base < R; base += (int64_t)kScanBatch * kScanThreads) {
+    int32_t v[kScanBatch];
+#pragma unroll
+    for (int j = 0; j < kScanBatch; ++j) {
+      const int64_t i = base + (int64_t)j * kScanThreads + tid;
+      v[j] = i < R ? counts[i] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kScanBatch; ++j) {
+      int32_t x = v[j];   // a chunk sums at most 1024 * 4095 blocks: int32 holds it
+      for (int off = 1; off < 32; off <<= 1) {
+        const int32_t o = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += o;
+      }
+      if (lane == 31) wsum[warp] = x;
+      __syncthreads();
+      if (warp == 0) {
+        int32_t y = wsum[lane];
+        for (int off = 1; off < 32; off <<= 1) {
+          const int32_t o = __shfl_up_sync(0xffffffffu, y, off);
+          if (lane >= off) y += o;
+        }
+        wsum[lane] = y;
+      }
+      __syncthreads();
+      const int64_t i = base + (int64_t)j * kScanThreads + tid;
+      const int64_t excl = carry + (warp > 0 ? wsum[warp - 1] : 0) + (x - v[j]);
+      if (i < R) row_ptr[i] = (int32_t)min64(excl, INT32_MAX);
+      carry += wsum[kScanThreads / 32 - 1];
+      __syncthreads();
+    }
   }
-  int64_t run = part[threadIdx.x] - s;
-  for (int64_t i = beg; i < end; ++i) {
-    row_ptr[i] = (int32_t)min64(run, INT32_MAX);
-    run += counts[i];
-  }
-  if (threadIdx.x == blockDim.x - 1) {
-    const int64_t tot = part[blockDim.x - 1];
-    row_ptr[R] = (int32_t)min64(tot, INT32_MAX);
-    *kept_total = tot;
-    if (tot > capacity || tot > INT32_MAX) raise_status(status, SA_ERR_CAPACITY);
+  if (tid == 0) {
+    row_ptr[R] = (int32_t)min64(carry, INT32_MAX);
+    *kept_total = carry;
+    if (carry > capacity || carry > INT32_MAX) raise_status(status, SA_ERR_CAPACITY);
   }
 }
 
@@ -538,46 +751,170 @@ __global__ void fill_cols_kernel(const uint8_t* __restrict__ mask, int64_t R, in
   }
 }
 
-// Work order: stable LSD radix sort of rows by key = 4095 - count (3 passes
-// of 4 bits), i.e. descending count, ties by ascending row index.  One CTA;
-// each thread owns a contiguous range of the current sequence and keeps its
-// 16 digit counts in a padded row of shared memory (stride 17: no bank
-// conflicts); the scatter offsets come from a scan in (digit, thread) order
-// done with warp shuffles, which keeps the scatter stable.  When the rows
-// fit (R <= kOrderSmemRows) the keys and the intermediate sequences live in
-// shared memory and only the final pass writes `order`.
+// The same for rows of a multiple of 16 blocks: a lane reads 16 flag bytes
+// at once (a warp covers 512 key blocks per load), and the lanes' kept
+// counts are placed by a warp exclusive scan.
+__global__ void fill_cols_vec_kernel(const uint8_t* __restrict__ mask, int64_t R, int64_t nkb,
+                                     const int32_t* __restrict__ row_ptr, int64_t capacity,
+                                     int32_t* __restrict__ col_idx) {
+  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= R) return;
+  const int64_t lo = row_ptr[warp];
+  const int64_t hi = row_ptr[warp + 1];
+  if (hi > capacity) return;  // capacity error already raised
+  const uint4* mrow = reinterpret_cast<const uint4*>(mask + warp * nkb);
+  const int64_t nv = nkb / 16;
+  int64_t pos = lo;
+  for (int64_t v0 = 0; v0 < nv; v0 += 32) {
+    const int64_t vi = v0 + lane;
+    const uint4 m = vi < nv ? __ldg(mrow + vi) : make_uint4(0, 0, 0, 0);
+    const uint32_t w[4] = {m.x, m.y, m.z, m.w};
+    uint32_t bits = 0;   // bit j: flag byte j of the 16 is set
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bits |= (((w[q] >> (8 * j)) & 0xFFu) != 0u ? 1u : 0u) << (4 * q + j);
+    const int c = __popc(bits);
+    int x = c;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += o;
+    }
+    int64_t p = pos + (x - c);
+    while (bits) {
+      const int j = __ffs(bits) - 1;
+      col_idx[p++] = (int32_t)(vi * 16 + j);
+      bits &= bits - 1u;
+    }
+    pos += __shfl_sync(0xffffffffu, x, 31);
+  }
+}
+
+// Work order: stable LSD radix sort of rows by key = 4095 - count, i.e.
+// descending count, ties by ascending row index.  One CTA.
+//
+// order_smem_kernel (R <= kOrderSmemRows): two passes of 6 bits, with the
+// keys and the intermediate sequence as 16-bit values in shared memory; only
+// the second pass writes `order`.  Warp w owns a contiguous range of the
+// current sequence and walks it 32 rows at a time: the lanes holding the same
+// digit find one another with a match, their leader adds the group's size to
+// the warp's count of that digit, and in the scatter each lane's slot is the
+// warp's running offset of its digit plus its rank among the lower lanes of
+// its group.  The offsets of entry (digit, warp) are every entry of smaller
+// digits plus the same digit's entries of smaller warps, so every pass is
+// stable.  With order_group = g > 0 one CTA sorts each group of g * nqb rows
+// (at most kOrderSmemRows).  order_kernel (one global order of more rows):
+// per-thread histograms and three passes of 4 bits through `tmp` and `order`
+// in global memory.
+constexpr int kOrderSmemRows = 32768;
+constexpr int kOrderSmemThreads = 1024;
+constexpr int kOrderSmemWarps = kOrderSmemThreads / 32;
+constexpr int kWhistStride = 65;   // a warp's 64 digit counts, padded
+
+size_t order_smem_bytes(int64_t R) {
+  return (size_t)kOrderSmemWarps * kWhistStride * 4 + (size_t)R * 2 * 2;
+}
+
+__global__ void __launch_bounds__(kOrderSmemThreads) order_smem_kernel(const int32_t* __restrict__ counts,
+                                                                       int64_t R, int64_t seg_rows,
+                                                                       int32_t* __restrict__ order) {
+  extern __shared__ uint32_t dyn[];
+  uint32_t* whist = dyn;                                                       // [warps][65]
+  uint16_t* skey = reinterpret_cast<uint16_t*>(dyn + kOrderSmemWarps * kWhistStride);   // [seg_rows]
+  uint16_t* seq = skey + seg_rows;                                             // [seg_rows] after pass 0
+  __shared__ uint32_t wsum[kOrderSmemWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // this CTA's segment: rows [base, base + n)
+  const int64_t base = (int64_t)blockIdx.x * seg_rows;
+  const int n = (int)min64(seg_rows, R - base);
+  counts += base;
+  order += base;
+  const int per = (n + kOrderSmemWarps - 1) / kOrderSmemWarps;
+  const int beg = min(n, warp * per), end = min(n, beg + per);
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t* wh = whist + warp * kWhistStride;
+  for (int i = tid; i < n; i += kOrderSmemThreads) skey[i] = (uint16_t)(4095u - (uint32_t)counts[i]);
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = 6 * pass;
+    wh[lane] = 0;
+    wh[lane + 32] = 0;
+    __syncthreads();   // keys (pass 0) or the sequence (pass 1) are complete
+    for (int i0 = beg; i0 < end; i0 += 32) {
+      const int i = i0 + lane;
+      const bool valid = i < end;
+      const int row = valid ? (pass == 0 ? i : (int)seq[i]) : 0;
+      const uint32_t dgt = valid ? ((uint32_t)skey[row] >> shift) & 63u : 64u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
+      if (valid && (peers & lt) == 0u) wh[dgt] += __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+    // Exclusive scan in (digit, warp) order: thread t holds entries 2t, 2t + 1.
+    {
+      const int e0 = 2 * tid, e1 = e0 + 1;
+      uint32_t* c0 = whist + (e0 & 31) * kWhistStride + (e0 >> 5);
+      uint32_t* c1 = whist + (e1 & 31) * kWhistStride + (e1 >> 5);
+      const uint32_t a = *c0, b = *c1;
+      uint32_t x = a + b;
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += o;
+      }
+      if (lane == 31) wsum[warp] = x;
+      __syncthreads();
+      if (warp == 0) {
+        uint32_t y = wsum[lane];
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t o = __shfl_up_sync(0xffffffffu, y, off);
+          if (lane >= off) y += o;
+        }
+        wsum[lane] = y;
+      }
+      __syncthreads();
+      const uint32_t ex = (warp > 0 ? wsum[warp - 1] : 0u) + x - (a + b);
+      *c0 = ex;
+      *c1 = ex + a;
+    }
+    __syncthreads();
+    for (int i0 = beg; i0 < end; i0 += 32) {
+      const int i = i0 + lane;
+      const bool valid = i < end;
+      const int row = valid ? (pass == 0 ? i : (int)seq[i]) : 0;
+      const uint32_t dgt = valid ? ((uint32_t)skey[row] >> shift) & 63u : 64u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
+      if (valid) {
+        const uint32_t slot = wh[dgt] + __popc(peers & lt);
+        if (pass == 0) seq[slot] = (uint16_t)row;
+        else order[slot] = (int32_t)(base + row);
+      }
+      __syncwarp();
+      if (valid && (peers & lt) == 0u) wh[dgt] += __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+  }
+}
+
 constexpr int kOrderThreads = 1024;
 constexpr int kOrderWarps = kOrderThreads / 32;
-constexpr int kOrderSmemRows = 8192;
-constexpr int kHistStride = 17;
+constexpr int kHistStride = 17;   // a thread's 16 digit counts, padded
 
 __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __restrict__ counts,
                                                               int64_t R, int32_t* __restrict__ tmp,
                                                               int32_t* __restrict__ order) {
-  extern __shared__ uint32_t dyn[];
-  uint32_t* hist = dyn;                                   // [kOrderThreads][17]
-  const bool in_smem = R <= kOrderSmemRows;
-  uint16_t* skey = reinterpret_cast<uint16_t*>(dyn + kHistStride * kOrderThreads);   // [R] key of row
-  int32_t* sa = reinterpret_cast<int32_t*>(skey + (in_smem ? kOrderSmemRows : 0));   // [R] sequences
-  int32_t* sb = sa + (in_smem ? kOrderSmemRows : 0);
+  extern __shared__ uint32_t hist[];                      // [thread][17]: 16 digits, padded
   __shared__ uint32_t wtot[kOrderWarps][16];              // per-warp digit totals, then warp offsets
   __shared__ uint32_t dtot[16];                           // digit totals
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t* my = hist + tid * kHistStride;
   const int64_t per = (R + kOrderThreads - 1) / kOrderThreads;
   const int64_t beg = tid * per, end = min(R, beg + per);
-  if (in_smem) {
-    for (int64_t i = tid; i < R; i += kOrderThreads) skey[i] = (uint16_t)(4095u - (uint32_t)counts[i]);
-    __syncthreads();
-  }
-  auto key_of = [&](int32_t row) -> uint32_t {
-    return in_smem ? (uint32_t)skey[row] : 4095u - (uint32_t)counts[row];
-  };
+  auto key_of = [&](int32_t row) -> uint32_t { return 4095u - (uint32_t)counts[row]; };
   for (int pass = 0; pass < 3; ++pass) {
-    // source and destination of this pass: rows in natural order first, the
-    // final pass writes `order`
-    const int32_t* src = pass == 0 ? nullptr : (in_smem ? (pass == 1 ? sa : sb) : (pass == 1 ? order : tmp));
-    int32_t* dst = pass == 2 ? order : (in_smem ? (pass == 0 ? sa : sb) : (pass == 0 ? order : tmp));
+    // rows in natural order first; pass 0 writes order, pass 1 tmp, pass 2 order
+    const int32_t* src = pass == 0 ? nullptr : (pass == 1 ? order : tmp);
+    int32_t* dst = pass == 1 ? tmp : order;
     const int shift = 4 * pass;
 #pragma unroll
     for (int dgt = 0; dgt < 16; ++dgt) my[dgt] = 0;
@@ -585,8 +922,6 @@ __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __r
       const int32_t row = src ? src[i] : (int32_t)i;
       my[(key_of(row) >> shift) & 15u] += 1;
     }
-    // Offsets: entry (digit, thread) starts after every entry of smaller
-    // digits and after the same digit's entries of smaller threads.
     uint32_t c[16], x[16];
 #pragma unroll
     for (int dgt = 0; dgt < 16; ++dgt) x[dgt] = c[dgt] = my[dgt];
@@ -629,20 +964,36 @@ __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __r
   }
 }
 
-sa_status launch_lists(const sa_shape& s, int bq, int bk, int32_t* counts, int32_t* tmp,
+sa_status launch_lists(const sa_shape& s, int bq, int bk, int order_group, int32_t* counts, int32_t* tmp,
                        sa_mask& out, cudaStream_t st) {
   const int64_t R = s.B * s.Hq * out.nqb;
   rows_scan_kernel<<<1, 1024, 0, st>>>(counts, R, out.col_capacity, out.row_ptr, out.kept_total,
                                        out.status);
   if (sa_status e = check_launch("rows_scan_kernel")) return e;
   const int64_t warps_per_block = 8;
-  fill_cols_kernel<<<(unsigned)ceil_div(R, warps_per_block), 32 * warps_per_block, 0, st>>>(
-      out.block_mask, R, out.nkb, out.row_ptr, out.col_capacity, out.col_idx);
+  const unsigned fill_grid = (unsigned)ceil_div(R, warps_per_block);
+  if (out.nkb % 16 == 0 && reinterpret_cast<uintptr_t>(out.block_mask) % 16 == 0)
+    fill_cols_vec_kernel<<<fill_grid, 32 * warps_per_block, 0, st>>>(out.block_mask, R, out.nkb, out.row_ptr,
+                                                                      out.col_capacity, out.col_idx);
+  else
+    fill_cols_kernel<<<fill_grid, 32 * warps_per_block, 0, st>>>(out.block_mask, R, out.nkb, out.row_ptr,
+                                                                  out.col_capacity, out.col_idx);
   if (sa_status e = check_launch("fill_cols_kernel")) return e;
-  size_t hist_bytes = (size_t)kHistStride * kOrderThreads * sizeof(uint32_t);
-  if (R <= kOrderSmemRows) hist_bytes += (size_t)kOrderSmemRows * (2 + 4 + 4);   // keys + two sequences
-  if (cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)hist_bytes) != cudaSuccess)
+  // Work order: one sort over all rows, or one per group of order_group heads.
+  const int64_t seg = order_group > 0 ? min64(R, (int64_t)order_group * out.nqb) : R;
+  const int64_t nseg = ceil_div(R, seg);
+  if (seg <= kOrderSmemRows) {
+    const size_t smem = order_smem_bytes(seg);
+    if (cudaFuncSetAttribute(order_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(order_smem_kernel) failed");
+    order_smem_kernel<<<(unsigned)nseg, kOrderSmemThreads, smem, st>>>(counts, R, seg, out.order);
+    return check_launch("order_smem_kernel");
+  }
+  if (nseg != 1) return set_error(SA_ERR_UNSUPPORTED, "order_group * nqb must be <= %d", kOrderSmemRows);
+  const size_t hist_bytes = (size_t)kHistStride * kOrderThreads * sizeof(uint32_t);
+  if (cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_bytes) !=
+      cudaSuccess)
     return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(order_kernel) failed");
   order_kernel<<<1, kOrderThreads, hist_bytes, st>>>(counts, R, tmp, out.order);
   return check_launch("order_kernel");
@@ -661,29 +1012,62 @@ RowRules make_rules(const sa_shape& s, const sa_mask_params& p) {
   return r;
 }
 
-template <typename T>
-sa_status launch_pool(const void* x, int64_t BH, int64_t N, int d, int b, int64_t nB, float* mean,
-                      float* sim, const int32_t* perm, void* y, int32_t* status, cudaStream_t st) {
-  dim3 grid((unsigned)nB, (unsigned)BH);
-  pool_cossim_kernel<T><<<grid, kPoolThreads, 0, st>>>(static_cast<const T*>(x), N, d, b, (int)nB,
-                                                       mean, sim, perm, static_cast<T*>(y), status);
+// Persistent grid: as many CTAs as fit on the device at once (at most one
+// per unit).
+template <typename K>
+sa_status pool_grid(K kernel, size_t smem, int64_t units, unsigned* grid) {
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(pool_cossim_kernel) failed");
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kPoolThreads, smem) != cudaSuccess ||
+      per_sm < 1)
+    return set_error(SA_ERR_CUDA, "pool_cossim_kernel does not fit on the device");
+  *grid = (unsigned)min64(units, (int64_t)sms * per_sm);
+  return SA_OK;
+}
+
+template <typename T, int CH, int QF>
+sa_status launch_pool_ch(const void* x, int64_t BH, int64_t N, int b, int64_t nB, float* mean,
+                         int64_t mean_tstride, float* sim, const int32_t* perm, void* y, int32_t* status,
+                         uint2* y8, float* qscale, cudaStream_t st) {
+  const size_t smem = pool_smem_bytes(CH * (16 / (int)sizeof(T)), b, (int)sizeof(T));
+  unsigned grid = 0;
+  if (sa_status e = pool_grid(pool_cossim_kernel<T, CH, QF>, smem, BH * nB, &grid)) return e;
+  pool_cossim_kernel<T, CH, QF><<<grid, kPoolThreads, smem, st>>>(static_cast<const T*>(x), BH, N, b, (int)nB,
+                                                                  mean, mean_tstride, sim, perm, static_cast<T*>(y),
+                                                                  status, y8, qscale);
   return check_launch("pool_cossim_kernel");
 }
 
-// Pooling with 8-bit codes and block scales instead of the reordered copy.
+template <typename T>
+sa_status launch_pool(const void* x, int64_t BH, int64_t N, int d, int b, int64_t nB, float* mean,
+                      int64_t mean_tstride, float* sim, const int32_t* perm, void* y, int32_t* status,
+                      cudaStream_t st) {
+  switch (d / (16 / (int)sizeof(T))) {   // 16-byte chunks per token (validated: a power of two <= 32)
+    case 1: return launch_pool_ch<T, 1, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
+    case 2: return launch_pool_ch<T, 2, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
+    case 4: return launch_pool_ch<T, 4, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
+    case 8: return launch_pool_ch<T, 8, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
+    case 16: return launch_pool_ch<T, 16, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
+    case 32: return launch_pool_ch<T, 32, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
+    default: return set_error(SA_ERR_UNSUPPORTED, "pooling: d must give a power-of-two count <= 32 of 16-byte chunks");
+  }
+}
+
+// Pooling with 8-bit codes and block scales instead of the reordered copy
+// (bf16, d = 128: 16 chunks).
 sa_status launch_pool_codes(const void* x, int64_t BH, int64_t N, int d, int b, int64_t nB, float* mean,
-                            float* sim, const int32_t* perm, int32_t fmt, void* y8, float* qscale, int32_t* status,
-                            cudaStream_t st) {
-  dim3 grid((unsigned)nB, (unsigned)BH);
+                            int64_t mean_tstride, float* sim, const int32_t* perm, int32_t fmt, void* y8,
+                            float* qscale, int32_t* status, cudaStream_t st) {
+  if (d != 128) return set_error(SA_ERR_UNSUPPORTED, "8-bit codes need d = 128");
   if (fmt == SA_Q_E4M3)
-    pool_cossim_kernel<uint16_t, 1 + SA_Q_E4M3><<<grid, kPoolThreads, 0, st>>>(
-        static_cast<const uint16_t*>(x), N, d, b, (int)nB, mean, sim, perm, nullptr, status,
-        static_cast<uint2*>(y8), qscale);
-  else
-    pool_cossim_kernel<uint16_t, 1 + SA_Q_INT8><<<grid, kPoolThreads, 0, st>>>(
-        static_cast<const uint16_t*>(x), N, d, b, (int)nB, mean, sim, perm, nullptr, status,
-        static_cast<uint2*>(y8), qscale);
-  return check_launch("pool_cossim_kernel");
+    return launch_pool_ch<uint16_t, 16, 1 + SA_Q_E4M3>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, nullptr,
+                                                        status, static_cast<uint2*>(y8), qscale, st);
+  return launch_pool_ch<uint16_t, 16, 1 + SA_Q_INT8>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, nullptr,
+                                                      status, static_cast<uint2*>(y8), qscale, st);
 }
 
 }  // namespace
@@ -692,7 +1076,8 @@ size_t predict_ws_bytes(const sa_shape& s, int bq, int bk, size_t off[6]) {
   const int64_t nqb = ceil_div(s.N, bq), nkb = ceil_div(s.N, bk);
   const int64_t R = s.B * s.Hq * nqb;
   size_t o = 0;
-  const size_t sizes[6] = {(size_t)(s.B * s.Hq * nqb * s.d) * 4, (size_t)(s.B * s.Hkv * nkb * s.d) * 4,
+  const int64_t nkb4 = (nkb + 3) / 4 * 4;
+  const size_t sizes[6] = {(size_t)(s.B * s.Hq * nqb * s.d) * 4, (size_t)(s.B * s.Hkv * nkb4 * s.d) * 4,
                            (size_t)(s.B * s.Hq * nqb) * 4,      (size_t)(s.B * s.Hkv * nkb) * 4,
                            (size_t)R * 4,                        (size_t)R * 4};
   for (int i = 0; i < 6; ++i) {
@@ -725,28 +1110,29 @@ sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
                          const sa_mask_params& p, const PredictWs& w, sa_mask& out,
                          cudaStream_t st, const int32_t* perm, void* q_r, void* k_r, const PoolCodes* codes) {
   const int64_t nqb = out.nqb, nkb = out.nkb;
+  const int64_t nkb4 = (nkb + 3) / 4 * 4;   // row stride of the transposed k_hat
   if (cudaMemsetAsync(out.status, 0, sizeof(int32_t), st) != cudaSuccess)
     return set_error(SA_ERR_CUDA, "cudaMemsetAsync(status) failed");
   sa_status e;
   if (codes) {   // bf16 input: codes and scales instead of reordered copies
-    if ((e = launch_pool_codes(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, perm, codes->format,
+    if ((e = launch_pool_codes(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, 0, w.sq, perm, codes->format,
                                codes->q8, codes->q_scales, out.status, st)))
       return e;
-    if ((e = launch_pool_codes(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, w.sk, perm, codes->format,
+    if ((e = launch_pool_codes(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, nkb4, w.sk, perm, codes->format,
                                codes->k8, codes->k_scales, out.status, st)))
       return e;
   } else if (s.dtype == SA_BF16) {
-    if ((e = launch_pool<uint16_t>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, perm, q_r,
+    if ((e = launch_pool<uint16_t>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, 0, w.sq, perm, q_r,
                                    out.status, st)))
       return e;
-    if ((e = launch_pool<uint16_t>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, w.sk, perm, k_r,
+    if ((e = launch_pool<uint16_t>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, nkb4, w.sk, perm, k_r,
                                    out.status, st)))
       return e;
   } else {
-    if ((e = launch_pool<float>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, w.sq, perm, q_r,
+    if ((e = launch_pool<float>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, 0, w.sq, perm, q_r,
                                 out.status, st)))
       return e;
-    if ((e = launch_pool<float>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, w.sk, perm, k_r,
+    if ((e = launch_pool<float>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, nkb4, w.sk, perm, k_r,
                                 out.status, st)))
       return e;
   }
@@ -764,7 +1150,7 @@ sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
       w.qhat, w.khat, w.sq, w.sk, s.Hq, s.Hkv, nqb, nkb, (int)s.d, P2, G, p.tau, p.theta,
       make_rules(s, p), out.block_mask, w.counts, out.status);
   if ((e = check_launch("score_topcdf_kernel"))) return e;
-  return launch_lists(s, p.bq, p.bk, w.counts, w.tmp, out, st);
+  return launch_lists(s, p.bq, p.bk, p.order_group, w.counts, w.tmp, out, st);
 }
 
 sa_status launch_mask_from_blocks(const uint8_t* in, const sa_shape& s, int bq, int bk, int causal,
@@ -785,7 +1171,7 @@ sa_status launch_mask_from_blocks(const uint8_t* in, const sa_shape& s, int bq, 
   mask_copy_kernel<<<(unsigned)R, kRowThreads, smem, st>>>(in, out.nqb, out.nkb, make_rules(s, p),
                                                           out.block_mask, counts, out.status);
   if (sa_status e = check_launch("mask_copy_kernel")) return e;
-  return launch_lists(s, bq, bk, counts, tmp, out, st);
+  return launch_lists(s, bq, bk, 0, counts, tmp, out, st);
 }
 
 }  // namespace sa

@@ -104,7 +104,7 @@ sa_status launch_reorder(const int32_t* perm, const void* src, void* dst, int64_
 
 struct PredictWs {
   float* qhat;     // [B*Hq, nqb, d]
-  float* khat;     // [B*Hkv, nkb, d]
+  float* khat;     // [B*Hkv, d, nkb4] (transposed; nkb4 = nkb rounded up to 4)
   float* sq;       // [B*Hq, nqb]
   float* sk;       // [B*Hkv, nkb]
   int32_t* counts; // [B*Hq*nqb]

@@ -32,7 +32,8 @@ STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3:
 
 EXPORTS = ["sa_version", "sa_last_error", "sa_attn_kernel_path", "sa_attn_workspace", "sa_layout_workspace",
            "sa_layout_build", "sa_reorder", "sa_unreorder", "sa_predict_mask_workspace",
-           "sa_predict_mask_ws_layout", "sa_predict_mask", "sa_reorder_predict_mask", "sa_predict_mask_noalloc",
+           "sa_predict_mask_ws_layout", "sa_order_group_hint", "sa_predict_mask", "sa_reorder_predict_mask",
+           "sa_predict_mask_noalloc",
            "sa_mask_from_blocks_workspace",
            "sa_mask_from_blocks", "sa_block_sparse_attn", "sa_dense_attn", "sa_read_status", "sa_l1_error",
            "sa_head_placement", "sa_reorder_heads", "sa_rows_attn", "sa_rows_mse",
@@ -63,7 +64,7 @@ class MaskParams(ctypes.Structure):
                 ("theta", ctypes.c_float), ("sink_tokens", ctypes.c_int64),
                 ("txt_len", ctypes.c_int64), ("local_window", ctypes.c_int64),
                 ("anchor_tokens", ctypes.c_int64), ("causal", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("order_group", ctypes.c_int32)]
 
 
 class Mask(ctypes.Structure):
@@ -99,6 +100,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sa_predict_mask_workspace": (SZ, [ctypes.POINTER(Shape), ctypes.POINTER(MaskParams)]),
         "sa_predict_mask_ws_layout": (I32, [ctypes.POINTER(Shape), ctypes.POINTER(MaskParams),
                                             ctypes.POINTER(SZ * 6)]),
+        "sa_order_group_hint": (I32, [ctypes.POINTER(Shape)]),
         "sa_predict_mask": (I32, [P, P, ctypes.POINTER(Shape), ctypes.POINTER(MaskParams), P, SZ,
                                   ctypes.POINTER(Mask), P]),
         "sa_reorder_predict_mask": (I32, [P, P, P, P, P, ctypes.POINTER(Shape), ctypes.POINTER(MaskParams), P,
@@ -172,9 +174,9 @@ def make_layout(T, H, W, txt_len=0, sink_frames=0, mode="identity", win=(1, 1, 1
 
 
 def make_params(bq, bk, tau, theta=0.0, sink_tokens=0, txt_len=0, local_window=0,
-                anchor_tokens=0, causal=False) -> MaskParams:
+                anchor_tokens=0, causal=False, order_group=0) -> MaskParams:
     return MaskParams(int(bq), int(bk), float(tau), float(theta), int(sink_tokens), int(txt_len),
-                      int(local_window), int(anchor_tokens), int(bool(causal)), 0)
+                      int(local_window), int(anchor_tokens), int(bool(causal)), int(order_group))
 
 
 # ---------------------------------------------------------------------------
@@ -221,6 +223,14 @@ def predict_mask_ws_layout(shape: Shape, params: MaskParams):
     off = (ctypes.c_size_t * 6)()
     _check(load().sa_predict_mask_ws_layout(ctypes.byref(shape), ctypes.byref(params), ctypes.byref(off)))
     return list(off)
+
+
+def order_group_hint(shape: Shape) -> int:
+    """The library's work-order grouping for a shape (MaskParams.order_group)."""
+    g = int(load().sa_order_group_hint(ctypes.byref(shape)))
+    if g < 0:
+        raise SAError(SA_ERR_INVALID_ARG, "sa_order_group_hint: invalid shape")
+    return g
 
 
 def predict_mask(q, k, shape: Shape, params: MaskParams, ws, mask: Mask, stream=None):
@@ -584,7 +594,8 @@ def host_pipeline_for(w, device="cuda", chunks=4, **kw) -> HostPipeline:
 def pipeline_for(w, device="cuda", **kw) -> Pipeline:
     """Pipeline for a workload description from ``inputs.WORKLOADS``."""
     lay = make_layout(w.T, w.H, w.W, w.txt_len, w.sink_frames, w.order, w.win)
+    shape = Shape(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, SA_BF16 if w.dtype == "bf16" else SA_FP32, 0)
     prm = make_params(w.bq, w.bk, w.tau, w.theta, w.sink_tokens, w.txt_len, w.local_window,
-                      w.anchor_tokens, w.causal)
+                      w.anchor_tokens, w.causal, order_group_hint(shape))
     return Pipeline(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, w.dtype, layout=lay, params=prm, lam=w.lam,
                     device=device, **kw)

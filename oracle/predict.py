@@ -19,7 +19,8 @@ Pipeline ([P3] section 2.2, with [P2] rf_v2 / ada_bsa and [P5] anchors):
      block-level local window keeps every block pair holding some (i, j)
      with 0 <= i - j < w; everything is then ANDed with causal validity.
   6. CSR lists (column indices ascending) and a work order (rows by
-     descending kept count, ties by ascending row index).
+     descending kept count, ties by ascending row index, optionally inside
+     groups of consecutive heads: a scheduling choice of this library).
 
 Readings where the pages are silent or garbled:
   * CosSim: the notes print mean(X X^T / |max(X X^T)|) while naming it a
@@ -232,20 +233,24 @@ def empty_rows(mask, n, bq, bk, causal):
     return bad
 
 
-def mask_to_csr(mask):
+def mask_to_csr(mask, order_group=0):
     """CSR form of a block mask [..., nQB, nKB] flattened over its leading axes
     in row-major order: row_ptr [R+1], col_idx ascending within a row, the
-    work order (rows by descending count, ties by ascending row index), and
-    the kept total."""
+    work order, and the kept total.  The work order (a scheduling choice of
+    this library, not the pages'): rows by descending count, ties by
+    ascending row index; with order_group = g > 0, the rows first form groups
+    of g consecutive heads (g * nQB rows each, the groups in order) and that
+    order applies inside each group."""
     mask = np.asarray(mask, dtype=bool)
-    nkb = mask.shape[-1]
+    nqb, nkb = mask.shape[-2], mask.shape[-1]
     flat = mask.reshape(-1, nkb)
     counts = flat.sum(axis=1).astype(np.int64)
     row_ptr = np.zeros(flat.shape[0] + 1, dtype=np.int64)
     row_ptr[1:] = np.cumsum(counts)
     col_idx = np.concatenate([np.flatnonzero(r) for r in flat]) if flat.size else np.zeros(0, np.int64)
     rows = np.arange(flat.shape[0])
-    order = np.lexsort((rows, -counts))
+    group = rows // (order_group * nqb) if order_group > 0 else np.zeros_like(rows)
+    order = np.lexsort((rows, -counts, group))
     return {"row_ptr": row_ptr, "col_idx": col_idx.astype(np.int64), "order": order,
             "counts": counts, "kept_total": int(counts.sum())}
 

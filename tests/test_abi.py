@@ -217,6 +217,22 @@ def test_workspace_queries_are_host_only(lib):
     assert sa.layout_workspace(sa.make_layout(13, 30, 52, 226, 1, "window", (2, 8, 8))) == 0
 
 
+def test_order_group_hint_and_check(lib):
+    # K and V of one KV head under 32 MiB: one global order (image, video)
+    assert sa.order_group_hint(_shape(B=2, Hq=24, Hkv=24, N=4096)) == 0
+    assert sa.order_group_hint(_shape(Hq=24, Hkv=24, N=20506)) == 0
+    # 38.7 MB per head: two heads (77 MB) fit in 96 MiB, four do not
+    assert sa.order_group_hint(_shape(Hq=24, Hkv=24, N=75600)) == 2
+    # GQA 32/8 at 131072: one KV head (67 MB) serves 4 query heads
+    assert sa.order_group_hint(_shape(Hq=32, Hkv=8, N=131072)) == 4
+    assert lib.sa_order_group_hint(ctypes.byref(_shape(Hq=3, Hkv=2))) == -1
+    p = sa.make_params(128, 64, 0.5, order_group=-1)
+    s, m, null = _shape(), _mask(), ctypes.c_void_p(None)
+    assert lib.sa_predict_mask(FAKE, FAKE, ctypes.byref(s), ctypes.byref(p), FAKE, 1 << 30,
+                               ctypes.byref(m), null) == sa.SA_ERR_INVALID_ARG
+    assert b"order_group" in lib.sa_last_error()
+
+
 def test_kernel_path_selection(lib):
     s = _shape()
     assert sa.attn_kernel_path(s, 128, 64, sa.SA_FLAG_FORCE_SIMT) == 0

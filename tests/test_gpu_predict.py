@@ -35,7 +35,7 @@ def run_gpu_predict(q_dev, k_dev, w, params, capacity=None):
     out = {
         "status": status,
         "qhat": view(0, B * Hq * nqb * d).reshape(B, Hq, nqb, d),
-        "khat": view(1, B * Hkv * nkb * d).reshape(B, Hkv, nkb, d),
+        "khat": khat_from_ws(ws, off, B, Hkv, nkb, d),
         "s_q": view(2, B * Hq * nqb).reshape(B, Hq, nqb),
         "s_k": view(3, B * Hkv * nkb).reshape(B, Hkv, nkb),
         "mask": mb.block_mask.cpu().numpy().reshape(B, Hq, nqb, nkb).astype(bool),
@@ -47,13 +47,21 @@ def run_gpu_predict(q_dev, k_dev, w, params, capacity=None):
     return out
 
 
+def khat_from_ws(ws, off, B, Hkv, nkb, d):
+    """k_hat from the prediction workspace, stored feature-major [B*Hkv, d, nkb4]."""
+    import torch
+    nkb4 = (nkb + 3) // 4 * 4
+    kt = ws[off[1]:off[1] + B * Hkv * d * nkb4 * 4].view(torch.float32).cpu().numpy()
+    return np.ascontiguousarray(kt.reshape(B, Hkv, d, nkb4)[..., :nkb].swapaxes(-1, -2))
+
+
 def oracle_predict(q, k, w):
     return Pr.predict_mask(q, k, w.bq, w.bk, w.tau, w.theta, w.causal, w.sink_tokens, w.txt_len,
                            w.local_window, w.anchor_tokens)
 
 
-def check_lists(g, mask):
-    c = Pr.mask_to_csr(mask)
+def check_lists(g, mask, order_group=0):
+    c = Pr.mask_to_csr(mask, order_group)
     assert g["kept_total"] == c["kept_total"]
     assert np.array_equal(g["row_ptr"], c["row_ptr"])
     assert np.array_equal(g["col_idx"][:c["kept_total"]], c["col_idx"])
@@ -90,6 +98,10 @@ SMALL = [
     ("causal_small_blocks", 1, 2, 1, 333, 32, 16, 8, 0.9, 0.0, True, 0, 0, 40, 5, "fp32"),
     ("toy", 1, 1, 1, 64, 16, 16, 16, 0.9, 0.5, False, 0, 0, 0, 0, "fp32"),
     ("tau_one", 1, 2, 2, 640, 128, 128, 64, 1.0, 0.0, False, 0, 0, 0, 0, "bf16"),
+    # more than 512 key blocks: TopCdf's threshold search instead of the arg-max loop
+    ("threshold_search", 1, 2, 2, 6000, 64, 32, 8, 0.9, 0.0, False, 0, 0, 0, 0, "bf16"),
+    ("threshold_causal", 1, 2, 1, 6000, 64, 32, 8, 0.95, 0.0, True, 0, 0, 64, 8, "bf16"),
+    ("threshold_low_tau", 1, 2, 2, 6000, 64, 32, 8, 0.25, 0.0, False, 0, 0, 0, 0, "bf16"),
 ]
 
 
@@ -131,6 +143,49 @@ def test_predict_full_size(name):
         assert abs(sp - w.target_sparsity) < 0.01
     else:
         assert sp == 0.0     # theta = 0.6 forces every block of this generator
+
+
+@pytest.mark.parametrize("order_group", [1, 2, 3])
+def test_work_order_in_head_groups(order_group):
+    """order_group > 0: the work order sorts each group of consecutive
+    (batch, head) rows on its own, bit-exact against the oracle's order."""
+    from long_context_mean_b200 import sa
+    B, Hq, Hkv, N, bq, bk = 2, 4, 2, 1500, 128, 64
+    w = I.Workload("groups", 99, B, Hq, Hkv, 1, 1, N, 0, 128, 128, "bf16", "lowrank", bq=bq, bk=bk, tau=0.8,
+                   causal=True, local_window=300, anchor_tokens=128, sigma_pos=20.0)
+    g = I.gen_qkv(w)
+    q_dev, k_dev, _ = P.qkv_dev(g, "bf16")
+    prm = sa.make_params(bq, bk, 0.8, 0.0, 0, 0, 300, 128, True, order_group)
+    gres = run_gpu_predict(q_dev, k_dev, w, prm)
+    assert gres["status"] == sa.SA_OK
+    check_lists(gres, gres["mask"], order_group)
+    # the grouped order differs from the global one on this mask
+    assert not np.array_equal(gres["order"], Pr.mask_to_csr(gres["mask"])["order"])
+
+
+def test_global_order_past_shared_memory_rows():
+    """More than 32768 rows: the work order comes from the global-memory
+    radix sort, bit-exact against the oracle."""
+    import torch
+    from long_context_mean_b200 import sa
+    rng = np.random.default_rng(11)
+    B, Hq, bq, bk = 1, 40, 128, 128
+    nqb = nkb = 1000
+    N = nqb * bq
+    dens = rng.random((B, Hq, nqb, 1)) * 0.6           # rows of many different lengths
+    m = rng.random((B, Hq, nqb, nkb)) < dens
+    m[..., 0] = True
+    shape = sa.Shape(B, Hq, Hq, N, 128, 128, sa.SA_BF16, 0)
+    blocks = torch.from_numpy(m.astype(np.uint8).ravel()).to("cuda")
+    mb = sa.MaskBuffers.allocate(B, Hq, N, bq, bk, "cuda", capacity=int(m.sum()))
+    ws = sa.workspace(sa.mask_from_blocks_workspace(shape, bq, bk), "cuda")
+    sa.mask_from_blocks(blocks, shape, bq, bk, False, ws, mb.struct)
+    assert sa.read_status(mb.status) == sa.SA_OK
+    c = Pr.mask_to_csr(m)
+    assert int(mb.kept_total.item()) == c["kept_total"]
+    assert np.array_equal(mb.row_ptr.cpu().numpy(), c["row_ptr"])
+    assert np.array_equal(mb.col_idx.cpu().numpy(), c["col_idx"])
+    assert np.array_equal(mb.order.cpu().numpy(), c["order"])
 
 
 def test_empty_row_status():
@@ -216,8 +271,11 @@ def _fused_vs_separate(w, perm_np, q_bits, k_bits):
     ref = run_gpu_predict(P.bf16_dev(qr_want), P.bf16_dev(kr_want), w, prm)
     off = sa.predict_mask_ws_layout(shape, prm)
     for i, key in ((0, "qhat"), (1, "khat"), (2, "s_q"), (3, "s_k")):
-        n = ref[key].size
-        got = ws[off[i]:off[i] + n * 4].view(torch.float32).cpu().numpy().reshape(ref[key].shape)
+        if key == "khat":
+            got = khat_from_ws(ws, off, shape.B, shape.Hkv, mb.struct.nkb, shape.d)
+        else:
+            n = ref[key].size
+            got = ws[off[i]:off[i] + n * 4].view(torch.float32).cpu().numpy().reshape(ref[key].shape)
         assert np.array_equal(got, ref[key]), key
     assert np.array_equal(mb.block_mask.cpu().numpy().reshape(ref["mask"].shape).astype(bool), ref["mask"])
     kt = int(mb.kept_total.item())

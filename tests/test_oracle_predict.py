@@ -208,6 +208,19 @@ def test_csr_and_order():
     assert c["kept_total"] == 7
 
 
+def test_work_order_in_head_groups():
+    # 2 heads x 2 query blocks, counts [1, 3 | 2, 2]: one global order puts
+    # the 3-block row first; groups of one head sort each head's rows alone.
+    m = np.array([[[1, 0, 0], [1, 1, 1]], [[1, 1, 0], [0, 1, 1]]], dtype=bool)
+    assert Pr.mask_to_csr(m)["order"].tolist() == [1, 2, 3, 0]
+    assert Pr.mask_to_csr(m, order_group=1)["order"].tolist() == [1, 0, 2, 3]
+    assert Pr.mask_to_csr(m, order_group=2)["order"].tolist() == [1, 2, 3, 0]
+    # a group larger than the heads is one global order; ragged last group
+    m3 = np.concatenate([m, m[:1]], axis=0)            # 3 heads, counts [1,3 | 2,2 | 1,3]
+    assert Pr.mask_to_csr(m3, order_group=2)["order"].tolist() == [1, 2, 3, 0, 5, 4]
+    assert Pr.mask_to_csr(m3, order_group=8)["order"].tolist() == Pr.mask_to_csr(m3)["order"].tolist()
+
+
 def test_empty_rows_element_level():
     # causal, bq = 4 > bk = 2: q-block 1 (rows 4..7) keeping only k-block 3
     # (keys 6, 7) leaves rows 4 and 5 with nothing.
