@@ -22,16 +22,7 @@ namespace {
 
 constexpr int kPoolThreads = 256;
 constexpr int kPoolWarps = kPoolThreads / 32;
-constexpr int kPoolStages = 3;   // blocks a CTA holds in shared memory: one in use, two arriving
-
-__device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_stages() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(kPoolStages - 1) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+constexpr int kPoolLoads = 4;   // 16-byte loads a lane has in flight
 
 // Two fp32 values in one 64-bit register for the packed fp32x2 pipe.
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
@@ -64,154 +55,111 @@ __device__ __forceinline__ void pairs16(const uint4& u, float, uint64_t* p) {
 }
 
 // ---------------------------------------------------------------------------
-// a2: block mean and mean pairwise cosine of every (head, block) unit.  A
-// persistent CTA takes units blockIdx.x, + gridDim.x, ... and streams their
-// tokens through a ring of kPoolStages blocks in shared memory with
-// cp.async, so two blocks are arriving while a third is reduced.  Thread i
-// owns chunk c = i % CH (CH = 16-byte pieces of a token) of tokens i / CH,
-// + 256 / CH, ...: it copies exactly the chunks it later reads, so the ring
-// needs no barrier of its own.  The arithmetic runs on fp32 pairs (packed
-// FMA/ADD), the token norm reduces inside the token's lane group and its
-// inverse is the hardware reciprocal square root; the block sums reduce
-// across lanes and warps.  With perm, token n of the block is read from row
-// perm[n] of x (an entry outside [0, N) raises SA_ERR_INVALID_ARG and the
-// token reads as zeros and is not written) and also written to row n of y
-// (a1 fused with a2: the reordered copy is produced by the same pass that
-// pools it).  The block mean goes to mean_out[(bh * nB + blk) * d + i], or
-// with mean_tstride > 0 to mean_out[(bh * d + i) * mean_tstride + blk]
-// (transposed: one row per feature, blocks contiguous).  QF = 1 + SA_Q_INT8
-// or 1 + SA_Q_E4M3 (bf16 input): instead of the copy, the pass writes the
-// block's 8-bit codes to row n of y8 and its scale (absmax / 127 or / 448)
-// to qscale, quantising from shared memory once the block's absmax is known.
-// Dynamic shared memory: ring [kPoolStages][b * CH] 16-byte chunks | block
-// sums [2][kPoolWarps][d] fp32 | token flags [kPoolStages][128].
+// a2: block mean and mean pairwise cosine of every (head, block) unit.  Each
+// warp owns whole units (unit = its global warp index, + the grid's warps,
+// ...), so no barrier couples the warps and the SM keeps as many of them in
+// flight as registers allow.  A token is CH lanes x 16 bytes (CH = chunks per
+// token, a template parameter); a warp step covers 32 / CH tokens and a lane
+// has kPoolLoads steps of loads in flight before it uses any.  The token norm
+// reduces inside the token's lane group (independent shuffle chains for the
+// loads in flight); Σx and Σx/‖x‖ (hardware reciprocal square root)
+// accumulate on the packed fp32x2 pipe and reduce across the token groups at
+// the end.  With perm, token n of the block is read from row perm[n] of x
+// (the block's rows staged in the warp's shared memory first; an entry
+// outside [0, N) raises SA_ERR_INVALID_ARG and the token reads as zeros and
+// is not written) and also written to row n of y (a1 fused with a2: the
+// reordered copy is produced by the same pass that pools it).  The block mean
+// goes to mean_out[(bh * nB + blk) * d + i], or with mean_tstride > 0 to
+// mean_out[(bh * d + i) * mean_tstride + blk] (transposed: one row per
+// feature, blocks contiguous).  QF = 1 + SA_Q_INT8 or 1 + SA_Q_E4M3 (bf16
+// input): instead of the copy, the pass writes the block's 8-bit codes to row
+// n of y8 and its scale (absmax / 127 or / 448) to qscale, reading the block
+// a second time (from L2) once its absmax is known.
 // ---------------------------------------------------------------------------
-size_t pool_smem_bytes(int d, int b, int elem) {
-  return (size_t)kPoolStages * b * d * elem + (size_t)2 * kPoolWarps * d * 4 + (size_t)kPoolStages * 128;
-}
-
 template <typename T, int CH, int QF = 0>
-__global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
+__global__ void __launch_bounds__(kPoolThreads, 4) pool_cossim_kernel(
     const T* __restrict__ x, int64_t BH, int64_t N, int b, int nB, float* __restrict__ mean_out,
     int64_t mean_tstride, float* __restrict__ s_out, const int32_t* __restrict__ perm, T* __restrict__ y,
     int32_t* status, uint2* __restrict__ y8 = nullptr, float* __restrict__ qscale = nullptr) {
   constexpr int EPL = 16 / sizeof(T);   // elements per chunk
   constexpr int NP = EPL / 2;           // fp32 pairs per chunk
   constexpr int d = CH * EPL;
-  constexpr int TPP = kPoolThreads / CH;   // tokens per pass of the CTA
+  constexpr int TPW = 32 / CH;          // tokens per warp step
   static_assert(CH >= 1 && CH <= 32 && (CH & (CH - 1)) == 0, "chunks per token: a power of two <= 32");
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint4* ring = reinterpret_cast<uint4*>(smem);
-  const int stage_chunks = b * CH;
-  float* sx = reinterpret_cast<float*>(ring + kPoolStages * stage_chunks);   // [kPoolWarps][d]
-  float* su = sx + kPoolWarps * d;
-  uint8_t* tok_ok = reinterpret_cast<uint8_t*>(su + kPoolWarps * d);        // [kPoolStages][128]
-  __shared__ float red[kPoolWarps];
-  __shared__ float wmax[kPoolWarps];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int sub = tid / CH, c = tid % CH;
+  __shared__ int32_t srow_all[kPoolWarps][128];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane / CH, c = lane % CH;
+  int32_t* srow = srow_all[warp];
   const int64_t units = BH * nB;
-
-  // Copies of this thread's chunks of unit `unit` into stage `st` (one
-  // commit group per call, empty past the last unit).
-  auto issue = [&](int64_t unit, int st) {
-    if (unit < units) {
-      const int64_t bh = unit / nB;
-      const int blk = (int)(unit - bh * nB);
-      const int64_t t0 = (int64_t)blk * b;
-      const int cnt = (int)min64(b, N - t0);
-      const uint4* xbh = reinterpret_cast<const uint4*>(x + bh * N * (int64_t)d) + c;
-      uint4* dst = ring + st * stage_chunks + c;
-      for (int tok = sub; tok < cnt; tok += TPP) {
-        const int64_t n = t0 + tok;
-        const int64_t src = perm ? (int64_t)__ldg(perm + n) : n;
-        const bool ok = (uint64_t)src < (uint64_t)N;
-        if (!ok) {   // not a permutation of [0, N)
-          if (c == 0) raise_status(status, SA_ERR_INVALID_ARG);
-          dst[tok * CH] = make_uint4(0, 0, 0, 0);
-        } else {
-          cp_async16((uint32_t)__cvta_generic_to_shared(dst + tok * CH), xbh + src * CH);
-        }
-        if (c == 0) tok_ok[st * 128 + tok] = ok ? 1 : 0;
-      }
-    }
-    cp_async_commit();
-  };
-
-  int64_t unit = blockIdx.x;
-#pragma unroll 1
-  for (int j = 0; j < kPoolStages - 1; ++j) issue(unit + (int64_t)j * gridDim.x, j);
-#pragma unroll 1
-  for (int it = 0; unit < units; ++it, unit += gridDim.x) {
-    const int st = it % kPoolStages;
-    issue(unit + (int64_t)(kPoolStages - 1) * gridDim.x, (it + kPoolStages - 1) % kPoolStages);
-    cp_async_wait_stages();   // this thread's copies of `unit` have landed
-    __syncthreads();          // token flags of `unit` written by other threads
+  const int64_t wstride = (int64_t)gridDim.x * kPoolWarps;
+  for (int64_t unit = (int64_t)blockIdx.x * kPoolWarps + warp; unit < units; unit += wstride) {
     const int64_t bh = unit / nB;
     const int blk = (int)(unit - bh * nB);
     const int64_t t0 = (int64_t)blk * b;
     const int cnt = (int)min64(b, N - t0);
-    const uint4* ring_st = ring + st * stage_chunks + c;
-    const uint8_t* ok_st = tok_ok + st * 128;
+    const uint4* xbh = reinterpret_cast<const uint4*>(x + bh * N * (int64_t)d) + c;
     uint4* ybh = y ? reinterpret_cast<uint4*>(y + bh * N * (int64_t)d) + t0 * CH + c : nullptr;
-    // Every token of this thread at once: the smem reads, then the norms
-    // (independent shuffle chains), then the sums.  The token loops have a
-    // uniform trip count: the shuffles need every lane.
-    constexpr int MAXP = (128 + TPP - 1) / TPP;
-    uint4 raw[MAXP];
-#pragma unroll
-    for (int ip = 0; ip < MAXP; ++ip) {
-      const int tok = ip * TPP + sub;
-      raw[ip] = tok < cnt ? ring_st[tok * CH] : make_uint4(0, 0, 0, 0);
-    }
-    if (ybh) {
-#pragma unroll
-      for (int ip = 0; ip < MAXP; ++ip) {
-        const int tok = ip * TPP + sub;
-        if (tok < cnt && ok_st[tok]) __stcs(ybh + tok * CH, raw[ip]);
+    if (perm) {
+      __syncwarp();   // the previous unit's rows are no longer read
+      for (int i = lane; i < cnt; i += 32) {
+        const int32_t s = __ldg(perm + t0 + i);
+        if ((uint32_t)s >= (uint64_t)N) raise_status(status, SA_ERR_INVALID_ARG);   // not a permutation of [0, N)
+        srow[i] = (uint32_t)s < (uint64_t)N ? s : -1;
       }
-    }
-    float ssum[MAXP];
-#pragma unroll
-    for (int ip = 0; ip < MAXP; ++ip) {
-      uint64_t v[NP];
-      pairs16(raw[ip], T(), v);
-      uint64_t s2 = f2(0.f, 0.f);
-#pragma unroll
-      for (int e = 0; e < NP; ++e) s2 = f2_fma(v[e], v[e], s2);
-      float s0, s1;
-      f2_split(s2, s0, s1);
-      ssum[ip] = s0 + s1;
-    }
-#pragma unroll
-    for (int off = CH >> 1; off > 0; off >>= 1) {
-#pragma unroll
-      for (int ip = 0; ip < MAXP; ++ip) ssum[ip] += __shfl_xor_sync(0xffffffffu, ssum[ip], off);
+      __syncwarp();
     }
     uint64_t ax[NP], au[NP];
 #pragma unroll
     for (int e = 0; e < NP; ++e) ax[e] = au[e] = f2(0.f, 0.f);
     float amax = 0.f;
+    for (int tb = 0; tb < cnt; tb += kPoolLoads * TPW) {   // uniform: the shuffles need every lane
+      uint4 raw[kPoolLoads];
+      uint32_t okm = 0;
 #pragma unroll
-    for (int ip = 0; ip < MAXP; ++ip) {
-      uint64_t v[NP];
-      pairs16(raw[ip], T(), v);
-      const float inv = ssum[ip] > 0.f ? rsqrtf(ssum[ip]) : 0.f;
-      const uint64_t inv2 = f2(inv, inv);
-#pragma unroll
-      for (int e = 0; e < NP; ++e) {
-        ax[e] = f2_add(ax[e], v[e]);
-        au[e] = f2_fma(v[e], inv2, au[e]);
+      for (int u = 0; u < kPoolLoads; ++u) {
+        const int tok = tb + u * TPW + sub;
+        int64_t src = -1;
+        if (tok < cnt) src = perm ? (int64_t)srow[tok] : t0 + tok;
+        if (src >= 0) okm |= 1u << u;
+        raw[u] = src >= 0 ? __ldg(xbh + src * CH) : make_uint4(0, 0, 0, 0);
       }
-      if constexpr (QF != 0) {
+      if (ybh) {
+#pragma unroll
+        for (int u = 0; u < kPoolLoads; ++u)
+          if ((okm >> u) & 1u) __stcs(ybh + (tb + u * TPW + sub) * CH, raw[u]);
+      }
+      // One token at a time from registers (the loads are all in flight):
+      // its norm over the token's lanes, then the sums.
+#pragma unroll
+      for (int u = 0; u < kPoolLoads; ++u) {
+        uint64_t v[NP];
+        pairs16(raw[u], T(), v);
+        uint64_t s2 = f2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < NP; ++e) s2 = f2_fma(v[e], v[e], s2);
+        float s0, s1;
+        f2_split(s2, s0, s1);
+        float ss = s0 + s1;
+#pragma unroll
+        for (int off = CH >> 1; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+        const uint64_t inv2 = f2(inv, inv);
 #pragma unroll
         for (int e = 0; e < NP; ++e) {
-          float lo, hi;
-          f2_split(v[e], lo, hi);
-          amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+          ax[e] = f2_add(ax[e], v[e]);
+          au[e] = f2_fma(v[e], inv2, au[e]);
+        }
+        if constexpr (QF != 0) {
+#pragma unroll
+          for (int e = 0; e < NP; ++e) {
+            float lo, hi;
+            f2_split(v[e], lo, hi);
+            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+          }
         }
       }
     }
+    // Lanes c, c + CH, ... hold the same features for different tokens.
     float axs[EPL], aus[EPL];
 #pragma unroll
     for (int e = 0; e < NP; ++e) {
@@ -226,58 +174,40 @@ __global__ void __launch_bounds__(kPoolThreads) pool_cossim_kernel(
         aus[e] += __shfl_xor_sync(0xffffffffu, aus[e], off);
       }
     }
+    float part = 0.f;
     if (lane < CH) {
+      const float invc = 1.0f / (float)cnt;
 #pragma unroll
       for (int e = 0; e < EPL; ++e) {
-        sx[warp * d + c * EPL + e] = axs[e];
-        su[warp * d + c * EPL + e] = aus[e];
+        const int i = c * EPL + e;
+        const float mv = axs[e] * invc;
+        if (mean_tstride > 0) mean_out[(bh * d + i) * mean_tstride + blk] = mv;
+        else mean_out[(bh * nB + blk) * (int64_t)d + i] = mv;
+        part = fmaf(aus[e], aus[e], part);
       }
-    }
-    if constexpr (QF != 0) {
-      for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      if (lane == 0) wmax[warp] = amax;
-    }
-    __syncthreads();
-    float part = 0.f;
-    for (int i = tid; i < d; i += kPoolThreads) {
-      float X = 0.f, U = 0.f;
-#pragma unroll
-      for (int w = 0; w < kPoolWarps; ++w) {
-        X += sx[w * d + i];
-        U += su[w * d + i];
-      }
-      const float mv = X / (float)cnt;
-      if (mean_tstride > 0) mean_out[(bh * d + i) * mean_tstride + blk] = mv;
-      else mean_out[(bh * nB + blk) * (int64_t)d + i] = mv;
-      part = fmaf(U, U, part);
     }
     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-    if (lane == 0) red[warp] = part;
+    if (lane == 0) s_out[bh * nB + blk] = part / ((float)cnt * (float)cnt);
     if constexpr (QF != 0) {
       static_assert(sizeof(T) == 2, "8-bit codes are written from bf16 input");
       constexpr int FMT = QF - 1;
-      float A = 0.f;
-#pragma unroll
-      for (int w = 0; w < kPoolWarps; ++w) A = fmaxf(A, wmax[w]);
+      for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       const float qmax = FMT == SA_Q_E4M3 ? 448.0f : 127.0f;
-      const float qinv = A > 0.f ? __fdiv_rn(qmax, A) : 0.f;
-      if (tid == 0) qscale[bh * nB + blk] = A > 0.f ? __fdiv_rn(A, qmax) : 0.f;
+      const float qinv = amax > 0.f ? __fdiv_rn(qmax, amax) : 0.f;
+      if (lane == 0) qscale[bh * nB + blk] = amax > 0.f ? __fdiv_rn(amax, qmax) : 0.f;
       uint2* y8bh = y8 + (bh * N + t0) * (int64_t)CH + c;
-      for (int tok = sub; tok < cnt; tok += TPP)
-        if (ok_st[tok]) y8bh[tok * CH] = quant8<FMT>(ring_st[tok * CH], qinv);
-    }
-    __syncthreads();
-    if (tid == 0) {
-      float tot = 0.f;
-      for (int w = 0; w < kPoolWarps; ++w) tot += red[w];
-      s_out[bh * nB + blk] = tot / ((float)cnt * (float)cnt);
+      for (int tok = sub; tok < cnt; tok += TPW) {
+        const int64_t src = perm ? (int64_t)srow[tok] : t0 + tok;
+        if (src >= 0) y8bh[tok * CH] = quant8<FMT>(__ldg(xbh + src * CH), qinv);
+      }
     }
   }
-  cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------
-// Shared row rules (structure-forced rows/columns, window, causal validity).
+// Row rules: the parameters of the structure-forced rows/columns, the local
+// window and causal validity (the score kernel turns them into key-block
+// ranges once per row).
 // ---------------------------------------------------------------------------
 struct RowRules {
   int64_t N, sink, txt, window, anchor;
@@ -285,16 +215,6 @@ struct RowRules {
   __device__ bool struct_row(int64_t qb) const {
     const int64_t i0 = qb * bq, i1 = min(N, (qb + 1) * bq);
     return i0 < sink || (txt > 0 && i1 - 1 >= N - txt);
-  }
-  __device__ bool struct_col(int64_t kb) const {
-    const int64_t j0 = kb * bk, j1 = min(N, (kb + 1) * bk);
-    return j0 < sink || j0 < anchor || (txt > 0 && j1 - 1 >= N - txt);
-  }
-  __device__ bool in_window(int64_t qb, int64_t kb) const {
-    if (window <= 0) return false;
-    const int64_t i0 = qb * bq, i1 = min(N, (qb + 1) * bq);
-    const int64_t j0 = kb * bk, j1 = min(N, (kb + 1) * bk);
-    return (i1 - 1 >= j0) && (i0 - (j1 - 1) < window);
   }
   __device__ bool valid(int64_t qb, int64_t kb) const {
     if (!causal) return true;
@@ -389,7 +309,7 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-__global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
+__global__ void __launch_bounds__(kRowThreads, 2) score_topcdf_kernel(
     const float* __restrict__ qhat, const float* __restrict__ khat, const float* __restrict__ sq,
     const float* __restrict__ sk, int64_t Hq, int64_t Hkv, int64_t nqb, int64_t nkb, int d,
     int P2, int G, float tau, float theta, RowRules rules, uint8_t* __restrict__ mask,
@@ -434,9 +354,9 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
     const float* kT = khat + g * (int64_t)d * nkb4;
     const float4* qs4 = reinterpret_cast<const float4*>(qs);
     const int nf4 = d / 4;
-    for (int kb = threadIdx.x; kb < nkb; kb += kRowThreads) {
+    for (int kb = threadIdx.x; kb < nkb4; kb += kRowThreads) {   // the padding gets -inf
       uint32_t need = 0;   // bit r: row r of the group scores this key block
-      if (!(guard && sk[g * nkb + kb] < theta)) {
+      if (kb < nkb && !(guard && sk[g * nkb + kb] < theta)) {
 #pragma unroll
         for (int r = 0; r < kMaxRowsPerCta; ++r)
           if (kb <= s_klim[r]) need |= 1u << r;
@@ -448,7 +368,7 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
       for (int r = 0; r < kMaxRowsPerCta; ++r) a[r] = f2(0.f, 0.f);
       if (need) {
         const float* kc = kT + kb;
-#pragma unroll 4
+#pragma unroll 8
         for (int e4 = 0; e4 < nf4; ++e4) {
           const uint64_t k01 = f2(__ldg(kc + (int64_t)(4 * e4) * nkb4), __ldg(kc + (int64_t)(4 * e4 + 1) * nkb4));
           const uint64_t k23 = f2(__ldg(kc + (int64_t)(4 * e4 + 2) * nkb4), __ldg(kc + (int64_t)(4 * e4 + 3) * nkb4));
@@ -480,11 +400,18 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
   const bool row_forced = s_forced[r] != 0;
   float* pr = sc + (size_t)r * nkb4;   // probabilities replace the scores (bisection)
   uint8_t* fl = flags + (size_t)r * nkb16;
-  for (int64_t kb = lane; kb < nkb; kb += 32) fl[kb] = 0;
+  for (int i = lane; i < nkb16 / 16; i += 32) reinterpret_cast<uint4*>(fl)[i] = make_uint4(0, 0, 0, 0);
+  // Float4 groups that can hold a finite score: key blocks past the row's
+  // last valid one (causal) and the padding are -inf.
+  const int nq_row = row_forced ? 0 : min(nkb4 / 4, (s_klim[r] + 4) / 4);
   if (!row_forced) {
     const float* srow = sc + r * nkb4;
+    const float4* srow4 = reinterpret_cast<const float4*>(srow);
     float mx = -INFINITY;
-    for (int64_t kb = lane; kb < nkb; kb += 32) mx = fmaxf(mx, srow[kb]);
+    for (int q = lane; q < nq_row; q += 32) {
+      const float4 v = srow4[q];
+      mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+    }
     mx = warp_max(mx);
     bool done = false;
     if (mx > -INFINITY && P2 <= 32 * kFastKeys) {
@@ -500,7 +427,7 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
         key[q] = 0ull;
         if (kb < nkb) {
           const float sv = srow[kb];
-          const float pv = (sv == -INFINITY) ? 0.f : expf(sv - mx);
+          const float pv = (sv == -INFINITY) ? 0.f : __expf(sv - mx);
           key[q] = ((uint64_t)__float_as_uint(pv) << 32) | (uint32_t)(~(uint32_t)kb);
           part += pv;
         }
@@ -544,15 +471,18 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
       // blocks whose p equals it are kept in index order while f(t*) + r p <
       // tau * total (r = rank among them).  t* is found by bisection over the
       // bit patterns of (0, 1] (p = exp(s - max) <= 1).
-      for (int kb = lane; kb < nkb4; kb += 32) {
-        const float sv = kb < nkb ? srow[kb] : -INFINITY;
-        pr[kb] = (sv == -INFINITY) ? 0.f : expf(sv - mx);
+      float4* pw4 = reinterpret_cast<float4*>(pr);
+      for (int q = lane; q < nq_row; q += 32) {
+        const float4 v = srow4[q];
+        float4 o;
+        o.x = v.x == -INFINITY ? 0.f : __expf(v.x - mx);
+        o.y = v.y == -INFINITY ? 0.f : __expf(v.y - mx);
+        o.z = v.z == -INFINITY ? 0.f : __expf(v.z - mx);
+        o.w = v.w == -INFINITY ? 0.f : __expf(v.w - mx);
+        pw4[q] = o;
       }
       __syncwarp();
       const float4* pr4 = reinterpret_cast<const float4*>(pr);
-      // Float4 groups that can hold a positive p: key blocks past the row's
-      // last valid one (causal) have p = 0.
-      const int nq_row = min(nkb4 / 4, (s_klim[r] + 4) / 4);
       // f(t) and the number of p whose bits exceed t, over the whole row.
       auto pass_full = [&](uint32_t t, int& count) -> float {
         float m0 = 0.f, m1 = 0.f;
@@ -625,12 +555,13 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
       const float above = f_hi;
       const float vstar = __uint_as_float(hi);
       uint32_t run = 0;
-      for (int64_t kb0 = 0; kb0 < nkb; kb0 += 32) {
-        const int64_t kb = kb0 + lane;
-        const uint32_t bits = kb < nkb ? __float_as_uint(pr[kb]) : 0u;
-        const bool tie = kb < nkb && bits == hi;
+      const int nrow = 4 * nq_row;   // p beyond this is 0: never kept (hi > 0)
+      for (int kb0 = 0; kb0 < nrow; kb0 += 32) {
+        const int kb = kb0 + lane;
+        const uint32_t bits = kb < nrow ? __float_as_uint(pr[kb]) : 0u;
+        const bool tie = kb < nrow && bits == hi;
         const unsigned bal = __ballot_sync(0xffffffffu, tie);
-        bool keep = kb < nkb && bits > hi;
+        bool keep = kb < nrow && bits > hi;
         if (tie) keep = above + (float)(run + __popc(bal & ((1u << lane) - 1u))) * vstar < limit;
         if (keep) fl[kb] = 1;
         run += __popc(bal);
@@ -638,15 +569,37 @@ __global__ void __launch_bounds__(kRowThreads) score_topcdf_kernel(
     }
   }
   __syncwarp();
+  // The row's key-block ranges, once: causally valid blocks kb <= klim; the
+  // local window [w0, w1]; the structural columns (sink, anchors) kb < c0 and
+  // (text) kb >= c1.
+  const int64_t i0 = qb * rules.bq, i1 = min64(rules.N, (qb + 1) * rules.bq);
+  const int klim = rules.causal ? (int)((i1 - 1) / rules.bk) : (int)nkb - 1;
+  int w0 = 1, w1 = 0;
+  if (rules.window > 0) {
+    // j1 - 1 >= i0 - window + 1 and j0 <= i1 - 1, with j0 = kb * bk, j1 = min(N, j0 + bk)
+    w0 = (int)max64(0, (i0 - rules.window + 1) / rules.bk);
+    while (w0 > 0 && min64(rules.N, (int64_t)(w0 - 1) * rules.bk + rules.bk) - 1 >= i0 - rules.window + 1) --w0;
+    while (w0 < nkb && min64(rules.N, (int64_t)w0 * rules.bk + rules.bk) - 1 < i0 - rules.window + 1) ++w0;
+    w1 = (int)min64(nkb - 1, (i1 - 1) / rules.bk);
+  }
+  const int64_t front = max64(rules.sink, rules.anchor);
+  const int c0 = (int)min64(nkb, (front + rules.bk - 1) / rules.bk);   // kb * bk < front
+  int c1 = (int)nkb;                                                 // last row of kb >= N - txt
+  if (rules.txt > 0) {
+    c1 = (int)max64(0, (rules.N - rules.txt) / rules.bk);
+    while (c1 > 0 && min64(rules.N, (int64_t)c1 * rules.bk) - 1 >= rules.N - rules.txt) --c1;
+    while (c1 < nkb && min64(rules.N, (int64_t)(c1 + 1) * rules.bk) - 1 < rules.N - rules.txt) ++c1;
+  }
   int cnt = 0, first = 0x7fffffff;
   uint8_t* mrow = mask + u * nkb;
-  for (int64_t kb = lane; kb < nkb; kb += 32) {
-    const bool col = rules.struct_col(kb) || (guard && sk[g * nkb + kb] < theta);
-    const bool keep = rules.valid(qb, kb) && (row_forced || fl[kb] || col || rules.in_window(qb, kb));
+  const float* skg = sk + g * nkb;
+  for (int kb = lane; kb < nkb; kb += 32) {
+    const bool col = kb < c0 || kb >= c1 || (guard && skg[kb] < theta);
+    const bool keep = kb <= klim && (row_forced || fl[kb] || col || (kb >= w0 && kb <= w1));
     mrow[kb] = keep ? 1 : 0;
     if (keep) {
       ++cnt;
-      first = min(first, (int)kb);
+      first = min(first, kb);
     }
   }
   for (int off = 16; off > 0; off >>= 1) {
@@ -1013,19 +966,16 @@ RowRules make_rules(const sa_shape& s, const sa_mask_params& p) {
 }
 
 // Persistent grid: as many CTAs as fit on the device at once (at most one
-// per unit).
+// warp per unit).
 template <typename K>
-sa_status pool_grid(K kernel, size_t smem, int64_t units, unsigned* grid) {
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(pool_cossim_kernel) failed");
+sa_status pool_grid(K kernel, int64_t units, unsigned* grid) {
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kPoolThreads, smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kPoolThreads, 0) != cudaSuccess ||
       per_sm < 1)
     return set_error(SA_ERR_CUDA, "pool_cossim_kernel does not fit on the device");
-  *grid = (unsigned)min64(units, (int64_t)sms * per_sm);
+  *grid = (unsigned)min64(ceil_div(units, kPoolWarps), (int64_t)sms * per_sm);
   return SA_OK;
 }
 
@@ -1033,12 +983,11 @@ template <typename T, int CH, int QF>
 sa_status launch_pool_ch(const void* x, int64_t BH, int64_t N, int b, int64_t nB, float* mean,
                          int64_t mean_tstride, float* sim, const int32_t* perm, void* y, int32_t* status,
                          uint2* y8, float* qscale, cudaStream_t st) {
-  const size_t smem = pool_smem_bytes(CH * (16 / (int)sizeof(T)), b, (int)sizeof(T));
   unsigned grid = 0;
-  if (sa_status e = pool_grid(pool_cossim_kernel<T, CH, QF>, smem, BH * nB, &grid)) return e;
-  pool_cossim_kernel<T, CH, QF><<<grid, kPoolThreads, smem, st>>>(static_cast<const T*>(x), BH, N, b, (int)nB,
-                                                                  mean, mean_tstride, sim, perm, static_cast<T*>(y),
-                                                                  status, y8, qscale);
+  if (sa_status e = pool_grid(pool_cossim_kernel<T, CH, QF>, BH * nB, &grid)) return e;
+  pool_cossim_kernel<T, CH, QF><<<grid, kPoolThreads, 0, st>>>(static_cast<const T*>(x), BH, N, b, (int)nB,
+                                                               mean, mean_tstride, sim, perm, static_cast<T*>(y),
+                                                               status, y8, qscale);
   return check_launch("pool_cossim_kernel");
 }
 

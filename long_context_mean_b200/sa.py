@@ -582,11 +582,18 @@ class HostPipeline:
         return read_status(self.status_word)
 
 
+def params_for(w) -> MaskParams:
+    """Mask parameters of a workload description, with the library's work-order
+    grouping for its shape."""
+    shape = Shape(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, SA_BF16 if w.dtype == "bf16" else SA_FP32, 0)
+    return make_params(w.bq, w.bk, w.tau, w.theta, w.sink_tokens, w.txt_len, w.local_window,
+                       w.anchor_tokens, w.causal, order_group_hint(shape))
+
+
 def host_pipeline_for(w, device="cuda", chunks=4, **kw) -> HostPipeline:
     """HostPipeline for a workload description from ``inputs.WORKLOADS``."""
     lay = make_layout(w.T, w.H, w.W, w.txt_len, w.sink_frames, w.order, w.win)
-    prm = make_params(w.bq, w.bk, w.tau, w.theta, w.sink_tokens, w.txt_len, w.local_window,
-                      w.anchor_tokens, w.causal)
+    prm = params_for(w)
     return HostPipeline(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, w.dtype, layout=lay, params=prm, lam=w.lam,
                         device=device, chunks=chunks, **kw)
 
@@ -594,8 +601,6 @@ def host_pipeline_for(w, device="cuda", chunks=4, **kw) -> HostPipeline:
 def pipeline_for(w, device="cuda", **kw) -> Pipeline:
     """Pipeline for a workload description from ``inputs.WORKLOADS``."""
     lay = make_layout(w.T, w.H, w.W, w.txt_len, w.sink_frames, w.order, w.win)
-    shape = Shape(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, SA_BF16 if w.dtype == "bf16" else SA_FP32, 0)
-    prm = make_params(w.bq, w.bk, w.tau, w.theta, w.sink_tokens, w.txt_len, w.local_window,
-                      w.anchor_tokens, w.causal, order_group_hint(shape))
+    prm = params_for(w)
     return Pipeline(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, w.dtype, layout=lay, params=prm, lam=w.lam,
                     device=device, **kw)
