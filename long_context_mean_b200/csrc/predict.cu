@@ -301,7 +301,7 @@ size_t score_smem_bytes(int d, int64_t nkb, int P2, int G) {
   const size_t nkb16 = (size_t)((nkb + 15) / 16) * 16;
   const size_t nkb4 = (size_t)((nkb + 3) / 4) * 4;
   return (size_t)kMaxRowsPerCta * d * 4 + (size_t)G * nkb4 * 4 + (size_t)G * nkb16 +
-         (size_t)kMaxRowsPerCta * kSelectRegs * 32 * 4;
+         (size_t)kMaxRowsPerCta * kSelectRegs * 32 * 4 + (size_t)nkb16;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -321,6 +321,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) score_topcdf_kernel(
   float* sc = reinterpret_cast<float*>(smem + (size_t)kMaxRowsPerCta * d * 4);
   uint8_t* flags = reinterpret_cast<uint8_t*>(sc + G * nkb4);
   float* cand = reinterpret_cast<float*>(flags + (size_t)G * nkb16);   // [8][kSelectRegs * 32]
+  uint8_t* colg = reinterpret_cast<uint8_t*>(cand + kMaxRowsPerCta * kSelectRegs * 32);   // [nkb16]
   __shared__ int s_forced[kMaxRowsPerCta];
   __shared__ int s_klim[kMaxRowsPerCta];   // last key block row r scores (-1: none)
 
@@ -343,6 +344,8 @@ __global__ void __launch_bounds__(kRowThreads, 2) score_topcdf_kernel(
                                             : (int)nkb - 1);
   }
   for (int i = threadIdx.x; i < rows * d; i += blockDim.x) qs[i] = qhat[(bh * nqb + qb0) * (int64_t)d + i];
+  // key blocks under the similarity guard (forced columns, out of the softmax)
+  for (int kb = threadIdx.x; kb < nkb; kb += blockDim.x) colg[kb] = (guard && sk[g * nkb + kb] < theta) ? 1 : 0;
   __syncthreads();
   int any_scored = 0;
   for (int r = 0; r < rows; ++r) any_scored |= !s_forced[r];
@@ -354,38 +357,105 @@ __global__ void __launch_bounds__(kRowThreads, 2) score_topcdf_kernel(
     const float* kT = khat + g * (int64_t)d * nkb4;
     const float4* qs4 = reinterpret_cast<const float4*>(qs);
     const int nf4 = d / 4;
-    for (int kb = threadIdx.x; kb < nkb4; kb += kRowThreads) {   // the padding gets -inf
-      uint32_t need = 0;   // bit r: row r of the group scores this key block
-      if (kb < nkb && !(guard && sk[g * nkb + kb] < theta)) {
+    // Two key blocks a thread per pass (kb and kb + 256): each shared read of
+    // q_hat feeds both, and their loads are in flight together.
+    auto need_of = [&](int kb) -> uint32_t {   // bit r: row r of the group scores key block kb
+      uint32_t need = 0;
+      if (kb < nkb && !colg[kb]) {
 #pragma unroll
         for (int r = 0; r < kMaxRowsPerCta; ++r)
           if (kb <= s_klim[r]) need |= 1u << r;
       }
-      // Row r's dot product as two packed partial sums: features (4e, 4e+1)
-      // and (4e+2, 4e+3) of each group of four.
-      uint64_t a[kMaxRowsPerCta];
+      return need;
+    };
+    if (nkb4 >= 8 * kRowThreads) {
+      // Long rows: four consecutive key blocks a thread, so a warp's 16-byte
+      // load of one feature covers 128 blocks; kb pairs share a packed FMA
+      // with the feature broadcast.
+      const int nq = nkb4 / 4;
+      const float4* kT4 = reinterpret_cast<const float4*>(kT);
+      for (int q = threadIdx.x; q < nq; q += kRowThreads) {
+        const uint32_t n0 = need_of(4 * q), n1 = need_of(4 * q + 1);
+        const uint32_t n2 = need_of(4 * q + 2), n3 = need_of(4 * q + 3);
+        uint64_t a01[kMaxRowsPerCta], a23[kMaxRowsPerCta];   // row r: blocks (4q, 4q+1), (4q+2, 4q+3)
 #pragma unroll
-      for (int r = 0; r < kMaxRowsPerCta; ++r) a[r] = f2(0.f, 0.f);
-      if (need) {
-        const float* kc = kT + kb;
-#pragma unroll 8
-        for (int e4 = 0; e4 < nf4; ++e4) {
-          const uint64_t k01 = f2(__ldg(kc + (int64_t)(4 * e4) * nkb4), __ldg(kc + (int64_t)(4 * e4 + 1) * nkb4));
-          const uint64_t k23 = f2(__ldg(kc + (int64_t)(4 * e4 + 2) * nkb4), __ldg(kc + (int64_t)(4 * e4 + 3) * nkb4));
+        for (int r = 0; r < kMaxRowsPerCta; ++r) a01[r] = a23[r] = f2(0.f, 0.f);
+        if (n0 | n1 | n2 | n3) {
+#pragma unroll 2
+          for (int e4 = 0; e4 < nf4; ++e4) {
+            float4 kf[4];   // features 4 e4 .. 4 e4 + 3 of the four blocks
 #pragma unroll
-          for (int r = 0; r < kMaxRowsPerCta; ++r) {
-            const float4 x = qs4[r * nf4 + e4];
-            a[r] = f2_fma(f2(x.x, x.y), k01, a[r]);
-            a[r] = f2_fma(f2(x.z, x.w), k23, a[r]);
+            for (int f = 0; f < 4; ++f) kf[f] = __ldg(kT4 + (int64_t)(4 * e4 + f) * nq + q);
+#pragma unroll
+            for (int r = 0; r < kMaxRowsPerCta; ++r) {
+              const float4 x = qs4[r * nf4 + e4];
+              const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int f = 0; f < 4; ++f) {
+                const uint64_t xx = f2(xv[f], xv[f]);
+                a01[r] = f2_fma(xx, f2(kf[f].x, kf[f].y), a01[r]);
+                a23[r] = f2_fma(xx, f2(kf[f].z, kf[f].w), a23[r]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < kMaxRowsPerCta; ++r) {
+          if (r < rows) {
+            float s0, s1, s2, s3;
+            f2_split(a01[r], s0, s1);
+            f2_split(a23[r], s2, s3);
+            float4 o;
+            o.x = ((n0 >> r) & 1u) ? s0 * scale : -INFINITY;
+            o.y = ((n1 >> r) & 1u) ? s1 * scale : -INFINITY;
+            o.z = ((n2 >> r) & 1u) ? s2 * scale : -INFINITY;
+            o.w = ((n3 >> r) & 1u) ? s3 * scale : -INFINITY;
+            reinterpret_cast<float4*>(sc + r * nkb4)[q] = o;
           }
         }
       }
+    } else {
+      for (int kb0 = threadIdx.x; kb0 < nkb4; kb0 += 2 * kRowThreads) {   // the padding gets -inf
+        const int kb1 = kb0 + kRowThreads;
+        const uint32_t need0 = need_of(kb0), need1 = kb1 < nkb4 ? need_of(kb1) : 0u;
+        // Row r's dot products as two packed partial sums each: features
+        // (4e, 4e+1) and (4e+2, 4e+3) of each group of four.
+        uint64_t a0[kMaxRowsPerCta], a1[kMaxRowsPerCta];
 #pragma unroll
-      for (int r = 0; r < kMaxRowsPerCta; ++r) {
-        if (r < rows) {
-          float lo, hi;
-          f2_split(a[r], lo, hi);
-          sc[r * nkb4 + kb] = ((need >> r) & 1u) ? (lo + hi) * scale : -INFINITY;
+        for (int r = 0; r < kMaxRowsPerCta; ++r) a0[r] = a1[r] = f2(0.f, 0.f);
+        if (need0 | need1) {
+          // a block no row needs reads block kb0 instead (in bounds, discarded)
+          const float* kc0 = kT + kb0;
+          const float* kc1 = kT + (need1 ? kb1 : kb0);
+#pragma unroll 4
+          for (int e4 = 0; e4 < nf4; ++e4) {
+            const int64_t o = (int64_t)(4 * e4) * nkb4;
+            const uint64_t p01 = f2(__ldg(kc0 + o), __ldg(kc0 + o + nkb4));
+            const uint64_t p23 = f2(__ldg(kc0 + o + 2 * nkb4), __ldg(kc0 + o + 3 * nkb4));
+            const uint64_t q01 = f2(__ldg(kc1 + o), __ldg(kc1 + o + nkb4));
+            const uint64_t q23 = f2(__ldg(kc1 + o + 2 * nkb4), __ldg(kc1 + o + 3 * nkb4));
+#pragma unroll
+            for (int r = 0; r < kMaxRowsPerCta; ++r) {
+              const float4 x = qs4[r * nf4 + e4];
+              const uint64_t x01 = f2(x.x, x.y), x23 = f2(x.z, x.w);
+              a0[r] = f2_fma(x01, p01, a0[r]);
+              a0[r] = f2_fma(x23, p23, a0[r]);
+              a1[r] = f2_fma(x01, q01, a1[r]);
+              a1[r] = f2_fma(x23, q23, a1[r]);
+            }
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < kMaxRowsPerCta; ++r) {
+          if (r < rows) {
+            float lo, hi;
+            f2_split(a0[r], lo, hi);
+            sc[r * nkb4 + kb0] = ((need0 >> r) & 1u) ? (lo + hi) * scale : -INFINITY;
+            if (kb1 < nkb4) {
+              f2_split(a1[r], lo, hi);
+              sc[r * nkb4 + kb1] = ((need1 >> r) & 1u) ? (lo + hi) * scale : -INFINITY;
+            }
+          }
         }
       }
     }
@@ -592,15 +662,26 @@ __global__ void __launch_bounds__(kRowThreads, 2) score_topcdf_kernel(
   }
   int cnt = 0, first = 0x7fffffff;
   uint8_t* mrow = mask + u * nkb;
-  const float* skg = sk + g * nkb;
-  for (int kb = lane; kb < nkb; kb += 32) {
-    const bool col = kb < c0 || kb >= c1 || (guard && skg[kb] < theta);
-    const bool keep = kb <= klim && (row_forced || fl[kb] || col || (kb >= w0 && kb <= w1));
-    mrow[kb] = keep ? 1 : 0;
+  auto keep_of = [&](int kb, bool picked) -> bool {
+    const bool col = kb < c0 || kb >= c1 || colg[kb];
+    const bool keep = kb <= klim && (row_forced || picked || col || (kb >= w0 && kb <= w1));
     if (keep) {
       ++cnt;
       first = min(first, kb);
     }
+    return keep;
+  };
+  if ((nkb & 3) == 0 && (reinterpret_cast<uintptr_t>(mask) & 3) == 0) {
+    // four blocks a lane: one 32-bit read of the picks, one 32-bit store
+    for (int q = lane; q < nkb / 4; q += 32) {
+      const uint32_t f4 = reinterpret_cast<const uint32_t*>(fl)[q];
+      uint32_t out = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out |= (keep_of(4 * q + j, ((f4 >> (8 * j)) & 0xFFu) != 0u) ? 1u : 0u) << (8 * j);
+      reinterpret_cast<uint32_t*>(mrow)[q] = out;
+    }
+  } else {
+    for (int kb = lane; kb < nkb; kb += 32) mrow[kb] = keep_of(kb, fl[kb] != 0) ? 1 : 0;
   }
   for (int off = 16; off > 0; off >>= 1) {
     cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
