@@ -228,7 +228,7 @@ def run_ours(args, rank, world, local_rank):
     host = {n: torch.from_numpy(g[n + "_bits"].view(np.int16)).view(torch.bfloat16).pin_memory() for n in "qkv"}
     q, k, v = (host[n].to(dev) for n in "qkv")
     stream = torch.cuda.current_stream(dev)
-    pipe = sa.pipeline_for(w, device=dev, log_skips=True, qk8=args.qk8)
+    pipe = sa.pipeline_for(w, device=dev, log_skips=True, qk8=args.qk8, order_group=args.order_group)
 
     # Calibration pass (untimed): mask, skip log, FLOPs, sparsity.
     pipe.run(q, k, v)
@@ -369,7 +369,7 @@ def run_ours(args, rank, world, local_rank):
     lse_host = torch.empty(pipe.lse.shape, dtype=pipe.lse.dtype).pin_memory()
     e2e_ms = float("nan")
     if not args.qk8:   # the host-buffer pass runs the bf16 path
-        hp = sa.host_pipeline_for(w, device=dev, chunks=args.e2e_chunks)
+        hp = sa.host_pipeline_for(w, device=dev, chunks=args.e2e_chunks, order_group=args.order_group)
 
         def e2e_step():
             hp.run(host["q"], host["k"], host["v"], out_host, lse_host, stream)
@@ -422,7 +422,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": f"bf16, QK {args.qk8} per block" if args.qk8 else "bf16",
         "data": "synthetic (seeded smooth-field generator, bf16)",
-        "config": workload_config(w, world),
+        "config": dict(workload_config(w, world), order_group=int(pipe.params.order_group)),
         "stages_ms": {"layout_reorder_predict": round(statistics.mean(pre_ms), 4),
                       "attention_with_fused_unreorder": round(statistics.mean(attn_ms), 4)},
         "timing_ms": {"step": spread(step_ms), "attention": spread(attn_ms), "prediction": spread(pre_ms)},
@@ -814,6 +814,9 @@ def main():
     ap.add_argument("--sweep", default=None,
                     help="attention throughput against block sparsity: 'all' or a comma list of workloads "
                          "(one JSON line per point instead of the headline line)")
+    ap.add_argument("--order-group", type=int, default=None,
+                    help="work-order grouping of the mask rows (sa_mask_params.order_group); "
+                         "default: the library's choice for the shape")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="head chunks of the end-to-end pass (copies overlap the kernels)")
     args = ap.parse_args()

@@ -582,25 +582,27 @@ class HostPipeline:
         return read_status(self.status_word)
 
 
-def params_for(w) -> MaskParams:
+def params_for(w, order_group=None) -> MaskParams:
     """Mask parameters of a workload description, with the library's work-order
-    grouping for its shape."""
-    shape = Shape(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, SA_BF16 if w.dtype == "bf16" else SA_FP32, 0)
+    grouping for its shape unless ``order_group`` is given."""
+    if order_group is None:
+        shape = Shape(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, SA_BF16 if w.dtype == "bf16" else SA_FP32, 0)
+        order_group = order_group_hint(shape)
     return make_params(w.bq, w.bk, w.tau, w.theta, w.sink_tokens, w.txt_len, w.local_window,
-                       w.anchor_tokens, w.causal, order_group_hint(shape))
+                       w.anchor_tokens, w.causal, order_group)
 
 
-def host_pipeline_for(w, device="cuda", chunks=4, **kw) -> HostPipeline:
+def host_pipeline_for(w, device="cuda", chunks=4, order_group=None, **kw) -> HostPipeline:
     """HostPipeline for a workload description from ``inputs.WORKLOADS``."""
     lay = make_layout(w.T, w.H, w.W, w.txt_len, w.sink_frames, w.order, w.win)
-    prm = params_for(w)
+    prm = params_for(w, order_group)
     return HostPipeline(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, w.dtype, layout=lay, params=prm, lam=w.lam,
                         device=device, chunks=chunks, **kw)
 
 
-def pipeline_for(w, device="cuda", **kw) -> Pipeline:
+def pipeline_for(w, device="cuda", order_group=None, **kw) -> Pipeline:
     """Pipeline for a workload description from ``inputs.WORKLOADS``."""
     lay = make_layout(w.T, w.H, w.W, w.txt_len, w.sink_frames, w.order, w.win)
-    prm = params_for(w)
+    prm = params_for(w, order_group)
     return Pipeline(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, w.dtype, layout=lay, params=prm, lam=w.lam,
                     device=device, **kw)
