@@ -255,15 +255,12 @@ def run_ours(args, rank, world, local_rank):
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
-    def step_timed():
-        """One step (the calls of Pipeline.run) with events around the
-        stages: [start, after predict, after attention]."""
-        e = [ev() for _ in range(3)]
-        e[0].record(stream)
+    def pred_stage(st):
+        """Layout, reorders and mask prediction (the calls of Pipeline.run) on st."""
         if not pipe.identity:
-            sa.layout_build(pipe.layout, pipe.perm, pipe.inv, pipe.layout_ws)
+            sa.layout_build(pipe.layout, pipe.perm, pipe.inv, pipe.layout_ws, st)
             # the V reorder on the pipeline's side stream, beside the prediction
-            pipe.ev_layout.record(stream)
+            pipe.ev_layout.record(st)
             pipe.side.wait_event(pipe.ev_layout)
             sa.reorder(pipe.perm, v, pipe.vr, pipe.side)
             pipe.ev_v.record(pipe.side)
@@ -271,28 +268,59 @@ def run_ours(args, rank, world, local_rank):
             # pass (the 8-bit path: reorder and quantisation)
             if args.qk8:
                 sa.reorder_predict_mask_q8(pipe.perm, q, k, args.qk8, pipe.q8, pipe.q_scales, pipe.k8,
-                                           pipe.k_scales, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
+                                           pipe.k_scales, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct, st)
             else:
                 sa.reorder_predict_mask(pipe.perm, q, k, pipe.qr, pipe.kr, pipe.shape, pipe.params, pipe.ws,
-                                        pipe.mask.struct)
-            stream.wait_event(pipe.ev_v)
-            qr, kr, vr = (q, k, pipe.vr) if args.qk8 else (pipe.qr, pipe.kr, pipe.vr)
+                                        pipe.mask.struct, st)
+            st.wait_event(pipe.ev_v)
         else:
-            qr, kr, vr = q, k, v
             if args.qk8:
                 sa.reorder_predict_mask_q8(None, q, k, args.qk8, pipe.q8, pipe.q_scales, pipe.k8, pipe.k_scales,
-                                           pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
+                                           pipe.shape, pipe.params, pipe.ws, pipe.mask.struct, st)
             else:
-                sa.predict_mask(qr, kr, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct)
-        e[1].record(stream)
-        # attention with the inverse reorder of O and LSE fused into its store
+                sa.predict_mask(q, k, pipe.shape, pipe.params, pipe.ws, pipe.mask.struct, st)
+
+    def attn_stage(st):
+        """Attention with the inverse reorder of O and LSE fused into its store."""
+        if pipe.identity:
+            qr, kr, vr = q, k, v
+        else:
+            qr, kr, vr = (q, k, pipe.vr) if args.qk8 else (pipe.qr, pipe.kr, pipe.vr)
         if args.qk8:
             sa.block_sparse_attn_qk8(pipe.q8, pipe.q_scales, pipe.k8, pipe.k_scales, vr, pipe.shape,
                                      pipe.mask.struct, pipe.lam, pipe.scale, pipe.out, pipe.attn_ws, pipe.lse,
-                                     out_perm=None if pipe.identity else pipe.perm, fmt=args.qk8)
+                                     stream=st, out_perm=None if pipe.identity else pipe.perm, fmt=args.qk8)
         else:
             sa.block_sparse_attn(qr, kr, vr, pipe.shape, pipe.mask.struct, pipe.lam, pipe.scale, pipe.out,
-                                 pipe.lse, ws=pipe.attn_ws, out_perm=None if pipe.identity else pipe.perm)
+                                 pipe.lse, stream=st, ws=pipe.attn_ws, out_perm=None if pipe.identity else pipe.perm)
+
+    # The two stages as CUDA graphs (the inputs and buffers are fixed): a
+    # replay launches every kernel of the stage without host gaps between them.
+    graphs = None
+    if not args.no_graphs:
+        pred_stage(stream)               # warm-up of the library's one-time setup outside capture
+        attn_stage(stream)
+        torch.cuda.synchronize(dev)
+        graphs = (torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph())
+        with torch.cuda.graph(graphs[0], capture_error_mode="relaxed"):
+            pred_stage(torch.cuda.current_stream(dev))
+        with torch.cuda.graph(graphs[1], capture_error_mode="relaxed"):
+            attn_stage(torch.cuda.current_stream(dev))
+        torch.cuda.synchronize(dev)
+
+    def step_timed():
+        """One step with events around the stages: [start, after predict, after attention]."""
+        e = [ev() for _ in range(3)]
+        e[0].record(stream)
+        if graphs:
+            graphs[0].replay()
+        else:
+            pred_stage(stream)
+        e[1].record(stream)
+        if graphs:
+            graphs[1].replay()
+        else:
+            attn_stage(stream)
         e[2].record(stream)
         return e
 
@@ -422,7 +450,8 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": f"bf16, QK {args.qk8} per block" if args.qk8 else "bf16",
         "data": "synthetic (seeded smooth-field generator, bf16)",
-        "config": dict(workload_config(w, world), order_group=int(pipe.params.order_group)),
+        "config": dict(workload_config(w, world), order_group=int(pipe.params.order_group),
+                       launch="cuda graph per stage" if graphs else "eager"),
         "stages_ms": {"layout_reorder_predict": round(statistics.mean(pre_ms), 4),
                       "attention_with_fused_unreorder": round(statistics.mean(attn_ms), 4)},
         "timing_ms": {"step": spread(step_ms), "attention": spread(attn_ms), "prediction": spread(pre_ms)},
@@ -814,6 +843,8 @@ def main():
     ap.add_argument("--sweep", default=None,
                     help="attention throughput against block sparsity: 'all' or a comma list of workloads "
                          "(one JSON line per point instead of the headline line)")
+    ap.add_argument("--no-graphs", action="store_true",
+                    help="launch each kernel from the host every step instead of replaying CUDA graphs")
     ap.add_argument("--order-group", type=int, default=None,
                     help="work-order grouping of the mask rows (sa_mask_params.order_group); "
                          "default: the library's choice for the shape")

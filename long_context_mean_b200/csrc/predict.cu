@@ -309,7 +309,8 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-__global__ void __launch_bounds__(kRowThreads, 2) score_topcdf_kernel(
+template <bool LONG>
+__global__ void __launch_bounds__(kRowThreads, LONG ? 2 : 3) score_topcdf_kernel(
     const float* __restrict__ qhat, const float* __restrict__ khat, const float* __restrict__ sq,
     const float* __restrict__ sk, int64_t Hq, int64_t Hkv, int64_t nqb, int64_t nkb, int d,
     int P2, int G, float tau, float theta, RowRules rules, uint8_t* __restrict__ mask,
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) score_topcdf_kernel(
       }
       return need;
     };
-    if (nkb4 >= 8 * kRowThreads) {
+    if (LONG) {   // rows of at least 8 * kRowThreads blocks (the launch checks)
       // Long rows: four consecutive key blocks a thread, so a warp's 16-byte
       // load of one feature covers 128 blocks; kb pairs share a packed FMA
       // with the feature broadcast.
@@ -1170,15 +1171,17 @@ sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
   while (P2 < nkb) P2 <<= 1;
   const int G = score_rows_per_cta(P2);
   const size_t smem = score_smem_bytes((int)s.d, nkb, P2, G);
+  // Rows of at least 2048 blocks (8 x 256, counted with the padding to 4)
+  // score four blocks a thread; shorter rows two.
+  const bool long_rows = nkb4 >= 8 * kRowThreads;
+  auto kern = long_rows ? score_topcdf_kernel<true> : score_topcdf_kernel<false>;
   if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(score_topcdf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return set_error(SA_ERR_CUDA, "cudaFuncSetAttribute(score_topcdf_kernel) failed");
   }
   dim3 grid((unsigned)ceil_div(nqb, G), (unsigned)(s.B * s.Hq));
-  score_topcdf_kernel<<<grid, kRowThreads, smem, st>>>(
-      w.qhat, w.khat, w.sq, w.sk, s.Hq, s.Hkv, nqb, nkb, (int)s.d, P2, G, p.tau, p.theta,
-      make_rules(s, p), out.block_mask, w.counts, out.status);
+  kern<<<grid, kRowThreads, smem, st>>>(w.qhat, w.khat, w.sq, w.sk, s.Hq, s.Hkv, nqb, nkb, (int)s.d, P2, G, p.tau,
+                                        p.theta, make_rules(s, p), out.block_mask, w.counts, out.status);
   if ((e = check_launch("score_topcdf_kernel"))) return e;
   return launch_lists(s, p.bq, p.bk, p.order_group, w.counts, w.tmp, out, st);
 }

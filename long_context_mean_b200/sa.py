@@ -497,7 +497,8 @@ class Pipeline:
             self.ev_layout.record(st)
             self.side.wait_event(self.ev_layout)
             reorder(self.perm, v, self.vr, self.side)
-            v.record_stream(self.side)   # the caller's v stays allocated until the side stream has read it
+            if not torch.cuda.is_current_stream_capturing():
+                v.record_stream(self.side)   # the caller's v stays allocated until the side stream has read it
             self.ev_v.record(self.side)
             # Q and K are reordered (or reordered and quantised) by the
             # pooling pass of the prediction.
@@ -520,6 +521,27 @@ class Pipeline:
             block_sparse_attn(qr, kr, vr, self.shape, self.mask.struct, self.lam, self.scale, out, lse,
                               self.skip_log, self.flags, stream, ws=self.attn_ws, out_perm=out_perm)
         return out, lse
+
+    def capture(self, q, k, v):
+        """Capture ``run(q, k, v)`` into a CUDA graph: the inputs and the
+        pipeline's buffers are fixed, so ``replay()`` re-runs the whole path
+        (every kernel, the side stream included) with one launch from the
+        host.  q, k, v must stay allocated and keep their addresses while the
+        graph is used; write new inputs into them in place."""
+        import torch
+        self.run(q, k, v)              # one-time library setup outside the capture
+        torch.cuda.synchronize(q.device)
+        self._graph_inputs = (q, k, v)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, capture_error_mode="relaxed"):
+            self.run(q, k, v)
+        torch.cuda.synchronize(q.device)
+        return self.graph
+
+    def replay(self):
+        """Re-run the captured path on the current stream (see ``capture``)."""
+        self.graph.replay()
+        return self.out, self.lse
 
     def _predict_codes(self, perm, q, k, stream):
         reorder_predict_mask_q8(perm, q, k, self.qk8, self.q8, self.q_scales, self.k8, self.k_scales, self.shape,
