@@ -227,7 +227,11 @@ def run_ours(args, rank, world, local_rank):
     g = I.gen_qkv(w)
     host = {n: torch.from_numpy(g[n + "_bits"].view(np.int16)).view(torch.bfloat16).pin_memory() for n in "qkv"}
     q, k, v = (host[n].to(dev) for n in "qkv")
-    stream = torch.cuda.current_stream(dev)
+    # The step runs on a high-priority stream: the V reorder on the pipeline's
+    # (default-priority) side stream then takes the SM slots the prediction
+    # leaves free instead of competing with its HBM-bound pooling.
+    stream = torch.cuda.Stream(device=dev, priority=torch.cuda.Stream.priority_range()[1])
+    torch.cuda.set_stream(stream)
     pipe = sa.pipeline_for(w, device=dev, log_skips=True, qk8=args.qk8, order_group=args.order_group)
 
     # Calibration pass (untimed): mask, skip log, FLOPs, sparsity.
@@ -302,9 +306,10 @@ def run_ours(args, rank, world, local_rank):
         attn_stage(stream)
         torch.cuda.synchronize(dev)
         graphs = (torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph())
-        with torch.cuda.graph(graphs[0], capture_error_mode="relaxed"):
+        cap = torch.cuda.Stream(device=dev, priority=stream.priority)
+        with torch.cuda.graph(graphs[0], stream=cap, capture_error_mode="relaxed"):
             pred_stage(torch.cuda.current_stream(dev))
-        with torch.cuda.graph(graphs[1], capture_error_mode="relaxed"):
+        with torch.cuda.graph(graphs[1], stream=cap, capture_error_mode="relaxed"):
             attn_stage(torch.cuda.current_stream(dev))
         torch.cuda.synchronize(dev)
 

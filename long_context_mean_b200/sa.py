@@ -533,7 +533,10 @@ class Pipeline:
         torch.cuda.synchronize(q.device)
         self._graph_inputs = (q, k, v)
         self.graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph, capture_error_mode="relaxed"):
+        # captured at high priority: the V reorder on the (default-priority)
+        # side stream then fills the SM slots the prediction leaves free
+        cap = torch.cuda.Stream(device=q.device, priority=torch.cuda.Stream.priority_range()[1])
+        with torch.cuda.graph(self.graph, stream=cap, capture_error_mode="relaxed"):
             self.run(q, k, v)
         torch.cuda.synchronize(q.device)
         return self.graph
