@@ -76,11 +76,24 @@ __device__ __forceinline__ void pairs16(const uint4& u, float, uint64_t* p) {
 // n of y8 and its scale (absmax / 127 or / 448) to qscale, reading the block
 // a second time (from L2) once its absmax is known.
 // ---------------------------------------------------------------------------
+// One pooled tensor of a launch (Q and K go through the same launch: their
+// units follow one another in one persistent grid).
+struct PoolJob {
+  const void* x;          // [BH, N, d]
+  int64_t BH;             // heads (batch x heads); 0: no job
+  int b, nB;              // block size, blocks per head
+  float* mean_out;        // block means, layout per mean_tstride
+  int64_t mean_tstride;   // 0: [BH, nB, d]; > 0: [BH, d, mean_tstride]
+  float* s_out;           // block similarities [BH, nB]
+  void* y;                // reordered copy (nullable)
+  uint2* y8;              // 8-bit codes (QF)
+  float* qscale;          // block scales (QF)
+};
+
 template <typename T, int CH, int QF = 0>
-__global__ void __launch_bounds__(kPoolThreads, 4) pool_cossim_kernel(
-    const T* __restrict__ x, int64_t BH, int64_t N, int b, int nB, float* __restrict__ mean_out,
-    int64_t mean_tstride, float* __restrict__ s_out, const int32_t* __restrict__ perm, T* __restrict__ y,
-    int32_t* status, uint2* __restrict__ y8 = nullptr, float* __restrict__ qscale = nullptr) {
+__global__ void __launch_bounds__(kPoolThreads, 4) pool_cossim_kernel(PoolJob j0, PoolJob j1, int64_t N,
+                                                                       const int32_t* __restrict__ perm,
+                                                                       int32_t* status) {
   constexpr int EPL = 16 / sizeof(T);   // elements per chunk
   constexpr int NP = EPL / 2;           // fp32 pairs per chunk
   constexpr int d = CH * EPL;
@@ -90,9 +103,21 @@ __global__ void __launch_bounds__(kPoolThreads, 4) pool_cossim_kernel(
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane / CH, c = lane % CH;
   int32_t* srow = srow_all[warp];
-  const int64_t units = BH * nB;
+  const int64_t units0 = j0.BH * j0.nB;
+  const int64_t units = units0 + j1.BH * j1.nB;
   const int64_t wstride = (int64_t)gridDim.x * kPoolWarps;
-  for (int64_t unit = (int64_t)blockIdx.x * kPoolWarps + warp; unit < units; unit += wstride) {
+  for (int64_t gunit = (int64_t)blockIdx.x * kPoolWarps + warp; gunit < units; gunit += wstride) {
+    const bool second = gunit >= units0;
+    const int64_t unit = second ? gunit - units0 : gunit;
+    const T* __restrict__ x = static_cast<const T*>(second ? j1.x : j0.x);
+    const int b = second ? j1.b : j0.b;
+    const int nB = second ? j1.nB : j0.nB;
+    float* __restrict__ mean_out = second ? j1.mean_out : j0.mean_out;
+    const int64_t mean_tstride = second ? j1.mean_tstride : j0.mean_tstride;
+    float* __restrict__ s_out = second ? j1.s_out : j0.s_out;
+    T* __restrict__ y = static_cast<T*>(second ? j1.y : j0.y);
+    uint2* __restrict__ y8 = second ? j1.y8 : j0.y8;
+    float* __restrict__ qscale = second ? j1.qscale : j0.qscale;
     const int64_t bh = unit / nB;
     const int blk = (int)(unit - bh * nB);
     const int64_t t0 = (int64_t)blk * b;
@@ -1062,43 +1087,36 @@ sa_status pool_grid(K kernel, int64_t units, unsigned* grid) {
 }
 
 template <typename T, int CH, int QF>
-sa_status launch_pool_ch(const void* x, int64_t BH, int64_t N, int b, int64_t nB, float* mean,
-                         int64_t mean_tstride, float* sim, const int32_t* perm, void* y, int32_t* status,
-                         uint2* y8, float* qscale, cudaStream_t st) {
+sa_status launch_pool_ch(const PoolJob& j0, const PoolJob& j1, int64_t N, const int32_t* perm, int32_t* status,
+                         cudaStream_t st) {
   unsigned grid = 0;
-  if (sa_status e = pool_grid(pool_cossim_kernel<T, CH, QF>, BH * nB, &grid)) return e;
-  pool_cossim_kernel<T, CH, QF><<<grid, kPoolThreads, 0, st>>>(static_cast<const T*>(x), BH, N, b, (int)nB,
-                                                               mean, mean_tstride, sim, perm, static_cast<T*>(y),
-                                                               status, y8, qscale);
+  if (sa_status e = pool_grid(pool_cossim_kernel<T, CH, QF>, j0.BH * j0.nB + j1.BH * j1.nB, &grid)) return e;
+  pool_cossim_kernel<T, CH, QF><<<grid, kPoolThreads, 0, st>>>(j0, j1, N, perm, status);
   return check_launch("pool_cossim_kernel");
 }
 
+// Q and K pooled in one launch (plain or with their reordered copies).
 template <typename T>
-sa_status launch_pool(const void* x, int64_t BH, int64_t N, int d, int b, int64_t nB, float* mean,
-                      int64_t mean_tstride, float* sim, const int32_t* perm, void* y, int32_t* status,
+sa_status launch_pool(const PoolJob& jq, const PoolJob& jk, int64_t N, int d, const int32_t* perm, int32_t* status,
                       cudaStream_t st) {
   switch (d / (16 / (int)sizeof(T))) {   // 16-byte chunks per token (validated: a power of two <= 32)
-    case 1: return launch_pool_ch<T, 1, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
-    case 2: return launch_pool_ch<T, 2, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
-    case 4: return launch_pool_ch<T, 4, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
-    case 8: return launch_pool_ch<T, 8, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
-    case 16: return launch_pool_ch<T, 16, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
-    case 32: return launch_pool_ch<T, 32, 0>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, y, status, nullptr, nullptr, st);
+    case 1: return launch_pool_ch<T, 1, 0>(jq, jk, N, perm, status, st);
+    case 2: return launch_pool_ch<T, 2, 0>(jq, jk, N, perm, status, st);
+    case 4: return launch_pool_ch<T, 4, 0>(jq, jk, N, perm, status, st);
+    case 8: return launch_pool_ch<T, 8, 0>(jq, jk, N, perm, status, st);
+    case 16: return launch_pool_ch<T, 16, 0>(jq, jk, N, perm, status, st);
+    case 32: return launch_pool_ch<T, 32, 0>(jq, jk, N, perm, status, st);
     default: return set_error(SA_ERR_UNSUPPORTED, "pooling: d must give a power-of-two count <= 32 of 16-byte chunks");
   }
 }
 
-// Pooling with 8-bit codes and block scales instead of the reordered copy
+// Pooling with 8-bit codes and block scales instead of the reordered copies
 // (bf16, d = 128: 16 chunks).
-sa_status launch_pool_codes(const void* x, int64_t BH, int64_t N, int d, int b, int64_t nB, float* mean,
-                            int64_t mean_tstride, float* sim, const int32_t* perm, int32_t fmt, void* y8,
-                            float* qscale, int32_t* status, cudaStream_t st) {
+sa_status launch_pool_codes(const PoolJob& jq, const PoolJob& jk, int64_t N, int d, const int32_t* perm,
+                            int32_t fmt, int32_t* status, cudaStream_t st) {
   if (d != 128) return set_error(SA_ERR_UNSUPPORTED, "8-bit codes need d = 128");
-  if (fmt == SA_Q_E4M3)
-    return launch_pool_ch<uint16_t, 16, 1 + SA_Q_E4M3>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, nullptr,
-                                                        status, static_cast<uint2*>(y8), qscale, st);
-  return launch_pool_ch<uint16_t, 16, 1 + SA_Q_INT8>(x, BH, N, b, nB, mean, mean_tstride, sim, perm, nullptr,
-                                                      status, static_cast<uint2*>(y8), qscale, st);
+  if (fmt == SA_Q_E4M3) return launch_pool_ch<uint16_t, 16, 1 + SA_Q_E4M3>(jq, jk, N, perm, status, st);
+  return launch_pool_ch<uint16_t, 16, 1 + SA_Q_INT8>(jq, jk, N, perm, status, st);
 }
 
 }  // namespace
@@ -1145,27 +1163,19 @@ sa_status launch_predict(const void* q, const void* k, const sa_shape& s,
   if (cudaMemsetAsync(out.status, 0, sizeof(int32_t), st) != cudaSuccess)
     return set_error(SA_ERR_CUDA, "cudaMemsetAsync(status) failed");
   sa_status e;
+  PoolJob jq{q, s.B * s.Hq, p.bq, (int)nqb, w.qhat, 0, w.sq, q_r, nullptr, nullptr};
+  PoolJob jk{k, s.B * s.Hkv, p.bk, (int)nkb, w.khat, nkb4, w.sk, k_r, nullptr, nullptr};
   if (codes) {   // bf16 input: codes and scales instead of reordered copies
-    if ((e = launch_pool_codes(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, 0, w.sq, perm, codes->format,
-                               codes->q8, codes->q_scales, out.status, st)))
-      return e;
-    if ((e = launch_pool_codes(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, nkb4, w.sk, perm, codes->format,
-                               codes->k8, codes->k_scales, out.status, st)))
-      return e;
+    jq.y = jk.y = nullptr;
+    jq.y8 = static_cast<uint2*>(codes->q8);
+    jq.qscale = codes->q_scales;
+    jk.y8 = static_cast<uint2*>(codes->k8);
+    jk.qscale = codes->k_scales;
+    if ((e = launch_pool_codes(jq, jk, s.N, (int)s.d, perm, codes->format, out.status, st))) return e;
   } else if (s.dtype == SA_BF16) {
-    if ((e = launch_pool<uint16_t>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, 0, w.sq, perm, q_r,
-                                   out.status, st)))
-      return e;
-    if ((e = launch_pool<uint16_t>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, nkb4, w.sk, perm, k_r,
-                                   out.status, st)))
-      return e;
+    if ((e = launch_pool<uint16_t>(jq, jk, s.N, (int)s.d, perm, out.status, st))) return e;
   } else {
-    if ((e = launch_pool<float>(q, s.B * s.Hq, s.N, (int)s.d, p.bq, nqb, w.qhat, 0, w.sq, perm, q_r,
-                                out.status, st)))
-      return e;
-    if ((e = launch_pool<float>(k, s.B * s.Hkv, s.N, (int)s.d, p.bk, nkb, w.khat, nkb4, w.sk, perm, k_r,
-                                out.status, st)))
-      return e;
+    if ((e = launch_pool<float>(jq, jk, s.N, (int)s.d, perm, out.status, st))) return e;
   }
   int P2 = 1;
   while (P2 < nkb) P2 <<= 1;
