@@ -329,8 +329,9 @@ def run_ours(args, rank, world, local_rank):
         e[2].record(stream)
         return e
 
-    # layout (1, Hilbert 3) + reorder V; pool Q, pool K, score, row scan, column fill, order; attention
-    launches_per_step = (0 if pipe.identity else (1 if w.order != "hilbert" else 3) + 1) + 6 + 1
+    # layout (1, Hilbert 3) + reorder V; pooling of Q and K (one launch), score, row scan, column
+    # fill, order; attention
+    launches_per_step = (0 if pipe.identity else (1 if w.order != "hilbert" else 3) + 1) + 5 + 1
     if args.qk8:
         launches_per_step += 1            # the tile-scale kernel (codes come from the pooling pass)
 
