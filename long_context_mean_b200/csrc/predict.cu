@@ -335,7 +335,7 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 template <bool LONG>
-__global__ void __launch_bounds__(kRowThreads, LONG ? 2 : 3) score_topcdf_kernel(
+__global__ void __launch_bounds__(kRowThreads, 2) score_topcdf_kernel(
     const float* __restrict__ qhat, const float* __restrict__ khat, const float* __restrict__ sq,
     const float* __restrict__ sk, int64_t Hq, int64_t Hkv, int64_t nqb, int64_t nkb, int d,
     int P2, int G, float tau, float theta, RowRules rules, uint8_t* __restrict__ mask,

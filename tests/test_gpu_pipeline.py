@@ -245,9 +245,17 @@ def test_video_large_hilbert_at_sparsity_085_sampled():
 
 
 def test_lm_causal_gqa_sampled():
+    """The causal 131K GQA workload: whole-head masks for four heads (KV heads
+    0, 2, 4 and 7), attention on seven query blocks of each, and the grouped
+    work order of all 32,768 rows bit-exact against the oracle's."""
     w = I.WORKLOADS["lm_causal"]
     nqb = -(-w.N // w.bq)
-    _sampled_heads_check(w, [(0, 0), (0, 29)], lambda h: h // (w.Hq // w.Hkv), [0, 1, 40, 513, nqb - 1])
+    pipe = _sampled_heads_check(w, [(0, 0), (0, 9), (0, 18), (0, 29)], lambda h: h // (w.Hq // w.Hkv),
+                                [0, 1, 40, 255, 513, 800, nqb - 1])
+    G = int(pipe.params.order_group)
+    assert G == 4
+    gmask = pipe.mask.block_mask.cpu().numpy().reshape(w.B, w.Hq, nqb, -1).astype(bool)
+    assert np.array_equal(pipe.mask.order.cpu().numpy(), Pr.mask_to_csr(gmask, G)["order"])
 
 
 @pytest.mark.parametrize("name,chunks", [("video", 4), ("lm_small", 2)])
