@@ -301,12 +301,13 @@ __device__ void finish_row(const uint8_t* flags, int64_t u, int64_t qb, int64_t 
 // for every row r of the group, reading k_hat (stored transposed, feature-
 // major, L2-resident, each element read once per group: a warp's load of a
 // feature is one 128-byte line) and the q_hat rows from shared memory (the
-// same address in every lane: broadcast, four features per load), so the
-// loop is bound by the FMA pipe.  Then warp r alone finishes row r: softmax and
-// TopCdf (an arg-max loop over register-resident keys when the row is short
-// and few blocks are picked, else a bisection for the last kept
-// probability), the union with the forced parts and the causal AND -- with
-// warp-level synchronisation only.
+// same address in every lane: broadcast, four features per load), with the
+// FMAs on the packed fp32x2 pipe.  Then warp r alone finishes row r: softmax
+// and TopCdf (an arg-max loop over register-resident keys when the row is
+// short and few blocks are picked, else a search for the last kept
+// probability: bisection over bit patterns while many candidates remain, then
+// steps that test the remaining candidates' own values), the union with the
+// forced parts and the causal AND -- with warp-level synchronisation only.
 // Dynamic shared memory: q_hat [8][d] | scores [G][nkb rounded to 4] (fp32;
 // the bisection turns a row's scores into its probabilities in place, the
 // padding holding zeros) | flags [G][nkb rounded to 16] (u8).
@@ -596,9 +597,33 @@ __global__ void __launch_bounds__(kRowThreads, 2) score_topcdf_kernel(
         count = __reduce_add_sync(0xffffffffu, c);
         return m;
       };
+      // The bisection starts at e = (1 - tau) / (4 n) instead of 0 (n = 4
+      // nq_row entries): the p <= e sum to at most (1 - tau) / 4, and total
+      // >= max p = 1, so f(e) >= tau * total + 0.75 (1 - tau) total -- above
+      // the limit by far more than the rounding of the sums while 1 - tau >=
+      // 1e-3 (otherwise the start stays 0).  The first pass takes the total,
+      // f(0), and the number of p above e together.
+      const uint32_t lo0 = (tau <= 0.999f) ? __float_as_uint(0.25f * (1.f - tau) / (float)(4 * nq_row)) : 0u;
       int c_lo = 0, c_hi = 0, c_mid = 0;   // how many p have bits above lo, hi
-      const float limit = tau * pass_full(0u, c_lo);
-      uint32_t lo = 0u, hi = 0x3F800000u;   // f(lo) >= limit (tau <= 1), f(hi) = 0 < limit
+      float total;
+      {
+        float m0 = 0.f, m1 = 0.f;
+        int c = 0;
+        for (int q = lane; q < nq_row; q += 32) {
+          const float4 v = pr4[q];
+          const bool g0 = __float_as_uint(v.x) > 0u, g1 = __float_as_uint(v.y) > 0u;
+          const bool g2 = __float_as_uint(v.z) > 0u, g3 = __float_as_uint(v.w) > 0u;
+          m0 += (g0 ? v.x : 0.f) + (g1 ? v.y : 0.f);
+          m1 += (g2 ? v.z : 0.f) + (g3 ? v.w : 0.f);
+          c += (int)(__float_as_uint(v.x) > lo0) + (int)(__float_as_uint(v.y) > lo0) +
+               (int)(__float_as_uint(v.z) > lo0) + (int)(__float_as_uint(v.w) > lo0);
+        }
+        total = m0 + m1;
+        for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
+        c_lo = __reduce_add_sync(0xffffffffu, c);
+      }
+      const float limit = tau * total;
+      uint32_t lo = lo0, hi = 0x3F800000u;   // f(lo) >= limit (tau <= 1), f(hi) = 0 < limit
       float f_hi = 0.f;                     // f(hi)
       while (hi - lo > 1u && c_lo - c_hi > kSelectRegs * 32) {
         const uint32_t mid = lo + (hi - lo) / 2u;
@@ -633,8 +658,28 @@ __global__ void __launch_bounds__(kRowThreads, 2) score_topcdf_kernel(
 #pragma unroll
         for (int j = 0; j < kSelectRegs; ++j) cv[j] = lane + 32 * j < n ? cbuf[lane + 32 * j] : 0.f;
         const float f_base = f_hi;   // f(hi) on entry: every gathered p is <= hi
-        while (hi - lo > 1u) {
-          const uint32_t mid = lo + (hi - lo) / 2u;
+        // f only changes at the gathered values, so the boundary is one of
+        // them (or hi): each step tests a candidate strictly inside (lo, hi),
+        // taken from a rotating lane, which then leaves the interval; the
+        // search ends when none is left (at most kSelectRegs * 32 steps) and
+        // reaches the same hi as a bisection over the bit patterns.
+        for (int step = 0;; ++step) {
+          float piv = 0.f;
+          bool has = false;
+#pragma unroll
+          for (int j = kSelectRegs - 1; j >= 0; --j) {
+            const uint32_t bj = __float_as_uint(cv[j]);
+            if (bj > lo && bj < hi) {
+              piv = cv[j];
+              has = true;
+            }
+          }
+          const unsigned bal = __ballot_sync(0xffffffffu, has);
+          if (bal == 0u) break;
+          const int rot = (step * 13) & 31;
+          const unsigned rb = (bal >> rot) | (bal << ((32 - rot) & 31));
+          const int src = (__ffs((int)rb) - 1 + rot) & 31;
+          const uint32_t mid = __float_as_uint(__shfl_sync(0xffffffffu, piv, src));
           float s = 0.f;
 #pragma unroll
           for (int j = 0; j < kSelectRegs; ++j) s += __float_as_uint(cv[j]) > mid ? cv[j] : 0.f;
