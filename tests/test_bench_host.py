@@ -53,3 +53,20 @@ def test_workload_config_names_the_sizes():
     assert c["seq_len"] == w.N == 20506 and c["global_batch"] == 2 * w.B
     assert "N=20506" in c["workload"] and "[13,30,52]+226" in c["workload"]
     assert c["parallelism"] == "replicas x2" and "flushed" in c["l2"]
+
+
+def test_cpu_baseline_samples_heads_in_turn():
+    """The CPU baseline walks query heads in turn and reads each one's own kv
+    head (GQA), timing only the oracle's attention."""
+    w = I.WORKLOADS["toy"].with_(Hq=4, Hkv=2, generator="lowrank", rank=4, sigma_pos=4.0)
+    g = I.gen_qkv(w)
+    q, k, v, m = bench.oracle_sample_setup(w, g, head=3)
+    from oracle import layout as Y
+    perm, _ = Y.build_layout(w.order, w.T, w.H, w.W, w.win, w.sink_frames, w.txt_len)
+    assert np.array_equal(q, Y.reorder(g["q"][:1, 3:4], perm))
+    assert np.array_equal(k, Y.reorder(g["k"][:1, 1:2], perm))
+    assert np.array_equal(v, Y.reorder(g["v"][:1, 1:2], perm))
+    r = bench.cpu_baseline(w, g, seconds=1e9)     # every block of every head
+    nqb = -(-w.N // w.bq)
+    assert f"of {4 * nqb} random query blocks of query heads 0-3" in r["sample"]
+    assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1
