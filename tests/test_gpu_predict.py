@@ -102,6 +102,8 @@ SMALL = [
     ("threshold_search", 1, 2, 2, 6000, 64, 32, 8, 0.9, 0.0, False, 0, 0, 0, 0, "bf16"),
     ("threshold_causal", 1, 2, 1, 6000, 64, 32, 8, 0.95, 0.0, True, 0, 0, 64, 8, "bf16"),
     ("threshold_low_tau", 1, 2, 2, 6000, 64, 32, 8, 0.25, 0.0, False, 0, 0, 0, 0, "bf16"),
+    # above tau = 0.999 the threshold search starts at 0 (no lower start)
+    ("threshold_near_one", 1, 2, 2, 6000, 64, 32, 8, 0.9995, 0.0, False, 0, 0, 0, 0, "bf16"),
     # 2048 key blocks: the scores of four consecutive blocks per thread
     ("long_rows", 1, 2, 1, 16384, 32, 64, 8, 0.9, 0.0, True, 0, 0, 128, 16, "bf16"),
 ]
